@@ -1,0 +1,68 @@
+"""Per-head mask construction for each workload kind (test infrastructure).
+
+``head_mask(wl, q, k, head)`` takes one head's q and k as float32 [N, d]
+(bf16 values, original token order) and returns the working order, the block
+mask and the intermediate values that decide it.
+"""
+import numpy as np
+
+from . import layout, masks
+
+
+def working_order(wl, head, tile=None):
+    """Slot -> original token for this head's working layout."""
+    if wl.kind in ("topk", "sta", "spade"):
+        bt, bh, bw = tile if tile is not None else wl.tile
+        return layout.tile_order(wl.T, wl.H, wl.W, bt, bh, bw)
+    if wl.kind == "spatiotemporal" and head in wl.temporal_heads:
+        return layout.frame_major_order(wl.T, wl.H, wl.W, wl.block)
+    return layout.identity_order(wl.T, wl.H, wl.W, wl.block)
+
+
+def head_mask(wl, q, k, head):
+    d = wl.head_dim
+    info = {}
+    if wl.kind == "fg":
+        s = masks.fg_scores(q, k, wl.fg_group)
+        tau, r = masks.fg_threshold(s, wl.fg_keep_fraction)
+        info.update(scores=s, tau=tau, rank=r)
+        return dict(keep_groups=masks.fg_keep(s, tau), info=info)
+
+    tile = None
+    if wl.kind == "spade":
+        totals = []
+        for cand in wl.candidates:
+            blk_c = layout.blocks(working_order(wl, head, cand), wl.block)
+            totals.append(float(masks.sics(k, blk_c).astype(np.float64).sum()))
+        choice = masks.choose_candidate(totals)
+        info.update(sics_totals=totals, choice=choice)
+        tile = wl.candidates[choice]
+
+    order = working_order(wl, head, tile)
+    blk = layout.blocks(order, wl.block)
+    valid = masks.valid_blocks(blk)
+
+    if wl.kind == "topk":
+        s = masks.pooled_scores(masks.block_means(q, blk), masks.block_means(k, blk), d)
+        info["scores"] = s
+        bm = masks.topk_with_diagonal(s, wl.topk, wl.keep_diagonal, valid, valid)
+    elif wl.kind == "sta":
+        dims = layout.tile_grid_dims(wl.T, wl.H, wl.W, *wl.tile)
+        bm = masks.tile_window(dims, wl.window, valid, valid)
+    elif wl.kind == "spatiotemporal":
+        if head in wl.temporal_heads:
+            bm = masks.temporal_rule(blk, wl.T, wl.H, wl.W)
+        else:
+            bm = masks.spatial_rule(blk, wl.T, wl.H, wl.W)
+        bm = masks.add_sinks(bm, blk, wl.sink_tokens, wl.block)
+    elif wl.kind == "spade":
+        s = masks.pooled_scores(masks.block_means(q, blk), masks.block_means(k, blk), d)
+        info["scores"] = s
+        dims = layout.tile_grid_dims(wl.T, wl.H, wl.W, *tile)
+        bm = masks.tile_window(dims, wl.window, valid, valid)
+        for i in range(blk.shape[0]):
+            if valid[i]:
+                bm[i] |= masks.top_p_row(s[i], valid, wl.top_p)
+    else:
+        raise ValueError(wl.kind)
+    return dict(order=order, order_blocks=blk, bmask=bm, tile=tile, info=info)

@@ -1,0 +1,273 @@
+"""Pins for the oracle's mask construction (CPU only).
+
+Closed forms (tests/golden/mask_counts.json), brute force on tiny inputs,
+library routines (torch.mean, torch.topk-free sorting by numpy argsort) and
+invariants (Top-P minimality, FG keep count) pin every rule.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import layout, masks, pipeline
+from synthetic import CONFIGS, make_qkv, bf16_bits_to_f32
+
+GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "mask_counts.json")))
+
+
+# ---------------------------------------------------------------- pooling
+def test_block_means_match_torch_mean_over_valid_tokens():
+    g = np.random.default_rng(0)
+    x = g.standard_normal((37, 8)).astype(np.float32)
+    order = np.full(48, -1)
+    order[:37] = g.permutation(37)
+    blk = order.reshape(6, 8)
+    got = masks.block_means(x, blk)
+    for b in range(6):
+        idx = blk[b][blk[b] >= 0]
+        if len(idx) == 0:
+            assert np.all(got[b] == 0.0)
+            continue
+        ref = torch.from_numpy(x[idx]).mean(dim=0).numpy()
+        np.testing.assert_allclose(got[b], ref, rtol=1e-6, atol=1e-7)
+
+
+def test_block_means_all_padding_block_is_zero():
+    x = np.ones((4, 3), np.float32)
+    blk = np.array([[0, 1], [-1, -1], [2, 3]])
+    np.testing.assert_array_equal(masks.block_means(x, blk)[1], 0.0)
+
+
+# ---------------------------------------------------------------- SICS
+def _sics_bruteforce(k, idx):
+    u = [k[i].astype(np.float64) / np.linalg.norm(k[i].astype(np.float64)) for i in idx]
+    return sum(float(np.dot(u[a], u[b])) for a in range(len(u)) for b in range(len(u)) if a != b)
+
+
+def test_sics_equals_pairwise_cosine_sum():
+    # SPADE review, Eqs. 3-5: the O(BS*d) partial-sum form equals the O(BS^2*d)
+    # sum of pairwise cosine similarities.
+    g = np.random.default_rng(1)
+    k = (g.standard_normal((70, 16)) + 0.7).astype(np.float32)
+    order = np.full(80, -1)
+    order[:70] = np.arange(70)
+    blk = order.reshape(5, 16)
+    got = masks.sics(k, blk)
+    for b in range(5):
+        idx = blk[b][blk[b] >= 0]
+        ref = _sics_bruteforce(k, idx)
+        assert abs(got[b] - ref) <= 1e-5 * max(1.0, abs(ref)), (b, got[b], ref)
+
+
+def test_sics_special_cases():
+    n, d = 10, 12
+    same = np.tile(np.arange(1, d + 1, dtype=np.float32), (n, 1))      # identical directions
+    scaled = same * np.arange(1, n + 1, dtype=np.float32)[:, None]      # positive rescales
+    ortho = np.eye(d, dtype=np.float32)[:n] * 3.0                       # orthogonal set
+    blk = np.arange(n)[None, :]
+    assert abs(masks.sics(same, blk)[0] - n * (n - 1)) < 1e-3
+    assert abs(masks.sics(scaled, blk)[0] - n * (n - 1)) < 1e-3
+    assert abs(masks.sics(ortho, blk)[0]) < 1e-5
+    anti = np.concatenate([same[:5], -same[:5]])                        # cancelling pairs
+    assert abs(masks.sics(anti, blk)[0] - (-10.0)) < 1e-3               # |0|^2 - 10
+
+
+def test_sics_zero_vector_contributes_nothing():
+    k = np.array([[1, 0], [0, 0], [1, 0]], np.float32)
+    assert abs(masks.sics(k, np.array([[0, 1, 2]]))[0] - 2.0) < 1e-6   # one ordered pair each way
+
+
+def test_choose_candidate_ties_and_order():
+    assert masks.choose_candidate([1.0, 3.0, 2.0]) == 1
+    assert masks.choose_candidate([5.0, 5.0 * (1 + 5e-5), 1.0]) == 0    # within 1e-4: first wins
+    assert masks.choose_candidate([5.0, 5.0 * (1 + 5e-4), 1.0]) == 1
+
+
+# ---------------------------------------------------------------- pooled scores / Top-K
+def test_pooled_scores_scale():
+    qb = np.array([[1, 2, 3, 4]], np.float32)
+    kb = np.array([[1, 1, 1, 1], [0, 0, 0, 2]], np.float32)
+    np.testing.assert_allclose(masks.pooled_scores(qb, kb, 4), [[5.0, 4.0]])
+
+
+def test_topk_matches_stable_argsort_and_diagonal():
+    g = np.random.default_rng(2)
+    s = g.standard_normal((6, 6)).astype(np.float32)
+    s[2, 4] = s[2, 1]                                  # a tie: lower index ranks first
+    valid = np.ones(6, bool)
+    m = masks.topk_with_diagonal(s, 2, True, valid, valid)
+    for i in range(6):
+        order = np.argsort(-s[i].astype(np.float64), kind="stable")
+        ref = set(order[:2].tolist()) | {i}
+        assert set(np.nonzero(m[i])[0].tolist()) == ref
+
+
+def test_tiny_config_brute_force_mask():
+    # Tiny workload: every token's tile found from its coordinates, tile means
+    # summed token by token, all 4 key tiles enumerated.
+    wl = CONFIGS["tiny_topk"]
+    x = make_qkv(wl)
+    for head in range(wl.heads):
+        q = bf16_bits_to_f32(x["q"][0, head])
+        k = bf16_bits_to_f32(x["k"][0, head])
+        res = pipeline.head_mask(wl, q, k, head)
+        qs = np.zeros((4, wl.head_dim)); ks = np.zeros((4, wl.head_dim)); cnt = np.zeros(4)
+        for t, h, w in itertools.product(range(4), range(8), range(8)):
+            tile = (t // 2) * 2 + (h // 4)                 # tile grid 2 x 2 x 1
+            n = (t * 8 + h) * 8 + w
+            qs[tile] += q[n]; ks[tile] += k[n]; cnt[tile] += 1
+        sc = (qs / cnt[:, None]) @ (ks / cnt[:, None]).T / 8.0
+        for i in range(4):
+            ranked = sorted(range(4), key=lambda j: (-sc[i, j], j))
+            ref = set(ranked[:2]) | {i}
+            assert set(np.nonzero(res["bmask"][i])[0].tolist()) == ref
+            assert 2 <= res["bmask"][i].sum() <= 3
+
+
+# ---------------------------------------------------------------- static rules
+def test_sta_closed_form_count():
+    wl = CONFIGS["sta_wan21_1p3b_480p"]
+    ref = GOLDEN["sta_wan21_1p3b_480p"]
+    res = pipeline.head_mask(wl, None, None, 0)
+    assert res["bmask"].shape == (ref["blocks_per_head"],) * 2
+    assert int(res["bmask"].sum()) == ref["kept_pairs_per_head"]
+    # "no mixed blocks": each kept tile pair is a full tile pair of the window
+    assert abs(res["bmask"].mean() - 0.0592) < 1e-4
+
+
+def test_sta_window_brute_force_on_small_grid():
+    dims = (3, 4, 2)
+    n = 24
+    valid = np.ones(n, bool)
+    m = masks.tile_window(dims, (3, 3, 3), valid, valid)
+    coords = list(itertools.product(range(3), range(4), range(2)))
+    for i, a in enumerate(coords):
+        for j, b in enumerate(coords):
+            assert m[i, j] == all(abs(x - y) <= 1 for x, y in zip(a, b))
+
+
+@pytest.mark.slow
+def test_spatial_temporal_closed_form_counts():
+    wl = CONFIGS["spatiotemporal_hunyuan_720p"]
+    sp = pipeline.head_mask(wl, None, None, 0)
+    tp = pipeline.head_mask(wl, None, None, 12)
+    assert int(sp["bmask"].sum()) == GOLDEN["spatiotemporal_hunyuan_720p_spatial"]["kept_pairs_per_head"]
+    assert int(tp["bmask"].sum()) == GOLDEN["spatiotemporal_hunyuan_720p_temporal"]["kept_pairs_per_head"]
+    # spatial: frame block-diagonal band; temporal: at most 3 overlap blocks + 2 sinks
+    assert tp["bmask"].sum(axis=1).max() <= 5
+    assert sp["bmask"][0, 0] and sp["bmask"][0, 59] and not sp["bmask"][0, 60]
+
+
+def test_temporal_rule_small_grid_brute_force():
+    T, H, W, bs = 3, 2, 5, 4
+    order = layout.frame_major_order(T, H, W, bs)
+    blk = layout.blocks(order, bs)
+    m = masks.temporal_rule(blk, T, H, W)
+    for i in range(blk.shape[0]):
+        for j in range(blk.shape[0]):
+            pi = {n % (H * W) for n in blk[i] if n >= 0}
+            pj = {n % (H * W) for n in blk[j] if n >= 0}
+            assert m[i, j] == bool(pi & pj)
+
+
+def test_sinks_are_whole_blocks_of_the_working_layout():
+    blk = np.arange(12).reshape(4, 3)
+    m = masks.add_sinks(np.eye(4, dtype=bool), blk, sink_tokens=4, block=3)
+    assert m[:, 0].all() and m[:, 1].all() and not m[3, 2]
+
+
+# ---------------------------------------------------------------- Top-P
+def _check_top_p(row, valid, p, kept):
+    cols = np.nonzero(valid)[0]
+    e = np.exp(row[cols].astype(np.float64) - row[cols].max())
+    prob = e / e.sum()
+    pk = prob[kept[cols]]
+    pn = prob[~kept[cols]]
+    assert pk.sum() >= p - 1e-5                                       # reaches p
+    assert pk.sum() - pk.min() < p + 1e-5                             # minimal prefix
+    if len(pn):
+        assert pk.min() >= pn.max() - 1e-7                            # a prefix of the order
+
+
+def test_top_p_invariants_random_rows():
+    g = np.random.default_rng(3)
+    for trial in range(200):
+        n = int(g.integers(1, 60))
+        row = (g.standard_normal(n) * g.uniform(0.1, 4)).astype(np.float32)
+        valid = g.random(n) < 0.8
+        if not valid.any():
+            valid[0] = True
+        kept = masks.top_p_row(row, valid, 0.9)
+        assert not kept[~valid].any()
+        _check_top_p(row, valid, 0.9, kept)
+
+
+def test_top_p_single_dominant_and_uniform():
+    row = np.array([10.0, 0.0, 0.0, 0.0], np.float32)
+    assert masks.top_p_row(row, np.ones(4, bool), 0.9).tolist() == [True, False, False, False]
+    row = np.zeros(10, np.float32)                                    # uniform: 9 of 10 reach 0.9
+    k = masks.top_p_row(row, np.ones(10, bool), 0.9)
+    assert k.sum() in (9, 10) and k[:9].all()                         # float32 sum of 0.1s
+
+
+# ---------------------------------------------------------------- FG slices
+def test_fg_threshold_keep_count_and_sort():
+    g = np.random.default_rng(4)
+    n, d, group = 300, 16, 8
+    q = g.standard_normal((n, d)).astype(np.float32)
+    k = g.standard_normal((n, d)).astype(np.float32)
+    s = masks.fg_scores(q, k, group)
+    assert s.shape == (math.ceil(n / group), n)
+    tau, r = masks.fg_threshold(s, 0.15)
+    assert r == math.ceil(0.15 * s.size)
+    srt = np.sort(s.reshape(-1))[::-1]
+    assert tau == srt[r - 1]
+    kept = masks.fg_keep(s, tau)
+    assert kept.sum() == r + int((srt[r:] == tau).sum())
+
+
+def test_fg_scores_use_group_mean_query():
+    g = np.random.default_rng(5)
+    q = g.standard_normal((10, 4)).astype(np.float32)
+    k = g.standard_normal((10, 4)).astype(np.float32)
+    s = masks.fg_scores(q, k, 4)                                      # groups 0-3, 4-7, 8-9
+    qbar = np.stack([q[0:4].mean(0), q[4:8].mean(0), q[8:10].mean(0)])
+    np.testing.assert_allclose(s, qbar @ k.T / 2.0, rtol=1e-5, atol=1e-6)
+
+
+# ---------------------------------------------------------------- SPADE pipeline on a small grid
+def test_spade_small_grid_pipeline_invariants():
+    from synthetic import Workload
+    wl = Workload(name="spade_small", config_id=99, T=5, H=9, W=16, heads=2, head_dim=32,
+                  kind="spade", block=32, candidates=((1, 4, 8), (4, 2, 4), (2, 4, 4)),
+                  top_p=0.9, window=(3, 3, 3))
+    x = make_qkv(wl)
+    for head in range(2):
+        q = bf16_bits_to_f32(x["q"][0, head]); k = bf16_bits_to_f32(x["k"][0, head])
+        res = pipeline.head_mask(wl, q, k, head)
+        info = res["info"]
+        # the choice is the argmax of the per-candidate SICS totals, each recomputed
+        # here by brute-force pairwise cosines
+        totals = []
+        for cand in wl.candidates:
+            blk = layout.blocks(pipeline.working_order(wl, head, cand), wl.block)
+            totals.append(sum(_sics_bruteforce(k, b[b >= 0]) for b in blk))
+        np.testing.assert_allclose(info["sics_totals"], totals, rtol=1e-4)
+        assert info["choice"] == int(np.argmax(totals))
+        blk = res["order_blocks"]
+        valid = masks.valid_blocks(blk)
+        dims = layout.tile_grid_dims(wl.T, wl.H, wl.W, *res["tile"])
+        win = masks.tile_window(dims, wl.window, valid, valid)
+        for i in range(blk.shape[0]):
+            if not valid[i]:
+                assert not res["bmask"][i].any()
+                continue
+            assert (res["bmask"][i] >= win[i]).all()
+            extra = res["bmask"][i]
+            tp = masks.top_p_row(info["scores"][i], valid, 0.9)
+            np.testing.assert_array_equal(extra, tp | win[i])
+            _check_top_p(info["scores"][i], valid, 0.9, tp)
