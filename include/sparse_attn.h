@@ -1,0 +1,228 @@
+/*
+ * sparse_attn.h - C ABI of the B200 (sm_100a) mask-driven sparse attention
+ * library for video diffusion transformers.
+ *
+ * The library computes, for every batch item b, head h and query token i of a
+ * T x H x W latent token grid,
+ *
+ *     O[b,h,i]   = sum_{j in K(i)} softmax_j(q_i . k_j / sqrt(d)) v_j
+ *     LSE[b,h,i] = ln sum_{j in K(i)} exp(q_i . k_j / sqrt(d))
+ *
+ * where K(i) is the set of keys the mask keeps for token i. The mask is built
+ * on the device by one of the policies below, then a flash-style attention
+ * kernel with online softmax visits only the kept key tiles (block masks) or
+ * the kept keys (M x 1 key slices).
+ *
+ * Sources of each policy (pith.science review pages of the papers):
+ *   SA_MASK_STA            "Fast Video Generation with Sliding Tile Attention"
+ *                          (arXiv 2502.04507), key machinery: 3D tiles equal to
+ *                          one attention block, fixed window of neighbour tiles.
+ *   SA_MASK_SPATIOTEMPORAL "Sparse VideoGen" (arXiv 2502.01776), key machinery
+ *                          and core discovery: spatial heads (own frame) and
+ *                          temporal heads (same position across frames, after a
+ *                          token-major to frame-major layout transform).
+ *   SA_MASK_TOPK, SA_MASK_SPADE
+ *                          "SPADE: An Input-Adaptive Sparse Attention Engine for
+ *                          Fast Video Diffusion Models Inference" (arXiv
+ *                          2608.03335), "Core claim" and "What carries the
+ *                          argument", Eqs. 3-5: 3D blocking candidates chosen by
+ *                          SICS, mean-pooled block summaries, head-wise
+ *                          Top-K/Top-P plus a local window.
+ *   SA_MASK_FG             "FG-Attn: Leveraging Fine-Grained Sparse Attention in
+ *                          Video Diffusion Models" (arXiv 2509.16518), skeptic
+ *                          critique and referee major comment 2 on Sec. 4.4:
+ *                          M x 1 key slices kept by k . q_avg / sqrt(D) against
+ *                          a threshold.
+ *
+ * Conventions for every entry point:
+ *   - Tensors Q, K, V, O are contiguous [batch, heads, N, head_dim] bf16 in the
+ *     original token order n = (t*H + h)*W + w, N = T*H*W. LSE is contiguous
+ *     [batch, heads, N] fp32, natural log. All are device pointers.
+ *   - head_dim is 64 or 128. N, and every tensor base pointer, is such that
+ *     rows are 16-byte aligned (always true for contiguous bf16 tensors with
+ *     these head dims and a 16-byte aligned base).
+ *   - The caller owns and allocates every buffer, including both workspaces,
+ *     whose sizes sparse_attn_workspace_size() returns. The library allocates
+ *     no device memory and keeps no global state between calls.
+ *   - ``stream`` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream. Work is enqueued asynchronously on it.
+ *   - Argument errors are detected on the host before anything is enqueued and
+ *     returned synchronously. Device-side failures (a bounded wait that ran
+ *     out, an index check that failed) set bits in a status word inside the
+ *     scratch workspace, read by sparse_attn_status(). No kernel traps.
+ *   - Not supported: backward, causal masking, grouped-query attention,
+ *     variable-length batches, dropout.
+ */
+#ifndef SPARSE_ATTN_H_
+#define SPARSE_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SA_API __attribute__((visibility("default")))
+#else
+#define SA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------- status */
+enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,     /* a null pointer, a bad size or a bad policy field   */
+  SA_ERR_UNSUPPORTED = 2,     /* valid but not implemented (e.g. head_dim 96)      */
+  SA_ERR_WORKSPACE = 3,       /* workspace pointer misaligned                      */
+  SA_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed                 */
+  SA_ERR_DEVICE_TIMEOUT = 5,  /* a kernel's bounded wait ran out (status word)     */
+  SA_ERR_DEVICE_BOUNDS = 6    /* a kernel's index check failed (status word)       */
+};
+
+/* ---------------------------------------------------------------- problem */
+typedef struct {
+  int batch;     /* >= 1                                                     */
+  int heads;     /* >= 1                                                     */
+  int T, H, W;   /* latent grid; N = T*H*W tokens                             */
+  int head_dim;  /* 64 or 128                                                */
+} sa_problem;
+
+/* ---------------------------------------------------------------- policy */
+enum {
+  SA_MASK_TOPK = 1,           /* diagonal + Top-K key tiles by mean-pooled q.k    */
+  SA_MASK_STA = 2,            /* sliding 3D tile window                           */
+  SA_MASK_SPATIOTEMPORAL = 3, /* spatial / temporal heads + sink blocks           */
+  SA_MASK_SPADE = 4,          /* SICS blocking choice + Top-P + tile window       */
+  SA_MASK_FG = 5,             /* M x 1 key slices by group-mean-query threshold   */
+  SA_MASK_EXPLICIT = 6        /* caller-supplied block bitmask                    */
+};
+
+enum {
+  SA_LAYOUT_IDENTITY = 0,     /* blocks of consecutive tokens in original order   */
+  SA_LAYOUT_FRAME_MAJOR = 1,  /* slot m = (h*W + w)*T + t                         */
+  SA_LAYOUT_TILE = 2          /* 3D tiles in raster order, raster inside a tile   */
+};
+
+typedef struct {
+  int kind;                   /* SA_MASK_*                                         */
+  int block;                  /* tokens per block: 128, or 64 (head_dim 64 only);
+                                 for tile layouts it must equal bt*bh*bw          */
+  int tile[3];                /* (bt, bh, bw): TOPK, STA, EXPLICIT+TILE            */
+  int topk;                   /* TOPK: number of key tiles by score (>= 1)         */
+  int keep_diagonal;          /* TOPK: also keep the query's own tile              */
+  int window[3];              /* STA, SPADE: odd window extents, in tiles          */
+  const int8_t* head_is_temporal; /* SPATIOTEMPORAL: host array [heads], 0 or 1    */
+  int sink_tokens;            /* SPATIOTEMPORAL: leading working-layout slots that
+                                 every query keeps, rounded up to whole blocks    */
+  int frame_radius;           /* SPATIOTEMPORAL: spatial heads keep +-radius frames */
+  int n_candidates;           /* SPADE: 1..4 blockings                             */
+  int candidates[4][3];       /* SPADE: (bt, bh, bw) of each blocking              */
+  float top_p;                /* SPADE: probability mass to keep, in (0, 1]        */
+  int fg_group;               /* FG: queries per group (M), a multiple of 64       */
+  float fg_keep_fraction;     /* FG: fraction of (group, key) slices kept, (0, 1]  */
+  int explicit_layout;        /* EXPLICIT: SA_LAYOUT_*                             */
+  const uint32_t* explicit_bits; /* EXPLICIT: device [batch*heads][nb][ceil(nb/32)],
+                                 bit j of row i keeps key block j for query block i */
+} sa_policy;
+
+/* ---------------------------------------------------------------- sizes
+ * Byte sizes of the two caller-owned device workspaces for this problem and
+ * policy. ``mask`` holds the built mask (position independent: it may be
+ * copied and reused by later forward calls with the same problem and policy).
+ * ``scratch`` holds intermediates and the status word. Both must be 256-byte
+ * aligned. Returns SA_OK or SA_ERR_INVALID_ARG / SA_ERR_UNSUPPORTED.
+ */
+SA_API int sparse_attn_workspace_size(const sa_problem* problem, const sa_policy* policy,
+                               size_t* mask_bytes, size_t* scratch_bytes);
+
+/* ---------------------------------------------------------------- mask
+ * Build the mask for ``policy`` from q and k (device, bf16, layout above) into
+ * mask_ws. Steps, by policy: mean pooling of Q and K per block and per-block
+ * SICS of K (SPADE, TOPK); per-head argmax of summed SICS over the candidate
+ * blockings (SPADE); pooled block scores qbar_i . kbar_j / sqrt(d) (SPADE,
+ * TOPK); selection (Top-K, Top-P with window, static windows, spatial/temporal
+ * rules with sinks); FG group means, slice scores, the exact per-head
+ * threshold and the slice bitmask (FG). q and k may be NULL for the static
+ * policies (STA, SPATIOTEMPORAL, EXPLICIT). Clears the status word.
+ * Asynchronous on ``stream``.
+ */
+SA_API int sparse_attn_build_mask(const sa_problem* problem, const sa_policy* policy,
+                           const void* q, const void* k,
+                           void* mask_ws, void* scratch_ws, void* stream);
+
+/* ---------------------------------------------------------------- attention
+ * O and LSE for the mask in mask_ws (built by sparse_attn_build_mask with the
+ * same problem and policy). Equivalent to sparse_attn_permute followed by
+ * sparse_attn_attend on the same stream. Outputs are written in original
+ * token order; rows whose kept key set is empty get O = 0 and LSE = -inf.
+ * ``lse`` may be NULL. Asynchronous on ``stream``.
+ */
+SA_API int sparse_attn_forward(const sa_problem* problem, const sa_policy* policy,
+                               const void* q, const void* k, const void* v,
+                               const void* mask_ws, void* scratch_ws,
+                               void* o, float* lse, void* stream);
+
+/* Layout step of the forward pass: copies Q, K, V of every head whose working
+ * layout is frame-major (slot m = (h*W + w)*T + t; Sparse VideoGen review, key
+ * machinery: the token-major to frame-major transform) into the scratch
+ * workspace, padded with zero rows to whole blocks. Does nothing for other
+ * layouts: identity blocks are read in place and 3D tiles are gathered by the
+ * attention kernel's 5-D TMA boxes. Reads the mask's per-head layouts, so it
+ * runs after sparse_attn_build_mask. Asynchronous on ``stream``. */
+SA_API int sparse_attn_permute(const sa_problem* problem, const sa_policy* policy,
+                               const void* q, const void* k, const void* v,
+                               const void* mask_ws, void* scratch_ws, void* stream);
+
+/* Attention step of the forward pass (the flash-style kernel with online
+ * softmax over the kept key blocks or key slices). Frame-major heads read the
+ * copies sparse_attn_permute left in scratch_ws. Asynchronous on ``stream``. */
+SA_API int sparse_attn_attend(const sa_problem* problem, const sa_policy* policy,
+                              const void* q, const void* k, const void* v,
+                              const void* mask_ws, void* scratch_ws,
+                              void* o, float* lse, void* stream);
+
+/* ---------------------------------------------------------------- inspection
+ * Copy one part of a built mask to host memory and wait for the copy.
+ *   SA_EXPORT_BLOCK_BITS   uint32 [batch*heads][nb][ceil(nb/32)]
+ *   SA_EXPORT_HEAD_INFO    sa_head_info [batch*heads]
+ *   SA_EXPORT_FG_BITS      uint32 [batch*heads][G][ceil(N/32)], G = ceil(N/fg_group)
+ *   SA_EXPORT_FG_TAU       float  [batch*heads]
+ * ``bytes`` must equal the size of that part (see sparse_attn_export_bytes).
+ */
+enum {
+  SA_EXPORT_BLOCK_BITS = 1,
+  SA_EXPORT_HEAD_INFO = 2,
+  SA_EXPORT_FG_BITS = 3,
+  SA_EXPORT_FG_TAU = 4
+};
+
+typedef struct {
+  int32_t layout;            /* SA_LAYOUT_* used by this head                     */
+  int32_t candidate;         /* SPADE: chosen blocking index; otherwise 0         */
+  int32_t bt, bh, bw;        /* tile of a tile layout (1,1,block otherwise)       */
+  int32_t nt, nh, nw;        /* tile grid of a tile layout                        */
+  int32_t nb;                /* blocks of this head's working layout              */
+  int32_t kept;              /* kept (query block, key block) pairs               */
+  float sics_total[4];       /* SPADE: summed SICS per candidate blocking         */
+  int32_t reserved[2];
+} sa_head_info;
+
+SA_API int sparse_attn_export_bytes(const sa_problem* problem, const sa_policy* policy, int what,
+                             size_t* bytes);
+SA_API int sparse_attn_mask_export(const sa_problem* problem, const sa_policy* policy,
+                            const void* mask_ws, int what, void* host_dst, size_t bytes,
+                            void* stream);
+
+/* Wait for ``stream`` and return the device status recorded in scratch_ws
+ * since the last sparse_attn_build_mask: SA_OK, SA_ERR_DEVICE_TIMEOUT or
+ * SA_ERR_DEVICE_BOUNDS. If ``clear`` is nonzero the word is reset. */
+SA_API int sparse_attn_status(void* scratch_ws, void* stream, int clear);
+
+/* Static description of a status code. Never NULL. */
+SA_API const char* sparse_attn_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPARSE_ATTN_H_ */

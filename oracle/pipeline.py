@@ -19,7 +19,9 @@ def working_order(wl, head, tile=None):
     return layout.identity_order(wl.T, wl.H, wl.W, wl.block)
 
 
-def head_mask(wl, q, k, head):
+def head_mask(wl, q, k, head, force_choice=None):
+    """``force_choice`` (SPADE) evaluates the given candidate instead of the
+    argmax, for a head whose summed SICS scores tie within the tolerance."""
     d = wl.head_dim
     info = {}
     if wl.kind == "fg":
@@ -36,6 +38,8 @@ def head_mask(wl, q, k, head):
             totals.append(float(masks.sics(k, blk_c).astype(np.float64).sum()))
         choice = masks.choose_candidate(totals)
         info.update(sics_totals=totals, choice=choice)
+        if force_choice is not None:
+            choice = force_choice
         tile = wl.candidates[choice]
 
     order = working_order(wl, head, tile)

@@ -1,0 +1,133 @@
+"""PyTorch-facing wrapper over the C ABI.
+
+PyTorch supplies device memory (the caller's tensors and the two workspaces)
+and the CUDA stream; every step of the computation runs in the native
+library. Nothing here computes on tensor values.
+"""
+import ctypes
+
+import numpy as np
+import torch
+
+from . import _native as N
+
+
+def make_policy(kind, block=128, tile=(1, 1, 128), topk=0, keep_diagonal=False,
+                window=(1, 1, 1), temporal_heads=None, heads=0, sink_tokens=0, frame_radius=1,
+                candidates=(), top_p=0.0, fg_group=64, fg_keep_fraction=0.15,
+                explicit_layout=N.SA_LAYOUT_IDENTITY, explicit_bits=None):
+    """Fill an ``sa_policy``. ``kind`` is a name ("topk", "sta", "spatiotemporal",
+    "spade", "fg", "explicit") or an SA_MASK_* code."""
+    names = {"topk": N.SA_MASK_TOPK, "sta": N.SA_MASK_STA,
+             "spatiotemporal": N.SA_MASK_SPATIOTEMPORAL, "spade": N.SA_MASK_SPADE,
+             "fg": N.SA_MASK_FG, "explicit": N.SA_MASK_EXPLICIT}
+    p = N.Policy()
+    p.kind = names.get(kind, kind)
+    p.block = block
+    p.tile[:] = list(tile)
+    p.topk = topk
+    p.keep_diagonal = 1 if keep_diagonal else 0
+    p.window[:] = list(window)
+    if temporal_heads is not None:
+        arr = (ctypes.c_int8 * max(1, heads))()
+        for h in temporal_heads:
+            arr[h] = 1
+        p.head_is_temporal = ctypes.cast(arr, ctypes.POINTER(ctypes.c_int8))
+        p._keep_alive = arr
+    p.sink_tokens = sink_tokens
+    p.frame_radius = frame_radius
+    p.n_candidates = len(candidates)
+    for i, c in enumerate(candidates):
+        p.candidates[i][:] = list(c)
+    p.top_p = top_p
+    p.fg_group = fg_group
+    p.fg_keep_fraction = fg_keep_fraction
+    p.explicit_layout = explicit_layout
+    if explicit_bits is not None:
+        p.explicit_bits = explicit_bits.data_ptr()
+        p._keep_bits = explicit_bits
+    return p
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_qkv(t, problem, name):
+    N_ = problem.T * problem.H * problem.W
+    want = (problem.batch, problem.heads, N_, problem.head_dim)
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != want:
+        raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {want}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+class SparseAttention:
+    """Caller-owned workspaces plus the build-mask / forward calls for one problem."""
+
+    def __init__(self, batch, heads, T, H, W, head_dim, policy, device="cuda"):
+        self.problem = N.Problem(batch, heads, T, H, W, head_dim)
+        self.policy = policy
+        self.mask_bytes, self.scratch_bytes = N.workspace_size(self.problem, policy)
+        self.device = torch.device(device)
+        self.mask_ws = torch.empty(self.mask_bytes, dtype=torch.uint8, device=self.device)
+        self.scratch_ws = torch.empty(max(self.scratch_bytes, 256), dtype=torch.uint8,
+                                      device=self.device)
+
+    @property
+    def n_tokens(self):
+        return self.problem.T * self.problem.H * self.problem.W
+
+    def build_mask(self, q, k, stream=None):
+        needs = self.policy.kind in (N.SA_MASK_TOPK, N.SA_MASK_SPADE, N.SA_MASK_FG)
+        if needs:
+            _check_qkv(q, self.problem, "q")
+            _check_qkv(k, self.problem, "k")
+        N.build_mask(self.problem, self.policy, q.data_ptr() if needs else None,
+                     k.data_ptr() if needs else None, self.mask_ws.data_ptr(),
+                     self.scratch_ws.data_ptr(), _stream_ptr(stream))
+
+    def forward(self, q, k, v, out=None, lse=None, stream=None):
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            _check_qkv(t, self.problem, n)
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+        N.forward(self.problem, self.policy, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                  self.mask_ws.data_ptr(), self.scratch_ws.data_ptr(), out.data_ptr(),
+                  lse.data_ptr(), _stream_ptr(stream))
+        return out, lse
+
+    def permute(self, q, k, v, stream=None):
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            _check_qkv(t, self.problem, n)
+        N.permute(self.problem, self.policy, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                  self.mask_ws.data_ptr(), self.scratch_ws.data_ptr(), _stream_ptr(stream))
+
+    def attend(self, q, k, v, out, lse, stream=None):
+        N.attend(self.problem, self.policy, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                 self.mask_ws.data_ptr(), self.scratch_ws.data_ptr(), out.data_ptr(),
+                 lse.data_ptr() if lse is not None else None, _stream_ptr(stream))
+        return out, lse
+
+    def __call__(self, q, k, v, stream=None):
+        self.build_mask(q, k, stream)
+        return self.forward(q, k, v, stream=stream)
+
+    def export(self, what, stream=None):
+        nbytes = N.export_bytes(self.problem, self.policy, what)
+        if what == N.SA_EXPORT_HEAD_INFO:
+            buf = (N.HeadInfo * (nbytes // ctypes.sizeof(N.HeadInfo)))()
+            N.mask_export(self.problem, self.policy, self.mask_ws.data_ptr(), what,
+                          ctypes.addressof(buf), nbytes, _stream_ptr(stream))
+            return list(buf)
+        dtype = np.float32 if what == N.SA_EXPORT_FG_TAU else np.uint32
+        arr = np.empty(nbytes // 4, dtype=dtype)
+        N.mask_export(self.problem, self.policy, self.mask_ws.data_ptr(), what,
+                      arr.ctypes.data, nbytes, _stream_ptr(stream))
+        return arr
+
+    def status(self, clear=False, stream=None):
+        return N.status(self.scratch_ws.data_ptr(), _stream_ptr(stream), clear)

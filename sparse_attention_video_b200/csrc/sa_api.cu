@@ -1,0 +1,536 @@
+// Host side of the C ABI declared in include/sparse_attn.h: argument checks,
+// workspace layouts, TMA tensor maps and the launch sequence of each call.
+// No device memory is allocated here; every buffer belongs to the caller.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "sa_attn.h"
+#include "sa_fg.h"
+#include "sa_internal.h"
+#include "sa_mask.h"
+
+using namespace sa;
+
+namespace {
+
+int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+bool is_tile_kind(int kind) { return kind == SA_MASK_TOPK || kind == SA_MASK_STA; }
+
+// Blocks of a 3D tiling of the problem's grid.
+int tile_blocks(const sa_problem& pr, const int* t) {
+  return ceil_div(pr.T, t[0]) * ceil_div(pr.H, t[1]) * ceil_div(pr.W, t[2]);
+}
+
+long long n_tokens(const sa_problem& pr) { return (long long)pr.T * pr.H * pr.W; }
+
+int check_problem(const sa_problem* pr) {
+  if (!pr) return SA_ERR_INVALID_ARG;
+  if (pr->batch < 1 || pr->heads < 1 || pr->T < 1 || pr->H < 1 || pr->W < 1)
+    return SA_ERR_INVALID_ARG;
+  if (pr->head_dim != 64 && pr->head_dim != 128) return SA_ERR_UNSUPPORTED;
+  if (n_tokens(*pr) > (1ll << 30) / pr->head_dim) return SA_ERR_UNSUPPORTED;
+  if ((long long)pr->batch * pr->heads > 65535) return SA_ERR_UNSUPPORTED;
+  return SA_OK;
+}
+
+int check_tile(const sa_problem& pr, const int* t, int block) {
+  if (t[0] < 1 || t[1] < 1 || t[2] < 1) return SA_ERR_INVALID_ARG;
+  if (t[0] * t[1] * t[2] != block) return SA_ERR_INVALID_ARG;
+  if (t[0] > 256 || t[1] > 256 || t[2] > 256) return SA_ERR_UNSUPPORTED;
+  if (tile_blocks(pr, t) > kMaxBlocks) return SA_ERR_UNSUPPORTED;
+  return SA_OK;
+}
+
+int check_policy(const sa_problem& pr, const sa_policy* po) {
+  if (!po) return SA_ERR_INVALID_ARG;
+  if (po->kind == SA_MASK_FG) {
+    if (po->fg_group != 64 && po->fg_group != 128) return SA_ERR_UNSUPPORTED;
+    if (!(po->fg_keep_fraction > 0.f && po->fg_keep_fraction <= 1.f)) return SA_ERR_INVALID_ARG;
+    return SA_OK;
+  }
+  if (po->block != 128 && !(po->block == 64 && pr.head_dim == 64)) return SA_ERR_UNSUPPORTED;
+  const long long N = n_tokens(pr);
+  switch (po->kind) {
+    case SA_MASK_TOPK:
+      if (po->topk < 1) return SA_ERR_INVALID_ARG;
+      return check_tile(pr, po->tile, po->block);
+    case SA_MASK_STA:
+      for (int i = 0; i < 3; ++i)
+        if (po->window[i] < 1 || po->window[i] % 2 == 0) return SA_ERR_INVALID_ARG;
+      return check_tile(pr, po->tile, po->block);
+    case SA_MASK_SPADE:
+      if (po->n_candidates < 1 || po->n_candidates > kMaxCand) return SA_ERR_INVALID_ARG;
+      if (!(po->top_p > 0.f && po->top_p <= 1.f)) return SA_ERR_INVALID_ARG;
+      for (int i = 0; i < 3; ++i)
+        if (po->window[i] < 1 || po->window[i] % 2 == 0) return SA_ERR_INVALID_ARG;
+      for (int c = 0; c < po->n_candidates; ++c) {
+        const int e = check_tile(pr, po->candidates[c], po->block);
+        if (e) return e;
+      }
+      return SA_OK;
+    case SA_MASK_SPATIOTEMPORAL:
+      if (!po->head_is_temporal) return SA_ERR_INVALID_ARG;
+      if (pr.heads > 256) return SA_ERR_UNSUPPORTED;
+      if (po->sink_tokens < 0 || po->frame_radius < 0) return SA_ERR_INVALID_ARG;
+      if (ceil_div(N, po->block) > kMaxBlocks) return SA_ERR_UNSUPPORTED;
+      return SA_OK;
+    case SA_MASK_EXPLICIT:
+      if (!po->explicit_bits) return SA_ERR_INVALID_ARG;
+      if (po->explicit_layout == SA_LAYOUT_TILE) return check_tile(pr, po->tile, po->block);
+      if (po->explicit_layout != SA_LAYOUT_IDENTITY && po->explicit_layout != SA_LAYOUT_FRAME_MAJOR)
+        return SA_ERR_INVALID_ARG;
+      if (ceil_div(N, po->block) > kMaxBlocks) return SA_ERR_UNSUPPORTED;
+      return SA_OK;
+    default:
+      return SA_ERR_INVALID_ARG;
+  }
+}
+
+// Max blocks per head over every layout the policy can use.
+int policy_nb(const sa_problem& pr, const sa_policy& po) {
+  switch (po.kind) {
+    case SA_MASK_TOPK:
+    case SA_MASK_STA:
+      return tile_blocks(pr, po.tile);
+    case SA_MASK_SPADE: {
+      int nb = 0;
+      for (int c = 0; c < po.n_candidates; ++c) nb = std::max(nb, tile_blocks(pr, po.candidates[c]));
+      return nb;
+    }
+    case SA_MASK_EXPLICIT:
+      if (po.explicit_layout == SA_LAYOUT_TILE) return tile_blocks(pr, po.tile);
+      return ceil_div(n_tokens(pr), po.block);
+    case SA_MASK_SPATIOTEMPORAL:
+      return ceil_div(n_tokens(pr), po.block);
+    default:
+      return 0;
+  }
+}
+
+bool needs_frame_major(const sa_problem& pr, const sa_policy& po) {
+  if (po.kind == SA_MASK_EXPLICIT) return po.explicit_layout == SA_LAYOUT_FRAME_MAJOR;
+  if (po.kind != SA_MASK_SPATIOTEMPORAL) return false;
+  for (int h = 0; h < pr.heads; ++h)
+    if (po.head_is_temporal[h]) return true;
+  return false;
+}
+
+int n_cand(const sa_policy& po) {
+  if (po.kind == SA_MASK_SPADE) return po.n_candidates;
+  if (po.kind == SA_MASK_TOPK) return 1;
+  return 0;
+}
+
+MaskLayout mask_layout(const sa_problem& pr, const sa_policy& po) {
+  MaskLayout L;
+  L.BH = pr.batch * pr.heads;
+  L.NB = policy_nb(pr, po);
+  L.W32 = (L.NB + 31) / 32;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+  L.off_head = take(sizeof(HeadGeom) * L.BH);
+  L.off_counts = take(sizeof(int) * (size_t)L.BH * L.NB);
+  L.off_cols = take(sizeof(int) * (size_t)L.BH * L.NB * L.NB);
+  L.off_bits = take(sizeof(uint32_t) * (size_t)L.BH * L.NB * L.W32);
+  if (po.kind == SA_MASK_FG) {
+    const long long N = n_tokens(pr);
+    L.G = ceil_div(N, po.fg_group);
+    L.WN = ceil_div(N, 32);
+    L.off_fg_bits = take(sizeof(uint32_t) * (size_t)L.BH * L.G * L.WN);
+    L.off_fg_tau = take(sizeof(float) * (size_t)L.BH);
+  }
+  L.total = std::max<size_t>(off, 256);
+  return L;
+}
+
+ScratchLayout scratch_layout(const sa_problem& pr, const sa_policy& po, const MaskLayout& M) {
+  ScratchLayout S;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+  S.off_status = take(256);
+  const int d = pr.head_dim;
+  if (needs_frame_major(pr, po)) {
+    const size_t n_pad = (size_t)ceil_div(n_tokens(pr), po.block) * po.block;
+    S.perm_stride = align_up((size_t)M.BH * n_pad * d * 2, 256);
+    S.off_perm = take(3 * S.perm_stride);
+  }
+  const int C = n_cand(po);
+  if (C > 0) {
+    S.off_qbar = take(sizeof(float) * (size_t)M.BH * C * M.NB * d);
+    S.off_kbar = take(sizeof(float) * (size_t)M.BH * C * M.NB * d);
+    S.off_sics = take(sizeof(float) * (size_t)M.BH * C * M.NB);
+    S.off_scores = take(sizeof(float) * (size_t)M.BH * M.NB * M.NB);
+  }
+  if (po.kind == SA_MASK_FG) {
+    S.off_fg_qbar = take(fg_qbar_bytes(M.BH, M.G, d));
+    S.off_fg_hist = take(fg_hist_bytes(M.BH));
+    S.off_fg_sel = take(fg_sel_bytes(M.BH));
+  }
+  S.total = off;
+  return S;
+}
+
+// ------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D map over [BH][rows][d] bf16 with a (64, box_rows, 1) box.
+bool map_3d(CUtensorMap* m, const void* base, int BH, long long rows, int d, int box_rows) {
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                     strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 5-D map over [BH][T][H][W][d] bf16 whose box is one (bt, bh, bw) tile x 64 columns.
+bool map_5d(CUtensorMap* m, const void* base, const sa_problem& pr, const int* tile) {
+  const int d = pr.head_dim;
+  const cuuint64_t e = 2;
+  cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)pr.W, (cuuint64_t)pr.H, (cuuint64_t)pr.T,
+                        (cuuint64_t)pr.batch * pr.heads};
+  cuuint64_t strides[4] = {d * e, (cuuint64_t)pr.W * d * e, (cuuint64_t)pr.H * pr.W * d * e,
+                           (cuuint64_t)pr.T * pr.H * pr.W * d * e};
+  cuuint32_t box[5] = {64, (cuuint32_t)tile[2], (cuuint32_t)tile[1], (cuuint32_t)tile[0], 1};
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims,
+                     strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int aligned(const void* p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
+
+}  // namespace
+
+// ======================================================================== API
+extern "C" int sparse_attn_workspace_size(const sa_problem* problem, const sa_policy* policy,
+                                          size_t* mask_bytes, size_t* scratch_bytes) {
+  int e = check_problem(problem);
+  if (e) return e;
+  e = check_policy(*problem, policy);
+  if (e) return e;
+  if (!mask_bytes || !scratch_bytes) return SA_ERR_INVALID_ARG;
+  const MaskLayout M = mask_layout(*problem, *policy);
+  const ScratchLayout S = scratch_layout(*problem, *policy, M);
+  *mask_bytes = M.total;
+  *scratch_bytes = S.total;
+  return SA_OK;
+}
+
+extern "C" int sparse_attn_build_mask(const sa_problem* problem, const sa_policy* policy,
+                                      const void* q, const void* k, void* mask_ws,
+                                      void* scratch_ws, void* stream) {
+  int e = check_problem(problem);
+  if (e) return e;
+  e = check_policy(*problem, policy);
+  if (e) return e;
+  const sa_problem& pr = *problem;
+  const sa_policy& po = *policy;
+  const bool needs_qk = po.kind == SA_MASK_TOPK || po.kind == SA_MASK_SPADE || po.kind == SA_MASK_FG;
+  if (needs_qk && (!aligned(q, 16) || !aligned(k, 16))) return SA_ERR_INVALID_ARG;
+  if (!aligned(mask_ws, 256) || !aligned(scratch_ws, 256)) return SA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const MaskLayout M = mask_layout(pr, po);
+  const ScratchLayout S = scratch_layout(pr, po, M);
+  uint8_t* mw = static_cast<uint8_t*>(mask_ws);
+  uint8_t* sw = static_cast<uint8_t*>(scratch_ws);
+  HeadGeom* heads = reinterpret_cast<HeadGeom*>(mw + M.off_head);
+  const int N = (int)n_tokens(pr);
+  const int d = pr.head_dim;
+  const int BH = M.BH;
+
+  if (cudaMemsetAsync(sw + S.off_status, 0, 256, st) != cudaSuccess) return SA_ERR_CUDA;
+
+  if (po.kind == SA_MASK_FG) {
+    FgBuildParams fp{};
+    fp.q = static_cast<const __nv_bfloat16*>(q);
+    fp.k = static_cast<const __nv_bfloat16*>(k);
+    fp.qbar = reinterpret_cast<float*>(sw + S.off_fg_qbar);
+    fp.hist = reinterpret_cast<uint32_t*>(sw + S.off_fg_hist);
+    fp.sel = reinterpret_cast<uint32_t*>(sw + S.off_fg_sel);
+    fp.bits = reinterpret_cast<uint32_t*>(mw + M.off_fg_bits);
+    fp.tau = reinterpret_cast<float*>(mw + M.off_fg_tau);
+    fp.status = reinterpret_cast<uint32_t*>(sw + S.off_status);
+    fp.BH = BH; fp.N = N; fp.d = d; fp.group = po.fg_group; fp.G = M.G; fp.WN = M.WN;
+    fp.keep_fraction = po.fg_keep_fraction;
+    return cuda_status(launch_fg_build(fp, st));
+  }
+
+  SelectParams sp{};
+  sp.heads = heads;
+  sp.bits = reinterpret_cast<uint32_t*>(mw + M.off_bits);
+  sp.counts = reinterpret_cast<int*>(mw + M.off_counts);
+  sp.cols = reinterpret_cast<int*>(mw + M.off_cols);
+  sp.kind = po.kind; sp.NB = M.NB; sp.W32 = M.W32; sp.T = pr.T; sp.H = pr.H; sp.W = pr.W;
+  sp.topk = po.topk; sp.keep_diagonal = po.keep_diagonal;
+  for (int i = 0; i < 3; ++i) sp.win[i] = po.window[i];
+  sp.top_p = po.top_p;
+  sp.frame_radius = po.frame_radius;
+  sp.sink_blocks = ceil_div(po.sink_tokens, po.block);
+
+  const int C = n_cand(po);
+  if (C > 0) {
+    PoolParams pp{};
+    pp.q = static_cast<const __nv_bfloat16*>(q);
+    pp.k = static_cast<const __nv_bfloat16*>(k);
+    pp.qbar = reinterpret_cast<float*>(sw + S.off_qbar);
+    pp.kbar = reinterpret_cast<float*>(sw + S.off_kbar);
+    pp.sics = reinterpret_cast<float*>(sw + S.off_sics);
+    for (int c = 0; c < C; ++c)
+      for (int i = 0; i < 3; ++i) pp.cand[c][i] = po.kind == SA_MASK_SPADE ? po.candidates[c][i] : po.tile[i];
+    pp.C = C; pp.NB = M.NB; pp.T = pr.T; pp.H = pr.H; pp.W = pr.W; pp.d = d;
+    if ((e = cuda_status(launch_pool_sics(pp, BH, M.NB, st)))) return e;
+    if (po.kind == SA_MASK_SPADE) {
+      ChooseParams cp{};
+      cp.sics = pp.sics; cp.heads = heads;
+      std::memcpy(cp.cand, pp.cand, sizeof(cp.cand));
+      cp.C = C; cp.NB = M.NB; cp.T = pr.T; cp.H = pr.H; cp.W = pr.W;
+      if ((e = cuda_status(launch_choose(cp, BH, st)))) return e;
+    }
+  }
+  if (po.kind != SA_MASK_SPADE) {
+    HeadInitParams hp{};
+    hp.geo = heads; hp.BH = BH; hp.heads = pr.heads;
+    hp.T = pr.T; hp.H = pr.H; hp.W = pr.W; hp.block = po.block;
+    hp.layout = po.kind == SA_MASK_EXPLICIT ? po.explicit_layout
+              : (is_tile_kind(po.kind) ? SA_LAYOUT_TILE : SA_LAYOUT_IDENTITY);
+    hp.bt = po.tile[0]; hp.bh = po.tile[1]; hp.bw = po.tile[2];
+    if (po.kind == SA_MASK_SPATIOTEMPORAL) {
+      hp.has_temporal_bits = 1;
+      for (int h = 0; h < pr.heads; ++h)
+        if (po.head_is_temporal[h]) hp.temporal_bits[h / 32] |= 1u << (h % 32);
+    }
+    if ((e = cuda_status(launch_head_init(hp, st)))) return e;
+  }
+  if (C > 0) {
+    ScoreParams sc{};
+    sc.heads = heads;
+    sc.qbar = reinterpret_cast<const float*>(sw + S.off_qbar);
+    sc.kbar = reinterpret_cast<const float*>(sw + S.off_kbar);
+    sc.scores = reinterpret_cast<float*>(sw + S.off_scores);
+    sc.C = C; sc.NB = M.NB; sc.sqrt_d = sqrtf((float)d);
+    if ((e = cuda_status(launch_pooled_scores(sc, BH, d, st)))) return e;
+    sp.scores = sc.scores;
+  }
+  if (po.kind == SA_MASK_EXPLICIT) sp.explicit_bits = po.explicit_bits;
+  return cuda_status(launch_select(sp, BH, st));
+}
+
+namespace {
+
+struct CallCtx {
+  MaskLayout M;
+  ScratchLayout S;
+  const uint8_t* mw;
+  uint8_t* sw;
+  cudaStream_t st;
+  int N, d, BH, n_pad;
+};
+
+int prepare_call(const sa_problem* problem, const sa_policy* policy, const void* q,
+                 const void* k, const void* v, const void* mask_ws, void* scratch_ws,
+                 void* stream, CallCtx* c) {
+  int e = check_problem(problem);
+  if (e) return e;
+  e = check_policy(*problem, policy);
+  if (e) return e;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return SA_ERR_INVALID_ARG;
+  if (!aligned(mask_ws, 256) || !aligned(scratch_ws, 256)) return SA_ERR_WORKSPACE;
+  c->M = mask_layout(*problem, *policy);
+  c->S = scratch_layout(*problem, *policy, c->M);
+  c->mw = static_cast<const uint8_t*>(mask_ws);
+  c->sw = static_cast<uint8_t*>(scratch_ws);
+  c->st = reinterpret_cast<cudaStream_t>(stream);
+  c->N = (int)n_tokens(*problem);
+  c->d = problem->head_dim;
+  c->BH = c->M.BH;
+  c->n_pad = policy->kind == SA_MASK_FG ? c->N : ceil_div(c->N, policy->block) * policy->block;
+  return SA_OK;
+}
+
+}  // namespace
+
+extern "C" int sparse_attn_permute(const sa_problem* problem, const sa_policy* policy,
+                                   const void* q, const void* k, const void* v,
+                                   const void* mask_ws, void* scratch_ws, void* stream) {
+  CallCtx c;
+  int e = prepare_call(problem, policy, q, k, v, mask_ws, scratch_ws, stream, &c);
+  if (e) return e;
+  if (!needs_frame_major(*problem, *policy)) return SA_OK;
+  PermuteParams pp{};
+  pp.heads = reinterpret_cast<const HeadGeom*>(c.mw + c.M.off_head);
+  const void* src[3] = {q, k, v};
+  for (int i = 0; i < 3; ++i) {
+    pp.src[i] = static_cast<const __nv_bfloat16*>(src[i]);
+    pp.dst[i] = reinterpret_cast<__nv_bfloat16*>(c.sw + c.S.off_perm + i * c.S.perm_stride);
+  }
+  pp.T = problem->T; pp.H = problem->H; pp.W = problem->W; pp.d = c.d; pp.n_pad = c.n_pad;
+  return cuda_status(launch_permute_fm(pp, c.BH, c.st));
+}
+
+extern "C" int sparse_attn_attend(const sa_problem* problem, const sa_policy* policy,
+                                  const void* q, const void* k, const void* v,
+                                  const void* mask_ws, void* scratch_ws, void* o, float* lse,
+                                  void* stream) {
+  CallCtx c;
+  int e = prepare_call(problem, policy, q, k, v, mask_ws, scratch_ws, stream, &c);
+  if (e) return e;
+  if (!aligned(o, 16) || (lse && !aligned(lse, 4))) return SA_ERR_INVALID_ARG;
+  if (!encode_fn()) return SA_ERR_CUDA;
+  const sa_problem& pr = *problem;
+  const sa_policy& po = *policy;
+  uint32_t* status = reinterpret_cast<uint32_t*>(c.sw + c.S.off_status);
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)c.d);
+
+  if (po.kind == SA_MASK_FG) {
+    FgAttnParams fp{};
+    fp.q = static_cast<const __nv_bfloat16*>(q);
+    fp.k = static_cast<const __nv_bfloat16*>(k);
+    fp.v = static_cast<const __nv_bfloat16*>(v);
+    fp.bits = reinterpret_cast<const uint32_t*>(c.mw + c.M.off_fg_bits);
+    fp.o = static_cast<__nv_bfloat16*>(o);
+    fp.lse = lse;
+    fp.status = status;
+    fp.BH = c.BH; fp.N = c.N; fp.d = c.d; fp.group = po.fg_group; fp.G = c.M.G; fp.WN = c.M.WN;
+    fp.scale_log2 = scale_log2;
+    return cuda_status(launch_fg_attn(fp, c.st));
+  }
+
+  const void* src[3] = {q, k, v};
+  const bool fm = needs_frame_major(pr, po);
+  AttnMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  CUtensorMap* sets[3] = {maps.q, maps.k, maps.v};
+  const bool tiled = po.kind == SA_MASK_SPADE || is_tile_kind(po.kind) ||
+                     (po.kind == SA_MASK_EXPLICIT && po.explicit_layout == SA_LAYOUT_TILE);
+  const int C = po.kind == SA_MASK_SPADE ? po.n_candidates : 1;
+  for (int i = 0; i < 3; ++i) {
+    if (!map_3d(&sets[i][0], src[i], c.BH, c.N, c.d, po.block)) return SA_ERR_CUDA;
+    if (fm) {
+      const void* perm = c.sw + c.S.off_perm + i * c.S.perm_stride;
+      if (!map_3d(&sets[i][1], perm, c.BH, c.n_pad, c.d, po.block)) return SA_ERR_CUDA;
+    } else {
+      sets[i][1] = sets[i][0];
+    }
+    for (int cc = 0; cc < C; ++cc) {
+      if (!tiled) { sets[i][2 + cc] = sets[i][0]; continue; }
+      const int* tile = po.kind == SA_MASK_SPADE ? po.candidates[cc] : po.tile;
+      if (!map_5d(&sets[i][2 + cc], src[i], pr, tile)) return SA_ERR_CUDA;
+    }
+  }
+  AttnParams ap{};
+  ap.heads = reinterpret_cast<const HeadGeom*>(c.mw + c.M.off_head);
+  ap.counts = reinterpret_cast<const int*>(c.mw + c.M.off_counts);
+  ap.cols = reinterpret_cast<const int*>(c.mw + c.M.off_cols);
+  ap.o = static_cast<__nv_bfloat16*>(o);
+  ap.lse = lse;
+  ap.status = status;
+  ap.BH = c.BH; ap.NB = c.M.NB; ap.T = pr.T; ap.H = pr.H; ap.W = pr.W; ap.N = c.N;
+  ap.scale_log2 = scale_log2;
+  return cuda_status(launch_attn_fwd(c.d, po.block, maps, ap, c.st));
+}
+
+extern "C" int sparse_attn_forward(const sa_problem* problem, const sa_policy* policy,
+                                   const void* q, const void* k, const void* v,
+                                   const void* mask_ws, void* scratch_ws, void* o, float* lse,
+                                   void* stream) {
+  int e = sparse_attn_permute(problem, policy, q, k, v, mask_ws, scratch_ws, stream);
+  if (e) return e;
+  return sparse_attn_attend(problem, policy, q, k, v, mask_ws, scratch_ws, o, lse, stream);
+}
+
+extern "C" int sparse_attn_export_bytes(const sa_problem* problem, const sa_policy* policy,
+                                        int what, size_t* bytes) {
+  int e = check_problem(problem);
+  if (e) return e;
+  e = check_policy(*problem, policy);
+  if (e) return e;
+  if (!bytes) return SA_ERR_INVALID_ARG;
+  const MaskLayout M = mask_layout(*problem, *policy);
+  switch (what) {
+    case SA_EXPORT_BLOCK_BITS: *bytes = sizeof(uint32_t) * (size_t)M.BH * M.NB * M.W32; break;
+    case SA_EXPORT_HEAD_INFO: *bytes = sizeof(HeadGeom) * (size_t)M.BH; break;
+    case SA_EXPORT_FG_BITS: *bytes = sizeof(uint32_t) * (size_t)M.BH * M.G * M.WN; break;
+    case SA_EXPORT_FG_TAU: *bytes = policy->kind == SA_MASK_FG ? sizeof(float) * M.BH : 0; break;
+    default: return SA_ERR_INVALID_ARG;
+  }
+  return SA_OK;
+}
+
+extern "C" int sparse_attn_mask_export(const sa_problem* problem, const sa_policy* policy,
+                                       const void* mask_ws, int what, void* host_dst,
+                                       size_t bytes, void* stream) {
+  size_t need = 0;
+  int e = sparse_attn_export_bytes(problem, policy, what, &need);
+  if (e) return e;
+  if (!host_dst || bytes != need || !aligned(mask_ws, 256)) return SA_ERR_INVALID_ARG;
+  const MaskLayout M = mask_layout(*problem, *policy);
+  size_t off = 0;
+  switch (what) {
+    case SA_EXPORT_BLOCK_BITS: off = M.off_bits; break;
+    case SA_EXPORT_HEAD_INFO: off = M.off_head; break;
+    case SA_EXPORT_FG_BITS: off = M.off_fg_bits; break;
+    case SA_EXPORT_FG_TAU: off = M.off_fg_tau; break;
+  }
+  if (need == 0) return SA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(host_dst, static_cast<const uint8_t*>(mask_ws) + off, need,
+                      cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return SA_ERR_CUDA;
+  return cuda_status(cudaStreamSynchronize(st));
+}
+
+extern "C" int sparse_attn_status(void* scratch_ws, void* stream, int clear) {
+  if (!aligned(scratch_ws, 256)) return SA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, scratch_ws, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return SA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SA_ERR_CUDA;
+  if (clear) {
+    if (cudaMemsetAsync(scratch_ws, 0, 256, st) != cudaSuccess) return SA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SA_ERR_CUDA;
+  }
+  if (word & SA_DEVFLAG_TIMEOUT) return SA_ERR_DEVICE_TIMEOUT;
+  if (word & SA_DEVFLAG_BOUNDS) return SA_ERR_DEVICE_BOUNDS;
+  return SA_OK;
+}
+
+extern "C" const char* sparse_attn_strerror(int status) {
+  switch (status) {
+    case SA_OK: return "ok";
+    case SA_ERR_INVALID_ARG: return "invalid argument";
+    case SA_ERR_UNSUPPORTED: return "unsupported problem or policy";
+    case SA_ERR_WORKSPACE: return "workspace pointer not 256-byte aligned";
+    case SA_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case SA_ERR_DEVICE_TIMEOUT: return "a device-side wait ran out (kernel gave up)";
+    case SA_ERR_DEVICE_BOUNDS: return "a device-side index check failed";
+    default: return "unknown status";
+  }
+}

@@ -1,0 +1,440 @@
+// Block-sparse flash attention on tcgen05 tensor cores (sm_100a).
+//
+// For one head and one query block of a working layout, the kernel visits the
+// kept key blocks in ascending order and computes
+//   S = Q K^T (tcgen05.mma, bf16 in, fp32 accumulate in tensor memory),
+//   P = exp(S / sqrt(d) - m) with a running row maximum m (online softmax),
+//   O += P V (tcgen05.mma, P staged in shared memory as bf16),
+// then writes O / l and LSE = ln(l) + m to the query tokens' original rows.
+// This is the flash block-sparse kernel with online softmax of the SPADE
+// review ("What carries the argument") and the dense-tile-only executor of the
+// Sliding Tile Attention review (key machinery: every computed block is dense,
+// the mask logic lives in the loader); online softmax is exact (SPADE review,
+// axiom ledger), so the result equals masked softmax attention.
+//
+// Roles (256 threads):
+//   warp 0      TMA producer: Q once, then K and V of each kept key block into
+//               a 2-stage ring. 3D tile layouts are gathered by one 5-D box per
+//               64 columns (no separate permutation pass); identity and
+//               frame-major layouts by a 3-D box.
+//   warp 1      allocates tensor memory; lane 0 issues all MMAs. S is double
+//               buffered so Q K_{j+1}^T runs while row j is in softmax.
+//   warps 4-7   softmax: thread r owns row r (tensor-memory lane r). The
+//               running maximum is only moved when it grows by more than 2^8,
+//               so O is rescaled rarely; P and l use the same reference, which
+//               keeps the result exact. Epilogue: O / l to bf16, scattered to
+//               original token rows (the inverse permutation is fused here).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "sa_attn.h"
+#include "sa_ptx.cuh"
+
+namespace sa {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kStages = 2;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows > 2^8
+
+template <int D, int BN>
+struct Smem {
+  static constexpr int kHalvesD = D / 64;                 // 64-column (128-byte) halves
+  static constexpr int kHalvesN = BN / 64;
+  static constexpr int kQBytes = kHalvesD * 128 * 128;    // 128 rows, M of the MMA
+  static constexpr int kKVHalf = BN * 128;                // one 64-column half of a K/V tile
+  static constexpr int kKVBytes = kHalvesD * kKVHalf;
+  static constexpr int kPBytes = kHalvesN * 128 * 128;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + kStages * kKVBytes;
+  static constexpr int kOffP = kOffV + kStages * kKVBytes;
+  static constexpr int kOffBar = kOffP + kPBytes;
+  static constexpr int kBytes = kOffBar + 256;
+  static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-byte alignment
+  static constexpr uint32_t kTmemCols = (2 * BN + D) <= 256 ? 256 : 512;
+};
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full;
+  uint64_t o_done;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Which tensor map and which coordinates fetch block ``blk`` of head ``bh``.
+__device__ __forceinline__ void block_source(const HeadGeom& g, int blk, int BN, int& map,
+                                             int& c1, int& c2, int& c3) {
+  if (g.layout == SA_LAYOUT_TILE) {
+    map = 2 + g.cand;
+    const int tw = blk % g.nw, th = (blk / g.nw) % g.nh, tt = blk / (g.nw * g.nh);
+    c1 = tw * g.bw; c2 = th * g.bh; c3 = tt * g.bt;
+  } else {
+    map = g.layout;  // 0 identity (original tensor), 1 frame-major (permuted copy)
+    c1 = blk * BN; c2 = 0; c3 = 0;
+  }
+}
+
+template <int D, int BN>
+__device__ __forceinline__ void load_block(const CUtensorMap* maps, const HeadGeom& g, int bh,
+                                           int blk, uint8_t* dst, uint64_t* bar) {
+  int map, c1, c2, c3;
+  block_source(g, blk, BN, map, c1, c2, c3);
+  const CUtensorMap* m = maps + map;
+#pragma unroll
+  for (int h = 0; h < D / 64; ++h) {
+    uint8_t* d = dst + h * (BN * 128);
+    if (map >= 2) tma_load_5d(d, m, bar, h * 64, c1, c2, c3, bh);
+    else tma_load_3d(d, m, bar, h * 64, c1, bh);
+  }
+}
+
+// Slot ``s`` of block ``blk`` -> original token index, or -1 for padding.
+__device__ __forceinline__ int slot_to_token(const HeadGeom& g, int blk, int s, int BN, int T,
+                                             int H, int W) {
+  const int N = T * H * W;
+  if (g.layout == SA_LAYOUT_TILE) {
+    const int tw = blk % g.nw, th = (blk / g.nw) % g.nh, tt = blk / (g.nw * g.nh);
+    const int lw = s % g.bw, lh = (s / g.bw) % g.bh, lt = s / (g.bw * g.bh);
+    const int t = tt * g.bt + lt, h = th * g.bh + lh, w = tw * g.bw + lw;
+    if (t >= T || h >= H || w >= W) return -1;
+    return (t * H + h) * W + w;
+  }
+  const int m = blk * BN + s;
+  if (m >= N) return -1;
+  if (g.layout == SA_LAYOUT_FRAME_MAJOR) {
+    const int pos = m / T, t = m - pos * T;
+    return t * (H * W) + pos;
+  }
+  return m;
+}
+
+// Validity of the BN slots of block ``blk`` as a bit mask (bit c = slot c holds
+// a token). Computed arithmetically from the block's position, so every
+// softmax thread can form it alone. Returns false when the block has no pad.
+template <int BN>
+__device__ __forceinline__ bool block_pad_mask(const HeadGeom& g, int blk, int T, int H, int W,
+                                               uint32_t (&bits)[BN / 32]) {
+#pragma unroll
+  for (int i = 0; i < BN / 32; ++i) bits[i] = 0u;
+  if (g.layout == SA_LAYOUT_TILE) {
+    const int tw = blk % g.nw, th = (blk / g.nw) % g.nh, tt = blk / (g.nw * g.nh);
+    const int lt_n = min(g.bt, T - tt * g.bt), lh_n = min(g.bh, H - th * g.bh);
+    const int lw_n = min(g.bw, W - tw * g.bw);
+    if (lt_n == g.bt && lh_n == g.bh && lw_n == g.bw) return false;
+    for (int lt = 0; lt < lt_n; ++lt)
+      for (int lh = 0; lh < lh_n; ++lh) {
+        const int a = (lt * g.bh + lh) * g.bw, b = a + lw_n;   // slots [a, b) are tokens
+#pragma unroll
+        for (int i = 0; i < BN / 32; ++i) {
+          const int lo = max(a, 32 * i), hi = min(b, 32 * i + 32);
+          if (hi > lo) {
+            const uint32_t width = (uint32_t)(hi - lo);
+            const uint32_t ones = width >= 32 ? 0xffffffffu : ((1u << width) - 1u);
+            bits[i] |= ones << (lo - 32 * i);
+          }
+        }
+      }
+    return true;
+  }
+  const int lim = T * H * W - blk * BN;                // slots [0, lim) are tokens
+  if (lim >= BN) return false;
+#pragma unroll
+  for (int i = 0; i < BN / 32; ++i) {
+    const int width = min(max(lim - 32 * i, 0), 32);
+    bits[i] = width >= 32 ? 0xffffffffu : ((1u << width) - 1u);
+  }
+  return true;
+}
+
+template <int D, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
+  using L = Smem<D, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem + L::kOffQ;
+  uint8_t* sK = smem + L::kOffK;
+  uint8_t* sV = smem + L::kOffV;
+  uint8_t* sP = smem + L::kOffP;
+  Bars* bars = reinterpret_cast<Bars*>(smem + L::kOffBar);
+
+  const int qb = blockIdx.x;
+  const int bh = blockIdx.y;
+  const HeadGeom g = p.heads[bh];
+  if (qb >= g.nb) return;  // uniform across the CTA, before any allocation
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const size_t row_base = ((size_t)bh * p.NB + qb);
+  const int n_keys = p.counts[row_base];
+  const int* cols = p.cols + row_base * p.NB;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->k_full[s], 1); mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1); mbar_init(&bars->v_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) { mbar_init(&bars->s_full[b], 1); mbar_init(&bars->s_free[b], 4); }
+    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if constexpr (BN < 128) {
+    // Rows BN..127 of the 128-row MMA operand carry no query; keep them finite.
+    constexpr int kVecPerHalf = (128 - BN) * 8;
+    for (int i = threadIdx.x; i < kVecPerHalf * L::kHalvesD; i += kThreads) {
+      const int h = i / kVecPerHalf, rem = i % kVecPerHalf;
+      reinterpret_cast<uint4*>(sQ + h * 16384 + BN * 128)[rem] = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const uint32_t tS[2] = {tmem, tmem + BN};
+  const uint32_t tO = tmem + 2 * BN;
+  volatile int* abort = &bars->abort;
+  uint32_t* status = p.status;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n_keys > 0) {
+      const CUtensorMap* qmaps = maps.q;
+      const CUtensorMap* kmaps = maps.k;
+      const CUtensorMap* vmaps = maps.v;
+      mbar_arrive_expect_tx(&bars->q_full, L::kHalvesD * BN * 128);
+      load_block<D, BN>(qmaps, g, bh, qb, sQ, &bars->q_full);
+      int issued = 0;
+      for (int j = 0; j < n_keys; ++j) {
+        const int st = j % kStages, rnd = j / kStages;
+        const int kb = cols[j];
+        if (kb < 0 || kb >= g.nb) { atomicOr(status, SA_DEVFLAG_BOUNDS); *abort = 1; break; }
+        if (!mbar_wait(&bars->k_empty[st], (rnd & 1) ^ 1, abort, status)) break;
+        mbar_arrive_expect_tx(&bars->k_full[st], L::kKVBytes);
+        load_block<D, BN>(kmaps, g, bh, kb, sK + st * L::kKVBytes, &bars->k_full[st]);
+        if (!mbar_wait(&bars->v_empty[st], (rnd & 1) ^ 1, abort, status)) { issued = j * 2 + 1; break; }
+        mbar_arrive_expect_tx(&bars->v_full[st], L::kKVBytes);
+        load_block<D, BN>(vmaps, g, bh, kb, sV + st * L::kKVBytes, &bars->v_full[st]);
+        issued = j * 2 + 2;
+      }
+      if (*abort) {
+        // Let copies already in flight land before the CTA's memory is released.
+        for (int j = (issued / 2 > kStages ? issued / 2 - kStages : 0); j < (issued + 1) / 2; ++j) {
+          const int st = j % kStages, par = (j / kStages) & 1;
+          for (uint32_t n = 0; n < kWaitPolls && !mbar_try_wait(&bars->k_full[st], par); ++n) {}
+          if (2 * j + 1 < issued)
+            for (uint32_t n = 0; n < kWaitPolls && !mbar_try_wait(&bars->v_full[st], par); ++n) {}
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_keys > 0) {
+      constexpr uint32_t idesc_qk = umma_idesc_bf16(128, BN, false, false);
+      constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, false, true);
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+      auto issue_pv = [&](int i) -> bool {
+        if (!mbar_wait(&bars->p_full, i & 1, abort, status)) return false;
+        if (!mbar_wait(&bars->v_full[i % kStages], (i / kStages) & 1, abort, status)) return false;
+        tc_fence_after();
+        const uint32_t vbase = aV + (i % kStages) * L::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // A = P (K-major, keys along K); B = V (MN-major: d contiguous).
+          const uint64_t da = umma_desc_sw128(aP + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+          const uint64_t db = umma_desc_sw128(vbase + kk * 16 * 128, L::kKVHalf, 1024);
+          umma_bf16_ss(tO, da, db, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&bars->o_done);
+        umma_commit(&bars->v_empty[i % kStages]);
+        return true;
+      };
+      bool ok = mbar_wait(&bars->q_full, 0, abort, status);
+      for (int j = 0; ok && j < n_keys; ++j) {
+        const int st = j % kStages, sb = j & 1;
+        if (!mbar_wait(&bars->k_full[st], (j / kStages) & 1, abort, status)) { ok = false; break; }
+        if (j >= 2 && !mbar_wait(&bars->s_free[sb], ((j - 2) >> 1) & 1, abort, status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kbase = aK + st * L::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk % 4) * 32;            // 16 bf16 along K inside a 128-byte row
+          const uint64_t da = umma_desc_sw128(aQ + (kk / 4) * 16384 + off, 16, 1024);
+          const uint64_t db = umma_desc_sw128(kbase + (kk / 4) * L::kKVHalf + off, 16, 1024);
+          umma_bf16_ss(tS[sb], da, db, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bars->s_full[sb]);
+        umma_commit(&bars->k_empty[st]);
+        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok) issue_pv(n_keys - 1);
+      // Every MMA issued above must finish before tensor memory is freed.
+      umma_commit(&bars->drain);
+      for (uint32_t n = 0; n < kWaitPolls && !mbar_try_wait(&bars->drain, 0); ++n) {}
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int r = threadIdx.x - 128;                  // row == tensor-memory lane
+    const uint32_t lane_off = (uint32_t)(32 * (warp - 4)) << 16;
+    const float scale = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    float s[BN];
+    bool ok = true;
+    for (int j = 0; j < n_keys; ++j) {
+      const int sb = j & 1;
+      const int kb = cols[j];
+      uint32_t pw[BN / 32];
+      const bool pad = block_pad_mask<BN>(g, kb, p.T, p.H, p.W, pw);
+      if (!mbar_wait(&bars->s_full[sb], (j >> 1) & 1, abort, status)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < BN; c += 32) tmem_ld32(tS[sb] + lane_off + c, s + c);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->s_free[sb]);
+
+      float mx = -INFINITY;
+      if (pad) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          s[c] = ((pw[c / 32] >> (c % 32)) & 1u) ? s[c] * scale : -INFINITY;
+          mx = fmaxf(mx, s[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) { s[c] *= scale; mx = fmaxf(mx, s[c]); }
+      }
+      const float m_new = fmaxf(m, mx);
+      const bool rescale = (m == -INFINITY) || (m_new > m + kRescaleThreshold);
+      const float m_use = rescale ? m_new : m;
+      float rs = 0.f;
+      if (m_use == -INFINITY) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) s[c] = 0.f;
+      } else {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) { s[c] = ex2_approx(s[c] - m_use); rs += s[c]; }
+      }
+      // P buffer and O are read/written by PV of the previous block: wait for it.
+      if (j >= 1) {
+        if (!mbar_wait(&bars->o_done, (j - 1) & 1, abort, status)) { ok = false; break; }
+        tc_fence_after();
+        if (rescale && m != -INFINITY) {
+          const float alpha = ex2_approx(m - m_use);
+          l *= alpha;
+          float o[32];
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            tmem_ld32(tO + lane_off + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(tO + lane_off + c, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      m = m_use;
+      l += rs;
+      // P row r into the 128-byte-swizzled K-major tile (keys along K).
+#pragma unroll
+      for (int h = 0; h < BN / 64; ++h) {
+        uint8_t* rowp = sP + h * 16384 + r * 128;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const float* x = s + h * 64 + ch * 8;
+          uint4 w;
+          w.x = pack_bf16x2(x[0], x[1]); w.y = pack_bf16x2(x[2], x[3]);
+          w.z = pack_bf16x2(x[4], x[5]); w.w = pack_bf16x2(x[6], x[7]);
+          *reinterpret_cast<uint4*>(rowp + ((ch ^ (r & 7)) << 4)) = w;
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full);
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok && n_keys > 0) {
+      ok = mbar_wait(&bars->o_done, (n_keys - 1) & 1, abort, status);
+      tc_fence_after();
+    }
+    const int tok = (r < BN) ? slot_to_token(g, qb, r, BN, p.T, p.H, p.W) : -1;
+    if (ok) {
+      const float inv_l = (n_keys > 0 && l > 0.f) ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (tok < 0 ? 0 : tok)) * D;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        float o[32];
+        if (n_keys > 0) {
+          tmem_ld32(tO + lane_off + c, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0.f;
+        }
+        if (tok >= 0) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w;
+            w.x = pack_bf16x2(o[e] * inv_l, o[e + 1] * inv_l);
+            w.y = pack_bf16x2(o[e + 2] * inv_l, o[e + 3] * inv_l);
+            w.z = pack_bf16x2(o[e + 4] * inv_l, o[e + 5] * inv_l);
+            w.w = pack_bf16x2(o[e + 6] * inv_l, o[e + 7] * inv_l);
+            *reinterpret_cast<uint4*>(orow + c + e) = w;
+          }
+        }
+      }
+      if (tok >= 0 && p.lse)
+        p.lse[(size_t)bh * p.N + tok] =
+            (n_keys > 0 && l > 0.f) ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace
+
+template <int D, int BN>
+static cudaError_t launch_one(const AttnMaps& maps, const AttnParams& p, cudaStream_t stream) {
+  using L = Smem<D, BN>;
+  auto kern = attn_fwd_kernel<D, BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.NB, p.BH);
+  kern<<<grid, kThreads, L::kAlloc, stream>>>(maps, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_fwd(int head_dim, int block, const AttnMaps& maps, const AttnParams& p,
+                            cudaStream_t stream) {
+  if (head_dim == 128 && block == 128) return launch_one<128, 128>(maps, p, stream);
+  if (head_dim == 64 && block == 128) return launch_one<64, 128>(maps, p, stream);
+  if (head_dim == 64 && block == 64) return launch_one<64, 64>(maps, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sa

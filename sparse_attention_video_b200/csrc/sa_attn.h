@@ -1,0 +1,36 @@
+// Launch interface of the block-sparse attention kernel (library-internal).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "sa_internal.h"
+
+namespace sa {
+
+// Tensor maps per source tensor. Index 0: the original [BH][N][d] tensor as a
+// 3-D map (identity layout); 1: the frame-major permuted copy [BH][N_pad][d];
+// 2 + c: the original tensor as a 5-D (d, W, H, T, BH) map whose box is the
+// 3D tile of blocking candidate c. All use 64-column boxes, 128-byte swizzle.
+constexpr int kMapsPerTensor = 6;
+struct AttnMaps {
+  CUtensorMap q[kMapsPerTensor];
+  CUtensorMap k[kMapsPerTensor];
+  CUtensorMap v[kMapsPerTensor];
+};
+
+struct AttnParams {
+  const HeadGeom* heads;   // [BH]
+  const int* counts;       // [BH][NB] kept key blocks per query block
+  const int* cols;         // [BH][NB][NB] kept key blocks, ascending
+  __nv_bfloat16* o;        // [BH][N][d]
+  float* lse;              // [BH][N]
+  uint32_t* status;        // device status word
+  int BH, NB, T, H, W, N;
+  float scale_log2;        // log2(e) / sqrt(d)
+};
+
+cudaError_t launch_attn_fwd(int head_dim, int block, const AttnMaps& maps, const AttnParams& p,
+                            cudaStream_t stream);
+
+}  // namespace sa

@@ -1,0 +1,514 @@
+// Mask construction kernels for block-sparse policies (sm_100a, CUDA cores).
+//
+//   head_init      per-head working-layout geometry for static policies
+//   permute_fm     token-major -> frame-major copy of Q, K, V for temporal heads
+//   pool_sics      per block: mean of Q, mean of K, and SICS of K, for every
+//                  blocking candidate (one pass over the block's tokens)
+//   choose         per head: argmax over candidates of summed SICS
+//   pooled_scores  per head: qbar_i . kbar_j / sqrt(d) over the chosen blocks
+//   select         per query block: Top-K / Top-P + window / static rules,
+//                  emitted as a bit row and an ascending list of key blocks
+//
+// All reductions run in a fixed order, so every result is deterministic.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "sa_mask.h"
+#include "sa_ptx.cuh"
+
+namespace sa {
+
+namespace {
+
+__device__ __forceinline__ int tile_slot_token(int bt, int bh, int bw, int nh, int nw, int blk,
+                                               int s, int T, int H, int W) {
+  const int tw = blk % nw, th = (blk / nw) % nh, tt = blk / (nw * nh);
+  const int lw = s % bw, lh = (s / bw) % bh, lt = s / (bw * bh);
+  const int t = tt * bt + lt, h = th * bh + lh, w = tw * bw + lw;
+  if (t >= T || h >= H || w >= W) return -1;
+  return (t * H + h) * W + w;
+}
+
+// ------------------------------------------------------------------ head_init
+__global__ void head_init_kernel(HeadInitParams p) {
+  const int bh = blockIdx.x * blockDim.x + threadIdx.x;
+  if (bh >= p.BH) return;
+  const int head = bh % p.heads;
+  HeadGeom g{};
+  const int N = p.T * p.H * p.W;
+  int layout = p.layout;
+  if (p.has_temporal_bits) {
+    const bool temporal = (p.temporal_bits[head / 32] >> (head % 32)) & 1u;
+    layout = temporal ? SA_LAYOUT_FRAME_MAJOR : SA_LAYOUT_IDENTITY;
+  }
+  g.layout = layout;
+  g.cand = 0;
+  if (layout == SA_LAYOUT_TILE) {
+    g.bt = p.bt; g.bh = p.bh; g.bw = p.bw;
+    g.nt = (p.T + p.bt - 1) / p.bt; g.nh = (p.H + p.bh - 1) / p.bh; g.nw = (p.W + p.bw - 1) / p.bw;
+    g.nb = g.nt * g.nh * g.nw;
+  } else {
+    g.bt = 1; g.bh = 1; g.bw = p.block;
+    g.nb = (N + p.block - 1) / p.block;
+    g.nt = 1; g.nh = 1; g.nw = g.nb;
+  }
+  g.kept = 0;
+  p.geo[bh] = g;
+}
+
+// ------------------------------------------------------------------ permute_fm
+// dst[bh][m] = src[bh][n(m)] for slot m of the frame-major order, zero rows for
+// slots m >= N. One 16-byte vector per thread; rows are 2*d bytes.
+__global__ void permute_fm_kernel(PermuteParams p) {
+  const int bh = blockIdx.y;
+  if (p.heads[bh].layout != SA_LAYOUT_FRAME_MAJOR) return;
+  const int vec_per_row = p.d / 8;
+  const int rows_per_cta = blockDim.x / vec_per_row;
+  const int r = blockIdx.x * rows_per_cta + threadIdx.x / vec_per_row;
+  const int c = threadIdx.x % vec_per_row;
+  if (r >= p.n_pad) return;
+  const int N = p.T * p.H * p.W;
+  uint4 val[3] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+  if (r < N) {
+    const int pos = r / p.T, t = r - pos * p.T;
+    const size_t src_row = (size_t)bh * N + (size_t)t * (p.H * p.W) + pos;
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+      val[i] = __ldg(reinterpret_cast<const uint4*>(p.src[i] + src_row * p.d) + c);
+  }
+  const size_t dst_row = (size_t)bh * p.n_pad + r;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) reinterpret_cast<uint4*>(p.dst[i] + dst_row * p.d)[c] = val[i];
+}
+
+// ------------------------------------------------------------------ pool_sics
+// One CTA per (block, candidate, head). Thread (token lane tl, chunk dc) loads
+// 8 dims of every (256 / (d/8))-th slot of the block.
+template <int D>
+__global__ void __launch_bounds__(256) pool_sics_kernel(PoolParams p) {
+  constexpr int CH = D / 8;            // 16-byte chunks per row
+  constexpr int TL = 256 / CH;         // token lanes
+  const int blk = blockIdx.x, c = blockIdx.y, bh = blockIdx.z;
+  const int bt = p.cand[c][0], bhh = p.cand[c][1], bw = p.cand[c][2];
+  const int nt = (p.T + bt - 1) / bt, nh = (p.H + bhh - 1) / bhh, nw = (p.W + bw - 1) / bw;
+  const int nb = nt * nh * nw;
+  if (blk >= nb) return;
+  const int BS = bt * bhh * bw;
+  const int tl = threadIdx.x / CH, dc = threadIdx.x % CH;
+  const int N = p.T * p.H * p.W;
+  const __nv_bfloat16* q = p.q + (size_t)bh * N * D;
+  const __nv_bfloat16* k = p.k + (size_t)bh * N * D;
+
+  float qs[8], ks[8], us[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) { qs[i] = 0.f; ks[i] = 0.f; us[i] = 0.f; }
+  int n_valid = 0, n_unit = 0;
+  // Both token lanes of a warp run the same number of iterations, and every
+  // lane joins the shuffles; pad slots contribute zeros.
+  for (int s = tl; s < BS; s += TL) {
+    const int tok = tile_slot_token(bt, bhh, bw, nh, nw, blk, s, p.T, p.H, p.W);
+    uint4 qv = make_uint4(0, 0, 0, 0), kv = make_uint4(0, 0, 0, 0);
+    if (tok >= 0) {
+      qv = __ldg(reinterpret_cast<const uint4*>(q + (size_t)tok * D) + dc);
+      kv = __ldg(reinterpret_cast<const uint4*>(k + (size_t)tok * D) + dc);
+    }
+    const __nv_bfloat16* qe = reinterpret_cast<const __nv_bfloat16*>(&qv);
+    const __nv_bfloat16* ke = reinterpret_cast<const __nv_bfloat16*>(&kv);
+    float kf[8], ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      kf[i] = __bfloat162float(ke[i]);
+      ss = fmaf(kf[i], kf[i], ss);
+    }
+#pragma unroll
+    for (int o = CH / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (tok < 0) continue;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      qs[i] += __bfloat162float(qe[i]);
+      ks[i] += kf[i];
+    }
+    ++n_valid;
+    if (ss > 0.f) {
+      const float nrm = sqrtf(ss);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) us[i] += kf[i] / nrm;
+      ++n_unit;
+    }
+  }
+  __shared__ float red[3][TL][D];
+  __shared__ int cnt[2][TL];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    red[0][tl][dc * 8 + i] = qs[i];
+    red[1][tl][dc * 8 + i] = ks[i];
+    red[2][tl][dc * 8 + i] = us[i];
+  }
+  if (dc == 0) { cnt[0][tl] = n_valid; cnt[1][tl] = n_unit; }
+  __syncthreads();
+  __shared__ float usq[D];
+  __shared__ int tot[2];
+  if (threadIdx.x < 2) {
+    int t = 0;
+    for (int i = 0; i < TL; ++i) t += cnt[threadIdx.x][i];
+    tot[threadIdx.x] = t;
+  }
+  __syncthreads();
+  const size_t base = (((size_t)bh * p.C + c) * p.NB + blk);
+  if (threadIdx.x < D) {
+    const int dd = threadIdx.x;
+    float a = 0.f, b = 0.f, u = 0.f;
+    for (int i = 0; i < TL; ++i) { a += red[0][i][dd]; b += red[1][i][dd]; u += red[2][i][dd]; }
+    const float nv = (float)tot[0];
+    p.qbar[base * D + dd] = tot[0] ? a / nv : 0.f;
+    p.kbar[base * D + dd] = tot[0] ? b / nv : 0.f;
+    usq[dd] = u * u;
+  }
+  __syncthreads();
+  // fixed-shape tree over the D squared components
+  for (int w = D / 2; w >= 1; w >>= 1) {
+    if (threadIdx.x < w) usq[threadIdx.x] += usq[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) p.sics[base] = usq[0] - (float)tot[1];
+}
+
+// ------------------------------------------------------------------ choose
+__global__ void choose_kernel(ChooseParams p) {
+  const int bh = blockIdx.x;
+  __shared__ double part[256];
+  __shared__ double totals[kMaxCand];
+  for (int c = 0; c < p.C; ++c) {
+    const int bt = p.cand[c][0], bhh = p.cand[c][1], bw = p.cand[c][2];
+    const int nb = ((p.T + bt - 1) / bt) * ((p.H + bhh - 1) / bhh) * ((p.W + bw - 1) / bw);
+    double s = 0.0;
+    for (int b = threadIdx.x; b < nb; b += blockDim.x)
+      s += (double)p.sics[((size_t)bh * p.C + c) * p.NB + b];
+    part[threadIdx.x] = s;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w >= 1; w >>= 1) {
+      if ((int)threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) totals[c] = part[0];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    int best = 0;
+    for (int c = 1; c < p.C; ++c) {
+      const double a = totals[best], b = totals[c];
+      if (b > a + 1e-4 * fmax(fabs(a), fabs(b))) best = c;
+    }
+    HeadGeom g{};
+    g.layout = SA_LAYOUT_TILE;
+    g.cand = best;
+    g.bt = p.cand[best][0]; g.bh = p.cand[best][1]; g.bw = p.cand[best][2];
+    g.nt = (p.T + g.bt - 1) / g.bt; g.nh = (p.H + g.bh - 1) / g.bh; g.nw = (p.W + g.bw - 1) / g.bw;
+    g.nb = g.nt * g.nh * g.nw;
+    g.kept = 0;
+    for (int c = 0; c < kMaxCand; ++c) g.sics_total[c] = c < p.C ? (float)totals[c] : 0.f;
+    p.heads[bh] = g;
+  }
+}
+
+// ------------------------------------------------------------------ pooled_scores
+// 64 x 64 output tile per CTA, 256 threads, 4 x 4 outputs per thread. Each
+// output is a sequential fp32 FMA chain over the d components.
+template <int D>
+__global__ void __launch_bounds__(256) pooled_scores_kernel(ScoreParams p) {
+  const int bh = blockIdx.z;
+  const HeadGeom g = p.heads[bh];
+  const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
+  if (i0 >= g.nb || j0 >= g.nb) return;
+  extern __shared__ float sm[];
+  float* sq = sm;              // [64][D+1]
+  float* sk = sm + 64 * (D + 1);
+  const size_t cbase = ((size_t)bh * p.C + g.cand) * p.NB;
+  for (int e = threadIdx.x; e < 64 * D; e += 256) {
+    const int r = e / D, c = e % D;
+    sq[r * (D + 1) + c] = (i0 + r < g.nb) ? p.qbar[(cbase + i0 + r) * D + c] : 0.f;
+    sk[r * (D + 1) + c] = (j0 + r < g.nb) ? p.kbar[(cbase + j0 + r) * D + c] : 0.f;
+  }
+  __syncthreads();
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+  for (int c = 0; c < D; ++c) {
+    float qa[4], kb[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) qa[a] = sq[(ty + 16 * a) * (D + 1) + c];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) kb[b] = sk[(tx + 16 * b) * (D + 1) + c];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(qa[a], kb[b], acc[a][b]);
+  }
+  const float rs = p.sqrt_d;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int i = i0 + ty + 16 * a, j = j0 + tx + 16 * b;
+      if (i < g.nb && j < g.nb) p.scores[((size_t)bh * p.NB + i) * p.NB + j] = acc[a][b] / rs;
+    }
+}
+
+// ------------------------------------------------------------------ select
+__device__ __forceinline__ bool block_valid(const HeadGeom& g, int blk, int T, int H, int W) {
+  if (g.layout == SA_LAYOUT_TILE) {
+    const int tw = blk % g.nw, th = (blk / g.nw) % g.nh, tt = blk / (g.nw * g.nh);
+    return tt * g.bt < T && th * g.bh < H && tw * g.bw < W;
+  }
+  return blk * g.bw < T * H * W;
+}
+
+// Block-wide reductions over 256 threads (fixed tree).
+__device__ __forceinline__ float block_max(float v, float* buf) {
+  for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (threadIdx.x % 32 == 0) buf[threadIdx.x / 32] = v;
+  __syncthreads();
+  float r = buf[0];
+  for (int i = 1; i < 8; ++i) r = fmaxf(r, buf[i]);
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ float block_sum(float v, float* buf) {
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (threadIdx.x % 32 == 0) buf[threadIdx.x / 32] = v;
+  __syncthreads();
+  float r = buf[0];
+  for (int i = 1; i < 8; ++i) r += buf[i];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
+  const int i = blockIdx.x, bh = blockIdx.y;
+  const HeadGeom g = p.heads[bh];
+  if (i >= g.nb) return;
+  __shared__ uint32_t bits[kMaxBlocks / 32];
+  __shared__ unsigned long long keys[kMaxBlocks];
+  __shared__ float fbuf[8];
+  __shared__ int s_count;
+  const int nb = g.nb, W32 = (nb + 31) / 32;
+  for (int w = threadIdx.x; w < W32; w += 256) bits[w] = 0u;
+  __syncthreads();
+  const bool qvalid = block_valid(g, i, p.T, p.H, p.W);
+  const float* srow = p.scores ? p.scores + ((size_t)bh * p.NB + i) * p.NB : nullptr;
+
+  if (qvalid) {
+    if (p.kind == SA_MASK_TOPK) {
+      // K rounds of block-wide argmax (score desc, index asc) over unchosen valid blocks.
+      for (int r = 0; r < p.topk; ++r) {
+        unsigned long long best = 0ull;
+        for (int j = threadIdx.x; j < nb; j += 256) {
+          if (!block_valid(g, j, p.T, p.H, p.W) || ((bits[j / 32] >> (j % 32)) & 1u)) continue;
+          uint32_t f = __float_as_uint(srow[j]);
+          f = (f & 0x80000000u) ? ~f : (f | 0x80000000u);         // order-preserving
+          // nonzero for every non-NaN score, so 0 can stand for "none"
+          const unsigned long long key = ((unsigned long long)f << 32) | (0xFFFFFFFFu - (uint32_t)j);
+          if (key > best) best = key;
+        }
+        for (int o = 16; o >= 1; o >>= 1) {
+          const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+          best = other > best ? other : best;
+        }
+        __shared__ unsigned long long wbest[8];
+        if (threadIdx.x % 32 == 0) wbest[threadIdx.x / 32] = best;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+          unsigned long long b = 0ull;
+          for (int w = 0; w < 8; ++w) b = wbest[w] > b ? wbest[w] : b;
+          if (b) {
+            const int j = (int)(0xFFFFFFFFu - (uint32_t)(b & 0xFFFFFFFFull));
+            bits[j / 32] |= 1u << (j % 32);
+          }
+        }
+        __syncthreads();
+      }
+      if (threadIdx.x == 0 && p.keep_diagonal && i < nb && block_valid(g, i, p.T, p.H, p.W))
+        bits[i / 32] |= 1u << (i % 32);
+    } else if (p.kind == SA_MASK_STA || p.kind == SA_MASK_SPADE) {
+      // clipped tile window around query tile i
+      const int rt = p.win[0] / 2, rh = p.win[1] / 2, rw = p.win[2] / 2;
+      const int iw = i % g.nw, ih = (i / g.nw) % g.nh, it = i / (g.nw * g.nh);
+      const int wt = 2 * rt + 1, wh = 2 * rh + 1, ww = 2 * rw + 1;
+      for (int e = threadIdx.x; e < wt * wh * ww; e += 256) {
+        const int jt = it - rt + e / (wh * ww), jh = ih - rh + (e / ww) % wh, jw = iw - rw + e % ww;
+        if (jt < 0 || jh < 0 || jw < 0 || jt >= g.nt || jh >= g.nh || jw >= g.nw) continue;
+        const int j = (jt * g.nh + jh) * g.nw + jw;
+        if (block_valid(g, j, p.T, p.H, p.W)) atomicOr(&bits[j / 32], 1u << (j % 32));
+      }
+      __syncthreads();
+      if (p.kind == SA_MASK_SPADE) {
+        // softmax over valid key blocks, then the shortest prefix by descending
+        // probability (ties to the lower index) whose fp32 running sum reaches top_p
+        float mx = -INFINITY;
+        for (int j = threadIdx.x; j < nb; j += 256)
+          if (block_valid(g, j, p.T, p.H, p.W)) mx = fmaxf(mx, srow[j]);
+        mx = block_max(mx, fbuf);
+        float se = 0.f;
+        for (int j = threadIdx.x; j < nb; j += 256)
+          if (block_valid(g, j, p.T, p.H, p.W)) se += expf(srow[j] - mx);
+        se = block_sum(se, fbuf);
+        int npow = 1;
+        while (npow < nb) npow <<= 1;
+        for (int j = threadIdx.x; j < npow; j += 256) {
+          unsigned long long key = 0ull;                 // invalid / padding sorts last
+          if (j < nb && block_valid(g, j, p.T, p.H, p.W)) {
+            const float pr = expf(srow[j] - mx) / se;
+            key = ((unsigned long long)__float_as_uint(pr) << 32) | (0xFFFFFFFFu - (uint32_t)j);
+          }
+          keys[j] = key;
+        }
+        __syncthreads();
+        // bitonic sort, descending
+        for (int size = 2; size <= npow; size <<= 1)
+          for (int stride = size / 2; stride >= 1; stride >>= 1) {
+            for (int a = threadIdx.x; a < npow; a += 256) {
+              const int b = a ^ stride;
+              if (b > a) {
+                const bool desc = (a & size) == 0;
+                const unsigned long long x = keys[a], y = keys[b];
+                if (desc ? (x < y) : (x > y)) { keys[a] = y; keys[b] = x; }
+              }
+            }
+            __syncthreads();
+          }
+        if (threadIdx.x == 0) {
+          float run = 0.f;
+          int c = 0;
+          while (c < npow && keys[c] != 0ull) {
+            run += __uint_as_float((uint32_t)(keys[c] >> 32));
+            ++c;
+            if (run >= p.top_p) break;
+          }
+          s_count = c;
+        }
+        __syncthreads();
+        for (int a = threadIdx.x; a < s_count; a += 256) {
+          const int j = (int)(0xFFFFFFFFu - (uint32_t)(keys[a] & 0xFFFFFFFFull));
+          atomicOr(&bits[j / 32], 1u << (j % 32));
+        }
+      }
+    } else if (p.kind == SA_MASK_SPATIOTEMPORAL) {
+      const int N = p.T * p.H * p.W, BS = g.bw, HW = p.H * p.W;
+      const int lo_i = i * BS, hi_i = min(N, lo_i + BS) - 1;
+      for (int j = threadIdx.x; j < nb; j += 256) {
+        const int lo_j = j * BS, hi_j = min(N, lo_j + BS) - 1;
+        bool keep;
+        if (g.layout == SA_LAYOUT_FRAME_MAJOR) {
+          // shared spatial position: slot m holds position m / T
+          keep = !(hi_j / p.T < lo_i / p.T || hi_i / p.T < lo_j / p.T);
+        } else {
+          // frame ranges within frame_radius
+          const int fi0 = lo_i / HW, fi1 = hi_i / HW, fj0 = lo_j / HW, fj1 = hi_j / HW;
+          const int gap = max(0, max(fj0 - fi1, fi0 - fj1));
+          keep = gap <= p.frame_radius;
+        }
+        if (j < p.sink_blocks) keep = true;
+        if (keep) atomicOr(&bits[j / 32], 1u << (j % 32));
+      }
+    } else if (p.kind == SA_MASK_EXPLICIT) {
+      const uint32_t* src = p.explicit_bits + ((size_t)bh * p.NB + i) * p.W32;
+      for (int w = threadIdx.x; w < W32; w += 256) {
+        uint32_t word = src[w];
+        if (32 * w + 32 > nb) word &= (nb - 32 * w) >= 32 ? 0xffffffffu : ((1u << (nb - 32 * w)) - 1u);
+        for (int b = 0; b < 32; ++b)
+          if (((word >> b) & 1u) && !block_valid(g, 32 * w + b, p.T, p.H, p.W)) word &= ~(1u << b);
+        bits[w] = word;
+      }
+    }
+  }
+  __syncthreads();
+  // emit: bit row, ascending list, count
+  uint32_t* brow = p.bits + ((size_t)bh * p.NB + i) * p.W32;
+  for (int w = threadIdx.x; w < p.W32; w += 256) brow[w] = w < W32 ? bits[w] : 0u;
+  __shared__ int wcount[kMaxBlocks / 32 + 1];
+  for (int w = threadIdx.x; w < W32; w += 256) wcount[w] = __popc(bits[w]);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int w = 0; w < W32; ++w) { const int c = wcount[w]; wcount[w] = run; run += c; }
+    wcount[W32] = run;
+    p.counts[(size_t)bh * p.NB + i] = run;
+    atomicAdd(&p.heads[bh].kept, run);
+  }
+  __syncthreads();
+  int* crow = p.cols + ((size_t)bh * p.NB + i) * p.NB;
+  for (int w = threadIdx.x; w < W32; w += 256) {
+    uint32_t word = bits[w];
+    int pos = wcount[w];
+    while (word) {
+      const int b = __ffs(word) - 1;
+      crow[pos++] = 32 * w + b;
+      word &= word - 1;
+    }
+  }
+}
+
+__global__ void zero_counts_kernel(int* counts, size_t n) {
+  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n;
+       e += (size_t)gridDim.x * blockDim.x)
+    counts[e] = 0;
+}
+
+}  // namespace
+
+cudaError_t launch_head_init(const HeadInitParams& p, cudaStream_t st) {
+  head_init_kernel<<<(p.BH + 127) / 128, 128, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_fm(const PermuteParams& p, int BH, cudaStream_t st) {
+  const int vec_per_row = p.d / 8;
+  const int rows_per_cta = 256 / vec_per_row;
+  dim3 grid((p.n_pad + rows_per_cta - 1) / rows_per_cta, BH);
+  permute_fm_kernel<<<grid, 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pool_sics(const PoolParams& p, int BH, int max_nb, cudaStream_t st) {
+  dim3 grid(max_nb, p.C, BH);
+  if (p.d == 128) pool_sics_kernel<128><<<grid, 256, 0, st>>>(p);
+  else if (p.d == 64) pool_sics_kernel<64><<<grid, 256, 0, st>>>(p);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_choose(const ChooseParams& p, int BH, cudaStream_t st) {
+  choose_kernel<<<BH, 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pooled_scores(const ScoreParams& p, int BH, int d, cudaStream_t st) {
+  dim3 grid((p.NB + 63) / 64, (p.NB + 63) / 64, BH);
+  const size_t sm = 2 * 64 * (d + 1) * sizeof(float);
+  if (d == 128) {
+    cudaFuncSetAttribute(pooled_scores_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    pooled_scores_kernel<128><<<grid, 256, sm, st>>>(p);
+  } else if (d == 64) {
+    pooled_scores_kernel<64><<<grid, 256, sm, st>>>(p);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const SelectParams& p, int BH, cudaStream_t st) {
+  dim3 grid(p.NB, BH);
+  select_kernel<<<grid, 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero_counts(int* counts, size_t n, cudaStream_t st) {
+  zero_counts_kernel<<<256, 256, 0, st>>>(counts, n);
+  return cudaGetLastError();
+}
+
+}  // namespace sa

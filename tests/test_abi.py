@@ -1,0 +1,90 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every
+symbol include/sparse_attn.h declares, sizes workspaces and rejects bad
+arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_video_b200 import _native as N
+from sparse_attention_video_b200 import make_policy
+from synthetic import CONFIGS
+from tests import _cases as C
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "sparse_attn.h")
+
+
+def _declared():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"SA_API\s+(?:const\s+)?\w+\*?\s+\**(sparse_attn_\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_exported_api():
+    assert _declared() == sorted(N.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    L = N.lib()
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_struct_sizes_match_header_layout():
+    # sa_problem: 6 ints; sa_head_info: 10 int32 + 4 float + 2 int32
+    assert ctypes.sizeof(N.Problem) == 24
+    assert ctypes.sizeof(N.HeadInfo) == 64
+
+
+@pytest.mark.parametrize("name", list(CONFIGS))
+def test_workspace_sizes_for_every_workload(name):
+    wl = CONFIGS[name]
+    pol = make_policy(**C.policy_kwargs(wl))
+    m, s = N.workspace_size(N.Problem(wl.batch, wl.heads, wl.T, wl.H, wl.W, wl.head_dim), pol)
+    assert m > 0 and s >= 256
+    assert m % 256 == 0 and s % 256 == 0
+
+
+def test_mask_workspace_holds_bits_and_lists():
+    wl = CONFIGS["sta_wan21_1p3b_480p"]
+    pol = make_policy(**C.policy_kwargs(wl))
+    pr = N.Problem(1, wl.heads, wl.T, wl.H, wl.W, wl.head_dim)
+    m, _ = N.workspace_size(pr, pol)
+    nb = 336
+    assert m >= wl.heads * nb * nb * 4                   # ascending key-block lists
+    assert N.export_bytes(pr, pol, N.SA_EXPORT_BLOCK_BITS) == wl.heads * nb * ((nb + 31) // 32) * 4
+    assert N.export_bytes(pr, pol, N.SA_EXPORT_HEAD_INFO) == wl.heads * 64
+
+
+def test_invalid_arguments_are_rejected_on_the_host():
+    L = N.lib()
+    wl = CONFIGS["sta_wan21_1p3b_480p"]
+    pol = make_policy(**C.policy_kwargs(wl))
+    m, s = ctypes.c_size_t(), ctypes.c_size_t()
+    bad_dim = N.Problem(1, 12, 21, 30, 52, 96)
+    assert L.sparse_attn_workspace_size(ctypes.byref(bad_dim), ctypes.byref(pol), ctypes.byref(m),
+                                        ctypes.byref(s)) == N.SA_ERR_UNSUPPORTED
+    zero = N.Problem(1, 0, 21, 30, 52, 128)
+    assert L.sparse_attn_workspace_size(ctypes.byref(zero), ctypes.byref(pol), ctypes.byref(m),
+                                        ctypes.byref(s)) == N.SA_ERR_INVALID_ARG
+    pr = N.Problem(1, 12, 21, 30, 52, 128)
+    even = make_policy("sta", tile=(4, 4, 8), window=(3, 2, 3))
+    assert L.sparse_attn_workspace_size(ctypes.byref(pr), ctypes.byref(even), ctypes.byref(m),
+                                        ctypes.byref(s)) == N.SA_ERR_INVALID_ARG
+    wrong_tile = make_policy("sta", tile=(4, 4, 4), window=(3, 3, 3))  # 64 tokens != block 128
+    assert L.sparse_attn_workspace_size(ctypes.byref(pr), ctypes.byref(wrong_tile), ctypes.byref(m),
+                                        ctypes.byref(s)) == N.SA_ERR_INVALID_ARG
+    # null / misaligned device pointers never reach the device
+    assert L.sparse_attn_forward(ctypes.byref(pr), ctypes.byref(pol), None, None, None, None, None,
+                                 None, None, None) == N.SA_ERR_INVALID_ARG
+    assert L.sparse_attn_build_mask(ctypes.byref(pr), ctypes.byref(pol), None, None, 0x1001, 0x2000,
+                                    None) == N.SA_ERR_WORKSPACE
+    st = make_policy("spatiotemporal", block=128)                     # head types missing
+    assert L.sparse_attn_workspace_size(ctypes.byref(pr), ctypes.byref(st), ctypes.byref(m),
+                                        ctypes.byref(s)) == N.SA_ERR_INVALID_ARG
+
+
+def test_strerror_covers_every_code():
+    for code in range(7):
+        assert N.strerror(code) and N.strerror(code) != "unknown status"
+    assert N.strerror(99) == "unknown status"
