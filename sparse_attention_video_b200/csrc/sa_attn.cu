@@ -154,6 +154,12 @@ __device__ __forceinline__ bool block_pad_mask(const HeadGeom& g, int blk, int T
   return true;
 }
 
+// Timeout site code recorded in status word 1: role (1 producer, 2 MMA,
+// 3 softmax), barrier id, key-block iteration.
+__device__ __forceinline__ uint32_t site(uint32_t role, uint32_t bar, int j) {
+  return (role << 24) | (bar << 16) | ((uint32_t)j & 0xFFFFu);
+}
+
 template <int D, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
@@ -170,7 +176,8 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   const int qb = blockIdx.x;
   const int bh = blockIdx.y;
   const HeadGeom g = p.heads[bh];
-  if (qb >= g.nb) return;  // uniform across the CTA, before any allocation
+  // uniform across the CTA, before any allocation
+  if (qb >= g.nb || grid_aborted(p.status)) return;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const size_t row_base = ((size_t)bh * p.NB + qb);
@@ -200,6 +207,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     fence_proxy_async_smem();
   }
   if (warp == 1) {
+    __syncwarp();
     tmem_alloc(&bars->tmem_base, L::kTmemCols);
     tmem_relinquish();
   }
@@ -225,10 +233,13 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         const int st = j % kStages, rnd = j / kStages;
         const int kb = cols[j];
         if (kb < 0 || kb >= g.nb) { atomicOr(status, SA_DEVFLAG_BOUNDS); *abort = 1; break; }
-        if (!mbar_wait(&bars->k_empty[st], (rnd & 1) ^ 1, abort, status)) break;
+        if (!mbar_wait(&bars->k_empty[st], (rnd & 1) ^ 1, abort, status, site(1, 1, j))) break;
         mbar_arrive_expect_tx(&bars->k_full[st], L::kKVBytes);
         load_block<D, BN>(kmaps, g, bh, kb, sK + st * L::kKVBytes, &bars->k_full[st]);
-        if (!mbar_wait(&bars->v_empty[st], (rnd & 1) ^ 1, abort, status)) { issued = j * 2 + 1; break; }
+        if (!mbar_wait(&bars->v_empty[st], (rnd & 1) ^ 1, abort, status, site(1, 2, j))) {
+          issued = j * 2 + 1;
+          break;
+        }
         mbar_arrive_expect_tx(&bars->v_full[st], L::kKVBytes);
         load_block<D, BN>(vmaps, g, bh, kb, sV + st * L::kKVBytes, &bars->v_full[st]);
         issued = j * 2 + 2;
@@ -237,9 +248,8 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         // Let copies already in flight land before the CTA's memory is released.
         for (int j = (issued / 2 > kStages ? issued / 2 - kStages : 0); j < (issued + 1) / 2; ++j) {
           const int st = j % kStages, par = (j / kStages) & 1;
-          for (uint32_t n = 0; n < kWaitPolls && !mbar_try_wait(&bars->k_full[st], par); ++n) {}
-          if (2 * j + 1 < issued)
-            for (uint32_t n = 0; n < kWaitPolls && !mbar_try_wait(&bars->v_full[st], par); ++n) {}
+          mbar_drain(&bars->k_full[st], par);
+          if (2 * j + 1 < issued) mbar_drain(&bars->v_full[st], par);
         }
       }
     }
@@ -250,8 +260,9 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, false, true);
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
       auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait(&bars->p_full, i & 1, abort, status)) return false;
-        if (!mbar_wait(&bars->v_full[i % kStages], (i / kStages) & 1, abort, status)) return false;
+        if (!mbar_wait(&bars->p_full, i & 1, abort, status, site(2, 3, i))) return false;
+        if (!mbar_wait(&bars->v_full[i % kStages], (i / kStages) & 1, abort, status, site(2, 4, i)))
+          return false;
         tc_fence_after();
         const uint32_t vbase = aV + (i % kStages) * L::kKVBytes;
 #pragma unroll
@@ -265,11 +276,17 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         umma_commit(&bars->v_empty[i % kStages]);
         return true;
       };
-      bool ok = mbar_wait(&bars->q_full, 0, abort, status);
+      bool ok = mbar_wait(&bars->q_full, 0, abort, status, site(2, 5, 0));
       for (int j = 0; ok && j < n_keys; ++j) {
         const int st = j % kStages, sb = j & 1;
-        if (!mbar_wait(&bars->k_full[st], (j / kStages) & 1, abort, status)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait(&bars->s_free[sb], ((j - 2) >> 1) & 1, abort, status)) { ok = false; break; }
+        if (!mbar_wait(&bars->k_full[st], (j / kStages) & 1, abort, status, site(2, 6, j))) {
+          ok = false;
+          break;
+        }
+        if (j >= 2 && !mbar_wait(&bars->s_free[sb], ((j - 2) >> 1) & 1, abort, status, site(2, 7, j))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t kbase = aK + st * L::kKVBytes;
 #pragma unroll
@@ -286,7 +303,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       if (ok) issue_pv(n_keys - 1);
       // Every MMA issued above must finish before tensor memory is freed.
       umma_commit(&bars->drain);
-      for (uint32_t n = 0; n < kWaitPolls && !mbar_try_wait(&bars->drain, 0); ++n) {}
+      mbar_drain(&bars->drain, 0);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
@@ -301,7 +318,12 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       const int kb = cols[j];
       uint32_t pw[BN / 32];
       const bool pad = block_pad_mask<BN>(g, kb, p.T, p.H, p.W, pw);
-      if (!mbar_wait(&bars->s_full[sb], (j >> 1) & 1, abort, status)) { ok = false; break; }
+      // a warp either waits out a barrier together or gives up together
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (j >> 1) & 1, abort, status,
+                                             site(3, 8, j)))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < BN; c += 32) tmem_ld32(tS[sb] + lane_off + c, s + c);
@@ -334,10 +356,17 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       }
       // P buffer and O are read/written by PV of the previous block: wait for it.
       if (j >= 1) {
-        if (!mbar_wait(&bars->o_done, (j - 1) & 1, abort, status)) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done, (j - 1) & 1, abort, status,
+                                               site(3, 9, j)))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        if (rescale && m != -INFINITY) {
-          const float alpha = ex2_approx(m - m_use);
+        // tcgen05.ld/st are warp-collective: the whole warp rescales when any
+        // of its rows needs it; rows that do not scale by 1.
+        const bool need = rescale && m != -INFINITY;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2_approx(m - m_use) : 1.f;
           l *= alpha;
           float o[32];
 #pragma unroll
@@ -373,7 +402,8 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     }
     // ------------------------------------------------------------ epilogue
     if (ok && n_keys > 0) {
-      ok = mbar_wait(&bars->o_done, (n_keys - 1) & 1, abort, status);
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (n_keys - 1) & 1, abort, status,
+                                             site(3, 10, n_keys)));
       tc_fence_after();
     }
     const int tok = (r < BN) ? slot_to_token(g, qb, r, BN, p.T, p.H, p.W) : -1;
@@ -411,6 +441,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }

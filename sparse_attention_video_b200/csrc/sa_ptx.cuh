@@ -46,26 +46,59 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Poll budget: each try_wait may itself block for a hardware time slice, so
-// this bound is several seconds of wall time on B200, far above any legal
-// wait inside one kernel.
-constexpr uint32_t kWaitPolls = 1u << 24;
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wall-time limit of one wait. Every legal wait inside these kernels lasts
+// microseconds to milliseconds; one second means an arrival was lost.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+
+// Record a timeout in the status word: flag bit, and in word 1 the first
+// site (caller-chosen code) that gave up.
+__device__ __forceinline__ void report_timeout(uint32_t* status, uint32_t site) {
+  if (!status) return;
+  atomicOr(status, (uint32_t)SA_DEVFLAG_TIMEOUT);
+  atomicCAS(status + 1, 0u, site);
+}
+
+__device__ __forceinline__ bool grid_aborted(const uint32_t* status) {
+  return status && (*reinterpret_cast<const volatile uint32_t*>(status) & SA_DEVFLAG_TIMEOUT);
+}
 
 // Bounded wait. ``abort`` is a shared flag: once any thread of the CTA gives
-// up, every later wait returns false at once.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort, uint32_t* status) {
+// up, every later wait of the CTA returns false at once; a timeout recorded by
+// another CTA in the status word ends the wait as well.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint32_t* status, uint32_t site = 0) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
   uint32_t polls = 0;
   while (!mbar_try_wait(bar, parity)) {
     if (*abort) return false;
-    if (++polls > kWaitPolls) {
-      *abort = 1;
-      if (status) atomicOr(status, (uint32_t)SA_DEVFLAG_TIMEOUT);
-      return false;
+    if ((++polls & 255u) == 0) {
+      if (grid_aborted(status)) { *abort = 1; return false; }
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        report_timeout(status, site ? site : 0xFFFFu);
+        return false;
+      }
     }
-    if (polls > 64) __nanosleep(32);
+    if (polls > 64) __nanosleep(64);
   }
   return true;
+}
+
+// Bounded wait that ignores the abort flags: used to let copies and MMAs that
+// are already in flight finish before a CTA that gave up releases its memory.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+    __nanosleep(256);
+  }
 }
 
 // ------------------------------------------------------------------ TMA

@@ -128,10 +128,21 @@ def make_qkv(wl, heads=None, threads=None):
         arr, b, j, key = job
         arr[b, j] = _one_head(grid, wl.head_dim, key)
 
-    if nthreads > 1 and len(jobs) > 1:
-        with ThreadPoolExecutor(nthreads) as ex:
-            list(ex.map(run, jobs))
-    else:
-        for job in jobs:
-            run(job)
+    # Each worker runs single-threaded BLAS: nesting a threaded BLAS inside a
+    # thread pool oversubscribes many-core hosts badly.
+    try:
+        from threadpoolctl import threadpool_limits
+        limit = threadpool_limits(limits=1, user_api="blas")
+    except Exception:
+        limit = None
+    try:
+        if nthreads > 1 and len(jobs) > 1:
+            with ThreadPoolExecutor(nthreads) as ex:
+                list(ex.map(run, jobs))
+        else:
+            for job in jobs:
+                run(job)
+    finally:
+        if limit is not None:
+            limit.unregister()
     return out
