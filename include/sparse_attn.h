@@ -184,7 +184,9 @@ SA_API int sparse_attn_attend(const sa_problem* problem, const sa_policy* policy
 
 /* ---------------------------------------------------------------- inspection
  * Copy one part of a built mask to host memory and wait for the copy.
- *   SA_EXPORT_BLOCK_BITS   uint32 [batch*heads][nb][ceil(nb/32)]
+ *   SA_EXPORT_BLOCK_BITS   uint32 [batch*heads][nb][ceil(nb/32)], nb the largest block
+ *                          count of the policy's layouts; rows at or past a head's own
+ *                          block count (sa_head_info.nb) are not written
  *   SA_EXPORT_HEAD_INFO    sa_head_info [batch*heads]
  *   SA_EXPORT_FG_BITS      uint32 [batch*heads][G][ceil(N/32)], G = ceil(N/fg_group)
  *   SA_EXPORT_FG_TAU       float  [batch*heads]
@@ -218,6 +220,33 @@ SA_API int sparse_attn_mask_export(const sa_problem* problem, const sa_policy* p
  * since the last sparse_attn_build_mask: SA_OK, SA_ERR_DEVICE_TIMEOUT or
  * SA_ERR_DEVICE_BOUNDS. If ``clear`` is nonzero the word is reset. */
 SA_API int sparse_attn_status(void* scratch_ws, void* stream, int clear);
+
+/* ---------------------------------------------------------------- no allocation
+ * The papers have no counterpart to this entry point. It is for callers that
+ * cannot allocate device memory when they build a mask: code running inside
+ * another framework's execute/enqueue callback (which is handed a stream and
+ * must not allocate), latency-critical paths where cudaMalloc/cudaFree may
+ * synchronize the device, and processes that reserve all of their device
+ * memory once at start-up.
+ *
+ * Same as sparse_attn_build_mask, except that the scratch workspace is a
+ * static device array of SA_STATIC_SCRATCH_BYTES inside the library, which
+ * every GPU that loads the library holds until the process exits. The caller
+ * still passes q, k and mask_ws. Problems whose scratch (the scratch_bytes of
+ * sparse_attn_workspace_size) exceeds SA_STATIC_SCRATCH_BYTES are rejected
+ * with SA_ERR_UNSUPPORTED before anything is enqueued. No device memory is
+ * allocated by this call.
+ *
+ * The first call on a device looks up the array's device address with that
+ * device current; make that first call before any stream capture. All calls
+ * share the one array: calls whose work can overlap on the GPU (unordered
+ * streams) race on it. The status word of this variant lives in the array and
+ * is not reported by sparse_attn_status. Asynchronous on ``stream``.
+ */
+#define SA_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
+SA_API int sparse_attn_build_mask_static(const sa_problem* problem, const sa_policy* policy,
+                                         const void* q, const void* k, void* mask_ws,
+                                         void* stream);
 
 /* Static description of a status code. Never NULL. */
 SA_API const char* sparse_attn_strerror(int status);

@@ -24,7 +24,9 @@ SA_EXPORT_BLOCK_BITS, SA_EXPORT_HEAD_INFO, SA_EXPORT_FG_BITS, SA_EXPORT_FG_TAU =
 EXPORTED = ("sparse_attn_workspace_size", "sparse_attn_build_mask", "sparse_attn_forward",
             "sparse_attn_permute", "sparse_attn_attend",
             "sparse_attn_export_bytes", "sparse_attn_mask_export", "sparse_attn_status",
-            "sparse_attn_strerror")
+            "sparse_attn_build_mask_static", "sparse_attn_strerror")
+
+SA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class Problem(ctypes.Structure):
@@ -78,6 +80,7 @@ def lib():
         L.sparse_attn_export_bytes.argtypes = [P, PP, ctypes.c_int, ctypes.POINTER(sz)]
         L.sparse_attn_mask_export.argtypes = [P, PP, vp, ctypes.c_int, vp, sz, vp]
         L.sparse_attn_status.argtypes = [vp, vp, ctypes.c_int]
+        L.sparse_attn_build_mask_static.argtypes = [P, PP, vp, vp, vp, vp]
         L.sparse_attn_strerror.argtypes = [ctypes.c_int]
         L.sparse_attn_strerror.restype = ctypes.c_char_p
         for name in EXPORTED[:-1]:
@@ -138,6 +141,13 @@ def mask_export(problem, policy, mask_ws, what, host_ptr, nbytes, stream=0):
     _check(lib().sparse_attn_mask_export(ctypes.byref(problem), ctypes.byref(policy), mask_ws,
                                          what, host_ptr, nbytes, stream),
            "sparse_attn_mask_export")
+
+
+def build_mask_static(problem, policy, q, k, mask_ws, stream=0):
+    """sparse_attn_build_mask with the library's static scratch array."""
+    _check(lib().sparse_attn_build_mask_static(ctypes.byref(problem), ctypes.byref(policy), q, k,
+                                               mask_ws, stream),
+           "sparse_attn_build_mask_static")
 
 
 def status(scratch_ws, stream=0, clear=False):
