@@ -44,6 +44,9 @@ def _args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-mask comparison")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run only this many heads (half of them temporal); for small "
+                         "profiler captures, not for bench lines")
     return ap.parse_args()
 
 
@@ -219,6 +222,8 @@ def main():
                                 device_id=dev)
 
     wl = CONFIGS[WORKLOAD]
+    if args.heads:
+        wl = wl.with_(heads=args.heads, temporal_heads=tuple(range(args.heads // 2, args.heads)))
     wl_r = wl.with_(config_id=wl.config_id + 1000 * rank)      # independent problem per rank
     log("generating inputs")
     x = make_qkv(wl_r)
