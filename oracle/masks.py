@@ -249,10 +249,11 @@ def fg_threshold(scores, keep_fraction):
     The printed pooling rule compares a monotone function of k . q_avg with an
     undefined tau_1; the workload fixes the threshold by the fraction of
     (group, key) slices to retain, so tau is the order statistic that keeps
-    that fraction.
+    that fraction. f is the keep fraction as a float32 value (the precision
+    in which it is specified to the kernels); the product is formed in float64.
     """
     flat = scores.reshape(-1)
-    r = int(math.ceil(keep_fraction * flat.size))
+    r = int(math.ceil(float(np.float32(keep_fraction)) * flat.size))
     return F32(np.partition(flat, flat.size - r)[flat.size - r]), r
 
 

@@ -140,8 +140,13 @@ MaskLayout mask_layout(const sa_problem& pr, const sa_policy& po) {
     const long long N = n_tokens(pr);
     L.G = ceil_div(N, po.fg_group);
     L.WN = ceil_div(N, 32);
+    L.P = ceil_div(N, 128);
+    L.cap = fg_list_cap_per_head(L.G, (int)N, po.fg_keep_fraction);
     L.off_fg_bits = take(sizeof(uint32_t) * (size_t)L.BH * L.G * L.WN);
     L.off_fg_tau = take(sizeof(float) * (size_t)L.BH);
+    L.off_fg_counts = take(sizeof(uint32_t) * (size_t)L.BH * L.P);
+    L.off_fg_offsets = take(sizeof(uint32_t) * (size_t)L.BH * (L.P + 1));
+    L.off_fg_list = take(sizeof(uint32_t) * (size_t)L.BH * L.cap);
   }
   L.total = std::max<size_t>(off, 256);
   return L;
@@ -166,7 +171,7 @@ ScratchLayout scratch_layout(const sa_problem& pr, const sa_policy& po, const Ma
     S.off_scores = take(sizeof(float) * (size_t)M.BH * M.NB * M.NB);
   }
   if (po.kind == SA_MASK_FG) {
-    S.off_fg_qbar = take(fg_qbar_bytes(M.BH, M.G, d));
+    S.off_fg_qsplit = take(fg_qsplit_bytes(M.BH, M.G, d));
     S.off_fg_hist = take(fg_hist_bytes(M.BH));
     S.off_fg_sel = take(fg_sel_bytes(M.BH));
   }
@@ -175,10 +180,7 @@ ScratchLayout scratch_layout(const sa_problem& pr, const sa_policy& po, const Ma
 }
 
 // ------------------------------------------------------------------ tensor maps
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+typedef EncodeFn EncodeTiledFn;
 
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
@@ -217,6 +219,19 @@ bool map_5d(CUtensorMap* m, const void* base, const sa_problem& pr, const int* t
   cuuint32_t box[5] = {64, (cuuint32_t)tile[2], (cuuint32_t)tile[1], (cuuint32_t)tile[0], 1};
   cuuint32_t es[5] = {1, 1, 1, 1, 1};
   return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims,
+                     strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over [rows][d] bf16 with a (64, 1) box: the tensor map a
+// tile::gather4 load needs (one-row boxes, four row coordinates per load).
+bool map_rows(CUtensorMap* m, const void* base, long long rows, int d) {
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t es[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                      strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -268,10 +283,11 @@ extern "C" int sparse_attn_build_mask(const sa_problem* problem, const sa_policy
   if (cudaMemsetAsync(sw + S.off_status, 0, 256, st) != cudaSuccess) return SA_ERR_CUDA;
 
   if (po.kind == SA_MASK_FG) {
+    if (!encode_fn()) return SA_ERR_CUDA;
     FgBuildParams fp{};
     fp.q = static_cast<const __nv_bfloat16*>(q);
     fp.k = static_cast<const __nv_bfloat16*>(k);
-    fp.qbar = reinterpret_cast<float*>(sw + S.off_fg_qbar);
+    fp.qsplit = reinterpret_cast<__nv_bfloat16*>(sw + S.off_fg_qsplit);
     fp.hist = reinterpret_cast<uint32_t*>(sw + S.off_fg_hist);
     fp.sel = reinterpret_cast<uint32_t*>(sw + S.off_fg_sel);
     fp.bits = reinterpret_cast<uint32_t*>(mw + M.off_fg_bits);
@@ -279,7 +295,15 @@ extern "C" int sparse_attn_build_mask(const sa_problem* problem, const sa_policy
     fp.status = reinterpret_cast<uint32_t*>(sw + S.off_status);
     fp.BH = BH; fp.N = N; fp.d = d; fp.group = po.fg_group; fp.G = M.G; fp.WN = M.WN;
     fp.keep_fraction = po.fg_keep_fraction;
-    return cuda_status(launch_fg_build(fp, st));
+    FgListParams& lp = fp.lists;
+    lp.bits = fp.bits;
+    lp.counts = reinterpret_cast<uint32_t*>(mw + M.off_fg_counts);
+    lp.offsets = reinterpret_cast<uint32_t*>(mw + M.off_fg_offsets);
+    lp.list = reinterpret_cast<uint32_t*>(mw + M.off_fg_list);
+    lp.status = fp.status;
+    lp.cap_per_head = M.cap;
+    lp.BH = BH; lp.P = M.P; lp.G = M.G; lp.WN = M.WN; lp.groups_per_tile = 128 / po.fg_group;
+    return cuda_status(launch_fg_build(fp, encode_fn(), st));
   }
 
   SelectParams sp{};
@@ -409,17 +433,22 @@ extern "C" int sparse_attn_attend(const sa_problem* problem, const sa_policy* po
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)c.d);
 
   if (po.kind == SA_MASK_FG) {
-    FgAttnParams fp{};
-    fp.q = static_cast<const __nv_bfloat16*>(q);
-    fp.k = static_cast<const __nv_bfloat16*>(k);
-    fp.v = static_cast<const __nv_bfloat16*>(v);
-    fp.bits = reinterpret_cast<const uint32_t*>(c.mw + c.M.off_fg_bits);
-    fp.o = static_cast<__nv_bfloat16*>(o);
-    fp.lse = lse;
-    fp.status = status;
-    fp.BH = c.BH; fp.N = c.N; fp.d = c.d; fp.group = po.fg_group; fp.G = c.M.G; fp.WN = c.M.WN;
-    fp.scale_log2 = scale_log2;
-    return cuda_status(launch_fg_attn(fp, c.st));
+    AttnMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (!map_3d(&maps.q[0], q, c.BH, c.N, c.d, 128)) return SA_ERR_CUDA;
+    if (!map_rows(&maps.k[0], k, (long long)c.BH * c.N, c.d)) return SA_ERR_CUDA;
+    if (!map_rows(&maps.v[0], v, (long long)c.BH * c.N, c.d)) return SA_ERR_CUDA;
+    AttnParams ap{};
+    ap.o = static_cast<__nv_bfloat16*>(o);
+    ap.lse = lse;
+    ap.status = status;
+    ap.BH = c.BH; ap.NB = c.M.P; ap.T = pr.T; ap.H = pr.H; ap.W = pr.W; ap.N = c.N;
+    ap.scale_log2 = scale_log2;
+    ap.fg_list = reinterpret_cast<const uint32_t*>(c.mw + c.M.off_fg_list);
+    ap.fg_offsets = reinterpret_cast<const uint32_t*>(c.mw + c.M.off_fg_offsets);
+    ap.fg_cap = c.M.cap;
+    ap.fg_groups_per_tile = 128 / po.fg_group;
+    return cuda_status(launch_attn_gather(c.d, maps, ap, c.st));
   }
 
   const void* src[3] = {q, k, v};

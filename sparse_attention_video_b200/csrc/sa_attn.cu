@@ -65,6 +65,8 @@ struct Bars {
   uint64_t p_full;
   uint64_t o_done;
   uint64_t drain;
+  uint64_t m_full[2], m_empty[2];   // gather mode: per-chunk group-membership masks
+  uint32_t masks[2][8];             // [chunk & 1][first group words 0-3, second group 4-7]
   uint32_t tmem_base;
   int abort;
 };
@@ -94,6 +96,17 @@ __device__ __forceinline__ void load_block(const CUtensorMap* maps, const HeadGe
     if (map >= 2) tma_load_5d(d, m, bar, h * 64, c1, c2, c3, bh);
     else tma_load_3d(d, m, bar, h * 64, c1, bh);
   }
+}
+
+// Four rows (row indices r0..r3 of a 2-D [rows][d] map) x 64 columns into
+// four consecutive 128-byte rows of shared memory.
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uint64_t* bar, int c0,
+                                            int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0),
+        "r"(r0), "r"(r1), "r"(r2), "r"(r3) : "memory");
 }
 
 // Slot ``s`` of block ``blk`` -> original token index, or -1 for padding.
@@ -160,7 +173,12 @@ __device__ __forceinline__ uint32_t site(uint32_t role, uint32_t bar, int j) {
   return (role << 24) | (bar << 16) | ((uint32_t)j & 0xFFFFu);
 }
 
-template <int D, int BN>
+// kGather = false: blocks of a working layout, kept key blocks from the mask's
+// ascending lists. kGather = true (M x 1 key slices): the query tile is 128
+// contiguous queries (one or two groups); its keys are the union list of those
+// groups, gathered 128 rows at a time with TMA tile::gather4, and each row
+// masks keys outside its own group.
+template <int D, int BN, bool kGather>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   using L = Smem<D, BN>;
@@ -175,14 +193,30 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
 
   const int qb = blockIdx.x;
   const int bh = blockIdx.y;
-  const HeadGeom g = p.heads[bh];
-  // uniform across the CTA, before any allocation
-  if (qb >= g.nb || grid_aborted(p.status)) return;
+  HeadGeom g{};
+  int n_keys = 0;
+  const int* cols = nullptr;
+  uint32_t list_count = 0;
+  const uint32_t* list = nullptr;
+  if constexpr (kGather) {
+    g.layout = SA_LAYOUT_IDENTITY;
+    g.bt = 1; g.bh = 1; g.bw = BN; g.nt = 1; g.nh = 1; g.nw = p.NB; g.nb = p.NB;
+    if (qb >= p.NB || grid_aborted(p.status)) return;
+    const uint32_t* off = p.fg_offsets + (size_t)bh * (p.NB + 1);
+    const uint32_t begin = off[qb];
+    list_count = off[qb + 1] - begin;
+    list = p.fg_list + (size_t)bh * p.fg_cap + begin;
+    n_keys = (int)((list_count + BN - 1) / BN);
+  } else {
+    g = p.heads[bh];
+    // uniform across the CTA, before any allocation
+    if (qb >= g.nb || grid_aborted(p.status)) return;
+    const size_t row_base = ((size_t)bh * p.NB + qb);
+    n_keys = p.counts[row_base];
+    cols = p.cols + row_base * p.NB;
+  }
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const size_t row_base = ((size_t)bh * p.NB + qb);
-  const int n_keys = p.counts[row_base];
-  const int* cols = p.cols + row_base * p.NB;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -194,6 +228,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     mbar_init(&bars->p_full, 4);
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->drain, 1);
+    for (int b = 0; b < 2; ++b) { mbar_init(&bars->m_full[b], 1); mbar_init(&bars->m_empty[b], 4); }
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -220,7 +255,86 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   volatile int* abort = &bars->abort;
   uint32_t* status = p.status;
 
-  if (warp == 0) {
+  if (warp == 0 && kGather) {
+    // ------------------------------------------------------------ producer (gather)
+    if (n_keys > 0) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars->q_full, L::kHalvesD * BN * 128);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_3d(sQ + h * (BN * 128), &maps.q[0], &bars->q_full, h * 64, qb * BN, bh);
+      }
+      const int row0 = bh * p.N;
+      int issued_k = 0, issued_v = 0;
+      for (int j = 0; j < n_keys; ++j) {
+        const int st = j % kStages, rnd = j / kStages, mb = j & 1;
+        // list entries j*128 + lane + 32*s; key index in the low 30 bits, one
+        // membership bit per group of the tile in bits 30 and 31
+        uint32_t e[4];
+        bool val[4];
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4) {
+          const uint32_t idx = (uint32_t)j * BN + lane + 32 * s4;
+          val[s4] = idx < list_count;
+          e[s4] = val[s4] ? __ldg(list + idx) : 0u;
+        }
+        uint32_t m0[4], m1[4];
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4) {
+          m0[s4] = __ballot_sync(0xffffffffu, val[s4] && ((e[s4] >> 30) & 1u));
+          m1[s4] = p.fg_groups_per_tile == 2
+                       ? __ballot_sync(0xffffffffu, val[s4] && ((e[s4] >> 31) & 1u)) : m0[s4];
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->m_empty[mb], ((j >> 1) & 1) ^ 1, abort,
+                                               status, site(1, 3, j))))
+          break;
+        if (lane == 0) {
+#pragma unroll
+          for (int s4 = 0; s4 < 4; ++s4) { bars->masks[mb][s4] = m0[s4]; bars->masks[mb][4 + s4] = m1[s4]; }
+          mbar_arrive(&bars->m_full[mb]);
+        }
+        // rows 4*lane .. 4*lane+3 of the chunk for this lane's gather4
+        int rows[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int src = (4 * lane + i) & 31;
+          const uint32_t x0 = __shfl_sync(0xffffffffu, e[0], src);
+          const uint32_t x1 = __shfl_sync(0xffffffffu, e[1], src);
+          const uint32_t x2 = __shfl_sync(0xffffffffu, e[2], src);
+          const uint32_t x3 = __shfl_sync(0xffffffffu, e[3], src);
+          const int sel = lane >> 3;
+          const uint32_t x = sel == 0 ? x0 : sel == 1 ? x1 : sel == 2 ? x2 : x3;
+          rows[i] = row0 + (int)(x & 0x3FFFFFFFu);
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->k_empty[st], (rnd & 1) ^ 1, abort, status,
+                                               site(1, 1, j))))
+          break;
+        if (lane == 0) mbar_arrive_expect_tx(&bars->k_full[st], L::kKVBytes);
+        __syncwarp();
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+          tma_gather4(sK + st * L::kKVBytes + h * (BN * 128) + lane * 512, &maps.k[0],
+                      &bars->k_full[st], h * 64, rows[0], rows[1], rows[2], rows[3]);
+        issued_k = j + 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->v_empty[st], (rnd & 1) ^ 1, abort, status,
+                                               site(1, 2, j))))
+          break;
+        if (lane == 0) mbar_arrive_expect_tx(&bars->v_full[st], L::kKVBytes);
+        __syncwarp();
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+          tma_gather4(sV + st * L::kKVBytes + h * (BN * 128) + lane * 512, &maps.v[0],
+                      &bars->v_full[st], h * 64, rows[0], rows[1], rows[2], rows[3]);
+        issued_v = j + 1;
+      }
+      if (*abort && lane == 0) {
+        for (int j = max(0, issued_k - kStages); j < issued_k; ++j)
+          mbar_drain(&bars->k_full[j % kStages], (j / kStages) & 1);
+        for (int j = max(0, issued_v - kStages); j < issued_v; ++j)
+          mbar_drain(&bars->v_full[j % kStages], (j / kStages) & 1);
+      }
+    }
+  } else if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n_keys > 0) {
       const CUtensorMap* qmaps = maps.q;
@@ -315,9 +429,22 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     bool ok = true;
     for (int j = 0; j < n_keys; ++j) {
       const int sb = j & 1;
-      const int kb = cols[j];
       uint32_t pw[BN / 32];
-      const bool pad = block_pad_mask<BN>(g, kb, p.T, p.H, p.W, pw);
+      bool pad = true;
+      if constexpr (kGather) {
+        // this row's group-membership bits for the chunk's 128 keys
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->m_full[sb], (j >> 1) & 1, abort, status,
+                                               site(3, 11, j)))) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int w = 0; w < BN / 32; ++w) pw[w] = bars->masks[sb][(r < 64 ? 0 : 4) + w];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->m_empty[sb]);
+      } else {
+        pad = block_pad_mask<BN>(g, cols[j], p.T, p.H, p.W, pw);
+      }
       // a warp either waits out a barrier together or gives up together
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (j >> 1) & 1, abort, status,
                                              site(3, 8, j)))) {
@@ -449,10 +576,10 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
 
 }  // namespace
 
-template <int D, int BN>
+template <int D, int BN, bool kGather>
 static cudaError_t launch_one(const AttnMaps& maps, const AttnParams& p, cudaStream_t stream) {
   using L = Smem<D, BN>;
-  auto kern = attn_fwd_kernel<D, BN>;
+  auto kern = attn_fwd_kernel<D, BN, kGather>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   dim3 grid(p.NB, p.BH);
@@ -462,9 +589,16 @@ static cudaError_t launch_one(const AttnMaps& maps, const AttnParams& p, cudaStr
 
 cudaError_t launch_attn_fwd(int head_dim, int block, const AttnMaps& maps, const AttnParams& p,
                             cudaStream_t stream) {
-  if (head_dim == 128 && block == 128) return launch_one<128, 128>(maps, p, stream);
-  if (head_dim == 64 && block == 128) return launch_one<64, 128>(maps, p, stream);
-  if (head_dim == 64 && block == 64) return launch_one<64, 64>(maps, p, stream);
+  if (head_dim == 128 && block == 128) return launch_one<128, 128, false>(maps, p, stream);
+  if (head_dim == 64 && block == 128) return launch_one<64, 128, false>(maps, p, stream);
+  if (head_dim == 64 && block == 64) return launch_one<64, 64, false>(maps, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_gather(int head_dim, const AttnMaps& maps, const AttnParams& p,
+                               cudaStream_t stream) {
+  if (head_dim == 128) return launch_one<128, 128, true>(maps, p, stream);
+  if (head_dim == 64) return launch_one<64, 128, true>(maps, p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -28,9 +28,17 @@ struct AttnParams {
   uint32_t* status;        // device status word
   int BH, NB, T, H, W, N;
   float scale_log2;        // log2(e) / sqrt(d)
+  // gather mode (M x 1 key slices): maps.q[0] is the 3-D query map, maps.k[0]
+  // and maps.v[0] are 2-D [BH*N][d] maps with one-row boxes for tile::gather4
+  const uint32_t* fg_list;     // [BH][fg_cap]
+  const uint32_t* fg_offsets;  // [BH][NB + 1]
+  long long fg_cap;
+  int fg_groups_per_tile;      // 2 for groups of 64, 1 for groups of 128
 };
 
 cudaError_t launch_attn_fwd(int head_dim, int block, const AttnMaps& maps, const AttnParams& p,
                             cudaStream_t stream);
+cudaError_t launch_attn_gather(int head_dim, const AttnMaps& maps, const AttnParams& p,
+                               cudaStream_t stream);
 
 }  // namespace sa

@@ -24,7 +24,10 @@ struct MaskLayout {
   int G = 0;         // FG groups per head
   int WN = 0;        // FG: ceil(N / 32)
   size_t off_head = 0, off_counts = 0, off_cols = 0, off_bits = 0;
-  size_t off_fg_bits = 0, off_fg_tau = 0, off_fg_order = 0;
+  int P = 0;         // FG: 128-query tiles per head
+  long long cap = 0; // FG: union-list capacity per head
+  size_t off_fg_bits = 0, off_fg_tau = 0;
+  size_t off_fg_counts = 0, off_fg_offsets = 0, off_fg_list = 0;
   size_t total = 0;
 };
 
@@ -35,7 +38,7 @@ struct ScratchLayout {
   size_t perm_stride = 0;          // bytes of one permuted tensor
   size_t off_qbar = 0, off_kbar = 0, off_sics = 0;  // [BH][C][NB][d] f32, [BH][C][NB] f32
   size_t off_scores = 0;           // [BH][NB][NB] f32
-  size_t off_fg_qbar = 0;          // [BH][G][d] f32
+  size_t off_fg_qsplit = 0;        // [3][BH][G_pad][d] bf16 terms of q_avg
   size_t off_fg_hist = 0;          // [BH][4096] u32 radix histogram
   size_t off_fg_sel = 0;           // [BH][4] u32 radix-select state
   size_t total = 0;

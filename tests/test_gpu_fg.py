@@ -1,0 +1,88 @@
+"""GPU parity of the fine-grained M x 1 key-slice path (B200 only).
+
+Through the C ABI: build the slice mask (group-mean queries, exact per-head
+threshold, bitmask), run the gather attention, then compare with the oracle:
+  - tau within 1e-4 relative of the oracle's R-th largest score;
+  - slice bits bit-exact, except slices whose score lies within 1e-4
+    relative of tau (either decision is correct there);
+  - O and LSE of the oracle's masked attention over the GPU's validated mask:
+    O max-abs <= 2e-2, mean-abs <= 2e-3, LSE max-abs <= 1e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention, masks
+from synthetic import CONFIGS, Workload, bf16_bits_to_f32, make_qkv
+from tests import _cases as C
+
+pytestmark = pytest.mark.gpu
+
+SMALL_FG = {
+    "fg_ragged_g64": Workload(name="fg_ragged_g64", config_id=111, T=6, H=12, W=20, heads=2,
+                              head_dim=128, kind="fg", fg_group=64, fg_keep_fraction=0.15),
+    "fg_g128_d64": Workload(name="fg_g128_d64", config_id=112, T=5, H=9, W=16, heads=2,
+                            head_dim=64, kind="fg", fg_group=128, fg_keep_fraction=0.2),
+    "fg_odd_groups": Workload(name="fg_odd_groups", config_id=113, T=3, H=7, W=19, heads=1,
+                              head_dim=128, kind="fg", fg_group=64, fg_keep_fraction=0.3),
+}
+
+
+def _dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def run_fg_case(wl, heads_check=None, groups_per_head=None, seed=0):
+    from sparse_attention_video_b200 import (SA_EXPORT_FG_BITS, SA_EXPORT_FG_TAU,
+                                             SparseAttention, make_policy)
+    x = make_qkv(wl)
+    q, k, v = (_dev(x[n]) for n in "qkv")
+    sa = SparseAttention(wl.batch, wl.heads, wl.T, wl.H, wl.W, wl.head_dim,
+                         make_policy(**C.policy_kwargs(wl)))
+    o, lse = sa(q, k, v)
+    torch.cuda.synchronize()
+    assert sa.status() == 0
+    N, M = wl.N, wl.fg_group
+    G, WN = math.ceil(N / M), math.ceil(N / 32)
+    tau = sa.export(SA_EXPORT_FG_TAU)
+    words = sa.export(SA_EXPORT_FG_BITS).reshape(wl.batch * wl.heads, G, WN)
+    o_np = bf16_bits_to_f32(o.view(torch.int16).cpu().numpy().view(np.uint16))
+    lse_np = lse.cpu().numpy()
+    rng = np.random.default_rng(seed)
+    heads_check = range(wl.heads) if heads_check is None else heads_check
+    for b in range(wl.batch):
+        for h in heads_check:
+            bh = b * wl.heads + h
+            qf, kf, vf = (bf16_bits_to_f32(x[n][b, h]) for n in "qkv")
+            s = masks.fg_scores(qf, kf, M)
+            tau_ref, r = masks.fg_threshold(s, wl.fg_keep_fraction)
+            assert abs(tau[bh] - tau_ref) <= C.REL_TIE * abs(tau_ref), (h, tau[bh], tau_ref)
+            keep_gpu = np.unpackbits(words[bh].view(np.uint8), bitorder="little").reshape(G, -1)[:, :N]
+            keep_gpu = keep_gpu.astype(bool)
+            keep_ref = masks.fg_keep(s, tau_ref)
+            diff = keep_gpu != keep_ref
+            if diff.any():
+                band = np.abs(s - tau_ref) <= C.REL_TIE * abs(tau_ref)
+                bad = diff & ~band
+                assert not bad.any(), (f"head {h}: {int(bad.sum())} slices differ outside the "
+                                       f"tie band; first {np.argwhere(bad)[:5].tolist()}")
+            kept = int(keep_gpu.sum())
+            n_band = int((np.abs(s - tau_ref) <= C.REL_TIE * abs(tau_ref)).sum())
+            assert abs(kept - r) <= n_band + int((s == tau_ref).sum()), (kept, r, n_band)
+            groups = range(G) if groups_per_head is None else rng.choice(
+                G, size=min(groups_per_head, G), replace=False)
+            o_ref, lse_ref = attention.slice_attention(qf, kf, vf, keep_gpu, M, groups)
+            rows = np.concatenate([np.arange(g * M, min(N, g * M + M)) for g in groups])
+            e = C.attention_errors(o_np[b, h, rows], lse_np[b, h, rows], o_ref[rows], lse_ref[rows])
+            C.check_errors(*e, where=f"{wl.name} head {h}")
+
+
+@pytest.mark.parametrize("name", list(SMALL_FG))
+def test_fg_small(name):
+    run_fg_case(SMALL_FG[name])
+
+
+def test_fg_full_size_sampled():
+    run_fg_case(CONFIGS["fg_slices_hunyuan_720p"], heads_check=[0, 23], groups_per_head=12)

@@ -223,7 +223,7 @@ def test_fg_threshold_keep_count_and_sort():
     s = masks.fg_scores(q, k, group)
     assert s.shape == (math.ceil(n / group), n)
     tau, r = masks.fg_threshold(s, 0.15)
-    assert r == math.ceil(0.15 * s.size)
+    assert r == math.ceil(float(np.float32(0.15)) * s.size)
     srt = np.sort(s.reshape(-1))[::-1]
     assert tau == srt[r - 1]
     kept = masks.fg_keep(s, tau)
