@@ -12,18 +12,22 @@
 // the mask logic lives in the loader); online softmax is exact (SPADE review,
 // axiom ledger), so the result equals masked softmax attention.
 //
-// Roles (256 threads):
-//   warp 0      TMA producer: Q once, then K and V of each kept key block into
+// Roles (320 threads):
+//   warps 0-7   softmax: two threads per row. Warp w reads tensor-memory lanes
+//               32*(w%4).. (row r = lane), and half w/4 of the row's columns.
+//               The two halves exchange their row maxima through shared
+//               memory and an mbarrier. The running maximum only moves when it
+//               grows by more than 2^8, so O is rescaled rarely; P and l use
+//               the same reference, which keeps the result exact. The 1/sqrt(d)
+//               scale is folded into one FFMA before exp2. Epilogue: O / l to
+//               bf16, each thread storing its half of the row at the query's
+//               original token row (the inverse permutation is fused here).
+//   warp 8      TMA producer: Q once, then K and V of each kept key block into
 //               a 2-stage ring. 3D tile layouts are gathered by one 5-D box per
 //               64 columns (no separate permutation pass); identity and
 //               frame-major layouts by a 3-D box.
-//   warp 1      allocates tensor memory; lane 0 issues all MMAs. S is double
+//   warp 9      allocates tensor memory; lane 0 issues all MMAs. S is double
 //               buffered so Q K_{j+1}^T runs while row j is in softmax.
-//   warps 4-7   softmax: thread r owns row r (tensor-memory lane r). The
-//               running maximum is only moved when it grows by more than 2^8,
-//               so O is rescaled rarely; P and l use the same reference, which
-//               keeps the result exact. Epilogue: O / l to bf16, scattered to
-//               original token rows (the inverse permutation is fused here).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -35,7 +39,10 @@ namespace sa {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 320;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr int kStages = 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows > 2^8
 
@@ -52,7 +59,7 @@ struct Smem {
   static constexpr int kOffV = kOffK + kStages * kKVBytes;
   static constexpr int kOffP = kOffV + kStages * kKVBytes;
   static constexpr int kOffBar = kOffP + kPBytes;
-  static constexpr int kBytes = kOffBar + 256;
+  static constexpr int kBytes = kOffBar + 4096;
   static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-byte alignment
   static constexpr uint32_t kTmemCols = (2 * BN + D) <= 256 ? 256 : 512;
 };
@@ -67,8 +74,11 @@ struct Bars {
   uint64_t drain;
   uint64_t m_full[2], m_empty[2];   // gather mode: per-chunk group-membership masks
   uint32_t masks[2][8];             // [chunk & 1][first group words 0-3, second group 4-7]
+  uint64_t x_bar;                   // the two halves of every row exchange values
   uint32_t tmem_base;
   int abort;
+  float xmax[2][2][128];            // [iteration & 1][half][row] partial row maxima
+  float xl[2][128];                 // [half][row] partial row sums
 };
 
 // Which tensor map and which coordinates fetch block ``blk`` of head ``bh``.
@@ -224,11 +234,18 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       mbar_init(&bars->k_full[s], 1); mbar_init(&bars->k_empty[s], 1);
       mbar_init(&bars->v_full[s], 1); mbar_init(&bars->v_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) { mbar_init(&bars->s_full[b], 1); mbar_init(&bars->s_free[b], 4); }
-    mbar_init(&bars->p_full, 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->s_full[b], 1);
+      mbar_init(&bars->s_free[b], kSoftmaxWarps);
+    }
+    mbar_init(&bars->p_full, kSoftmaxWarps);
+    mbar_init(&bars->x_bar, kSoftmaxWarps);
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->drain, 1);
-    for (int b = 0; b < 2; ++b) { mbar_init(&bars->m_full[b], 1); mbar_init(&bars->m_empty[b], 4); }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->m_full[b], 1);
+      mbar_init(&bars->m_empty[b], kSoftmaxWarps);
+    }
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -241,7 +258,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     }
     fence_proxy_async_smem();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tmem_alloc(&bars->tmem_base, L::kTmemCols);
     tmem_relinquish();
@@ -255,7 +272,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   volatile int* abort = &bars->abort;
   uint32_t* status = p.status;
 
-  if (warp == 0 && kGather) {
+  if (warp == kProducerWarp && kGather) {
     // ------------------------------------------------------------ producer (gather)
     if (n_keys > 0) {
       if (lane == 0) {
@@ -334,7 +351,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
           mbar_drain(&bars->v_full[j % kStages], (j / kStages) & 1);
       }
     }
-  } else if (warp == 0) {
+  } else if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n_keys > 0) {
       const CUtensorMap* qmaps = maps.q;
@@ -367,7 +384,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_keys > 0) {
       constexpr uint32_t idesc_qk = umma_idesc_bf16(128, BN, false, false);
@@ -419,31 +436,39 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       umma_commit(&bars->drain);
       mbar_drain(&bars->drain, 0);
     }
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int r = threadIdx.x - 128;                  // row == tensor-memory lane
-    const uint32_t lane_off = (uint32_t)(32 * (warp - 4)) << 16;
+    constexpr int HC = BN / 2;                        // S columns per thread
+    constexpr int HD = D / 2;                         // O columns per thread
+    const int half = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;             // row == tensor-memory lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const float scale = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
-    float s[BN];
+    float m = -INFINITY;                              // reference maximum, log2 units
+    float l = 0.f;                                    // this half's share of the row sum
+    float s[HC];
     bool ok = true;
     for (int j = 0; j < n_keys; ++j) {
       const int sb = j & 1;
-      uint32_t pw[BN / 32];
+      uint32_t pw[HC / 32];
       bool pad = true;
       if constexpr (kGather) {
-        // this row's group-membership bits for the chunk's 128 keys
+        // this row's group-membership bits for its half of the chunk's keys
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->m_full[sb], (j >> 1) & 1, abort, status,
                                                site(3, 11, j)))) {
           ok = false;
           break;
         }
 #pragma unroll
-        for (int w = 0; w < BN / 32; ++w) pw[w] = bars->masks[sb][(r < 64 ? 0 : 4) + w];
+        for (int w = 0; w < HC / 32; ++w)
+          pw[w] = bars->masks[sb][(r < 64 ? 0 : 4) + half * (HC / 32) + w];
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->m_empty[sb]);
       } else {
-        pad = block_pad_mask<BN>(g, cols[j], p.T, p.H, p.W, pw);
+        uint32_t full[BN / 32];
+        pad = block_pad_mask<BN>(g, cols[j], p.T, p.H, p.W, full);
+#pragma unroll
+        for (int w = 0; w < HC / 32; ++w) pw[w] = full[half * (HC / 32) + w];
       }
       // a warp either waits out a barrier together or gives up together
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (j >> 1) & 1, abort, status,
@@ -453,7 +478,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       }
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < BN; c += 32) tmem_ld32(tS[sb] + lane_off + c, s + c);
+      for (int c = 0; c < HC; c += 32) tmem_ld32(tS[sb] + lane_off + half * HC + c, s + c);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -462,24 +487,34 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       float mx = -INFINITY;
       if (pad) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          s[c] = ((pw[c / 32] >> (c % 32)) & 1u) ? s[c] * scale : -INFINITY;
+        for (int c = 0; c < HC; ++c) {
+          s[c] = ((pw[c / 32] >> (c % 32)) & 1u) ? s[c] : -INFINITY;
           mx = fmaxf(mx, s[c]);
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) { s[c] *= scale; mx = fmaxf(mx, s[c]); }
+        for (int c = 0; c < HC; ++c) mx = fmaxf(mx, s[c]);
       }
-      const float m_new = fmaxf(m, mx);
+      // row maximum over both halves
+      bars->xmax[sb][half][r] = mx;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->x_bar);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->x_bar, j & 1, abort, status, site(3, 12, j)))) {
+        ok = false;
+        break;
+      }
+      mx = fmaxf(mx, bars->xmax[sb][half ^ 1][r]);
+      const float m_new = fmaxf(m, mx * scale);
       const bool rescale = (m == -INFINITY) || (m_new > m + kRescaleThreshold);
       const float m_use = rescale ? m_new : m;
       float rs = 0.f;
       if (m_use == -INFINITY) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) s[c] = 0.f;
+        for (int c = 0; c < HC; ++c) s[c] = 0.f;
       } else {
+        const float neg = -m_use;
 #pragma unroll
-        for (int c = 0; c < BN; ++c) { s[c] = ex2_approx(s[c] - m_use); rs += s[c]; }
+        for (int c = 0; c < HC; ++c) { s[c] = ex2_approx(fmaf(s[c], scale, neg)); rs += s[c]; }
       }
       // P buffer and O are read/written by PV of the previous block: wait for it.
       if (j >= 1) {
@@ -497,30 +532,28 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
           l *= alpha;
           float o[32];
 #pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            tmem_ld32(tO + lane_off + c, o);
+          for (int c = 0; c < HD; c += 32) {
+            tmem_ld32(tO + lane_off + half * HD + c, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(tO + lane_off + c, o);
+            tmem_st32(tO + lane_off + half * HD + c, o);
           }
           tmem_wait_st();
         }
       }
       m = m_use;
       l += rs;
-      // P row r into the 128-byte-swizzled K-major tile (keys along K).
+      // This half of P row r into the 128-byte-swizzled K-major tile (keys along K).
 #pragma unroll
-      for (int h = 0; h < BN / 64; ++h) {
-        uint8_t* rowp = sP + h * 16384 + r * 128;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const float* x = s + h * 64 + ch * 8;
-          uint4 w;
-          w.x = pack_bf16x2(x[0], x[1]); w.y = pack_bf16x2(x[2], x[3]);
-          w.z = pack_bf16x2(x[4], x[5]); w.w = pack_bf16x2(x[6], x[7]);
-          *reinterpret_cast<uint4*>(rowp + ((ch ^ (r & 7)) << 4)) = w;
-        }
+      for (int ch = 0; ch < HC / 8; ++ch) {
+        const int key0 = half * HC + ch * 8;            // first of the 8 keys of this chunk
+        uint8_t* rowp = sP + (key0 / 64) * 16384 + r * 128;
+        const float* x = s + ch * 8;
+        uint4 w;
+        w.x = pack_bf16x2(x[0], x[1]); w.y = pack_bf16x2(x[2], x[3]);
+        w.z = pack_bf16x2(x[4], x[5]); w.w = pack_bf16x2(x[6], x[7]);
+        *reinterpret_cast<uint4*>(rowp + ((((key0 % 64) / 8) ^ (r & 7)) << 4)) = w;
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -533,15 +566,24 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
                                              site(3, 10, n_keys)));
       tc_fence_after();
     }
+    if (ok) {
+      // row sum over both halves
+      bars->xl[half][r] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->x_bar);
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->x_bar, n_keys & 1, abort, status,
+                                             site(3, 13, n_keys)));
+    }
     const int tok = (r < BN) ? slot_to_token(g, qb, r, BN, p.T, p.H, p.W) : -1;
     if (ok) {
-      const float inv_l = (n_keys > 0 && l > 0.f) ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (tok < 0 ? 0 : tok)) * D;
+      const float l_tot = l + bars->xl[half ^ 1][r];
+      const float inv_l = (n_keys > 0 && l_tot > 0.f) ? 1.f / l_tot : 0.f;
+      __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (tok < 0 ? 0 : tok)) * D + half * HD;
 #pragma unroll
-      for (int c = 0; c < D; c += 32) {
+      for (int c = 0; c < HD; c += 32) {
         float o[32];
         if (n_keys > 0) {
-          tmem_ld32(tO + lane_off + c, o);
+          tmem_ld32(tO + lane_off + half * HD + c, o);
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -559,15 +601,15 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
           }
         }
       }
-      if (tok >= 0 && p.lse)
+      if (tok >= 0 && half == 0 && p.lse)
         p.lse[(size_t)bh * p.N + tok] =
-            (n_keys > 0 && l > 0.f) ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+            (n_keys > 0 && l_tot > 0.f) ? (m + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
