@@ -4,7 +4,7 @@
 // kept key blocks in ascending order and computes
 //   S = Q K^T (tcgen05.mma, bf16 in, fp32 accumulate in tensor memory),
 //   P = exp(S / sqrt(d) - m) with a running row maximum m (online softmax),
-//   O += P V (tcgen05.mma, P staged in shared memory as bf16),
+//   O += P V (tcgen05.mma, P written back over S in tensor memory as bf16),
 // then writes O / l and LSE = ln(l) + m to the query tokens' original rows.
 // This is the flash block-sparse kernel with online softmax of the SPADE
 // review ("What carries the argument") and the dense-tile-only executor of the
@@ -57,12 +57,10 @@ struct Smem {
   static constexpr int kQBytes = kHalvesD * 128 * 128;    // 128 rows, M of the MMA
   static constexpr int kKVHalf = BN * 128;                // one 64-column half of a K/V tile
   static constexpr int kKVBytes = kHalvesD * kKVHalf;
-  static constexpr int kPBytes = kHalvesN * 128 * 128;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + kStages * kKVBytes;
-  static constexpr int kOffP = kOffV + kStages * kKVBytes;
-  static constexpr int kOffBar = kOffP + kPBytes;
+  static constexpr int kOffBar = kOffV + kStages * kKVBytes;
   static constexpr int kBytes = kOffBar + 4096;
   static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-byte alignment
   static constexpr uint32_t kTmemCols = (2 * BN + D) <= 256 ? 256 : 512;
@@ -202,7 +200,6 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   uint8_t* sQ = smem + L::kOffQ;
   uint8_t* sK = smem + L::kOffK;
   uint8_t* sV = smem + L::kOffV;
-  uint8_t* sP = smem + L::kOffP;
   Bars* bars = reinterpret_cast<Bars*>(smem + L::kOffBar);
 
   const int qb = blockIdx.x;
@@ -393,7 +390,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     if (lane == 0 && n_keys > 0) {
       constexpr uint32_t idesc_qk = umma_idesc_bf16(128, BN, false, false);
       constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, false, true);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
       auto issue_pv = [&](int i) -> bool {
         if (!mbar_wait(&bars->p_full, i & 1, abort, status, site(2, 3, i))) return false;
         if (!mbar_wait(&bars->v_full[i % kStages], (i / kStages) & 1, abort, status, site(2, 4, i)))
@@ -402,10 +399,10 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         const uint32_t vbase = aV + (i % kStages) * L::kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          // A = P (K-major, keys along K); B = V (MN-major: d contiguous).
-          const uint64_t da = umma_desc_sw128(aP + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+          // A = P in tensor memory (16 keys = 8 packed columns per step);
+          // B = V (MN-major: d contiguous).
           const uint64_t db = umma_desc_sw128(vbase + kk * 16 * 128, L::kKVHalf, 1024);
-          umma_bf16_ss(tO, da, db, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(tO, tS[i & 1] + kk * 8, db, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&bars->o_done);
         umma_commit(&bars->v_empty[i % kStages]);
@@ -564,18 +561,18 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       }
       m = m_use;
       l += rs;
-      // This half of P row r into the 128-byte-swizzled K-major tile (keys along K).
+      // P as packed bf16 pairs over this half's share of the first BN/2 columns
+      // of S (the A operand of the PV MMA is read from tensor memory). Packed
+      // in place: entry c only reads entries 2c and 2c+1, not yet overwritten.
 #pragma unroll
-      for (int ch = 0; ch < HC / 8; ++ch) {
-        const int key0 = half * HC + ch * 8;            // first of the 8 keys of this chunk
-        uint8_t* rowp = sP + (key0 / 64) * 16384 + r * 128;
-        const float* x = s + ch * 8;
-        uint4 w;
-        w.x = pack_bf16x2(x[0], x[1]); w.y = pack_bf16x2(x[2], x[3]);
-        w.z = pack_bf16x2(x[4], x[5]); w.w = pack_bf16x2(x[6], x[7]);
-        *reinterpret_cast<uint4*>(rowp + ((((key0 % 64) / 8) ^ (r & 7)) << 4)) = w;
+      for (int c = 0; c < HC / 2; ++c) s[c] = __uint_as_float(pack_bf16x2(s[2 * c], s[2 * c + 1]));
+      if constexpr (HC / 2 >= 32) {
+#pragma unroll
+        for (int c = 0; c < HC / 2; c += 32) tmem_st32(tS[sb] + lane_off + half * (HC / 2) + c, s + c);
+      } else {
+        tmem_st16(tS[sb] + lane_off + half * (HC / 2), s);
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full);
