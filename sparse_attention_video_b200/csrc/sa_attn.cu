@@ -70,13 +70,13 @@ struct Bars {
   uint64_t q_full;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], s_free[2];
+  uint64_t s_full[2];
   uint64_t p_full;
   uint64_t o_done;
   uint64_t drain;
   uint64_t m_full[2], m_empty[2];   // gather mode: per-chunk group-membership masks
   uint32_t masks[2][8];             // [chunk & 1][first group words 0-3, second group 4-7]
-  uint64_t x_bar;                   // the two halves of every row exchange values
+  uint64_t x_bar[4];                // warps w and w+4 (same rows) exchange values
   uint32_t tmem_base;
   int abort;
   float xmax[2][2][128];            // [iteration & 1][half][row] partial row maxima
@@ -235,12 +235,9 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       mbar_init(&bars->k_full[s], 1); mbar_init(&bars->k_empty[s], 1);
       mbar_init(&bars->v_full[s], 1); mbar_init(&bars->v_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_free[b], kSoftmaxWarps);
-    }
+    for (int b = 0; b < 2; ++b) mbar_init(&bars->s_full[b], 1);
     mbar_init(&bars->p_full, kSoftmaxWarps);
-    mbar_init(&bars->x_bar, kSoftmaxWarps);
+    for (int qd = 0; qd < 4; ++qd) mbar_init(&bars->x_bar[qd], 2);
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->drain, 1);
     for (int b = 0; b < 2; ++b) {
@@ -415,10 +412,8 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
           ok = false;
           break;
         }
-        if (j >= 2 && !mbar_wait(&bars->s_free[sb], ((j - 2) >> 1) & 1, abort, status, site(2, 7, j))) {
-          ok = false;
-          break;
-        }
+        // S buffer sb was last read as P_{j-2} by PV_{j-2}, which was issued
+        // before this QK; tcgen05 MMAs of one thread run in issue order.
         tc_fence_after();
         const uint32_t kbase = aK + st * L::kKVBytes;
 #pragma unroll
@@ -481,9 +476,6 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
 #pragma unroll
       for (int c = 0; c < HC; c += 32) tmem_ld32(tS[sb] + lane_off + half * HC + c, s + c);
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->s_free[sb]);
 
       // row maximum of this half: four independent chains, then combined
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -501,8 +493,9 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       // row maximum over both halves
       bars->xmax[sb][half][r] = mx;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->x_bar);
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->x_bar, j & 1, abort, status, site(3, 12, j)))) {
+      if (lane == 0) mbar_arrive(&bars->x_bar[warp & 3]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->x_bar[warp & 3], j & 1, abort, status,
+                                             site(3, 12, j)))) {
         ok = false;
         break;
       }
@@ -587,8 +580,8 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       // row sum over both halves
       bars->xl[half][r] = l;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->x_bar);
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->x_bar, n_keys & 1, abort, status,
+      if (lane == 0) mbar_arrive(&bars->x_bar[warp & 3]);
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->x_bar[warp & 3], n_keys & 1, abort, status,
                                              site(3, 13, n_keys)));
     }
     const int tok = (r < BN) ? slot_to_token(g, qb, r, BN, p.T, p.H, p.W) : -1;
