@@ -44,6 +44,8 @@ def _args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-mask comparison")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="workload name (synthetic.CONFIGS); the bench line uses the default")
     ap.add_argument("--heads", type=int, default=0,
                     help="run only this many heads (half of them temporal); for small "
                          "profiler captures, not for bench lines")
@@ -82,6 +84,19 @@ def cpu_oracle_sample(wl, x, budget_s=20.0):
     flops = 0.0
     n_blocks = 0
     t0 = time.perf_counter()
+    if wl.kind == "fg":
+        q, k, v = (bf16_bits_to_f32(x[n][0, 0]) for n in "qkv")
+        keep = pipeline.head_mask(wl, q, k, 0)["keep_groups"]
+        for g in rng.permutation(keep.shape[0]):
+            attention.slice_attention(q, k, v, keep, wl.fg_group, [int(g)])
+            flops += 4.0 * wl.head_dim * float(keep[g].sum()) * wl.fg_group
+            n_blocks += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+        desc = (f"oracle on head 0: slice scores, threshold and mask of the head + masked "
+                f"attention (float64) for {n_blocks} query groups of {wl.fg_group}")
+        return flops / dt / 1e12, desc, threads
     for h in heads:
         q, k, v = (bf16_bits_to_f32(x[n][0, h]) for n in "qkv")
         ref = pipeline.head_mask(wl, q, k, h)
@@ -168,6 +183,27 @@ def _traffic_per_launch():
         return None
 
 
+def policy_kwargs(wl):
+    """The workload's mask policy as make_policy() arguments."""
+    if wl.kind == "topk":
+        return dict(kind="topk", block=wl.block, tile=wl.tile, topk=wl.topk,
+                    keep_diagonal=wl.keep_diagonal)
+    if wl.kind == "sta":
+        return dict(kind="sta", block=wl.block, tile=wl.tile, window=wl.window)
+    if wl.kind == "spatiotemporal":
+        return dict(kind="spatiotemporal", block=wl.block, temporal_heads=wl.temporal_heads,
+                    heads=wl.heads, sink_tokens=wl.sink_tokens, frame_radius=1)
+    if wl.kind == "spade":
+        return dict(kind="spade", block=wl.block, candidates=wl.candidates, top_p=wl.top_p,
+                    window=wl.window)
+    return dict(kind="fg", block=wl.block, fg_group=wl.fg_group,
+                fg_keep_fraction=wl.fg_keep_fraction)
+
+
+# kernels of ours launched by one step (build_mask + permute + attend)
+LAUNCHES_PER_STEP = {"topk": 5, "sta": 3, "spatiotemporal": 4, "spade": 5, "fg": 13}
+
+
 # ---------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
     if rank != 0:
@@ -221,17 +257,17 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=600),
                                 device_id=dev)
 
-    wl = CONFIGS[WORKLOAD]
+    wl = CONFIGS[args.workload]
     if args.heads:
-        wl = wl.with_(heads=args.heads, temporal_heads=tuple(range(args.heads // 2, args.heads)))
+        th = tuple(range(args.heads // 2, args.heads)) if wl.temporal_heads else ()
+        wl = wl.with_(heads=args.heads, temporal_heads=th)
     wl_r = wl.with_(config_id=wl.config_id + 1000 * rank)      # independent problem per rank
     log("generating inputs")
     x = make_qkv(wl_r)
     log("inputs ready")
     host = {n: torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in "qkv"}
     q, k, v = (host[n].to(dev) for n in "qkv")
-    pol = make_policy("spatiotemporal", block=wl.block, temporal_heads=wl.temporal_heads,
-                      heads=wl.heads, sink_tokens=wl.sink_tokens, frame_radius=1)
+    pol = make_policy(**policy_kwargs(wl))
     sa = SparseAttention(1, wl.heads, wl.T, wl.H, wl.W, wl.head_dim, pol, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
@@ -255,8 +291,14 @@ def main():
     torch.cuda.synchronize(dev)
     log("warm-up done")
     assert sa.status() == 0, "device status word set during warm-up"
-    kept = sum(h.kept for h in sa.export(2))
-    flops_call = 4.0 * wl.head_dim * kept * wl.block * wl.block
+    if wl.kind == "fg":
+        # executed work: every 128-query tile against the union of its groups' kept keys
+        from sparse_attention_video_b200 import SA_EXPORT_FG_TILE_KEYS
+        keys = float(sa.export(SA_EXPORT_FG_TILE_KEYS).astype(np.float64).sum())
+        flops_call = 4.0 * wl.head_dim * keys * 128
+    else:
+        kept = sum(h.kept for h in sa.export(2))
+        flops_call = 4.0 * wl.head_dim * kept * wl.block * wl.block
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -311,7 +353,7 @@ def main():
 
     # ---- the same kernel with every block kept
     dense = {}
-    if not args.no_dense:
+    if not args.no_dense and wl.head_dim == 128 and wl.block == 128:
         nb = (wl.N + wl.block - 1) // wl.block
         w32 = (nb + 31) // 32
         words = torch.full((wl.heads, nb, w32), -1, dtype=torch.int32, device=dev)
@@ -354,22 +396,25 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "grid": "30x48x80", "tokens": wl.N, "heads": wl.heads,
-                   "head_dim": wl.head_dim, "batch": 1, "block": wl.block,
+        "config": {"workload": wl.name, "grid": f"{wl.T}x{wl.H}x{wl.W}", "tokens": wl.N,
+                   "heads": wl.heads, "head_dim": wl.head_dim, "batch": 1, "block": wl.block,
                    "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (Q, K, V = 2.12 GB per step)"},
+                   "l2": (f"inputs larger than L2 (Q, K, V = {h2d / 1e9:.2f} GB per step)"
+                          if h2d > 126e6 else "inputs smaller than L2: not flushed")},
         "step_breakdown_ms": {"build_mask": mask_ms, "permute": perm_ms, "attention": attn_ms},
         "attended_tflop_per_call": flops_call / 1e12,
         "attention_ms_per_call": attn_ms,
-        "roofline": {"kernel": "attn_fwd_kernel<128,128>", "bound": "tensor",
+        "roofline": {"kernel": "attn_fwd_kernel<%d,%d,%s>" % (wl.head_dim, wl.block,
+                                                               "gather" if wl.kind == "fg" else "block"),
+                     "bound": "tensor",
                      "achieved": achieved, "peak": peak_sust, "unit": "TFLOP/s",
                      "frac": achieved / peak_sust,
                      "peak_note": f"{peak_src} sustained cuBLAS bf16 (burst {peak_burst})",
-                     "traffic": traffic},
+                     "traffic": traffic if wl.name == WORKLOAD and not args.heads else None},
         "cpu_baseline": cpu,
         "e2e": {"value": world * flops_call / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": LAUNCHES_PER_STEP[wl.kind] * args.steps,
         "clocks": clk,
         **dense,
     }

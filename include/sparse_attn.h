@@ -190,13 +190,17 @@ SA_API int sparse_attn_attend(const sa_problem* problem, const sa_policy* policy
  *   SA_EXPORT_HEAD_INFO    sa_head_info [batch*heads]
  *   SA_EXPORT_FG_BITS      uint32 [batch*heads][G][ceil(N/32)], G = ceil(N/fg_group)
  *   SA_EXPORT_FG_TAU       float  [batch*heads]
+ *   SA_EXPORT_FG_TILE_KEYS uint32 [batch*heads][ceil(N/128)]: keys the slice attention
+ *                          visits for each 128-query tile (the union of the kept
+ *                          keys of the groups in the tile)
  * ``bytes`` must equal the size of that part (see sparse_attn_export_bytes).
  */
 enum {
   SA_EXPORT_BLOCK_BITS = 1,
   SA_EXPORT_HEAD_INFO = 2,
   SA_EXPORT_FG_BITS = 3,
-  SA_EXPORT_FG_TAU = 4
+  SA_EXPORT_FG_TAU = 4,
+  SA_EXPORT_FG_TILE_KEYS = 5
 };
 
 typedef struct {

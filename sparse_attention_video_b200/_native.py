@@ -20,6 +20,7 @@ SA_MASK_SPADE, SA_MASK_FG, SA_MASK_EXPLICIT = 4, 5, 6
 SA_LAYOUT_IDENTITY, SA_LAYOUT_FRAME_MAJOR, SA_LAYOUT_TILE = 0, 1, 2
 
 SA_EXPORT_BLOCK_BITS, SA_EXPORT_HEAD_INFO, SA_EXPORT_FG_BITS, SA_EXPORT_FG_TAU = 1, 2, 3, 4
+SA_EXPORT_FG_TILE_KEYS = 5
 
 EXPORTED = ("sparse_attn_workspace_size", "sparse_attn_build_mask", "sparse_attn_forward",
             "sparse_attn_permute", "sparse_attn_attend",

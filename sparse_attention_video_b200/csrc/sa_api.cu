@@ -507,6 +507,7 @@ extern "C" int sparse_attn_export_bytes(const sa_problem* problem, const sa_poli
     case SA_EXPORT_HEAD_INFO: *bytes = sizeof(HeadGeom) * (size_t)M.BH; break;
     case SA_EXPORT_FG_BITS: *bytes = sizeof(uint32_t) * (size_t)M.BH * M.G * M.WN; break;
     case SA_EXPORT_FG_TAU: *bytes = policy->kind == SA_MASK_FG ? sizeof(float) * M.BH : 0; break;
+    case SA_EXPORT_FG_TILE_KEYS: *bytes = sizeof(uint32_t) * (size_t)M.BH * M.P; break;
     default: return SA_ERR_INVALID_ARG;
   }
   return SA_OK;
@@ -526,6 +527,7 @@ extern "C" int sparse_attn_mask_export(const sa_problem* problem, const sa_polic
     case SA_EXPORT_HEAD_INFO: off = M.off_head; break;
     case SA_EXPORT_FG_BITS: off = M.off_fg_bits; break;
     case SA_EXPORT_FG_TAU: off = M.off_fg_tau; break;
+    case SA_EXPORT_FG_TILE_KEYS: off = M.off_fg_counts; break;
   }
   if (need == 0) return SA_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -43,7 +43,7 @@ constexpr int kThreads = 320;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows > 2^8
 // One exp2 in kPolyEvery on the FMA pipe (0 = all on MUFU). Measured on the
 // 115,200-token workload, moving a quarter of them was slower (12.04 vs
@@ -61,9 +61,11 @@ struct Smem {
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + kStages * kKVBytes;
   static constexpr int kOffBar = kOffV + kStages * kKVBytes;
-  static constexpr int kBytes = kOffBar + 4096;
+  static constexpr int kBytes = kOffBar + 512;
   static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-byte alignment
-  static constexpr uint32_t kTmemCols = (2 * BN + D) <= 256 ? 256 : 512;
+  // S (two buffers), O, and 6 columns where the two halves of a row exchange
+  // their partial maxima (by iteration parity) and partial sums
+  static constexpr uint32_t kTmemCols = (2 * BN + D + 6) <= 256 ? 256 : 512;
 };
 
 struct Bars {
@@ -79,9 +81,9 @@ struct Bars {
   uint64_t x_bar[4];                // warps w and w+4 (same rows) exchange values
   uint32_t tmem_base;
   int abort;
-  float xmax[2][2][128];            // [iteration & 1][half][row] partial row maxima
-  float xl[2][128];                 // [half][row] partial row sums
 };
+
+static_assert(sizeof(Bars) <= 512, "barrier block must fit its shared-memory slot");
 
 // Which tensor map and which coordinates fetch block ``blk`` of head ``bh``.
 __device__ __forceinline__ void block_source(const HeadGeom& g, int blk, int BN, int& map,
@@ -267,6 +269,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   const uint32_t tmem = bars->tmem_base;
   const uint32_t tS[2] = {tmem, tmem + BN};
   const uint32_t tO = tmem + 2 * BN;
+  const uint32_t tX = tmem + 2 * BN + D;          // exchange columns
   volatile int* abort = &bars->abort;
   uint32_t* status = p.status;
 
@@ -281,17 +284,26 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       }
       const int row0 = bh * p.N;
       int issued_k = 0, issued_v = 0;
+      // list entries j*128 + lane + 32*s; key index in the low 30 bits, one
+      // membership bit per group of the tile in bits 30 and 31. The next
+      // chunk's entries are loaded while this chunk waits on its barriers.
+      uint32_t en[4];
+#pragma unroll
+      for (int s4 = 0; s4 < 4; ++s4) {
+        const uint32_t idx = (uint32_t)lane + 32 * s4;
+        en[s4] = idx < list_count ? __ldg(list + idx) : 0u;
+      }
       for (int j = 0; j < n_keys; ++j) {
         const int st = j % kStages, rnd = j / kStages, mb = j & 1;
-        // list entries j*128 + lane + 32*s; key index in the low 30 bits, one
-        // membership bit per group of the tile in bits 30 and 31
         uint32_t e[4];
         bool val[4];
 #pragma unroll
         for (int s4 = 0; s4 < 4; ++s4) {
           const uint32_t idx = (uint32_t)j * BN + lane + 32 * s4;
           val[s4] = idx < list_count;
-          e[s4] = val[s4] ? __ldg(list + idx) : 0u;
+          e[s4] = en[s4];
+          const uint32_t nidx = idx + BN;
+          en[s4] = nidx < list_count ? __ldg(list + nidx) : 0u;
         }
         uint32_t m0[4], m1[4];
 #pragma unroll
@@ -490,8 +502,11 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         for (int c = 0; c < HC; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
       }
       float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      // row maximum over both halves
-      bars->xmax[sb][half][r] = mx;
+      // row maximum over both halves, exchanged through spare tensor-memory
+      // columns (the two warps of a pair read and write the same lanes)
+      tmem_st1(tX + lane_off + 2 * sb + half, mx);
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->x_bar[warp & 3]);
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->x_bar[warp & 3], j & 1, abort, status,
@@ -499,7 +514,9 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         ok = false;
         break;
       }
-      mx = fmaxf(mx, bars->xmax[sb][half ^ 1][r]);
+      tc_fence_after();
+      mx = fmaxf(mx, tmem_ld1(tX + lane_off + 2 * sb + (half ^ 1)));
+      tmem_wait_ld();
       const float m_new = fmaxf(m, mx * scale);
       const bool rescale = (m == -INFINITY) || (m_new > m + kRescaleThreshold);
       const float m_use = rescale ? m_new : m;
@@ -578,15 +595,23 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     }
     if (ok) {
       // row sum over both halves
-      bars->xl[half][r] = l;
+      tmem_st1(tX + lane_off + 4 + half, l);
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->x_bar[warp & 3]);
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->x_bar[warp & 3], n_keys & 1, abort, status,
                                              site(3, 13, n_keys)));
     }
     const int tok = (r < BN) ? slot_to_token(g, qb, r, BN, p.T, p.H, p.W) : -1;
+    float l_other = 0.f;
     if (ok) {
-      const float l_tot = l + bars->xl[half ^ 1][r];
+      tc_fence_after();
+      l_other = tmem_ld1(tX + lane_off + 4 + (half ^ 1));
+      tmem_wait_ld();
+    }
+    if (ok) {
+      const float l_tot = l + l_other;
       const float inv_l = (n_keys > 0 && l_tot > 0.f) ? 1.f / l_tot : 0.f;
       __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (tok < 0 ? 0 : tok)) * D + half * HD;
 #pragma unroll
