@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 
@@ -237,6 +238,34 @@ bool map_rows(CUtensorMap* m, const void* base, long long rows, int d) {
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int gcd_i(int a, int b) { return b ? gcd_i(b, a % b) : a; }
+int lcm_i(int a, int b) { return a / gcd_i(a, b) * b; }
+
+// Regions for the pooling kernel: the least common multiple of the candidate
+// tiles along each axis, so every region holds whole blocks of every
+// candidate; then grown along w, h, t (by doubling while it stays inside the
+// grid) until the smallest candidate count per region reaches 8 blocks, one
+// per warp of the CTA, without exceeding 8 for any candidate.
+void pool_regions(PoolParams& pp) {
+  int R[3] = {1, 1, 1};
+  for (int c = 0; c < pp.C; ++c)
+    for (int a = 0; a < 3; ++a) R[a] = lcm_i(R[a], pp.cand[c][a]);
+  auto blocks = [&](int c) {
+    return (R[0] / pp.cand[c][0]) * (R[1] / pp.cand[c][1]) * (R[2] / pp.cand[c][2]);
+  };
+  const int ext[3] = {pp.T, pp.H, pp.W};
+  for (bool grew = true; grew;) {
+    grew = false;
+    int mx = 0, mn = 1 << 30;
+    for (int c = 0; c < pp.C; ++c) { mx = std::max(mx, blocks(c)); mn = std::min(mn, blocks(c)); }
+    if (mn >= 8 || 2 * mx > 8) break;
+    for (int a = 2; a >= 0 && !grew; --a)
+      if (2 * R[a] <= ext[a] + R[a] - 1) { R[a] *= 2; grew = true; }
+  }
+  pp.Rt = R[0]; pp.Rh = R[1]; pp.Rw = R[2];
+  pp.nRt = ceil_div(pp.T, R[0]); pp.nRh = ceil_div(pp.H, R[1]); pp.nRw = ceil_div(pp.W, R[2]);
+}
+
 int aligned(const void* p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
@@ -329,6 +358,7 @@ extern "C" int sparse_attn_build_mask(const sa_problem* problem, const sa_policy
     for (int c = 0; c < C; ++c)
       for (int i = 0; i < 3; ++i) pp.cand[c][i] = po.kind == SA_MASK_SPADE ? po.candidates[c][i] : po.tile[i];
     pp.C = C; pp.NB = M.NB; pp.T = pr.T; pp.H = pr.H; pp.W = pr.W; pp.d = d;
+    pool_regions(pp);
     if ((e = cuda_status(launch_pool_sics(pp, BH, M.NB, st)))) return e;
     if (po.kind == SA_MASK_SPADE) {
       ChooseParams cp{};

@@ -82,95 +82,131 @@ __global__ void permute_fm_kernel(PermuteParams p) {
 }
 
 // ------------------------------------------------------------------ pool_sics
-// One CTA per (block, candidate, head). Thread (token lane tl, chunk dc) loads
-// 8 dims of every (256 / (d/8))-th slot of the block.
+// One warp per (block, candidate, head), 8 warps per CTA. Half-warp h of the
+// warp takes tokens h, h+2, h+4, ... of the block; lane i of a half-warp owns
+// dimensions 8i..8i+7 (16-byte loads, one 256-byte row per half-warp), four
+// token pairs in flight per step. Row norms come from shuffles inside the
+// half-warp; the two halves are combined by one shuffle at the end. Every sum
+// runs in a fixed order.
+constexpr int kMaxPoolBlock = 128;   // tokens per block (64 or 128)
+
 template <int D>
 __global__ void __launch_bounds__(256) pool_sics_kernel(PoolParams p) {
-  constexpr int CH = D / 8;            // 16-byte chunks per row
-  constexpr int TL = 256 / CH;         // token lanes
-  const int blk = blockIdx.x, c = blockIdx.y, bh = blockIdx.z;
+  static_assert(D == 128 || D == 64, "head_dim");
+  constexpr int CH = D / 8;                 // lanes per token (16 or 8)
+  constexpr int TPW = 32 / CH;              // tokens per warp step (2 or 4)
+  constexpr int UNROLL = 4;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int c = blockIdx.x, region = blockIdx.y, bh = blockIdx.z;
   const int bt = p.cand[c][0], bhh = p.cand[c][1], bw = p.cand[c][2];
   const int nt = (p.T + bt - 1) / bt, nh = (p.H + bhh - 1) / bhh, nw = (p.W + bw - 1) / bw;
-  const int nb = nt * nh * nw;
-  if (blk >= nb) return;
+  // Local block ``warp`` of this candidate inside the region (regions are the
+  // least common multiple of every candidate's tile, so each holds whole
+  // blocks of every candidate; the candidates' CTAs of one region run next to
+  // each other and read the same tokens while they are in L2).
+  const int rw = region % p.nRw, rh = (region / p.nRw) % p.nRh, rt = region / (p.nRw * p.nRh);
+  const int mt = p.Rt / bt, mh = p.Rh / bhh, mw = p.Rw / bw;
+  __shared__ int slot_tok[8][kMaxPoolBlock];
+  for (int lb = warp; lb < mt * mh * mw; lb += 8) {
+  const int lw = lb % mw, lh = (lb / mw) % mh, lt = lb / (mw * mh);
+  const int tt = rt * mt + lt, th = rh * mh + lh, tw = rw * mw + lw;
+  if (tt >= nt || th >= nh || tw >= nw) continue;
+  const int blk = (tt * nh + th) * nw + tw;
   const int BS = bt * bhh * bw;
-  const int tl = threadIdx.x / CH, dc = threadIdx.x % CH;
+  const int tl = lane / CH, dc = lane % CH;
   const int N = p.T * p.H * p.W;
   const __nv_bfloat16* q = p.q + (size_t)bh * N * D;
   const __nv_bfloat16* k = p.k + (size_t)bh * N * D;
+  // token index of every slot of this warp's block, computed once (the
+  // divisions by runtime tile sizes stay out of the streaming loop)
+  int* st = slot_tok[warp];
+  __syncwarp();
+  for (int s = lane; s < BS; s += 32) st[s] = tile_slot_token(bt, bhh, bw, nh, nw, blk, s, p.T, p.H, p.W);
+  __syncwarp();
 
   float qs[8], ks[8], us[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) { qs[i] = 0.f; ks[i] = 0.f; us[i] = 0.f; }
   int n_valid = 0, n_unit = 0;
-  // Both token lanes of a warp run the same number of iterations, and every
-  // lane joins the shuffles; pad slots contribute zeros.
-  for (int s = tl; s < BS; s += TL) {
-    const int tok = tile_slot_token(bt, bhh, bw, nh, nw, blk, s, p.T, p.H, p.W);
-    uint4 qv = make_uint4(0, 0, 0, 0), kv = make_uint4(0, 0, 0, 0);
-    if (tok >= 0) {
-      qv = __ldg(reinterpret_cast<const uint4*>(q + (size_t)tok * D) + dc);
-      kv = __ldg(reinterpret_cast<const uint4*>(k + (size_t)tok * D) + dc);
+  for (int s0 = 0; s0 < BS; s0 += TPW * UNROLL) {
+    uint4 qv[UNROLL], kv[UNROLL];
+    int tok[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int s = s0 + u * TPW + tl;
+      tok[u] = s < BS ? st[s] : -1;
+      qv[u] = make_uint4(0, 0, 0, 0);
+      kv[u] = make_uint4(0, 0, 0, 0);
+      if (tok[u] >= 0) {
+        qv[u] = __ldg(reinterpret_cast<const uint4*>(q + (size_t)tok[u] * D) + dc);
+        kv[u] = __ldg(reinterpret_cast<const uint4*>(k + (size_t)tok[u] * D) + dc);
+      }
     }
-    const __nv_bfloat16* qe = reinterpret_cast<const __nv_bfloat16*>(&qv);
-    const __nv_bfloat16* ke = reinterpret_cast<const __nv_bfloat16*>(&kv);
-    float kf[8], ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const __nv_bfloat16* qe = reinterpret_cast<const __nv_bfloat16*>(&qv[u]);
+      const __nv_bfloat16* ke = reinterpret_cast<const __nv_bfloat16*>(&kv[u]);
+      float kf[8], ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        kf[i] = __bfloat162float(ke[i]);
+        ss = fmaf(kf[i], kf[i], ss);
+      }
+      // every lane joins; pad slots carry zeros
+#pragma unroll
+      for (int o = CH / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (tok[u] < 0) continue;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        qs[i] += __bfloat162float(qe[i]);
+        ks[i] += kf[i];
+      }
+      ++n_valid;
+      if (ss > 0.f) {
+        // one correctly rounded 1/||k|| per token, then products: within about
+        // one ulp of k_i / ||k|| per component
+        const float rn = 1.0f / sqrtf(ss);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) us[i] = fmaf(kf[i], rn, us[i]);
+        ++n_unit;
+      }
+    }
+  }
+  // combine the token lanes of the warp (same dimensions, lanes dc + CH*t)
+#pragma unroll
+  for (int o = CH; o < 32; o <<= 1) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      kf[i] = __bfloat162float(ke[i]);
-      ss = fmaf(kf[i], kf[i], ss);
+      qs[i] += __shfl_xor_sync(0xffffffffu, qs[i], o);
+      ks[i] += __shfl_xor_sync(0xffffffffu, ks[i], o);
+      us[i] += __shfl_xor_sync(0xffffffffu, us[i], o);
     }
-#pragma unroll
-    for (int o = CH / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (tok < 0) continue;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      qs[i] += __bfloat162float(qe[i]);
-      ks[i] += kf[i];
-    }
-    ++n_valid;
-    if (ss > 0.f) {
-      const float nrm = sqrtf(ss);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) us[i] += kf[i] / nrm;
-      ++n_unit;
-    }
+    n_valid += __shfl_xor_sync(0xffffffffu, n_valid, o);
+    n_unit += __shfl_xor_sync(0xffffffffu, n_unit, o);
   }
-  __shared__ float red[3][TL][D];
-  __shared__ int cnt[2][TL];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    red[0][tl][dc * 8 + i] = qs[i];
-    red[1][tl][dc * 8 + i] = ks[i];
-    red[2][tl][dc * 8 + i] = us[i];
-  }
-  if (dc == 0) { cnt[0][tl] = n_valid; cnt[1][tl] = n_unit; }
-  __syncthreads();
-  __shared__ float usq[D];
-  __shared__ int tot[2];
-  if (threadIdx.x < 2) {
-    int t = 0;
-    for (int i = 0; i < TL; ++i) t += cnt[threadIdx.x][i];
-    tot[threadIdx.x] = t;
-  }
-  __syncthreads();
+  // every lane of a token group counted that group's tokens, so summing over
+  // the groups gives each lane the block's counts
   const size_t base = (((size_t)bh * p.C + c) * p.NB + blk);
-  if (threadIdx.x < D) {
-    const int dd = threadIdx.x;
-    float a = 0.f, b = 0.f, u = 0.f;
-    for (int i = 0; i < TL; ++i) { a += red[0][i][dd]; b += red[1][i][dd]; u += red[2][i][dd]; }
-    const float nv = (float)tot[0];
-    p.qbar[base * D + dd] = tot[0] ? a / nv : 0.f;
-    p.kbar[base * D + dd] = tot[0] ? b / nv : 0.f;
-    usq[dd] = u * u;
+  float usq = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) usq = fmaf(us[i], us[i], usq);
+#pragma unroll
+  for (int o = CH / 2; o >= 1; o >>= 1) usq += __shfl_xor_sync(0xffffffffu, usq, o);
+  if (tl == 0) {
+    const float nv = (float)n_valid;
+    float4* qo = reinterpret_cast<float4*>(p.qbar + base * D + dc * 8);
+    float4* ko = reinterpret_cast<float4*>(p.kbar + base * D + dc * 8);
+    if (n_valid) {
+      qo[0] = make_float4(qs[0] / nv, qs[1] / nv, qs[2] / nv, qs[3] / nv);
+      qo[1] = make_float4(qs[4] / nv, qs[5] / nv, qs[6] / nv, qs[7] / nv);
+      ko[0] = make_float4(ks[0] / nv, ks[1] / nv, ks[2] / nv, ks[3] / nv);
+      ko[1] = make_float4(ks[4] / nv, ks[5] / nv, ks[6] / nv, ks[7] / nv);
+    } else {
+      qo[0] = qo[1] = ko[0] = ko[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (dc == 0) p.sics[base] = usq - (float)n_unit;
   }
-  __syncthreads();
-  // fixed-shape tree over the D squared components
-  for (int w = D / 2; w >= 1; w >>= 1) {
-    if (threadIdx.x < w) usq[threadIdx.x] += usq[threadIdx.x + w];
-    __syncthreads();
   }
-  if (threadIdx.x == 0) p.sics[base] = usq[0] - (float)tot[1];
 }
 
 // ------------------------------------------------------------------ choose
@@ -292,12 +328,18 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
   const HeadGeom g = p.heads[bh];
   if (i >= g.nb) return;
   __shared__ uint32_t bits[kMaxBlocks / 32];
+  __shared__ uint32_t vbits[kMaxBlocks / 32];
   __shared__ unsigned long long keys[kMaxBlocks];
   __shared__ float fbuf[8];
   __shared__ int s_count;
   const int nb = g.nb, W32 = (nb + 31) / 32;
-  for (int w = threadIdx.x; w < W32; w += 256) bits[w] = 0u;
+  for (int w = threadIdx.x; w < W32; w += 256) { bits[w] = 0u; vbits[w] = 0u; }
   __syncthreads();
+  // which key blocks hold at least one token, computed once per row
+  for (int j = threadIdx.x; j < nb; j += 256)
+    if (block_valid(g, j, p.T, p.H, p.W)) atomicOr(&vbits[j / 32], 1u << (j % 32));
+  __syncthreads();
+  auto kvalid = [&](int j) { return (vbits[j >> 5] >> (j & 31)) & 1u; };
   const bool qvalid = block_valid(g, i, p.T, p.H, p.W);
   const float* srow = p.scores ? p.scores + ((size_t)bh * p.NB + i) * p.NB : nullptr;
 
@@ -307,7 +349,7 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
       for (int r = 0; r < p.topk; ++r) {
         unsigned long long best = 0ull;
         for (int j = threadIdx.x; j < nb; j += 256) {
-          if (!block_valid(g, j, p.T, p.H, p.W) || ((bits[j / 32] >> (j % 32)) & 1u)) continue;
+          if (!kvalid(j) || ((bits[j / 32] >> (j % 32)) & 1u)) continue;
           uint32_t f = __float_as_uint(srow[j]);
           f = (f & 0x80000000u) ? ~f : (f | 0x80000000u);         // order-preserving
           // nonzero for every non-NaN score, so 0 can stand for "none"
@@ -342,7 +384,7 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
         const int jt = it - rt + e / (wh * ww), jh = ih - rh + (e / ww) % wh, jw = iw - rw + e % ww;
         if (jt < 0 || jh < 0 || jw < 0 || jt >= g.nt || jh >= g.nh || jw >= g.nw) continue;
         const int j = (jt * g.nh + jh) * g.nw + jw;
-        if (block_valid(g, j, p.T, p.H, p.W)) atomicOr(&bits[j / 32], 1u << (j % 32));
+        if (kvalid(j)) atomicOr(&bits[j / 32], 1u << (j % 32));
       }
       __syncthreads();
       if (p.kind == SA_MASK_SPADE) {
@@ -350,17 +392,17 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
         // probability (ties to the lower index) whose fp32 running sum reaches top_p
         float mx = -INFINITY;
         for (int j = threadIdx.x; j < nb; j += 256)
-          if (block_valid(g, j, p.T, p.H, p.W)) mx = fmaxf(mx, srow[j]);
+          if (kvalid(j)) mx = fmaxf(mx, srow[j]);
         mx = block_max(mx, fbuf);
         float se = 0.f;
         for (int j = threadIdx.x; j < nb; j += 256)
-          if (block_valid(g, j, p.T, p.H, p.W)) se += expf(srow[j] - mx);
+          if (kvalid(j)) se += expf(srow[j] - mx);
         se = block_sum(se, fbuf);
         int npow = 1;
         while (npow < nb) npow <<= 1;
         for (int j = threadIdx.x; j < npow; j += 256) {
           unsigned long long key = 0ull;                 // invalid / padding sorts last
-          if (j < nb && block_valid(g, j, p.T, p.H, p.W)) {
+          if (j < nb && kvalid(j)) {
             const float pr = expf(srow[j] - mx) / se;
             key = ((unsigned long long)__float_as_uint(pr) << 32) | (0xFFFFFFFFu - (uint32_t)j);
           }
@@ -380,15 +422,48 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
             }
             __syncthreads();
           }
-        if (threadIdx.x == 0) {
-          float run = 0.f;
-          int c = 0;
-          while (c < npow && keys[c] != 0ull) {
-            run += __uint_as_float((uint32_t)(keys[c] >> 32));
-            ++c;
-            if (run >= p.top_p) break;
-          }
-          s_count = c;
+        // Shortest prefix of the sorted order whose fp32 running sum reaches
+        // top_p: a block-wide inclusive scan (thread t sums its 16 consecutive
+        // entries, then a scan over the thread totals), then the first
+        // position whose running sum reaches top_p. Running sums in another
+        // order than one left-to-right pass differ only in the last bits.
+        constexpr int kPer = kMaxBlocks / 256;
+        float cum[kPer];
+        float run = 0.f;
+        const int base = threadIdx.x * kPer;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) {
+          const int a = base + e;
+          const float pr = (a < npow && keys[a] != 0ull) ? __uint_as_float((uint32_t)(keys[a] >> 32)) : 0.f;
+          run += pr;
+          cum[e] = run;
+        }
+        // exclusive scan of the thread totals (warp shuffles, then warp totals)
+        float incl = run;
+        for (int o = 1; o < 32; o <<= 1) {
+          const float t = __shfl_up_sync(0xffffffffu, incl, o);
+          if ((threadIdx.x & 31) >= o) incl += t;
+        }
+        __shared__ float wsum[8];
+        if ((threadIdx.x & 31) == 31) wsum[threadIdx.x >> 5] = incl;
+        if (threadIdx.x == 0) s_count = 0x7fffffff;
+        __syncthreads();
+        float wpre = 0.f;
+        for (int w = 0; w < (int)(threadIdx.x >> 5); ++w) wpre += wsum[w];
+        const float excl = wpre + incl - run;
+        int first = 0x7fffffff;
+#pragma unroll
+        for (int e = kPer - 1; e >= 0; --e) {
+          const int a = base + e;
+          if (a < npow && keys[a] != 0ull && excl + cum[e] >= p.top_p) first = a;
+        }
+        if (first != 0x7fffffff) atomicMin(&s_count, first + 1);
+        __syncthreads();
+        if (threadIdx.x == 0 && s_count == 0x7fffffff) {
+          // the sum never reached top_p (rounding): keep every valid block
+          int nvalid = 0;
+          while (nvalid < npow && keys[nvalid] != 0ull) ++nvalid;
+          s_count = nvalid;
         }
         __syncthreads();
         for (int a = threadIdx.x; a < s_count; a += 256) {
@@ -420,7 +495,7 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
         uint32_t word = src[w];
         if (32 * w + 32 > nb) word &= (nb - 32 * w) >= 32 ? 0xffffffffu : ((1u << (nb - 32 * w)) - 1u);
         for (int b = 0; b < 32; ++b)
-          if (((word >> b) & 1u) && !block_valid(g, 32 * w + b, p.T, p.H, p.W)) word &= ~(1u << b);
+          if (((word >> b) & 1u) && !kvalid(32 * w + b)) word &= ~(1u << b);
         bits[w] = word;
       }
     }
@@ -474,7 +549,8 @@ cudaError_t launch_permute_fm(const PermuteParams& p, int BH, cudaStream_t st) {
 }
 
 cudaError_t launch_pool_sics(const PoolParams& p, int BH, int max_nb, cudaStream_t st) {
-  dim3 grid(max_nb, p.C, BH);
+  (void)max_nb;
+  dim3 grid(p.C, p.nRt * p.nRh * p.nRw, BH);
   if (p.d == 128) pool_sics_kernel<128><<<grid, 256, 0, st>>>(p);
   else if (p.d == 64) pool_sics_kernel<64><<<grid, 256, 0, st>>>(p);
   else return cudaErrorInvalidValue;

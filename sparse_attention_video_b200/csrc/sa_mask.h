@@ -32,6 +32,8 @@ struct PoolParams {
   float* sics;                      // [BH][C][NB]
   int cand[kMaxCand][3];
   int C, NB, T, H, W, d;
+  int Rt, Rh, Rw;                   // region: lcm of the candidates' tiles, <= 8 blocks each
+  int nRt, nRh, nRw;                // regions covering every candidate's tile grid
 };
 
 struct ChooseParams {
