@@ -204,6 +204,29 @@ def policy_kwargs(wl):
 LAUNCHES_PER_STEP = {"topk": 5, "sta": 3, "spatiotemporal": 4, "spade": 5, "fg": 13}
 
 
+# ---------------------------------------------------------------- multi-rank helpers
+def rank_workload(wl, rank):
+    """Rank r runs its own problem of the same shape (weak scaling, no data
+    exchange): the seeds differ by rank."""
+    return wl.with_(config_id=wl.config_id + 1000 * rank)
+
+
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise maximum of a list of floats over all ranks (the step time of
+    a multi-GPU run is its slowest rank)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return list(values)
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_tflops(world, flops_per_rank_step, ms_per_step):
+    """Whole-job throughput: every rank's work over the slowest rank's time."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
     if rank != 0:
@@ -261,7 +284,7 @@ def main():
     if args.heads:
         th = tuple(range(args.heads // 2, args.heads)) if wl.temporal_heads else ()
         wl = wl.with_(heads=args.heads, temporal_heads=th)
-    wl_r = wl.with_(config_id=wl.config_id + 1000 * rank)      # independent problem per rank
+    wl_r = rank_workload(wl, rank)
     log("generating inputs")
     x = make_qkv(wl_r)
     log("inputs ready")
@@ -320,13 +343,11 @@ def main():
     mask_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     perm_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    if world > 1:
-        t = torch.tensor([ms_total, attn_ms, mask_ms, perm_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total, attn_ms, mask_ms, perm_ms = t.tolist()
+    ms_total, attn_ms, mask_ms, perm_ms = max_over_ranks([ms_total, attn_ms, mask_ms, perm_ms],
+                                                          dist, dev)
     assert sa.status() == 0, "device status word set during the timed steps"
     ms_step = ms_total / args.steps
-    value = world * flops_call / (ms_step * 1e-3) / 1e12
+    value = aggregate_tflops(world, flops_call, ms_step)
 
     # ---- end to end through the public API with host buffers
     o_host = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
@@ -344,10 +365,7 @@ def main():
     torch.cuda.synchronize(dev)
     log("end-to-end steps done")
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
+    e2e_ms = max_over_ranks([e2e_ms], dist, dev)[0]
     h2d = sum(host[n].numel() * 2 for n in "qkv")
     d2h = o_host.numel() * 2 + lse_host.numel() * 4
 
@@ -412,7 +430,7 @@ def main():
                      "peak_note": f"{peak_src} sustained cuBLAS bf16 (burst {peak_burst})",
                      "traffic": traffic if wl.name == WORKLOAD and not args.heads else None},
         "cpu_baseline": cpu,
-        "e2e": {"value": world * flops_call / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": aggregate_tflops(world, flops_call, e2e_ms), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": LAUNCHES_PER_STEP[wl.kind] * args.steps,
         "clocks": clk,

@@ -225,6 +225,15 @@ SA_API int sparse_attn_mask_export(const sa_problem* problem, const sa_policy* p
  * SA_ERR_DEVICE_BOUNDS. If ``clear`` is nonzero the word is reset. */
 SA_API int sparse_attn_status(void* scratch_ws, void* stream, int clear);
 
+/* Failure-path self-test: launches one CTA on ``stream`` that waits, with the
+ * bounded wait every kernel of this library uses, on a barrier that nothing
+ * completes. After about one second the wait gives up and records
+ * SA_ERR_DEVICE_TIMEOUT in the status word of ``scratch_ws`` (read it with
+ * sparse_attn_status); the context stays usable. While that status is not
+ * cleared, later kernels that share the status word exit at once. Returns
+ * SA_OK once the launch is enqueued. */
+SA_API int sparse_attn_selftest_wait_timeout(void* scratch_ws, void* stream);
+
 /* ---------------------------------------------------------------- no allocation
  * The papers have no counterpart to this entry point. It is for callers that
  * cannot allocate device memory when they build a mask: code running inside

@@ -25,7 +25,8 @@ SA_EXPORT_FG_TILE_KEYS = 5
 EXPORTED = ("sparse_attn_workspace_size", "sparse_attn_build_mask", "sparse_attn_forward",
             "sparse_attn_permute", "sparse_attn_attend",
             "sparse_attn_export_bytes", "sparse_attn_mask_export", "sparse_attn_status",
-            "sparse_attn_build_mask_static", "sparse_attn_strerror")
+            "sparse_attn_build_mask_static", "sparse_attn_selftest_wait_timeout",
+            "sparse_attn_strerror")
 
 SA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
 
@@ -82,6 +83,7 @@ def lib():
         L.sparse_attn_mask_export.argtypes = [P, PP, vp, ctypes.c_int, vp, sz, vp]
         L.sparse_attn_status.argtypes = [vp, vp, ctypes.c_int]
         L.sparse_attn_build_mask_static.argtypes = [P, PP, vp, vp, vp, vp]
+        L.sparse_attn_selftest_wait_timeout.argtypes = [vp, vp]
         L.sparse_attn_strerror.argtypes = [ctypes.c_int]
         L.sparse_attn_strerror.restype = ctypes.c_char_p
         for name in EXPORTED[:-1]:
