@@ -32,7 +32,8 @@ namespace sa {
 
 namespace {
 
-constexpr int kScoreThreads = 256;
+constexpr int kScoreThreads = 640;   // warps 4-19: epilogue, four per key lane quarter
+constexpr int kEpiParts = 4;         // group columns split into 128 / kEpiParts per warp
 constexpr int kKeyTilesPerCta = 64;      // 8192 keys per CTA
 constexpr int kBins = 4096;
 
@@ -117,7 +118,7 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
     mbar_init(&bars->q_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->k_full[i], 1); mbar_init(&bars->k_empty[i], 1);
-      mbar_init(&bars->acc_full[i], 1); mbar_init(&bars->acc_free[i], 4);
+      mbar_init(&bars->acc_full[i], 1); mbar_init(&bars->acc_free[i], 4 * kEpiParts);
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -189,10 +190,14 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
     }
   } else if (warp >= 4) {
     // ---------------------------------------------------------- epilogue
-    const int r = threadIdx.x - 128;                  // key lane within the tile
-    const int w4 = warp - 4;
-    const uint32_t lane_off = (uint32_t)(32 * w4) << 16;
-    uint32_t* whist = hist + w4 * kBins;
+    // Warp w reads tensor-memory lanes 32*(w%4).. (its keys) and part
+    // (w-4)/4 of the 128 group columns; the warps of a lane quarter share one
+    // histogram.
+    constexpr int kCols = 128 / kEpiParts;
+    const int quarter = warp & 3, half = (warp - 4) >> 2;
+    const int r = 32 * quarter + lane;                 // key lane within the tile
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    uint32_t* whist = hist + quarter * kBins;
     const int g_base = gt * 128;
     const int g_lim = min(128, p.G - g_base);
     for (int j = 0; j < n_tiles; ++j) {
@@ -203,9 +208,12 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       tc_fence_after();
       const int key = (tile0 + j) * 128 + r;
       const bool kvalid = key < p.N;
-      uint32_t words[4] = {0u, 0u, 0u, 0u};
+      uint32_t words[kCols / 32];
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int i = 0; i < kCols / 32; ++i) words[i] = 0u;
+#pragma unroll
+      for (int cc = 0; cc < kCols; cc += 32) {
+        const int c0 = half * kCols + cc;
         float v[32];
         tmem_ld32(tmem + ab * 128 + lane_off + c0, v);
         tmem_wait_ld();
@@ -222,7 +230,7 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
           for (int e = 0; e < 32; ++e) {
             const bool keep = kvalid && (c0 + e < g_lim) && order_key(v[e]) >= tau_key;
             const uint32_t ballot = __ballot_sync(0xffffffffu, keep);
-            if (lane == e) words[c0 / 32] = ballot;
+            if (lane == e) words[cc / 32] = ballot;
           }
         }
       }
@@ -230,11 +238,11 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->acc_free[ab]);
       if (p.mode == FG_MODE_BITS) {
-        // lane e holds the 32 keys of this warp for groups e, e+32, e+64, e+96
-        const int kw = ((tile0 + j) * 128 + 32 * w4) / 32;
+        // lane e holds this warp's 32 keys for groups half*kCols + 32*i + e
+        const int kw = ((tile0 + j) * 128 + 32 * quarter) / 32;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int gl = lane + 32 * i;
+        for (int i = 0; i < kCols / 32; ++i) {
+          const int gl = half * kCols + lane + 32 * i;
           if (gl < g_lim && kw < p.WN)
             p.bits[((size_t)bh * p.G + g_base + gl) * p.WN + kw] = words[i];
         }
