@@ -225,19 +225,6 @@ bool map_5d(CUtensorMap* m, const void* base, const sa_problem& pr, const int* t
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2-D map over [rows][d] bf16 with a (64, 1) box: the tensor map a
-// tile::gather4 load needs (one-row boxes, four row coordinates per load).
-bool map_rows(CUtensorMap* m, const void* base, long long rows, int d) {
-  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-  cuuint32_t box[2] = {64, 1};
-  cuuint32_t es[2] = {1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                     strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int gcd_i(int a, int b) { return b ? gcd_i(b, a % b) : a; }
 int lcm_i(int a, int b) { return a / gcd_i(a, b) * b; }
 
@@ -466,14 +453,14 @@ extern "C" int sparse_attn_attend(const sa_problem* problem, const sa_policy* po
     AttnMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     if (!map_3d(&maps.q[0], q, c.BH, c.N, c.d, 128)) return SA_ERR_CUDA;
-    if (!map_rows(&maps.k[0], k, (long long)c.BH * c.N, c.d)) return SA_ERR_CUDA;
-    if (!map_rows(&maps.v[0], v, (long long)c.BH * c.N, c.d)) return SA_ERR_CUDA;
     AttnParams ap{};
     ap.o = static_cast<__nv_bfloat16*>(o);
     ap.lse = lse;
     ap.status = status;
     ap.BH = c.BH; ap.NB = c.M.P; ap.T = pr.T; ap.H = pr.H; ap.W = pr.W; ap.N = c.N;
     ap.scale_log2 = scale_log2;
+    ap.k_rows = static_cast<const __nv_bfloat16*>(k);
+    ap.v_rows = static_cast<const __nv_bfloat16*>(v);
     ap.fg_list = reinterpret_cast<const uint32_t*>(c.mw + c.M.off_fg_list);
     ap.fg_offsets = reinterpret_cast<const uint32_t*>(c.mw + c.M.off_fg_offsets);
     ap.fg_cap = c.M.cap;

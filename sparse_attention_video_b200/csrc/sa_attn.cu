@@ -28,6 +28,8 @@
 //               frame-major layouts by a 3-D box.
 //   warp 9      allocates tensor memory; lane 0 issues all MMAs. S is double
 //               buffered so Q K_{j+1}^T runs while row j is in softmax.
+//   warps 10-11 (M x 1 slices only) copy the kept keys' K and V rows with
+//               cp.async; warp 8 then only builds the per-group masks.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -43,6 +45,7 @@ constexpr int kThreads = 320;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kCopyWarp0 = 10;             // gather mode: warps 10-11 copy K/V rows
 constexpr int kStages = 3;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows > 2^8
 // One exp2 in kPolyEvery on the FMA pipe (0 = all on MUFU). Measured on the
@@ -110,17 +113,6 @@ __device__ __forceinline__ void load_block(const CUtensorMap* maps, const HeadGe
     if (map >= 2) tma_load_5d(d, m, bar, h * 64, c1, c2, c3, bh);
     else tma_load_3d(d, m, bar, h * 64, c1, bh);
   }
-}
-
-// Four rows (row indices r0..r3 of a 2-D [rows][d] map) x 64 columns into
-// four consecutive 128-byte rows of shared memory.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uint64_t* bar, int c0,
-                                            int r0, int r1, int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
-      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0),
-        "r"(r0), "r"(r1), "r"(r2), "r"(r3) : "memory");
 }
 
 // Slot ``s`` of block ``blk`` -> original token index, or -1 for padding.
@@ -193,7 +185,7 @@ __device__ __forceinline__ uint32_t site(uint32_t role, uint32_t bar, int j) {
 // groups, gathered 128 rows at a time with TMA tile::gather4, and each row
 // masks keys outside its own group.
 template <int D, int BN, bool kGather>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kGather ? kThreads + 64 : kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   using L = Smem<D, BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -233,9 +225,11 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
+    // gather mode: K/V stages are filled by the two copy warps, not by TMA
+    const uint32_t fill_arrivals = kGather ? 2u : 1u;
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->k_full[s], 1); mbar_init(&bars->k_empty[s], 1);
-      mbar_init(&bars->v_full[s], 1); mbar_init(&bars->v_empty[s], 1);
+      mbar_init(&bars->k_full[s], fill_arrivals); mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], fill_arrivals); mbar_init(&bars->v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) mbar_init(&bars->s_full[b], 1);
     mbar_init(&bars->p_full, kSoftmaxWarps);
@@ -252,7 +246,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   if constexpr (BN < 128) {
     // Rows BN..127 of the 128-row MMA operand carry no query; keep them finite.
     constexpr int kVecPerHalf = (128 - BN) * 8;
-    for (int i = threadIdx.x; i < kVecPerHalf * L::kHalvesD; i += kThreads) {
+    for (int i = threadIdx.x; i < kVecPerHalf * L::kHalvesD; i += blockDim.x) {
       const int h = i / kVecPerHalf, rem = i % kVecPerHalf;
       reinterpret_cast<uint4*>(sQ + h * 16384 + BN * 128)[rem] = make_uint4(0, 0, 0, 0);
     }
@@ -282,8 +276,6 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         for (int h = 0; h < D / 64; ++h)
           tma_load_3d(sQ + h * (BN * 128), &maps.q[0], &bars->q_full, h * 64, qb * BN, bh);
       }
-      const int row0 = bh * p.N;
-      int issued_k = 0, issued_v = 0;
       // list entries j*128 + lane + 32*s; key index in the low 30 bits, one
       // membership bit per group of the tile in bits 30 and 31. The next
       // chunk's entries are loaded while this chunk waits on its barriers.
@@ -294,7 +286,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         en[s4] = idx < list_count ? __ldg(list + idx) : 0u;
       }
       for (int j = 0; j < n_keys; ++j) {
-        const int st = j % kStages, rnd = j / kStages, mb = j & 1;
+        const int mb = j & 1;
         uint32_t e[4];
         bool val[4];
 #pragma unroll
@@ -320,45 +312,6 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
           for (int s4 = 0; s4 < 4; ++s4) { bars->masks[mb][s4] = m0[s4]; bars->masks[mb][4 + s4] = m1[s4]; }
           mbar_arrive(&bars->m_full[mb]);
         }
-        // rows 4*lane .. 4*lane+3 of the chunk for this lane's gather4
-        int rows[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int src = (4 * lane + i) & 31;
-          const uint32_t x0 = __shfl_sync(0xffffffffu, e[0], src);
-          const uint32_t x1 = __shfl_sync(0xffffffffu, e[1], src);
-          const uint32_t x2 = __shfl_sync(0xffffffffu, e[2], src);
-          const uint32_t x3 = __shfl_sync(0xffffffffu, e[3], src);
-          const int sel = lane >> 3;
-          const uint32_t x = sel == 0 ? x0 : sel == 1 ? x1 : sel == 2 ? x2 : x3;
-          rows[i] = row0 + (int)(x & 0x3FFFFFFFu);
-        }
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->k_empty[st], (rnd & 1) ^ 1, abort, status,
-                                               site(1, 1, j))))
-          break;
-        if (lane == 0) mbar_arrive_expect_tx(&bars->k_full[st], L::kKVBytes);
-        __syncwarp();
-#pragma unroll
-        for (int h = 0; h < D / 64; ++h)
-          tma_gather4(sK + st * L::kKVBytes + h * (BN * 128) + lane * 512, &maps.k[0],
-                      &bars->k_full[st], h * 64, rows[0], rows[1], rows[2], rows[3]);
-        issued_k = j + 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->v_empty[st], (rnd & 1) ^ 1, abort, status,
-                                               site(1, 2, j))))
-          break;
-        if (lane == 0) mbar_arrive_expect_tx(&bars->v_full[st], L::kKVBytes);
-        __syncwarp();
-#pragma unroll
-        for (int h = 0; h < D / 64; ++h)
-          tma_gather4(sV + st * L::kKVBytes + h * (BN * 128) + lane * 512, &maps.v[0],
-                      &bars->v_full[st], h * 64, rows[0], rows[1], rows[2], rows[3]);
-        issued_v = j + 1;
-      }
-      if (*abort && lane == 0) {
-        for (int j = max(0, issued_k - kStages); j < issued_k; ++j)
-          mbar_drain(&bars->k_full[j % kStages], (j / kStages) & 1);
-        for (int j = max(0, issued_v - kStages); j < issued_v; ++j)
-          mbar_drain(&bars->v_full[j % kStages], (j / kStages) & 1);
       }
     }
   } else if (warp == kProducerWarp) {
@@ -443,6 +396,63 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       // Every MMA issued above must finish before tensor memory is freed.
       umma_commit(&bars->drain);
       mbar_drain(&bars->drain, 0);
+    }
+  } else if (kGather && warp >= kCopyWarp0) {
+    // ------------------------------------------------------------ K/V row copies (gather)
+    // Thread t copies rows t and t+64 of every chunk: 16-byte cp.async pieces
+    // straight into the 128-byte-swizzled tiles the MMA reads. Chunk j is
+    // announced once chunk j+1 is in flight: wait for this thread's older
+    // group, make the generic-proxy writes visible to the tensor core's async
+    // proxy, then arrive.
+    const int t = (warp - kCopyWarp0) * 32 + lane;
+    const __nv_bfloat16* kbase = p.k_rows + (size_t)bh * p.N * D;
+    const __nv_bfloat16* vbase = p.v_rows + (size_t)bh * p.N * D;
+    bool okc = true;
+    for (int j = 0; j < n_keys; ++j) {
+      const int st = j % kStages, rnd = j / kStages;
+      int key[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const uint32_t idx = (uint32_t)j * BN + t + 64 * i;
+        key[i] = idx < list_count ? (int)(__ldg(list + idx) & 0x3FFFFFFFu) : 0;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->k_empty[st], (rnd & 1) ^ 1, abort, status,
+                                             site(4, 1, j))) ||
+          !__all_sync(0xffffffffu, mbar_wait(&bars->v_empty[st], (rnd & 1) ^ 1, abort, status,
+                                             site(4, 2, j)))) {
+        okc = false;
+        break;
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int r = t + 64 * i;
+        const __nv_bfloat16* ks = kbase + (size_t)key[i] * D;
+        const __nv_bfloat16* vs = vbase + (size_t)key[i] * D;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          const int off = (c / 8) * (BN * 128) + r * 128 + (((c % 8) ^ (r & 7)) << 4);
+          cp_async16(sK + st * L::kKVBytes + off, ks + c * 8);
+          cp_async16(sV + st * L::kKVBytes + off, vs + c * 8);
+        }
+      }
+      cp_async_commit();
+      if (j >= 1) {
+        cp_async_wait<1>();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bars->k_full[(j - 1) % kStages]);
+          mbar_arrive(&bars->v_full[(j - 1) % kStages]);
+        }
+      }
+    }
+    // own copies land before anything else (also on the abort path)
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (okc && n_keys > 0 && lane == 0) {
+      mbar_arrive(&bars->k_full[(n_keys - 1) % kStages]);
+      mbar_arrive(&bars->v_full[(n_keys - 1) % kStages]);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -660,7 +670,7 @@ static cudaError_t launch_one(const AttnMaps& maps, const AttnParams& p, cudaStr
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   dim3 grid(p.NB, p.BH);
-  kern<<<grid, kThreads, L::kAlloc, stream>>>(maps, p);
+  kern<<<grid, kGather ? kThreads + 64 : kThreads, L::kAlloc, stream>>>(maps, p);
   return cudaGetLastError();
 }
 

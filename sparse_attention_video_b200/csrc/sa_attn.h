@@ -28,8 +28,9 @@ struct AttnParams {
   uint32_t* status;        // device status word
   int BH, NB, T, H, W, N;
   float scale_log2;        // log2(e) / sqrt(d)
-  // gather mode (M x 1 key slices): maps.q[0] is the 3-D query map, maps.k[0]
-  // and maps.v[0] are 2-D [BH*N][d] maps with one-row boxes for tile::gather4
+  // gather mode (M x 1 key slices): maps.q[0] is the 3-D query map
+  const __nv_bfloat16* k_rows; // gather mode: K and V [BH][N][d], rows copied by key index
+  const __nv_bfloat16* v_rows;
   const uint32_t* fg_list;     // [BH][fg_cap]
   const uint32_t* fg_offsets;  // [BH][NB + 1]
   long long fg_cap;
