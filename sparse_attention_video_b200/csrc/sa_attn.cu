@@ -14,16 +14,20 @@
 //
 // Roles (320 threads):
 //   warps 0-7   softmax: two threads per row. Warp w reads tensor-memory lanes
-//               32*(w%4).. (row r = lane), and half w/4 of the row's columns.
-//               The two halves exchange their row maxima through shared
-//               memory and an mbarrier. The running maximum only moves when it
-//               grows by more than 2^8, so O is rescaled rarely; P and l use
-//               the same reference, which keeps the result exact. The 1/sqrt(d)
-//               scale is folded into one FFMA before exp2. Epilogue: O / l to
-//               bf16, each thread storing its half of the row at the query's
-//               original token row (the inverse permutation is fused here).
+//               32*(w%4).. (row r = lane), and half w/4 of each key block.
+//               Each half is a softmax of its own: its own running maximum and
+//               sum, and its own O accumulator that the PV MMA fills from that
+//               half's keys, so the two never wait on each other per block.
+//               The running maximum only moves when it grows by more than
+//               2^8, so O is rescaled rarely; P and l use the same reference,
+//               which keeps the result exact. The 1/sqrt(d) scale is folded
+//               into one FFMA before exp2. Epilogue: the halves trade (m, l)
+//               through shared memory, and each thread writes half of the
+//               row's columns of (a0 O_0 + a1 O_1) / (a0 l0 + a1 l1) in bf16 at
+//               the query's original token row (the inverse permutation is
+//               fused here).
 //   warp 8      TMA producer: Q once, then K and V of each kept key block into
-//               a 2-stage ring. 3D tile layouts are gathered by one 5-D box per
+//               a 3-stage ring. 3D tile layouts are gathered by one 5-D box per
 //               64 columns (no separate permutation pass); identity and
 //               frame-major layouts by a 3-D box.
 //   warp 9      allocates tensor memory; lane 0 issues all MMAs. S is double
@@ -66,9 +70,8 @@ struct Smem {
   static constexpr int kOffBar = kOffV + kStages * kKVBytes;
   static constexpr int kBytes = kOffBar + 512;
   static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-byte alignment
-  // S (two buffers), O, and 6 columns where the two halves of a row exchange
-  // their partial maxima (by iteration parity) and partial sums
-  static constexpr uint32_t kTmemCols = (2 * BN + D + 6) <= 256 ? 256 : 512;
+  // S (two buffers) and one O accumulator per half of the key block
+  static constexpr uint32_t kTmemCols = (2 * BN + 2 * D) <= 256 ? 256 : 512;
 };
 
 struct Bars {
@@ -76,12 +79,14 @@ struct Bars {
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
   uint64_t s_full[2];
-  uint64_t p_full;
+  // P_j written into S buffer j & 1. One barrier per buffer: a softmax warp
+  // that finishes block j early may arrive for block j + 1 before the others
+  // arrive for j, and that arrival must not count toward block j.
+  uint64_t p_full[2];
   uint64_t o_done;
   uint64_t drain;
   uint64_t m_full[2], m_empty[2];   // gather mode: per-chunk group-membership masks
   uint32_t masks[2][8];             // [chunk & 1][first group words 0-3, second group 4-7]
-  uint64_t x_bar[4];                // warps w and w+4 (same rows) exchange values
   uint32_t tmem_base;
   int abort;
 };
@@ -232,8 +237,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       mbar_init(&bars->v_full[s], fill_arrivals); mbar_init(&bars->v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) mbar_init(&bars->s_full[b], 1);
-    mbar_init(&bars->p_full, kSoftmaxWarps);
-    for (int qd = 0; qd < 4; ++qd) mbar_init(&bars->x_bar[qd], 2);
+    for (int b = 0; b < 2; ++b) mbar_init(&bars->p_full[b], kSoftmaxWarps);
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->drain, 1);
     for (int b = 0; b < 2; ++b) {
@@ -262,8 +266,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const uint32_t tS[2] = {tmem, tmem + BN};
-  const uint32_t tO = tmem + 2 * BN;
-  const uint32_t tX = tmem + 2 * BN + D;          // exchange columns
+  const uint32_t tO = tmem + 2 * BN;              // O_0 at tO, O_1 at tO + D
   volatile int* abort = &bars->abort;
   uint32_t* status = p.status;
 
@@ -352,42 +355,59 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     if (lane == 0 && n_keys > 0) {
       constexpr uint32_t idesc_qk = umma_idesc_bf16(128, BN, false, false);
       constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, false, true);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+      // Descriptors are formed once; each MMA only advances a base by a
+      // compile-time offset, so the issuing thread spends its time issuing.
+      const uint64_t dQ = umma_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dK0 = umma_desc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dV0 = umma_desc_sw128(smem_u32(sV), L::kKVHalf, 1024);
+      uint64_t da[D / 16];
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)        // 16 bf16 along K inside a 128-byte row
+        da[kk] = umma_desc_advance(dQ, (kk / 4) * 16384 + (kk % 4) * 32);
       auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait(&bars->p_full, i & 1, abort, status, site(2, 3, i))) return false;
-        if (!mbar_wait(&bars->v_full[i % kStages], (i / kStages) & 1, abort, status, site(2, 4, i)))
+        if (!mbar_wait<false>(&bars->p_full[i & 1], (i >> 1) & 1, abort, status, site(2, 3, i)))
           return false;
+        if (!mbar_wait<false>(&bars->v_full[i % kStages], (i / kStages) & 1, abort, status,
+                              site(2, 4, i)))
+          return false;
+        const uint64_t dv = umma_desc_advance(dV0, (i % kStages) * L::kKVBytes);
+        const uint32_t ta = tS[i & 1];
+        uint64_t db[BN / 16];
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) db[kk] = umma_desc_advance(dv, kk * 16 * 128);
         tc_fence_after();
-        const uint32_t vbase = aV + (i % kStages) * L::kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           // A = P in tensor memory (16 keys = 8 packed columns per step);
-          // B = V (MN-major: d contiguous).
-          const uint64_t db = umma_desc_sw128(vbase + kk * 16 * 128, L::kKVHalf, 1024);
-          umma_bf16_ts(tO, tS[i & 1] + kk * 8, db, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          // each half's P sits at the start of that half's own S columns.
+          // B = V (MN-major: d contiguous). Keys of the first half of the
+          // block accumulate into O_0, keys of the second half into O_1.
+          constexpr int kPerHalf = BN / 32;
+          const int hk = kk / kPerHalf, sk = kk % kPerHalf;
+          umma_bf16_ts(tO + hk * D, ta + hk * (BN / 2) + sk * 8, db[kk], idesc_pv,
+                       (i > 0 || sk > 0) ? 1u : 0u);
         }
         umma_commit(&bars->o_done);
         umma_commit(&bars->v_empty[i % kStages]);
         return true;
       };
-      bool ok = mbar_wait(&bars->q_full, 0, abort, status, site(2, 5, 0));
+      bool ok = mbar_wait<false>(&bars->q_full, 0, abort, status, site(2, 5, 0));
       for (int j = 0; ok && j < n_keys; ++j) {
         const int st = j % kStages, sb = j & 1;
-        if (!mbar_wait(&bars->k_full[st], (j / kStages) & 1, abort, status, site(2, 6, j))) {
+        if (!mbar_wait<false>(&bars->k_full[st], (j / kStages) & 1, abort, status, site(2, 6, j))) {
           ok = false;
           break;
         }
+        const uint64_t dk = umma_desc_advance(dK0, st * L::kKVBytes);
+        uint64_t db[D / 16];
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          db[kk] = umma_desc_advance(dk, (kk / 4) * L::kKVHalf + (kk % 4) * 32);
         // S buffer sb was last read as P_{j-2} by PV_{j-2}, which was issued
         // before this QK; tcgen05 MMAs of one thread run in issue order.
         tc_fence_after();
-        const uint32_t kbase = aK + st * L::kKVBytes;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk % 4) * 32;            // 16 bf16 along K inside a 128-byte row
-          const uint64_t da = umma_desc_sw128(aQ + (kk / 4) * 16384 + off, 16, 1024);
-          const uint64_t db = umma_desc_sw128(kbase + (kk / 4) * L::kKVHalf + off, 16, 1024);
-          umma_bf16_ss(tS[sb], da, db, idesc_qk, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk) umma_bf16_ss(tS[sb], da[kk], db[kk], idesc_qk, kk > 0 ? 1u : 0u);
         umma_commit(&bars->s_full[sb]);
         umma_commit(&bars->k_empty[st]);
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
@@ -456,16 +476,24 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    // Thread (half, r) owns keys [half*HC, half*HC + HC) of every block for row
+    // r: its own running maximum m and sum l, and its own accumulator
+    // O_half = sum over its keys of P V, which the PV MMA writes to a separate
+    // tensor-memory region. The two halves never wait on each other inside the
+    // loop; the epilogue merges them as two partial softmaxes:
+    //   O = (a0 O_0 + a1 O_1) / (a0 l0 + a1 l1),  a_h = 2^(m_h - max(m0, m1)).
     constexpr int HC = BN / 2;                        // S columns per thread
-    constexpr int HD = D / 2;                         // O columns per thread
     const int half = warp >> 2;
     const int r = (warp & 3) * 32 + lane;             // row == tensor-memory lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tOh = tO + half * D + lane_off;    // this half's accumulator
     const float scale = p.scale_log2;
     float m = -INFINITY;                              // reference maximum, log2 units
-    float l = 0.f;                                    // this half's share of the row sum
+    float l = 0.f;                                    // sum of P over this half's keys
     float s[HC];
     bool ok = true;
+    // key block of the next iteration, loaded one iteration ahead
+    int kb_next = (!kGather && n_keys > 0) ? cols[0] : 0;
     for (int j = 0; j < n_keys; ++j) {
       const int sb = j & 1;
       uint32_t pw[HC / 32];
@@ -483,8 +511,10 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->m_empty[sb]);
       } else {
+        const int kb = kb_next;
+        if (j + 1 < n_keys) kb_next = cols[j + 1];
         uint32_t full[BN / 32];
-        pad = block_pad_mask<BN>(g, cols[j], p.T, p.H, p.W, full);
+        pad = block_pad_mask<BN>(g, kb, p.T, p.H, p.W, full);
 #pragma unroll
         for (int w = 0; w < HC / 32; ++w) pw[w] = full[half * (HC / 32) + w];
       }
@@ -499,34 +529,20 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       for (int c = 0; c < HC; c += 32) tmem_ld32(tS[sb] + lane_off + half * HC + c, s + c);
       tmem_wait_ld();
 
-      // row maximum of this half: four independent chains, then combined
+      // maximum over this half's keys: three-input max, four independent chains
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (pad) {
 #pragma unroll
-        for (int c = 0; c < HC; ++c) {
-          s[c] = ((pw[c / 32] >> (c % 32)) & 1u) ? s[c] : -INFINITY;
-          mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
-        }
-      } else {
+        for (int c = 0; c < HC; ++c) s[c] = ((pw[c / 32] >> (c % 32)) & 1u) ? s[c] : -INFINITY;
+      }
 #pragma unroll
-        for (int c = 0; c < HC; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
+      for (int c = 0; c < HC; c += 8) {
+        mx4[0] = fmax3(mx4[0], s[c], s[c + 1]);
+        mx4[1] = fmax3(mx4[1], s[c + 2], s[c + 3]);
+        mx4[2] = fmax3(mx4[2], s[c + 4], s[c + 5]);
+        mx4[3] = fmax3(mx4[3], s[c + 6], s[c + 7]);
       }
-      float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      // row maximum over both halves, exchanged through spare tensor-memory
-      // columns (the two warps of a pair read and write the same lanes)
-      tmem_st1(tX + lane_off + 2 * sb + half, mx);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->x_bar[warp & 3]);
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->x_bar[warp & 3], j & 1, abort, status,
-                                             site(3, 12, j)))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      mx = fmaxf(mx, tmem_ld1(tX + lane_off + 2 * sb + (half ^ 1)));
-      tmem_wait_ld();
+      const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
       const float m_new = fmaxf(m, mx * scale);
       const bool rescale = (m == -INFINITY) || (m_new > m + kRescaleThreshold);
       const float m_use = rescale ? m_new : m;
@@ -535,8 +551,8 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
 #pragma unroll
         for (int c = 0; c < HC; ++c) s[c] = 0.f;
       } else {
-        // exp2 of every kPolyEvery-th column on the FMA pipe, the rest on MUFU,
-        // to balance the two pipes; four independent partial sums
+        // exp2 of every kPolyEvery-th column on the FMA pipe, the rest on MUFU;
+        // four independent partial sums
         const float neg = -m_use;
         float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -545,110 +561,121 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
           s[c] = (kPolyEvery > 0 && c % kPolyEvery == kPolyEvery - 1) ? exp2_poly(x) : ex2_approx(x);
           rs4[c & 3] += s[c];
         }
-        if (pad) {
-          // masked keys: exactly zero (the polynomial floors at 2^-125)
+        if (kPolyEvery > 0 && pad) {
+          // masked keys: exactly zero. ex2.approx(-inf) is already +0; only
+          // the polynomial (which floors at 2^-125) needs this.
 #pragma unroll
           for (int c = 0; c < HC; ++c)
             if (!((pw[c / 32] >> (c % 32)) & 1u)) { rs4[c & 3] -= s[c]; s[c] = 0.f; }
         }
         rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       }
-      // P buffer and O are read/written by PV of the previous block: wait for it.
+      // O_half is accumulated by PV of the previous block, so a rescale waits
+      // for it; without one nothing here touches O and no wait is needed.
+      // The wait is unambiguous by parity: S_j was committed after PV_{j-2}
+      // was issued, so PV_{j-2} is complete and o_done is at most one phase
+      // behind PV_{j-1}. tcgen05.ld/st are warp-collective, so the whole warp
+      // rescales when any of its rows needs it; rows that do not scale by 1.
       if (j >= 1) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done, (j - 1) & 1, abort, status,
-                                               site(3, 9, j)))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // tcgen05.ld/st are warp-collective: the whole warp rescales when any
-        // of its rows needs it; rows that do not scale by 1.
         const bool need = rescale && m != -INFINITY;
         if (__any_sync(0xffffffffu, need)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done, (j - 1) & 1, abort, status,
+                                                 site(3, 9, j)))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
           const float alpha = need ? ex2_approx(m - m_use) : 1.f;
           l *= alpha;
           float o[32];
 #pragma unroll
-          for (int c = 0; c < HD; c += 32) {
-            tmem_ld32(tO + lane_off + half * HD + c, o);
+          for (int c = 0; c < D; c += 32) {
+            tmem_ld32(tOh + c, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(tO + lane_off + half * HD + c, o);
+            tmem_st32(tOh + c, o);
           }
           tmem_wait_st();
         }
       }
       m = m_use;
       l += rs;
-      // P as packed bf16 pairs over this half's share of the first BN/2 columns
-      // of S (the A operand of the PV MMA is read from tensor memory). Packed
-      // in place: entry c only reads entries 2c and 2c+1, not yet overwritten.
+      // P as packed bf16 pairs over the first HC/2 of this half's own S
+      // columns (the A operand of the PV MMA is read from tensor memory). The
+      // other half never reads these columns, so no ordering between the two
+      // halves is needed. Packed in place: entry c only reads entries 2c and
+      // 2c+1, not yet overwritten.
 #pragma unroll
       for (int c = 0; c < HC / 2; ++c) s[c] = __uint_as_float(pack_bf16x2(s[2 * c], s[2 * c + 1]));
       if constexpr (HC / 2 >= 32) {
 #pragma unroll
-        for (int c = 0; c < HC / 2; c += 32) tmem_st32(tS[sb] + lane_off + half * (HC / 2) + c, s + c);
+        for (int c = 0; c < HC / 2; c += 32) tmem_st32(tS[sb] + lane_off + half * HC + c, s + c);
       } else {
-        tmem_st16(tS[sb] + lane_off + half * (HC / 2), s);
+        tmem_st16(tS[sb] + lane_off + half * HC, s);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full);
+      if (lane == 0) mbar_arrive(&bars->p_full[sb]);
     }
     // ------------------------------------------------------------ epilogue
+    // Once ``drain`` completes every MMA of the CTA has completed, so the Q
+    // tile is free: the two halves of each row trade (m, l) through it.
     if (ok && n_keys > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (n_keys - 1) & 1, abort, status,
-                                             site(3, 10, n_keys)));
+      // the MMA warp commits ``drain`` after its last PV
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->drain, 0, abort, status, site(3, 10, n_keys)));
       tc_fence_after();
     }
-    if (ok) {
-      // row sum over both halves
-      tmem_st1(tX + lane_off + 4 + half, l);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->x_bar[warp & 3]);
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->x_bar[warp & 3], n_keys & 1, abort, status,
-                                             site(3, 13, n_keys)));
-    }
+    float* xch = reinterpret_cast<float*>(sQ);        // [half][m, l][128 rows]
+    xch[(half * 2 + 0) * 128 + r] = m;
+    xch[(half * 2 + 1) * 128 + r] = l;
+    named_barrier_sync(1, kSoftmaxWarps * 32);
+    const float m_o = xch[((half ^ 1) * 2 + 0) * 128 + r];
+    const float l_o = xch[((half ^ 1) * 2 + 1) * 128 + r];
     const int tok = (r < BN) ? slot_to_token(g, qb, r, BN, p.T, p.H, p.W) : -1;
-    float l_other = 0.f;
     if (ok) {
-      tc_fence_after();
-      l_other = tmem_ld1(tX + lane_off + 4 + (half ^ 1));
-      tmem_wait_ld();
-    }
-    if (ok) {
-      const float l_tot = l + l_other;
+      // half 0 holds (m0, l0); the other half's values came through shared memory
+      const float m0 = half == 0 ? m : m_o, l0 = half == 0 ? l : l_o;
+      const float m1 = half == 0 ? m_o : m, l1 = half == 0 ? l_o : l;
+      const float mm = fmaxf(m0, m1);
+      const float a0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mm);
+      const float a1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mm);
+      const float l_tot = a0 * l0 + a1 * l1;
       const float inv_l = (n_keys > 0 && l_tot > 0.f) ? 1.f / l_tot : 0.f;
+      const float w0 = a0 * inv_l, w1 = a1 * inv_l;
+      // this thread writes output columns [half*D/2, half*D/2 + D/2)
+      constexpr int HD = D / 2;
       __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (tok < 0 ? 0 : tok)) * D + half * HD;
 #pragma unroll
-      for (int c = 0; c < HD; c += 32) {
-        float o[32];
+      for (int c = 0; c < HD; c += 16) {
+        float o0[16], o1[16];
         if (n_keys > 0) {
-          tmem_ld32(tO + lane_off + half * HD + c, o);
+          tmem_ld16(tO + lane_off + half * HD + c, o0);
+          tmem_ld16(tO + D + lane_off + half * HD + c, o1);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0.f;
+          for (int e = 0; e < 16; ++e) { o0[e] = 0.f; o1[e] = 0.f; }
         }
         if (tok >= 0) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
+          for (int e = 0; e < 16; e += 8) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = fmaf(o0[e + u], w0, o1[e + u] * w1);
             uint4 w;
-            w.x = pack_bf16x2(o[e] * inv_l, o[e + 1] * inv_l);
-            w.y = pack_bf16x2(o[e + 2] * inv_l, o[e + 3] * inv_l);
-            w.z = pack_bf16x2(o[e + 4] * inv_l, o[e + 5] * inv_l);
-            w.w = pack_bf16x2(o[e + 6] * inv_l, o[e + 7] * inv_l);
+            w.x = pack_bf16x2(v[0], v[1]);
+            w.y = pack_bf16x2(v[2], v[3]);
+            w.z = pack_bf16x2(v[4], v[5]);
+            w.w = pack_bf16x2(v[6], v[7]);
             *reinterpret_cast<uint4*>(orow + c + e) = w;
           }
         }
       }
       if (tok >= 0 && half == 0 && p.lse)
         p.lse[(size_t)bh * p.N + tok] =
-            (n_keys > 0 && l_tot > 0.f) ? (m + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
+            (n_keys > 0 && l_tot > 0.f) ? (mm + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
     }
   }
 

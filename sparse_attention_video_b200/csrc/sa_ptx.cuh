@@ -72,6 +72,10 @@ __device__ __forceinline__ bool grid_aborted(const uint32_t* status) {
 // Bounded wait. ``abort`` is a shared flag: once any thread of the CTA gives
 // up, every later wait of the CTA returns false at once; a timeout recorded by
 // another CTA in the status word ends the wait as well.
+// ``kSleep`` = false keeps polling without __nanosleep (try_wait already
+// suspends in hardware): for the MMA issuer, whose wake-up latency is on the
+// critical path.
+template <bool kSleep = true>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint32_t* status, uint32_t site = 0) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -87,7 +91,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         return false;
       }
     }
-    if (polls > 64) __nanosleep(64);
+    if (kSleep && polls > 64) __nanosleep(64);
   }
   return true;
 }
@@ -257,6 +261,14 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn, 
          ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Descriptor of the same tile ``byte_off`` bytes further on: the start
+// address field (address >> 4, 14 bits) is the low end of the descriptor, and
+// every shared-memory address here is below 2^18, so plain addition never
+// carries into the next field.
+__device__ __forceinline__ uint64_t umma_desc_advance(uint64_t desc, uint32_t byte_off) {
+  return desc + (uint64_t)(byte_off >> 4);
+}
+
 __device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                              uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -315,6 +327,18 @@ __device__ __forceinline__ float exp2_poly(float x) {
   const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
   const int n = __float_as_int(t) - __float_as_int(magic);
   return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
+// max(a, b, c) in one instruction (three-input max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Named barrier ``id`` (1..15) over ``count`` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
