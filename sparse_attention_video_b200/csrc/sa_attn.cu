@@ -13,25 +13,26 @@
 // axiom ledger), so the result equals masked softmax attention.
 //
 // Roles (320 threads):
-//   warps 0-7   softmax: two threads per row. Warp w reads tensor-memory lanes
-//               32*(w%4).. (row r = lane), and half w/4 of each key block.
-//               Each half is a softmax of its own: its own running maximum and
-//               sum, and its own O accumulator that the PV MMA fills from that
-//               half's keys, so the two never wait on each other per block.
-//               The running maximum only moves when it grows by more than
-//               2^8, so O is rescaled rarely; P and l use the same reference,
-//               which keeps the result exact. The 1/sqrt(d) scale is folded
-//               into one FFMA before exp2. Epilogue: the halves trade (m, l)
-//               through shared memory, and each thread writes half of the
-//               row's columns of (a0 O_0 + a1 O_1) / (a0 l0 + a1 l1) in bf16 at
-//               the query's original token row (the inverse permutation is
-//               fused here).
+//   warps 0-7   softmax, two groups of four warps. Group g takes the key
+//               blocks j with j % 2 == g, one thread per row (warp w reads
+//               tensor-memory lanes 32*(w%4)..): its own running maximum and
+//               sum, and its own O accumulator that the PV MMAs of its blocks
+//               fill. While one group waits for its next S, the other is in
+//               its exponentials. The running maximum only moves when it
+//               grows by more than 2^8, so O is rescaled rarely; P and l use
+//               the same reference, which keeps the result exact. The
+//               1/sqrt(d) scale is folded into one FFMA before exp2.
+//               Epilogue: the groups trade (m, l) through shared memory, and
+//               each thread writes half of its row's columns of
+//               (a0 O_0 + a1 O_1) / (a0 l0 + a1 l1) in bf16 at the query's
+//               original token row (the inverse permutation is fused here).
 //   warp 8      TMA producer: Q once, then K and V of each kept key block into
 //               a 3-stage ring. 3D tile layouts are gathered by one 5-D box per
 //               64 columns (no separate permutation pass); identity and
 //               frame-major layouts by a 3-D box.
-//   warp 9      allocates tensor memory; lane 0 issues all MMAs. S is double
-//               buffered so Q K_{j+1}^T runs while row j is in softmax.
+//   warp 9      allocates tensor memory; lane 0 issues all MMAs: QK_0, QK_1,
+//               then PV_j, QK_{j+2} for every j. S_j goes to buffer j % 2,
+//               O_j % 2 accumulates P_j V_j.
 //   warps 10-11 (M x 1 slices only) copy the kept keys' K and V rows with
 //               cp.async; warp 8 then only builds the per-group masks.
 #include <cuda.h>
@@ -70,7 +71,7 @@ struct Smem {
   static constexpr int kOffBar = kOffV + kStages * kKVBytes;
   static constexpr int kBytes = kOffBar + 512;
   static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-byte alignment
-  // S (two buffers) and one O accumulator per half of the key block
+  // S (one buffer per softmax group) and one O accumulator per group
   static constexpr uint32_t kTmemCols = (2 * BN + 2 * D) <= 256 ? 256 : 512;
 };
 
@@ -79,11 +80,7 @@ struct Bars {
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
   uint64_t s_full[2];
-  // P_j written into S buffer j & 1. One barrier per buffer: a softmax warp
-  // that finishes block j early may arrive for block j + 1 before the others
-  // arrive for j, and that arrival must not count toward block j.
-  uint64_t p_full[2];
-  uint64_t o_done;
+  uint64_t p_full[2];               // P_j written into S buffer j & 1 (by group j & 1)
   uint64_t drain;
   uint64_t m_full[2], m_empty[2];   // gather mode: per-chunk group-membership masks
   uint32_t masks[2][8];             // [chunk & 1][first group words 0-3, second group 4-7]
@@ -237,12 +234,11 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       mbar_init(&bars->v_full[s], fill_arrivals); mbar_init(&bars->v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) mbar_init(&bars->s_full[b], 1);
-    for (int b = 0; b < 2; ++b) mbar_init(&bars->p_full[b], kSoftmaxWarps);
-    mbar_init(&bars->o_done, 1);
+    for (int b = 0; b < 2; ++b) mbar_init(&bars->p_full[b], kSoftmaxWarps / 2);
     mbar_init(&bars->drain, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->m_full[b], 1);
-      mbar_init(&bars->m_empty[b], kSoftmaxWarps);
+      mbar_init(&bars->m_empty[b], kSoftmaxWarps / 2);
     }
     bars->abort = 0;
     fence_barrier_init();
@@ -364,6 +360,25 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)        // 16 bf16 along K inside a 128-byte row
         da[kk] = umma_desc_advance(dQ, (kk / 4) * 16384 + (kk % 4) * 32);
+      // QK_j into S buffer j & 1 (softmax group j & 1 reads it).
+      auto issue_qk = [&](int j) -> bool {
+        const int st = j % kStages;
+        if (!mbar_wait<false>(&bars->k_full[st], (j / kStages) & 1, abort, status, site(2, 6, j)))
+          return false;
+        const uint64_t dk = umma_desc_advance(dK0, st * L::kKVBytes);
+        uint64_t db[D / 16];
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          db[kk] = umma_desc_advance(dk, (kk / 4) * L::kKVHalf + (kk % 4) * 32);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16_ss(tS[j & 1], da[kk], db[kk], idesc_qk, kk > 0 ? 1u : 0u);
+        umma_commit(&bars->s_full[j & 1]);
+        umma_commit(&bars->k_empty[st]);
+        return true;
+      };
+      // PV_j: O_{j&1} += P_j V_j, P_j read from S buffer j & 1.
       auto issue_pv = [&](int i) -> bool {
         if (!mbar_wait<false>(&bars->p_full[i & 1], (i >> 1) & 1, abort, status, site(2, 3, i)))
           return false;
@@ -371,48 +386,32 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
                               site(2, 4, i)))
           return false;
         const uint64_t dv = umma_desc_advance(dV0, (i % kStages) * L::kKVBytes);
-        const uint32_t ta = tS[i & 1];
         uint64_t db[BN / 16];
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) db[kk] = umma_desc_advance(dv, kk * 16 * 128);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          // A = P in tensor memory (16 keys = 8 packed columns per step);
-          // each half's P sits at the start of that half's own S columns.
-          // B = V (MN-major: d contiguous). Keys of the first half of the
-          // block accumulate into O_0, keys of the second half into O_1.
-          constexpr int kPerHalf = BN / 32;
-          const int hk = kk / kPerHalf, sk = kk % kPerHalf;
-          umma_bf16_ts(tO + hk * D, ta + hk * (BN / 2) + sk * 8, db[kk], idesc_pv,
-                       (i > 0 || sk > 0) ? 1u : 0u);
+          // A = P in tensor memory: 16 keys = 8 packed columns per step. The
+          // P of keys 64c..64c+63 sits at the start of their own S columns
+          // 64c.. (where their scores were). B = V (MN-major: d contiguous).
+          // O_{i&1} is first written by block i & 1.
+          umma_bf16_ts(tO + (i & 1) * D, tS[i & 1] + (kk / 4) * 64 + (kk % 4) * 8, db[kk],
+                       idesc_pv, (i > 1 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&bars->o_done);
         umma_commit(&bars->v_empty[i % kStages]);
         return true;
       };
+      // Order: QK_0, QK_1, then PV_j, QK_{j+2} for every j. S buffer j & 1
+      // is rewritten by QK_{j+2} only after PV_j (issued first) read P_j, and
+      // the commit of S_{j+2} also covers PV_j: once a softmax group sees
+      // S_{j+2}, its O accumulator holds every block before j + 2.
       bool ok = mbar_wait<false>(&bars->q_full, 0, abort, status, site(2, 5, 0));
+      for (int j = 0; ok && j < 2 && j < n_keys; ++j) ok = issue_qk(j);
       for (int j = 0; ok && j < n_keys; ++j) {
-        const int st = j % kStages, sb = j & 1;
-        if (!mbar_wait<false>(&bars->k_full[st], (j / kStages) & 1, abort, status, site(2, 6, j))) {
-          ok = false;
-          break;
-        }
-        const uint64_t dk = umma_desc_advance(dK0, st * L::kKVBytes);
-        uint64_t db[D / 16];
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          db[kk] = umma_desc_advance(dk, (kk / 4) * L::kKVHalf + (kk % 4) * 32);
-        // S buffer sb was last read as P_{j-2} by PV_{j-2}, which was issued
-        // before this QK; tcgen05 MMAs of one thread run in issue order.
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) umma_bf16_ss(tS[sb], da[kk], db[kk], idesc_qk, kk > 0 ? 1u : 0u);
-        umma_commit(&bars->s_full[sb]);
-        umma_commit(&bars->k_empty[st]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        ok = issue_pv(j);
+        if (ok && j + 2 < n_keys) ok = issue_qk(j + 2);
       }
-      if (ok) issue_pv(n_keys - 1);
       // Every MMA issued above must finish before tensor memory is freed.
       umma_commit(&bars->drain);
       mbar_drain(&bars->drain, 0);
@@ -476,194 +475,184 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    // Thread (half, r) owns keys [half*HC, half*HC + HC) of every block for row
-    // r: its own running maximum m and sum l, and its own accumulator
-    // O_half = sum over its keys of P V, which the PV MMA writes to a separate
-    // tensor-memory region. The two halves never wait on each other inside the
-    // loop; the epilogue merges them as two partial softmaxes:
-    //   O = (a0 O_0 + a1 O_1) / (a0 l0 + a1 l1),  a_h = 2^(m_h - max(m0, m1)).
-    constexpr int HC = BN / 2;                        // S columns per thread
-    const int half = warp >> 2;
+    // Group grp = warp / 4 takes the key blocks j with j % 2 == grp; thread r
+    // of a group owns row r of those blocks: its own running maximum m, sum
+    // l and accumulator O_grp. The two groups work on different blocks at the
+    // same time, so one group's loads, reductions and barrier waits overlap
+    // the other's exponentials. The epilogue merges the two partial softmaxes:
+    //   O = (a0 O_0 + a1 O_1) / (a0 l0 + a1 l1),  a_g = 2^(m_g - max(m0, m1)).
+    // A row is processed 64 columns at a time (registers hold one chunk): the
+    // maximum over every chunk first, then exp2 chunk by chunk from the last,
+    // which is still in registers, reloading the others from tensor memory.
+    constexpr int kChunks = BN / 64;
+    const int grp = warp >> 2;
     const int r = (warp & 3) * 32 + lane;             // row == tensor-memory lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tOh = tO + half * D + lane_off;    // this half's accumulator
+    const uint32_t tSg = tS[grp] + lane_off;
+    const uint32_t tOg = tO + grp * D + lane_off;
     const float scale = p.scale_log2;
     float m = -INFINITY;                              // reference maximum, log2 units
-    float l = 0.f;                                    // sum of P over this half's keys
-    float s[HC];
+    float l = 0.f;                                    // sum of P over this group's blocks
+    float s[64];
     bool ok = true;
-    // key block of the next iteration, loaded one iteration ahead
-    int kb_next = (!kGather && n_keys > 0) ? cols[0] : 0;
-    for (int j = 0; j < n_keys; ++j) {
-      const int sb = j & 1;
-      uint32_t pw[HC / 32];
+    // key block of this group's next block, loaded one block ahead
+    int kb_next = (!kGather && grp < n_keys) ? cols[grp] : 0;
+    for (int j = grp; j < n_keys; j += 2) {
+      const uint32_t par = (uint32_t)(j >> 1) & 1u;
+      uint32_t pw[BN / 32];
       bool pad = true;
       if constexpr (kGather) {
-        // this row's group-membership bits for its half of the chunk's keys
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars->m_full[sb], (j >> 1) & 1, abort, status,
+        // this row's group-membership bits for the chunk's keys
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->m_full[grp], par, abort, status,
                                                site(3, 11, j)))) {
           ok = false;
           break;
         }
 #pragma unroll
-        for (int w = 0; w < HC / 32; ++w)
-          pw[w] = bars->masks[sb][(r < 64 ? 0 : 4) + half * (HC / 32) + w];
+        for (int w = 0; w < BN / 32; ++w) pw[w] = bars->masks[grp][(r < 64 ? 0 : 4) + w];
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->m_empty[sb]);
+        if (lane == 0) mbar_arrive(&bars->m_empty[grp]);
       } else {
         const int kb = kb_next;
-        if (j + 1 < n_keys) kb_next = cols[j + 1];
-        uint32_t full[BN / 32];
-        pad = block_pad_mask<BN>(g, kb, p.T, p.H, p.W, full);
-#pragma unroll
-        for (int w = 0; w < HC / 32; ++w) pw[w] = full[half * (HC / 32) + w];
+        if (j + 2 < n_keys) kb_next = cols[j + 2];
+        pad = block_pad_mask<BN>(g, kb, p.T, p.H, p.W, pw);
       }
       // a warp either waits out a barrier together or gives up together
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (j >> 1) & 1, abort, status,
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[grp], par, abort, status,
                                              site(3, 8, j)))) {
         ok = false;
         break;
       }
       tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < HC; c += 32) tmem_ld32(tS[sb] + lane_off + half * HC + c, s + c);
-      tmem_wait_ld();
-
-      // maximum over this half's keys: three-input max, four independent chains
+      // row maximum: three-input max, four independent chains
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (pad) {
 #pragma unroll
-        for (int c = 0; c < HC; ++c) s[c] = ((pw[c / 32] >> (c % 32)) & 1u) ? s[c] : -INFINITY;
-      }
+      for (int ch = 0; ch < kChunks; ++ch) {
+        tmem_ld32(tSg + ch * 64, s);
+        tmem_ld32(tSg + ch * 64 + 32, s + 32);
+        tmem_wait_ld();
+        if (pad) {
 #pragma unroll
-      for (int c = 0; c < HC; c += 8) {
-        mx4[0] = fmax3(mx4[0], s[c], s[c + 1]);
-        mx4[1] = fmax3(mx4[1], s[c + 2], s[c + 3]);
-        mx4[2] = fmax3(mx4[2], s[c + 4], s[c + 5]);
-        mx4[3] = fmax3(mx4[3], s[c + 6], s[c + 7]);
+          for (int c = 0; c < 64; ++c)
+            s[c] = ((pw[ch * 2 + c / 32] >> (c % 32)) & 1u) ? s[c] : -INFINITY;
+        }
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) {
+          mx4[0] = fmax3(mx4[0], s[c], s[c + 1]);
+          mx4[1] = fmax3(mx4[1], s[c + 2], s[c + 3]);
+          mx4[2] = fmax3(mx4[2], s[c + 4], s[c + 5]);
+          mx4[3] = fmax3(mx4[3], s[c + 6], s[c + 7]);
+        }
       }
       const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
       const float m_new = fmaxf(m, mx * scale);
       const bool rescale = (m == -INFINITY) || (m_new > m + kRescaleThreshold);
       const float m_use = rescale ? m_new : m;
-      float rs = 0.f;
-      if (m_use == -INFINITY) {
+      const float neg = -m_use;
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < HC; ++c) s[c] = 0.f;
-      } else {
-        // exp2 of every kPolyEvery-th column on the FMA pipe, the rest on MUFU;
-        // four independent partial sums
-        const float neg = -m_use;
-        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int ch = kChunks - 1; ch >= 0; --ch) {
+        if (ch != kChunks - 1) {
+          tmem_ld32(tSg + ch * 64, s);
+          tmem_ld32(tSg + ch * 64 + 32, s + 32);
+          tmem_wait_ld();
+          if (pad) {
 #pragma unroll
-        for (int c = 0; c < HC; ++c) {
-          const float x = fmaf(s[c], scale, neg);
-          s[c] = (kPolyEvery > 0 && c % kPolyEvery == kPolyEvery - 1) ? exp2_poly(x) : ex2_approx(x);
-          rs4[c & 3] += s[c];
+            for (int c = 0; c < 64; ++c)
+              s[c] = ((pw[ch * 2 + c / 32] >> (c % 32)) & 1u) ? s[c] : -INFINITY;
+          }
         }
-        if (kPolyEvery > 0 && pad) {
-          // masked keys: exactly zero. ex2.approx(-inf) is already +0; only
-          // the polynomial (which floors at 2^-125) needs this.
+        if (m_use == -INFINITY) {
 #pragma unroll
-          for (int c = 0; c < HC; ++c)
-            if (!((pw[c / 32] >> (c % 32)) & 1u)) { rs4[c & 3] -= s[c]; s[c] = 0.f; }
+          for (int c = 0; c < 64; ++c) s[c] = 0.f;
+        } else {
+          // exp2 of every kPolyEvery-th column on the FMA pipe, the rest on
+          // MUFU; masked keys (-inf) give exactly +0 on MUFU
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const float x = fmaf(s[c], scale, neg);
+            s[c] = (kPolyEvery > 0 && c % kPolyEvery == kPolyEvery - 1) ? exp2_poly(x) : ex2_approx(x);
+            if (kPolyEvery > 0 && pad && !((pw[ch * 2 + c / 32] >> (c % 32)) & 1u)) s[c] = 0.f;
+            rs4[c & 3] += s[c];
+          }
         }
-        rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+        // P as packed bf16 pairs over the first 32 of the chunk's own 64 S
+        // columns (the A operand of the PV MMA is read from tensor memory);
+        // packed in place: entry c only reads entries 2c and 2c+1
+#pragma unroll
+        for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(pack_bf16x2(s[2 * c], s[2 * c + 1]));
+        tmem_st32(tSg + ch * 64, s);
       }
-      // O_half is accumulated by PV of the previous block, so a rescale waits
-      // for it; without one nothing here touches O and no wait is needed.
-      // The wait is unambiguous by parity: S_j was committed after PV_{j-2}
-      // was issued, so PV_{j-2} is complete and o_done is at most one phase
-      // behind PV_{j-1}. tcgen05.ld/st are warp-collective, so the whole warp
+      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      // O_grp holds blocks up to j - 2, all complete (S_j was committed after
+      // PV_{j-2}), and PV_j waits for this group's arrival below: a rescale
+      // needs no wait. tcgen05.ld/st are warp-collective, so the whole warp
       // rescales when any of its rows needs it; rows that do not scale by 1.
-      if (j >= 1) {
-        const bool need = rescale && m != -INFINITY;
-        if (__any_sync(0xffffffffu, need)) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_done, (j - 1) & 1, abort, status,
-                                                 site(3, 9, j)))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const float alpha = need ? ex2_approx(m - m_use) : 1.f;
-          l *= alpha;
-          float o[32];
+      const bool need = rescale && m != -INFINITY;
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha = need ? ex2_approx(m - m_use) : 1.f;
+        l *= alpha;
+        float o[32];
 #pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            tmem_ld32(tOh + c, o);
-            tmem_wait_ld();
+        for (int c = 0; c < D; c += 32) {
+          tmem_ld32(tOg + c, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(tOh + c, o);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) o[e] *= alpha;
+          tmem_st32(tOg + c, o);
         }
       }
       m = m_use;
       l += rs;
-      // P as packed bf16 pairs over the first HC/2 of this half's own S
-      // columns (the A operand of the PV MMA is read from tensor memory). The
-      // other half never reads these columns, so no ordering between the two
-      // halves is needed. Packed in place: entry c only reads entries 2c and
-      // 2c+1, not yet overwritten.
-#pragma unroll
-      for (int c = 0; c < HC / 2; ++c) s[c] = __uint_as_float(pack_bf16x2(s[2 * c], s[2 * c + 1]));
-      if constexpr (HC / 2 >= 32) {
-#pragma unroll
-        for (int c = 0; c < HC / 2; c += 32) tmem_st32(tS[sb] + lane_off + half * HC + c, s + c);
-      } else {
-        tmem_st16(tS[sb] + lane_off + half * HC, s);
-      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[sb]);
+      if (lane == 0) mbar_arrive(&bars->p_full[grp]);
     }
     // ------------------------------------------------------------ epilogue
     // Once ``drain`` completes every MMA of the CTA has completed, so the Q
-    // tile is free: the two halves of each row trade (m, l) through it.
+    // tile is free: the two groups trade (m, l) of each row through it.
     if (ok && n_keys > 0) {
       // the MMA warp commits ``drain`` after its last PV
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->drain, 0, abort, status, site(3, 10, n_keys)));
       tc_fence_after();
     }
-    float* xch = reinterpret_cast<float*>(sQ);        // [half][m, l][128 rows]
-    xch[(half * 2 + 0) * 128 + r] = m;
-    xch[(half * 2 + 1) * 128 + r] = l;
+    float* xch = reinterpret_cast<float*>(sQ);        // [group][m, l][128 rows]
+    xch[(grp * 2 + 0) * 128 + r] = m;
+    xch[(grp * 2 + 1) * 128 + r] = l;
     named_barrier_sync(1, kSoftmaxWarps * 32);
-    const float m_o = xch[((half ^ 1) * 2 + 0) * 128 + r];
-    const float l_o = xch[((half ^ 1) * 2 + 1) * 128 + r];
+    const float m_o = xch[((grp ^ 1) * 2 + 0) * 128 + r];
+    const float l_o = xch[((grp ^ 1) * 2 + 1) * 128 + r];
     const int tok = (r < BN) ? slot_to_token(g, qb, r, BN, p.T, p.H, p.W) : -1;
     if (ok) {
-      // half 0 holds (m0, l0); the other half's values came through shared memory
-      const float m0 = half == 0 ? m : m_o, l0 = half == 0 ? l : l_o;
-      const float m1 = half == 0 ? m_o : m, l1 = half == 0 ? l_o : l;
+      const float m0 = grp == 0 ? m : m_o, l0 = grp == 0 ? l : l_o;
+      const float m1 = grp == 0 ? m_o : m, l1 = grp == 0 ? l_o : l;
       const float mm = fmaxf(m0, m1);
+      // a group with no block (or only masked keys) has m = -inf and an O
+      // that was never written: weight 0, and its O is not read
       const float a0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mm);
       const float a1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mm);
       const float l_tot = a0 * l0 + a1 * l1;
       const float inv_l = (n_keys > 0 && l_tot > 0.f) ? 1.f / l_tot : 0.f;
       const float w0 = a0 * inv_l, w1 = a1 * inv_l;
-      // this thread writes output columns [half*D/2, half*D/2 + D/2)
+      const bool use0 = n_keys > 0 && w0 != 0.f, use1 = n_keys > 1 && w1 != 0.f;
+      // this thread writes output columns [grp*D/2, grp*D/2 + D/2)
       constexpr int HD = D / 2;
-      __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (tok < 0 ? 0 : tok)) * D + half * HD;
+      __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (tok < 0 ? 0 : tok)) * D + grp * HD;
 #pragma unroll
       for (int c = 0; c < HD; c += 16) {
         float o0[16], o1[16];
-        if (n_keys > 0) {
-          tmem_ld16(tO + lane_off + half * HD + c, o0);
-          tmem_ld16(tO + D + lane_off + half * HD + c, o1);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) { o0[e] = 0.f; o1[e] = 0.f; }
-        }
+        // tcgen05.ld is warp-collective: load whenever any lane needs it
+        if (__any_sync(0xffffffffu, use0)) tmem_ld16(tO + lane_off + grp * HD + c, o0);
+        if (__any_sync(0xffffffffu, use1)) tmem_ld16(tO + D + lane_off + grp * HD + c, o1);
+        tmem_wait_ld();
         if (tok >= 0) {
 #pragma unroll
           for (int e = 0; e < 16; e += 8) {
             float v[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = fmaf(o0[e + u], w0, o1[e + u] * w1);
+            for (int u = 0; u < 8; ++u)
+              v[u] = (use0 ? o0[e + u] * w0 : 0.f) + (use1 ? o1[e + u] * w1 : 0.f);
             uint4 w;
             w.x = pack_bf16x2(v[0], v[1]);
             w.y = pack_bf16x2(v[2], v[3]);
@@ -673,7 +662,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
           }
         }
       }
-      if (tok >= 0 && half == 0 && p.lse)
+      if (tok >= 0 && grp == 0 && p.lse)
         p.lse[(size_t)bh * p.N + tok] =
             (n_keys > 0 && l_tot > 0.f) ? (mm + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
     }
