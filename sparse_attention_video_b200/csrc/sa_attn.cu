@@ -53,10 +53,9 @@ constexpr int kMmaWarp = 9;
 constexpr int kCopyWarp0 = 10;             // gather mode: warps 10-11 copy K/V rows
 constexpr int kStages = 3;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows > 2^8
-// One exp2 in kPolyEvery on the FMA pipe (0 = all on MUFU). Measured on the
-// 115,200-token workload, moving a quarter of them was slower (12.04 vs
-// 11.79 ms): the MUFU pipe is not what bounds this kernel.
-constexpr int kPolyEvery = 0;
+// Every exp2 runs on MUFU. Moving one in four (or eight) to the FMA-pipe
+// polynomial of sa_ptx.cuh was measured slower on the 115,200-token workload
+// (12.3 / 11.3 against 9.0 ms per call): issue slots, not MUFU, bound it.
 
 template <int D, int BN>
 struct Smem {
@@ -77,8 +76,8 @@ struct Smem {
 
 struct Bars {
   uint64_t q_full;
-  uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t k_full[kStages], v_full[kStages];
+  uint64_t kv_empty[kStages];       // stage free: PV of its block (hence its QK) completed
   uint64_t s_full[2];
   uint64_t p_full[2];               // P_j written into S buffer j & 1 (by group j & 1)
   uint64_t drain;
@@ -230,8 +229,8 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     // gather mode: K/V stages are filled by the two copy warps, not by TMA
     const uint32_t fill_arrivals = kGather ? 2u : 1u;
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->k_full[s], fill_arrivals); mbar_init(&bars->k_empty[s], 1);
-      mbar_init(&bars->v_full[s], fill_arrivals); mbar_init(&bars->v_empty[s], 1);
+      mbar_init(&bars->k_full[s], fill_arrivals); mbar_init(&bars->v_full[s], fill_arrivals);
+      mbar_init(&bars->kv_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) mbar_init(&bars->s_full[b], 1);
     for (int b = 0; b < 2; ++b) mbar_init(&bars->p_full[b], kSoftmaxWarps / 2);
@@ -326,13 +325,9 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         const int st = j % kStages, rnd = j / kStages;
         const int kb = cols[j];
         if (kb < 0 || kb >= g.nb) { atomicOr(status, SA_DEVFLAG_BOUNDS); *abort = 1; break; }
-        if (!mbar_wait(&bars->k_empty[st], (rnd & 1) ^ 1, abort, status, site(1, 1, j))) break;
+        if (!mbar_wait(&bars->kv_empty[st], (rnd & 1) ^ 1, abort, status, site(1, 1, j))) break;
         mbar_arrive_expect_tx(&bars->k_full[st], L::kKVBytes);
         load_block<D, BN>(kmaps, g, bh, kb, sK + st * L::kKVBytes, &bars->k_full[st]);
-        if (!mbar_wait(&bars->v_empty[st], (rnd & 1) ^ 1, abort, status, site(1, 2, j))) {
-          issued = j * 2 + 1;
-          break;
-        }
         mbar_arrive_expect_tx(&bars->v_full[st], L::kKVBytes);
         load_block<D, BN>(vmaps, g, bh, kb, sV + st * L::kKVBytes, &bars->v_full[st]);
         issued = j * 2 + 2;
@@ -375,7 +370,6 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         for (int kk = 0; kk < D / 16; ++kk)
           umma_bf16_ss(tS[j & 1], da[kk], db[kk], idesc_qk, kk > 0 ? 1u : 0u);
         umma_commit(&bars->s_full[j & 1]);
-        umma_commit(&bars->k_empty[st]);
         return true;
       };
       // PV_j: O_{j&1} += P_j V_j, P_j read from S buffer j & 1.
@@ -399,7 +393,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
           umma_bf16_ts(tO + (i & 1) * D, tS[i & 1] + (kk / 4) * 64 + (kk % 4) * 8, db[kk],
                        idesc_pv, (i > 1 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&bars->v_empty[i % kStages]);
+        umma_commit(&bars->kv_empty[i % kStages]);
         return true;
       };
       // Order: QK_0, QK_1, then PV_j, QK_{j+2} for every j. S buffer j & 1
@@ -435,10 +429,8 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         const uint32_t idx = (uint32_t)j * BN + t + 64 * i;
         key[i] = idx < list_count ? (int)(__ldg(list + idx) & 0x3FFFFFFFu) : 0;
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->k_empty[st], (rnd & 1) ^ 1, abort, status,
-                                             site(4, 1, j))) ||
-          !__all_sync(0xffffffffu, mbar_wait(&bars->v_empty[st], (rnd & 1) ^ 1, abort, status,
-                                             site(4, 2, j)))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_empty[st], (rnd & 1) ^ 1, abort, status,
+                                             site(4, 1, j)))) {
         okc = false;
         break;
       }
@@ -508,10 +500,8 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
           ok = false;
           break;
         }
-#pragma unroll
-        for (int w = 0; w < BN / 32; ++w) pw[w] = bars->masks[grp][(r < 64 ? 0 : 4) + w];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->m_empty[grp]);
+        // the words stay in shared memory until this block is done (they are
+        // read chunk by chunk below; m_empty is signalled after the block)
       } else {
         const int kb = kb_next;
         if (j + 2 < n_keys) kb_next = cols[j + 2];
@@ -524,18 +514,29 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         break;
       }
       tc_fence_after();
-      // row maximum: three-input max, four independent chains
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      // One pass over the row, 64 columns at a time: load, chunk maximum,
+      // exp2 against the running reference m, P back into tensor memory. The
+      // reference moves only when a chunk's maximum passes it by more than
+      // 2^8; then everything already summed against the old reference (l,
+      // this block's partial sum, this block's stored P chunks and O) is
+      // scaled by 2^(m_old - m_new). O holds blocks up to j - 2, all
+      // complete (S_j was committed after PV_{j-2}), and PV_j waits for this
+      // group's arrival below, so touching O needs no wait.
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int ch = 0; ch < kChunks; ++ch) {
         tmem_ld32(tSg + ch * 64, s);
         tmem_ld32(tSg + ch * 64 + 32, s + 32);
         tmem_wait_ld();
         if (pad) {
+          uint32_t w2[2];
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            s[c] = ((pw[ch * 2 + c / 32] >> (c % 32)) & 1u) ? s[c] : -INFINITY;
+          for (int w = 0; w < 2; ++w)
+            w2[w] = kGather ? bars->masks[grp][(r < 64 ? 0 : 4) + ch * 2 + w] : pw[ch * 2 + w];
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[c] = ((w2[c / 32] >> (c % 32)) & 1u) ? s[c] : -INFINITY;
         }
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < 64; c += 8) {
           mx4[0] = fmax3(mx4[0], s[c], s[c + 1]);
@@ -543,38 +544,58 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
           mx4[2] = fmax3(mx4[2], s[c + 4], s[c + 5]);
           mx4[3] = fmax3(mx4[3], s[c + 6], s[c + 7]);
         }
-      }
-      const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
-      const float m_new = fmaxf(m, mx * scale);
-      const bool rescale = (m == -INFINITY) || (m_new > m + kRescaleThreshold);
-      const float m_use = rescale ? m_new : m;
-      const float neg = -m_use;
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+        const float cm = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]) * scale;
+        // m = -inf and cm finite counts as moving (the first key of the row)
+        const bool move = cm > m + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, move)) {
+          // warp-collective tensor-memory traffic: lanes that keep their
+          // reference scale by 1
+          const bool had = move && m != -INFINITY;
+          const float alpha = had ? ex2_approx(m - cm) : 1.f;
+          l *= alpha;
 #pragma unroll
-      for (int ch = kChunks - 1; ch >= 0; --ch) {
-        if (ch != kChunks - 1) {
-          tmem_ld32(tSg + ch * 64, s);
-          tmem_ld32(tSg + ch * 64 + 32, s + 32);
-          tmem_wait_ld();
-          if (pad) {
+          for (int e = 0; e < 4; ++e) rs4[e] *= alpha;
+          if (__any_sync(0xffffffffu, had)) {
+            float o[32];
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-              s[c] = ((pw[ch * 2 + c / 32] >> (c % 32)) & 1u) ? s[c] : -INFINITY;
+            for (int c = 0; c < D; c += 32) {
+              tmem_ld32(tOg + c, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] *= alpha;
+              tmem_st32(tOg + c, o);
+            }
+#pragma unroll
+            for (int pc = 0; pc < ch; ++pc) {
+              // this block's P chunks stored so far: packed bf16 pairs
+              tmem_ld32(tSg + pc * 64, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const uint32_t b = __float_as_uint(o[e]);
+                o[e] = __uint_as_float(pack_bf16x2(__uint_as_float(b << 16) * alpha,
+                                                   __uint_as_float(b & 0xFFFF0000u) * alpha));
+              }
+              tmem_st32(tSg + pc * 64, o);
+            }
           }
+          if (move) m = cm;
         }
-        if (m_use == -INFINITY) {
+        // masked keys are -inf and give exactly +0 on MUFU; a row whose
+        // reference is still -inf has only masked keys so far. Scale and
+        // shift, and the partial sums, run two columns per instruction.
+        const float neg = m == -INFINITY ? 0.f : -m;
 #pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = 0.f;
-        } else {
-          // exp2 of every kPolyEvery-th column on the FMA pipe, the rest on
-          // MUFU; masked keys (-inf) give exactly +0 on MUFU
+        for (int c = 0; c < 64; c += 2) {
+          float x0, x1;
+          fma2(s[c], s[c + 1], scale, scale, neg, neg, x0, x1);
+          s[c] = ex2_approx(x0);
+          s[c + 1] = ex2_approx(x1);
+        }
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const float x = fmaf(s[c], scale, neg);
-            s[c] = (kPolyEvery > 0 && c % kPolyEvery == kPolyEvery - 1) ? exp2_poly(x) : ex2_approx(x);
-            if (kPolyEvery > 0 && pad && !((pw[ch * 2 + c / 32] >> (c % 32)) & 1u)) s[c] = 0.f;
-            rs4[c & 3] += s[c];
-          }
+        for (int c = 0; c < 64; c += 4) {
+          add2(rs4[0], rs4[1], s[c], s[c + 1]);
+          add2(rs4[2], rs4[3], s[c + 2], s[c + 3]);
         }
         // P as packed bf16 pairs over the first 32 of the chunk's own 64 S
         // columns (the A operand of the PV MMA is read from tensor memory);
@@ -583,27 +604,11 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(pack_bf16x2(s[2 * c], s[2 * c + 1]));
         tmem_st32(tSg + ch * 64, s);
       }
-      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-      // O_grp holds blocks up to j - 2, all complete (S_j was committed after
-      // PV_{j-2}), and PV_j waits for this group's arrival below: a rescale
-      // needs no wait. tcgen05.ld/st are warp-collective, so the whole warp
-      // rescales when any of its rows needs it; rows that do not scale by 1.
-      const bool need = rescale && m != -INFINITY;
-      if (__any_sync(0xffffffffu, need)) {
-        const float alpha = need ? ex2_approx(m - m_use) : 1.f;
-        l *= alpha;
-        float o[32];
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          tmem_ld32(tOg + c, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tmem_st32(tOg + c, o);
-        }
+      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      if constexpr (kGather) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->m_empty[grp]);
       }
-      m = m_use;
-      l += rs;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();

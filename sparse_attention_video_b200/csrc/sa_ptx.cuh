@@ -329,6 +329,26 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (n << 23));
 }
 
+// Two fp32 lanes per instruction (packed f32x2 FMA / add, sm_100): halves
+// the issue slots of elementwise softmax arithmetic.
+__device__ __forceinline__ void fma2(float a0, float a1, float b0, float b1, float c0, float c1,
+                                     float& d0, float& d1) {
+  unsigned long long A, B, C, Dd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(B) : "f"(b0), "f"(b1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(C) : "f"(c0), "f"(c1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(Dd) : "l"(A), "l"(B), "l"(C));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(Dd));
+}
+// (a0, a1) += (b0, b1)
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  unsigned long long A, B, Dd;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(B) : "f"(b0), "f"(b1));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(Dd) : "l"(A), "l"(B));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(Dd));
+}
+
 // max(a, b, c) in one instruction (three-input max.f32, sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
