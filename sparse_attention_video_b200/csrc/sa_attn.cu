@@ -412,39 +412,44 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     }
   } else if (kGather && warp >= kCopyWarp0) {
     // ------------------------------------------------------------ K/V row copies (gather)
-    // Thread t copies rows t and t+64 of every chunk: 16-byte cp.async pieces
-    // straight into the 128-byte-swizzled tiles the MMA reads. Chunk j is
-    // announced once chunk j+1 is in flight: wait for this thread's older
-    // group, make the generic-proxy writes visible to the tensor core's async
-    // proxy, then arrive.
-    const int t = (warp - kCopyWarp0) * 32 + lane;
-    const __nv_bfloat16* kbase = p.k_rows + (size_t)bh * p.N * D;
-    const __nv_bfloat16* vbase = p.v_rows + (size_t)bh * p.N * D;
+    // Copy warp cw fills rows 64cw..64cw+63 of every chunk with 16-byte
+    // cp.async pieces straight into the 128-byte-swizzled tiles the MMA
+    // reads. D/8 consecutive lanes copy one whole row (coalesced: a warp
+    // instruction moves 32/(D/8) full rows), the key index of each row comes
+    // by shuffle from the lane that loaded it. Chunk j is announced once
+    // chunk j+1 is in flight: wait for this thread's older group, make the
+    // generic-proxy writes visible to the tensor core's async proxy, arrive.
+    constexpr int kPieces = D / 8;                  // 16-byte pieces per row
+    constexpr int kRowsPerStep = 32 / kPieces;      // rows per warp instruction
+    const int cw = warp - kCopyWarp0;
+    const int piece = lane % kPieces, sub = lane / kPieces;
+    const __nv_bfloat16* kbase = p.k_rows + (size_t)bh * p.N * D + piece * 8;
+    const __nv_bfloat16* vbase = p.v_rows + (size_t)bh * p.N * D + piece * 8;
     bool okc = true;
     for (int j = 0; j < n_keys; ++j) {
       const int st = j % kStages, rnd = j / kStages;
-      int key[2];
+      // lane l holds the keys of rows 64cw + l and 64cw + 32 + l
+      int kl[2];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const uint32_t idx = (uint32_t)j * BN + t + 64 * i;
-        key[i] = idx < list_count ? (int)(__ldg(list + idx) & 0x3FFFFFFFu) : 0;
+        const uint32_t idx = (uint32_t)j * BN + 64 * cw + 32 * i + lane;
+        kl[i] = idx < list_count ? (int)(__ldg(list + idx) & 0x3FFFFFFFu) : 0;
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_empty[st], (rnd & 1) ^ 1, abort, status,
                                              site(4, 1, j)))) {
         okc = false;
         break;
       }
+      uint8_t* dk = sK + st * L::kKVBytes + (piece / 8) * (BN * 128);
+      uint8_t* dv = sV + st * L::kKVBytes + (piece / 8) * (BN * 128);
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int r = t + 64 * i;
-        const __nv_bfloat16* ks = kbase + (size_t)key[i] * D;
-        const __nv_bfloat16* vs = vbase + (size_t)key[i] * D;
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          const int off = (c / 8) * (BN * 128) + r * 128 + (((c % 8) ^ (r & 7)) << 4);
-          cp_async16(sK + st * L::kKVBytes + off, ks + c * 8);
-          cp_async16(sV + st * L::kKVBytes + off, vs + c * 8);
-        }
+      for (int i = 0; i < 64 / kRowsPerStep; ++i) {
+        const int rl = i * kRowsPerStep + sub;       // row within this warp's 64
+        const int key = __shfl_sync(0xffffffffu, kl[(i * kRowsPerStep) / 32], rl % 32);
+        const int r = 64 * cw + rl;
+        const int off = r * 128 + (((piece % 8) ^ (r & 7)) << 4);
+        cp_async16(dk + off, kbase + (size_t)key * D);
+        cp_async16(dv + off, vbase + (size_t)key * D);
       }
       cp_async_commit();
       if (j >= 1) {
@@ -473,9 +478,6 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     // same time, so one group's loads, reductions and barrier waits overlap
     // the other's exponentials. The epilogue merges the two partial softmaxes:
     //   O = (a0 O_0 + a1 O_1) / (a0 l0 + a1 l1),  a_g = 2^(m_g - max(m0, m1)).
-    // A row is processed 64 columns at a time (registers hold one chunk): the
-    // maximum over every chunk first, then exp2 chunk by chunk from the last,
-    // which is still in registers, reloading the others from tensor memory.
     constexpr int kChunks = BN / 64;
     const int grp = warp >> 2;
     const int r = (warp & 3) * 32 + lane;             // row == tensor-memory lane
