@@ -36,10 +36,13 @@ constexpr int kScoreThreads = 640;   // warps 4-19: epilogue, four per key lane 
 constexpr int kEpiParts = 4;         // group columns split into 128 / kEpiParts per warp
 constexpr int kKeyTilesPerCta = 64;      // 8192 keys per CTA
 constexpr int kBins = 4096;
+constexpr int kAcc = 4;              // score tiles in tensor memory (128 columns each)
 
+// Unsigned key with the order of the floats: negative values have every bit
+// flipped, non-negative ones only the sign bit (two instructions).
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
 }
 __device__ __forceinline__ float key_to_float(uint32_t k) {
   const uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
@@ -85,7 +88,7 @@ struct ScoreSmem {
 struct ScoreBars {
   uint64_t q_full;
   uint64_t k_full[2], k_empty[2];
-  uint64_t acc_full[2], acc_free[2];
+  uint64_t acc_full[kAcc], acc_free[kAcc];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -116,8 +119,8 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->k_full[i], 1); mbar_init(&bars->k_empty[i], 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(&bars->k_full[i], 1); mbar_init(&bars->k_empty[i], 1); }
+    for (int i = 0; i < kAcc; ++i) {
       mbar_init(&bars->acc_full[i], 1); mbar_init(&bars->acc_free[i], 4 * kEpiParts);
     }
     mbar_init(&bars->drain, 1);
@@ -128,7 +131,7 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
     for (int i = threadIdx.x; i < 4 * kBins; i += kScoreThreads) hist[i] = 0u;
   if (warp == 1) {
     __syncwarp();
-    tmem_alloc(&bars->tmem_base, 256);
+    tmem_alloc(&bars->tmem_base, 128 * kAcc);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -162,26 +165,35 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc_bf16(128, 128, false, false);
-      const uint32_t aK = smem_u32(sK), aQ = smem_u32(sQ);
-      bool ok = mbar_wait(&bars->q_full, 0, abort, status, 0x05050000u);
+      // Descriptors formed once: the q_avg terms' are fixed, a K stage's
+      // differ from stage 0's by a constant; each MMA adds a compile-time
+      // offset, so the issuing thread spends its time issuing.
+      const uint64_t dK0 = umma_desc_sw128(smem_u32(sK), 16, 1024);
+      uint64_t dq[3][D / 16];
+#pragma unroll
+      for (int t = 0; t < 3; ++t)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          dq[t][kk] = umma_desc_sw128(smem_u32(sQ) + t * L::kTerm + (kk / 4) * 16384 + (kk % 4) * 32,
+                                      16, 1024);
+      bool ok = mbar_wait<false>(&bars->q_full, 0, abort, status, 0x05050000u);
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int st = j & 1, ab = j & 1;
-        if (!mbar_wait(&bars->k_full[st], (j >> 1) & 1, abort, status, 0x05060000u | j)) break;
-        if (j >= 2 && !mbar_wait(&bars->acc_free[ab], ((j - 2) >> 1) & 1, abort, status, 0x05070000u | j))
+        const int st = j & 1, ab = j % kAcc;
+        if (!mbar_wait<false>(&bars->k_full[st], (j >> 1) & 1, abort, status, 0x05060000u | j)) break;
+        if (j >= kAcc && !mbar_wait<false>(&bars->acc_free[ab], ((j / kAcc) - 1) & 1, abort, status,
+                                        0x05070000u | j))
           break;
+        const uint64_t dk = umma_desc_advance(dK0, st * L::kKTile);
+        uint64_t da[D / 16];
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) da[kk] = umma_desc_advance(dk, (kk / 4) * 16384 + (kk % 4) * 32);
         tc_fence_after();
         const uint32_t d_tmem = tmem + ab * 128;
-        int first = 1;
-        for (int t = 0; t < 3; ++t) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-            const uint64_t da = umma_desc_sw128(aK + st * L::kKTile + off, 16, 1024);
-            const uint64_t db = umma_desc_sw128(aQ + t * L::kTerm + off, 16, 1024);
-            umma_bf16_ss(d_tmem, da, db, idesc, first ? 0u : 1u);
-            first = 0;
-          }
-        }
+        for (int t = 0; t < 3; ++t)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_bf16_ss(d_tmem, da[kk], dq[t][kk], idesc, (t > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&bars->acc_full[ab]);
         umma_commit(&bars->k_empty[st]);
       }
@@ -201,8 +213,8 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
     const int g_base = gt * 128;
     const int g_lim = min(128, p.G - g_base);
     for (int j = 0; j < n_tiles; ++j) {
-      const int ab = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->acc_full[ab], (j >> 1) & 1, abort, status,
+      const int ab = j % kAcc;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->acc_full[ab], (j / kAcc) & 1, abort, status,
                                              0x06080000u | j)))
         break;
       tc_fence_after();
@@ -217,18 +229,27 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         float v[32];
         tmem_ld32(tmem + ab * 128 + lane_off + c0, v);
         tmem_wait_ld();
+        // all 32 columns real (the usual case): no per-score bounds tests
+        const int n_ok = kvalid ? min(32, g_lim - c0) : 0;
         if (p.mode == FG_MODE_HIST) {
+          if (n_ok == 32) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if (!kvalid || c0 + e >= g_lim) continue;
-            const uint32_t kk = order_key(v[e]);
-            if ((kk & p.match_mask) != prefix) continue;
-            atomicAdd(&whist[(kk >> p.bin_shift) & p.bin_mask], 1u);
+            for (int e = 0; e < 32; ++e) {
+              const uint32_t kk = order_key(v[e]);
+              if ((kk & p.match_mask) == prefix) atomicAdd(&whist[(kk >> p.bin_shift) & p.bin_mask], 1u);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const uint32_t kk = order_key(v[e]);
+              if (e < n_ok && (kk & p.match_mask) == prefix)
+                atomicAdd(&whist[(kk >> p.bin_shift) & p.bin_mask], 1u);
+            }
           }
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const bool keep = kvalid && (c0 + e < g_lim) && order_key(v[e]) >= tau_key;
+            const bool keep = e < n_ok && order_key(v[e]) >= tau_key;
             const uint32_t ballot = __ballot_sync(0xffffffffu, keep);
             if (lane == e) words[cc / 32] = ballot;
           }
@@ -261,7 +282,7 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 128 * kAcc);
   }
 }
 
