@@ -416,16 +416,15 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     // cp.async pieces straight into the 128-byte-swizzled tiles the MMA
     // reads. D/8 consecutive lanes copy one whole row (coalesced: a warp
     // instruction moves 32/(D/8) full rows), the key index of each row comes
-    // by shuffle from the lane that loaded it. Chunk j is announced once
-    // chunk j+1 is in flight: wait for this thread's older group, make the
-    // generic-proxy writes visible to the tensor core's async proxy, arrive.
+    // by shuffle from the lane that loaded it. Before each announcement the
+    // warp waits for its own copies and makes the generic-proxy writes
+    // visible to the tensor core's async proxy.
     constexpr int kPieces = D / 8;                  // 16-byte pieces per row
     constexpr int kRowsPerStep = 32 / kPieces;      // rows per warp instruction
     const int cw = warp - kCopyWarp0;
     const int piece = lane % kPieces, sub = lane / kPieces;
     const __nv_bfloat16* kbase = p.k_rows + (size_t)bh * p.N * D + piece * 8;
     const __nv_bfloat16* vbase = p.v_rows + (size_t)bh * p.N * D + piece * 8;
-    bool okc = true;
     for (int j = 0; j < n_keys; ++j) {
       const int st = j % kStages, rnd = j / kStages;
       // lane l holds the keys of rows 64cw + l and 64cw + 32 + l
@@ -437,39 +436,40 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_empty[st], (rnd & 1) ^ 1, abort, status,
                                              site(4, 1, j)))) {
-        okc = false;
         break;
       }
       uint8_t* dk = sK + st * L::kKVBytes + (piece / 8) * (BN * 128);
       uint8_t* dv = sV + st * L::kKVBytes + (piece / 8) * (BN * 128);
+      // K first, then V, as two cp.async groups: QK_j needs only K_j, so K is
+      // announced as soon as it has landed; V follows.
+      int keys[64 / kRowsPerStep];
 #pragma unroll
       for (int i = 0; i < 64 / kRowsPerStep; ++i) {
         const int rl = i * kRowsPerStep + sub;       // row within this warp's 64
-        const int key = __shfl_sync(0xffffffffu, kl[(i * kRowsPerStep) / 32], rl % 32);
+        keys[i] = __shfl_sync(0xffffffffu, kl[(i * kRowsPerStep) / 32], rl % 32);
         const int r = 64 * cw + rl;
-        const int off = r * 128 + (((piece % 8) ^ (r & 7)) << 4);
-        cp_async16(dk + off, kbase + (size_t)key * D);
-        cp_async16(dv + off, vbase + (size_t)key * D);
+        cp_async16(dk + r * 128 + (((piece % 8) ^ (r & 7)) << 4), kbase + (size_t)keys[i] * D);
       }
       cp_async_commit();
-      if (j >= 1) {
-        cp_async_wait<1>();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bars->k_full[(j - 1) % kStages]);
-          mbar_arrive(&bars->v_full[(j - 1) % kStages]);
-        }
+#pragma unroll
+      for (int i = 0; i < 64 / kRowsPerStep; ++i) {
+        const int r = 64 * cw + i * kRowsPerStep + sub;
+        cp_async16(dv + r * 128 + (((piece % 8) ^ (r & 7)) << 4), vbase + (size_t)keys[i] * D);
       }
+      cp_async_commit();
+      cp_async_wait<1>();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->k_full[st]);
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->v_full[st]);
     }
     // own copies land before anything else (also on the abort path)
     cp_async_wait<0>();
     fence_proxy_async_smem();
     __syncwarp();
-    if (okc && n_keys > 0 && lane == 0) {
-      mbar_arrive(&bars->k_full[(n_keys - 1) % kStages]);
-      mbar_arrive(&bars->v_full[(n_keys - 1) % kStages]);
-    }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     // Group grp = warp / 4 takes the key blocks j with j % 2 == grp; thread r
