@@ -175,6 +175,7 @@ ScratchLayout scratch_layout(const sa_problem& pr, const sa_policy& po, const Ma
     S.off_fg_qsplit = take(fg_qsplit_bytes(M.BH, M.G, d));
     S.off_fg_hist = take(fg_hist_bytes(M.BH));
     S.off_fg_sel = take(fg_sel_bytes(M.BH));
+    S.off_fg_cand = take(fg_cand_bytes(M.BH));
   }
   S.total = off;
   return S;
@@ -306,6 +307,9 @@ extern "C" int sparse_attn_build_mask(const sa_problem* problem, const sa_policy
     fp.qsplit = reinterpret_cast<__nv_bfloat16*>(sw + S.off_fg_qsplit);
     fp.hist = reinterpret_cast<uint32_t*>(sw + S.off_fg_hist);
     fp.sel = reinterpret_cast<uint32_t*>(sw + S.off_fg_sel);
+    fp.cand = reinterpret_cast<uint2*>(sw + S.off_fg_cand);
+    fp.cand_count = reinterpret_cast<uint32_t*>(sw + S.off_fg_cand + sizeof(uint2) * (size_t)M.BH * kFgCandCap);
+    fp.fallback = fp.cand_count + M.BH;
     fp.bits = reinterpret_cast<uint32_t*>(mw + M.off_fg_bits);
     fp.tau = reinterpret_cast<float*>(mw + M.off_fg_tau);
     fp.status = reinterpret_cast<uint32_t*>(sw + S.off_status);

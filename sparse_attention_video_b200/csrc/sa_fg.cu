@@ -37,6 +37,8 @@ constexpr int kEpiParts = 4;         // group columns split into 128 / kEpiParts
 constexpr int kKeyTilesPerCta = 64;      // 8192 keys per CTA
 constexpr int kBins = 4096;
 constexpr int kAcc = 4;              // score tiles in tensor memory (128 columns each)
+constexpr int kKStages = 3;          // key tiles in flight
+constexpr int kHists = 2;            // shared-memory histogram copies (two lane quarters each)
 
 // Unsigned key with the order of the floats: negative values have every bit
 // flipped, non-negative ones only the sign bit (two instructions).
@@ -80,14 +82,14 @@ struct ScoreSmem {
   static constexpr int kKTile = kHalves * 128 * 128;          // 128 keys
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = 3 * kTerm;
-  static constexpr int kOffHist = kOffK + 2 * kKTile;
-  static constexpr int kOffBar = kOffHist + 4 * kBins * 4;
+  static constexpr int kOffHist = kOffK + kKStages * kKTile;
+  static constexpr int kOffBar = kOffHist + kHists * kBins * 4;
   static constexpr int kAlloc = kOffBar + 256 + 1024;
 };
 
 struct ScoreBars {
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2];
+  uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t acc_full[kAcc], acc_free[kAcc];
   uint64_t drain;
   uint32_t tmem_base;
@@ -112,14 +114,25 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   const int tile0 = chunk * kKeyTilesPerCta;
   const int n_tiles = min(kKeyTilesPerCta, n_tiles_total - tile0);
   if (n_tiles <= 0 || grid_aborted(p.status)) return;
+  if (p.only_heads && p.only_heads[bh] == 0u) return;     // uniform across the CTA
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   // Selection state of this head (HIST level > 0 and BITS read the prefix).
-  const uint32_t prefix = p.mode == FG_MODE_BITS ? 0u : p.sel[bh * 4 + 0];
+  const uint32_t prefix = p.mode == FG_MODE_HIST ? p.sel[bh * 4 + 0] : 0u;
   const uint32_t tau_key = p.sel[bh * 4 + 0];
+  // Bitmask thresholds as floats: the order key is monotonic in the float
+  // value, so key >= t  <=>  value >= key_to_float(t) (zeros aside: -0 and
+  // +0 compare equal as floats, which only matters when the threshold is a
+  // zero, a tie either way).
+  // BITS: keep >= tau. BITS_COLLECT: keep >= the first key above the 24-bit
+  // prefix bin, list the scores inside the bin.
+  const float f_tau = key_to_float(tau_key);
+  const uint32_t hi24 = tau_key >> 8;
+  const float f_bin_lo = key_to_float(hi24 << 8);
+  const float f_bin_hi = hi24 >= 0xFFFFFFu ? INFINITY : key_to_float((hi24 + 1u) << 8);
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int i = 0; i < 2; ++i) { mbar_init(&bars->k_full[i], 1); mbar_init(&bars->k_empty[i], 1); }
+    for (int i = 0; i < kKStages; ++i) { mbar_init(&bars->k_full[i], 1); mbar_init(&bars->k_empty[i], 1); }
     for (int i = 0; i < kAcc; ++i) {
       mbar_init(&bars->acc_full[i], 1); mbar_init(&bars->acc_free[i], 4 * kEpiParts);
     }
@@ -128,7 +141,7 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
     fence_barrier_init();
   }
   if (p.mode == FG_MODE_HIST)
-    for (int i = threadIdx.x; i < 4 * kBins; i += kScoreThreads) hist[i] = 0u;
+    for (int i = threadIdx.x; i < kHists * kBins; i += kScoreThreads) hist[i] = 0u;
   if (warp == 1) {
     __syncwarp();
     tmem_alloc(&bars->tmem_base, 128 * kAcc);
@@ -151,8 +164,9 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
                       t * p.BH + bh);
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait(&bars->k_empty[st], ((j >> 1) & 1) ^ 1, abort, status, 0x04010000u | j)) break;
+        const int st = j % kKStages;
+        if (!mbar_wait(&bars->k_empty[st], ((j / kKStages) & 1) ^ 1, abort, status, 0x04010000u | j))
+          break;
         mbar_arrive_expect_tx(&bars->k_full[st], L::kKTile);
         for (int h = 0; h < L::kHalves; ++h)
           tma_load_3d(sK + st * L::kKTile + h * 16384, &kmap, &bars->k_full[st], h * 64,
@@ -160,7 +174,8 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         issued = j + 1;
       }
       if (*abort)
-        for (int j = max(0, issued - 2); j < issued; ++j) mbar_drain(&bars->k_full[j & 1], (j >> 1) & 1);
+        for (int j = max(0, issued - kKStages); j < issued; ++j)
+          mbar_drain(&bars->k_full[j % kKStages], (j / kKStages) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -178,8 +193,9 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
                                       16, 1024);
       bool ok = mbar_wait<false>(&bars->q_full, 0, abort, status, 0x05050000u);
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int st = j & 1, ab = j % kAcc;
-        if (!mbar_wait<false>(&bars->k_full[st], (j >> 1) & 1, abort, status, 0x05060000u | j)) break;
+        const int st = j % kKStages, ab = j % kAcc;
+        if (!mbar_wait<false>(&bars->k_full[st], (j / kKStages) & 1, abort, status, 0x05060000u | j))
+          break;
         if (j >= kAcc && !mbar_wait<false>(&bars->acc_free[ab], ((j / kAcc) - 1) & 1, abort, status,
                                         0x05070000u | j))
           break;
@@ -203,13 +219,13 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   } else if (warp >= 4) {
     // ---------------------------------------------------------- epilogue
     // Warp w reads tensor-memory lanes 32*(w%4).. (its keys) and part
-    // (w-4)/4 of the 128 group columns; the warps of a lane quarter share one
-    // histogram.
+    // (w-4)/4 of the 128 group columns; the warps of lane quarters q and
+    // q + 2 share one histogram.
     constexpr int kCols = 128 / kEpiParts;
     const int quarter = warp & 3, half = (warp - 4) >> 2;
     const int r = 32 * quarter + lane;                 // key lane within the tile
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
-    uint32_t* whist = hist + quarter * kBins;
+    uint32_t* whist = hist + (quarter % kHists) * kBins;
     const int g_base = gt * 128;
     const int g_lim = min(128, p.G - g_base);
     for (int j = 0; j < n_tiles; ++j) {
@@ -247,18 +263,34 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
             }
           }
         } else {
+          const float f_keep = p.mode == FG_MODE_BITS ? f_tau : f_bin_hi;
+          bool any_cand = false;
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const bool keep = e < n_ok && order_key(v[e]) >= tau_key;
+            const bool ok_e = e < n_ok;
+            const bool keep = ok_e && v[e] >= f_keep;
             const uint32_t ballot = __ballot_sync(0xffffffffu, keep);
             if (lane == e) words[cc / 32] = ballot;
+            any_cand |= ok_e && v[e] >= f_bin_lo && !(v[e] >= f_keep);
+          }
+          if (p.mode == FG_MODE_BITS_COLLECT && __any_sync(0xffffffffu, any_cand)) {
+            // rare: scores that share their top 24 bits with the threshold
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (e < n_ok && v[e] >= f_bin_lo && !(v[e] >= f_keep)) {
+                const uint32_t pos = atomicAdd(p.cand_count + bh, 1u);
+                if (pos < kFgCandCap)
+                  p.cand[(size_t)bh * kFgCandCap + pos] = make_uint2(
+                      (uint32_t)key, ((uint32_t)(g_base + c0 + e) << 8) | (order_key(v[e]) & 0xFFu));
+              }
+            }
           }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->acc_free[ab]);
-      if (p.mode == FG_MODE_BITS) {
+      if (p.mode != FG_MODE_HIST) {
         // lane e holds this warp's 32 keys for groups half*kCols + 32*i + e
         const int kw = ((tile0 + j) * 128 + 32 * quarter) / 32;
 #pragma unroll
@@ -275,7 +307,9 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   if (p.mode == FG_MODE_HIST) {
     uint32_t* gh = p.hist + (size_t)bh * kBins;
     for (int b = threadIdx.x; b <= (int)p.bin_mask; b += kScoreThreads) {
-      const uint32_t c = hist[b] + hist[kBins + b] + hist[2 * kBins + b] + hist[3 * kBins + b];
+      uint32_t c = 0;
+#pragma unroll
+      for (int h = 0; h < kHists; ++h) c += hist[h * kBins + b];
       if (c) atomicAdd(&gh[b], c);
     }
   }
@@ -290,15 +324,21 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
 // sel[bh*4 + 0] prefix key so far, [1] rank left (1-based, counted from the
 // largest), [2] number of slices kept (after the final level: R plus ties is
 // only known after BITS; [2] holds R).
-__global__ void fg_select_init_kernel(uint32_t* sel, uint32_t* hist, int BH, uint32_t rank) {
+__global__ void fg_select_init_kernel(uint32_t* sel, uint32_t* hist, uint32_t* cand_count,
+                                      int BH, uint32_t rank) {
   const int bh = blockIdx.x;
-  if (threadIdx.x == 0) { sel[bh * 4 + 0] = 0u; sel[bh * 4 + 1] = rank; sel[bh * 4 + 2] = rank; }
+  if (threadIdx.x == 0) {
+    sel[bh * 4 + 0] = 0u; sel[bh * 4 + 1] = rank; sel[bh * 4 + 2] = rank;
+    cand_count[bh] = 0u;
+  }
   for (int b = threadIdx.x; b < kBins; b += blockDim.x) hist[(size_t)bh * kBins + b] = 0u;
 }
 
 __global__ void fg_select_kernel(uint32_t* sel, uint32_t* hist, int nbins, int shift,
-                                 float* tau, float inv_sqrt_d, int final_level) {
+                                 float* tau, float inv_sqrt_d, int final_level,
+                                 const uint32_t* only_heads) {
   const int bh = blockIdx.x;
+  if (only_heads && only_heads[bh] == 0u) return;
   __shared__ uint32_t counts[kBins];
   uint32_t* h = hist + (size_t)bh * kBins;
   for (int b = threadIdx.x; b < nbins; b += blockDim.x) { counts[b] = h[b]; h[b] = 0u; }
@@ -314,6 +354,50 @@ __global__ void fg_select_kernel(uint32_t* sel, uint32_t* hist, int nbins, int s
     sel[bh * 4 + 0] |= (uint32_t)b << shift;
     sel[bh * 4 + 1] = rank - acc;
     if (final_level) tau[bh] = key_to_float(sel[bh * 4 + 0]) * inv_sqrt_d;
+  }
+}
+
+// Last select level over the collected candidates (keys sharing the top 24
+// bits decided so far): histogram of their low 8 bits, the bin holding the
+// rank left is tau's low byte; candidates at or above it get their bit. A
+// head whose list overflowed is flagged for the full third level instead.
+__global__ void fg_fixup_kernel(uint32_t* sel, const uint2* cand, const uint32_t* cand_count,
+                                uint32_t* fallback, uint32_t* bits, float* tau, float inv_sqrt_d,
+                                int G, int WN) {
+  const int bh = blockIdx.x;
+  __shared__ uint32_t counts[256];
+  __shared__ uint32_t low;
+  const uint32_t n = cand_count[bh];
+  if (n > kFgCandCap) {
+    if (threadIdx.x == 0) fallback[bh] = 1u;
+    return;
+  }
+  for (int b = threadIdx.x; b < 256; b += blockDim.x) counts[b] = 0u;
+  __syncthreads();
+  const uint2* c = cand + (size_t)bh * kFgCandCap;
+  for (uint32_t i = threadIdx.x; i < n; i += blockDim.x) atomicAdd(&counts[c[i].y & 0xFFu], 1u);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    fallback[bh] = 0u;
+    const uint32_t rank = sel[bh * 4 + 1];
+    uint32_t acc = 0;
+    int b = 255;
+    for (; b > 0; --b) {                     // from the largest keys down
+      if (acc + counts[b] >= rank) break;
+      acc += counts[b];
+    }
+    low = (uint32_t)b;
+    sel[bh * 4 + 0] |= (uint32_t)b;
+    sel[bh * 4 + 1] = rank - acc;
+    tau[bh] = key_to_float(sel[bh * 4 + 0]) * inv_sqrt_d;
+  }
+  __syncthreads();
+  for (uint32_t i = threadIdx.x; i < n; i += blockDim.x) {
+    const uint2 e = c[i];
+    if ((e.y & 0xFFu) < low) continue;
+    const uint32_t g = e.y >> 8, key = e.x;
+    if ((int)g < G && (int)(key >> 5) < WN)
+      atomicOr(bits + ((size_t)bh * G + g) * WN + (key >> 5), 1u << (key & 31u));
   }
 }
 
@@ -417,6 +501,9 @@ int fg_g_pad(int G) { return (G + 127) / 128 * 128; }
 size_t fg_qsplit_bytes(int BH, int G, int d) { return 3ull * BH * fg_g_pad(G) * d * 2; }
 size_t fg_hist_bytes(int BH) { return sizeof(uint32_t) * (size_t)BH * kBins; }
 size_t fg_sel_bytes(int BH) { return sizeof(uint32_t) * (size_t)BH * 4; }
+size_t fg_cand_bytes(int BH) {
+  return sizeof(uint2) * (size_t)BH * kFgCandCap + 2 * sizeof(uint32_t) * (size_t)BH;
+}
 long long fg_list_cap_per_head(int G, int N, float f) {
   return (long long)ceil((double)f * (double)G * (double)N) + N + 32;
 }
@@ -436,30 +523,48 @@ cudaError_t launch_fg_build(const FgBuildParams& b, EncodeFn enc, cudaStream_t s
 
   const double total = (double)b.G * (double)b.N;
   const uint32_t rank = (uint32_t)ceil((double)b.keep_fraction * total);
-  fg_select_init_kernel<<<b.BH, 256, 0, st>>>(b.sel, b.hist, b.BH, rank);
+  fg_select_init_kernel<<<b.BH, 256, 0, st>>>(b.sel, b.hist, b.cand_count, b.BH, rank);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   FgScoreParams sp{};
   sp.bits = b.bits; sp.hist = b.hist; sp.sel = b.sel; sp.status = b.status;
+  sp.cand = b.cand; sp.cand_count = b.cand_count;
   sp.BH = b.BH; sp.N = b.N; sp.G = b.G; sp.WN = b.WN;
   const float inv_sqrt_d = 1.0f / sqrtf((float)b.d);
-  // radix select of the rank-th largest key: bits 31..20, 19..8, 7..0
+  auto score = [&]() {
+    return b.d == 128 ? launch_score<128>(km, qm, sp, st) : launch_score<64>(km, qm, sp, st);
+  };
+  // Radix select of the rank-th largest key: bits 31..20, 19..8, then 7..0.
   const int shifts[3] = {20, 8, 0};
   const int widths[3] = {12, 12, 8};
-  for (int lv = 0; lv < 3; ++lv) {
+  auto hist_level = [&](int lv, const uint32_t* only) -> cudaError_t {
     sp.mode = FG_MODE_HIST;
     sp.bin_shift = shifts[lv];
     sp.bin_mask = (1u << widths[lv]) - 1u;
     sp.match_mask = lv == 0 ? 0u : (0xFFFFFFFFu << shifts[lv - 1]);
-    e = b.d == 128 ? launch_score<128>(km, qm, sp, st) : launch_score<64>(km, qm, sp, st);
-    if (e != cudaSuccess) return e;
+    sp.only_heads = only;
+    cudaError_t err = score();
+    if (err != cudaSuccess) return err;
     fg_select_kernel<<<b.BH, 256, 0, st>>>(b.sel, b.hist, 1 << widths[lv], shifts[lv], b.tau,
-                                           inv_sqrt_d, lv == 2);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
+                                           inv_sqrt_d, lv == 2, only);
+    return cudaGetLastError();
+  };
+  for (int lv = 0; lv < 2; ++lv)
+    if ((e = hist_level(lv, nullptr)) != cudaSuccess) return e;
+  // The bitmask pass settles every score outside the 24-bit prefix bin and
+  // lists the few inside it; fg_fixup selects the last 8 bits among them.
+  sp.mode = FG_MODE_BITS_COLLECT;
+  sp.only_heads = nullptr;
+  if ((e = score()) != cudaSuccess) return e;
+  fg_fixup_kernel<<<b.BH, 256, 0, st>>>(b.sel, b.cand, b.cand_count, b.fallback, b.bits, b.tau,
+                                        inv_sqrt_d, b.G, b.WN);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // Heads whose candidate list overflowed: the full third level and the plain
+  // bitmask pass (every other head's CTAs return at once).
+  if ((e = hist_level(2, b.fallback)) != cudaSuccess) return e;
   sp.mode = FG_MODE_BITS;
-  e = b.d == 128 ? launch_score<128>(km, qm, sp, st) : launch_score<64>(km, qm, sp, st);
-  if (e != cudaSuccess) return e;
+  sp.only_heads = b.fallback;
+  if ((e = score()) != cudaSuccess) return e;
   return launch_fg_lists(b.lists, st);
 }
 

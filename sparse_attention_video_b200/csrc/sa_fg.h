@@ -13,7 +13,16 @@ typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void
                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-enum { FG_MODE_HIST = 0, FG_MODE_BITS = 1 };
+// HIST: histogram level of the radix select. BITS: slice bitmask key >= tau.
+// BITS_COLLECT: bitmask of the keys whose top 24 bits exceed the prefix the
+// first two levels decided, plus a list of the keys that share it (the last
+// 8 bits are then selected among those few by fg_fixup).
+enum { FG_MODE_HIST = 0, FG_MODE_BITS = 1, FG_MODE_BITS_COLLECT = 2 };
+
+// Candidate slots per head for the last select level; more than this (only
+// with very many scores equal in their top 24 bits) falls back to the full
+// third histogram pass.
+constexpr uint32_t kFgCandCap = 65536;
 
 struct FgQbarParams {
   const __nv_bfloat16* q;
@@ -30,6 +39,9 @@ struct FgScoreParams {
   int bin_shift;           // HIST: bin = (key >> bin_shift) & bin_mask
   uint32_t bin_mask;
   uint32_t match_mask;     // HIST: count only keys with (key & match_mask) == prefix
+  uint2* cand;             // BITS_COLLECT: [BH][kFgCandCap] (key index, group << 8 | low 8 bits)
+  uint32_t* cand_count;    // [BH]
+  const uint32_t* only_heads;  // if set: heads whose flag is 0 do nothing
   int BH, N, G, WN;
 };
 
@@ -49,6 +61,9 @@ struct FgBuildParams {
   __nv_bfloat16* qsplit;
   uint32_t* hist;
   uint32_t* sel;
+  uint2* cand;             // [BH][kFgCandCap]
+  uint32_t* cand_count;    // [BH]
+  uint32_t* fallback;      // [BH]: 1 where the candidate list overflowed
   uint32_t* bits;
   float* tau;
   uint32_t* status;
@@ -61,6 +76,7 @@ int fg_g_pad(int G);
 size_t fg_qsplit_bytes(int BH, int G, int d);
 size_t fg_hist_bytes(int BH);
 size_t fg_sel_bytes(int BH);
+size_t fg_cand_bytes(int BH);
 long long fg_list_cap_per_head(int G, int N, float keep_fraction);
 cudaError_t launch_fg_build(const FgBuildParams& p, EncodeFn enc, cudaStream_t st);
 cudaError_t launch_fg_lists(const FgListParams& p, cudaStream_t st);

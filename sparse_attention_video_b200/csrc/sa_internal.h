@@ -41,6 +41,7 @@ struct ScratchLayout {
   size_t off_fg_qsplit = 0;        // [3][BH][G_pad][d] bf16 terms of q_avg
   size_t off_fg_hist = 0;          // [BH][4096] u32 radix histogram
   size_t off_fg_sel = 0;           // [BH][4] u32 radix-select state
+  size_t off_fg_cand = 0;          // [BH][kFgCandCap] uint2 candidates, then [BH] count, [BH] fallback
   size_t total = 0;
 };
 
