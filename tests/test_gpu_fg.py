@@ -15,7 +15,7 @@ import pytest
 import torch
 
 from oracle import attention, masks
-from synthetic import CONFIGS, Workload, bf16_bits_to_f32, make_qkv
+from synthetic import CONFIGS, Workload, bf16_bits_to_f32, f32_to_bf16_bits, make_qkv
 from tests import _cases as C
 
 pytestmark = pytest.mark.gpu
@@ -34,10 +34,12 @@ def _dev(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def run_fg_case(wl, heads_check=None, groups_per_head=None, seed=0):
+def run_fg_case(wl, heads_check=None, groups_per_head=None, seed=0, transform=None):
     from sparse_attention_video_b200 import (SA_EXPORT_FG_BITS, SA_EXPORT_FG_TAU,
                                              SparseAttention, make_policy)
     x = make_qkv(wl)
+    if transform is not None:
+        transform(x)
     q, k, v = (_dev(x[n]) for n in "qkv")
     sa = SparseAttention(wl.batch, wl.heads, wl.T, wl.H, wl.W, wl.head_dim,
                          make_policy(**C.policy_kwargs(wl)))
@@ -86,3 +88,21 @@ def test_fg_small(name):
 
 def test_fg_full_size_sampled():
     run_fg_case(CONFIGS["fg_slices_hunyuan_720p"], heads_check=[0, 23], groups_per_head=12)
+
+
+def test_fg_threshold_ties_fallback():
+    """Keys 64.. are copies of key 0 and the first group's queries are 4 x
+    key 0, so that group's 73,664 equal scores are the largest of the head:
+    with f = 0.0005 the R-th largest (R = 42,467) is that score. Everything
+    sharing the threshold's top 24 bits is more than the library's candidate
+    list holds, so the mask must come out exact through the full third select
+    level, with every tie kept (and the kept count still fits the key lists)."""
+    wl = Workload(name="fg_ties", config_id=114, T=16, H=64, W=72, heads=1, head_dim=128,
+                  kind="fg", fg_group=64, fg_keep_fraction=0.0005)
+
+    def tie_keys(x):
+        k0 = bf16_bits_to_f32(x["k"][:, :, :1, :])
+        x["q"][:, :, :64, :] = f32_to_bf16_bits(4.0 * k0)
+        x["k"][:, :, 64:, :] = x["k"][:, :, :1, :]
+
+    run_fg_case(wl, groups_per_head=3, transform=tie_keys)
