@@ -116,20 +116,6 @@ __device__ __forceinline__ void load_block(const CUtensorMap* maps, const HeadGe
   }
 }
 
-// Pull block ``blk`` of head ``bh`` into L2 (same boxes as load_block).
-template <int D, int BN>
-__device__ __forceinline__ void prefetch_block(const CUtensorMap* maps, const HeadGeom& g, int bh,
-                                               int blk) {
-  int map, c1, c2, c3;
-  block_source(g, blk, BN, map, c1, c2, c3);
-  const CUtensorMap* m = maps + map;
-#pragma unroll
-  for (int h = 0; h < D / 64; ++h) {
-    if (map >= 2) tma_prefetch_l2_5d(m, h * 64, c1, c2, c3, bh);
-    else tma_prefetch_l2_3d(m, h * 64, c1, bh);
-  }
-}
-
 // Slot ``s`` of block ``blk`` -> original token index, or -1 for padding.
 __device__ __forceinline__ int slot_to_token(const HeadGeom& g, int blk, int s, int BN, int T,
                                              int H, int W) {
@@ -287,13 +273,6 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
 #pragma unroll
         for (int h = 0; h < D / 64; ++h)
           tma_load_3d(sQ + h * (BN * 128), &maps.q[0], &bars->q_full, h * 64, qb * BN, bh);
-        // Q tile of the CTA about one wave later, into L2
-        const long long lin = (long long)bh * p.NB + qb + p.prefetch_ahead;
-        if (p.prefetch_ahead > 0 && lin < (long long)p.BH * p.NB) {
-#pragma unroll
-          for (int h = 0; h < D / 64; ++h)
-            tma_prefetch_l2_3d(&maps.q[0], h * 64, (int)(lin % p.NB) * BN, (int)(lin / p.NB));
-        }
       }
       // list entries j*128 + lane + 32*s; key index in the low 30 bits, one
       // membership bit per group of the tile in bits 30 and 31. The next
@@ -341,16 +320,6 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       const CUtensorMap* vmaps = maps.v;
       mbar_arrive_expect_tx(&bars->q_full, L::kHalvesD * BN * 128);
       load_block<D, BN>(qmaps, g, bh, qb, sQ, &bars->q_full);
-      // The CTA that starts about one wave later reads its Q tile from HBM
-      // first thing; pull that tile into L2 now.
-      if (p.prefetch_ahead > 0) {
-        const long long lin = (long long)bh * p.NB + qb + p.prefetch_ahead;
-        if (lin < (long long)p.BH * p.NB) {
-          const int pbh = (int)(lin / p.NB), pqb = (int)(lin % p.NB);
-          const HeadGeom pg = p.heads[pbh];
-          if (pqb < pg.nb) prefetch_block<D, BN>(qmaps, pg, pbh, pqb);
-        }
-      }
       int issued = 0;
       for (int j = 0; j < n_keys; ++j) {
         const int st = j % kStages, rnd = j / kStages;
@@ -674,56 +643,35 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       const float inv_l = (n_keys > 0 && l_tot > 0.f) ? 1.f / l_tot : 0.f;
       const float w0 = a0 * inv_l, w1 = a1 * inv_l;
       const bool use0 = n_keys > 0 && w0 != 0.f, use1 = n_keys > 1 && w1 != 0.f;
-      // This thread's output columns [grp*D/2, grp*D/2 + D/2), all loaded
-      // from tensor memory before one wait, go to a staging tile in the first
-      // K stage (every load and MMA of the CTA has completed): [128 rows]
-      // [D bf16], 16-byte chunks XOR-swizzled by row. The rows then leave in
-      // coalesced 16-lanes-per-row stores (a thread per row would write 32
-      // scattered rows per instruction).
+      // this thread writes output columns [grp*D/2, grp*D/2 + D/2)
       constexpr int HD = D / 2;
-      float o0[HD], o1[HD];
-      // tcgen05.ld is warp-collective: load whenever any lane needs it
-      if (__any_sync(0xffffffffu, use0)) {
+      __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (tok < 0 ? 0 : tok)) * D + grp * HD;
 #pragma unroll
-        for (int c = 0; c < HD; c += 32) tmem_ld32(tO + lane_off + grp * HD + c, o0 + c);
-      }
-      if (__any_sync(0xffffffffu, use1)) {
+      for (int c = 0; c < HD; c += 16) {
+        float o0[16], o1[16];
+        // tcgen05.ld is warp-collective: load whenever any lane needs it
+        if (__any_sync(0xffffffffu, use0)) tmem_ld16(tO + lane_off + grp * HD + c, o0);
+        if (__any_sync(0xffffffffu, use1)) tmem_ld16(tO + D + lane_off + grp * HD + c, o1);
+        tmem_wait_ld();
+        if (tok >= 0) {
 #pragma unroll
-        for (int c = 0; c < HD; c += 32) tmem_ld32(tO + D + lane_off + grp * HD + c, o1 + c);
-      }
-      tmem_wait_ld();
+          for (int e = 0; e < 16; e += 8) {
+            float v[8];
 #pragma unroll
-      for (int e = 0; e < HD; e += 8) {
-        float v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          v[u] = (use0 ? o0[e + u] * w0 : 0.f) + (use1 ? o1[e + u] * w1 : 0.f);
-        uint4 w;
-        w.x = pack_bf16x2(v[0], v[1]);
-        w.y = pack_bf16x2(v[2], v[3]);
-        w.z = pack_bf16x2(v[4], v[5]);
-        w.w = pack_bf16x2(v[6], v[7]);
-        const int ci = (grp * HD + e) / 8;             // 16-byte chunk of the row
-        *reinterpret_cast<uint4*>(sK + r * (D * 2) + ((ci ^ (r % (D / 8))) << 4)) = w;
+            for (int u = 0; u < 8; ++u)
+              v[u] = (use0 ? o0[e + u] * w0 : 0.f) + (use1 ? o1[e + u] * w1 : 0.f);
+            uint4 w;
+            w.x = pack_bf16x2(v[0], v[1]);
+            w.y = pack_bf16x2(v[2], v[3]);
+            w.z = pack_bf16x2(v[4], v[5]);
+            w.w = pack_bf16x2(v[6], v[7]);
+            *reinterpret_cast<uint4*>(orow + c + e) = w;
+          }
+        }
       }
       if (tok >= 0 && grp == 0 && p.lse)
         p.lse[(size_t)bh * p.N + tok] =
             (n_keys > 0 && l_tot > 0.f) ? (mm + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
-    }
-    int* tok_s = reinterpret_cast<int*>(sV);          // row -> token, in the first V stage
-    if (grp == 0) tok_s[r] = tok;
-    named_barrier_sync(1, kSoftmaxWarps * 32);
-    if (ok) {
-      constexpr int kChunksRow = D / 8;                // 16-byte chunks per row
-      constexpr int kRowsPerPass = kSoftmaxWarps * 32 / kChunksRow;
-      const int t = threadIdx.x, c = t % kChunksRow;
-      for (int rr = t / kChunksRow; rr < BN; rr += kRowsPerPass) {
-        const int tk = tok_s[rr];
-        if (tk < 0) continue;
-        const uint4 v = *reinterpret_cast<const uint4*>(sK + rr * (D * 2) +
-                                                        ((c ^ (rr % kChunksRow)) << 4));
-        *reinterpret_cast<uint4*>(p.o + ((size_t)bh * p.N + tk) * D + c * 8) = v;
-      }
     }
   }
 
@@ -744,13 +692,8 @@ static cudaError_t launch_one(const AttnMaps& maps, const AttnParams& p, cudaStr
   auto kern = attn_fwd_kernel<D, BN, kGather>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  AttnParams pp = p;
-  pp.prefetch_ahead = sms;
   dim3 grid(p.NB, p.BH);
-  kern<<<grid, kGather ? kThreads + 64 : kThreads, L::kAlloc, stream>>>(maps, pp);
+  kern<<<grid, kGather ? kThreads + 64 : kThreads, L::kAlloc, stream>>>(maps, p);
   return cudaGetLastError();
 }
 

@@ -35,8 +35,6 @@ struct AttnParams {
   const uint32_t* fg_offsets;  // [BH][NB + 1]
   long long fg_cap;
   int fg_groups_per_tile;      // 2 for groups of 64, 1 for groups of 128
-  int prefetch_ahead;          // set by the launcher: SM count (CTA (qb, bh) pulls into L2 the
-                               // Q tile of the CTA that many places later in launch order)
 };
 
 cudaError_t launch_attn_fwd(int head_dim, int block, const AttnMaps& maps, const AttnParams& p,
