@@ -252,6 +252,13 @@ void pool_regions(PoolParams& pp) {
   }
   pp.Rt = R[0]; pp.Rh = R[1]; pp.Rw = R[2];
   pp.nRt = ceil_div(pp.T, R[0]); pp.nRh = ceil_div(pp.H, R[1]); pp.nRw = ceil_div(pp.W, R[2]);
+  // atoms: greatest common divisor of the tiles along each axis
+  int A[3] = {pp.cand[0][0], pp.cand[0][1], pp.cand[0][2]};
+  for (int c = 1; c < pp.C; ++c)
+    for (int a = 0; a < 3; ++a) A[a] = gcd_i(A[a], pp.cand[c][a]);
+  pp.At = A[0]; pp.Ah = A[1]; pp.Aw = A[2];
+  const long long nA = (long long)(R[0] / A[0]) * (R[1] / A[1]) * (R[2] / A[2]);
+  pp.nA = nA <= kMaxPoolAtoms ? (int)nA : 0;    // else the per-candidate kernel
 }
 
 int aligned(const void* p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }

@@ -209,6 +209,152 @@ __global__ void __launch_bounds__(256) pool_sics_kernel(PoolParams p) {
   }
 }
 
+// One pass over Q and K for every blocking candidate at once. A region (the
+// least common multiple of the candidates' tiles) is cut into atoms, the
+// greatest common divisor of the tiles along each axis: every atom lies in
+// exactly one block of every candidate. Warps stream the atoms' tokens once
+// (q, k, and the unit vector k / ||k|| with one correctly rounded reciprocal
+// square root per token), keep per-atom sums in shared memory, then every
+// candidate block adds up its atoms: its mean q, mean k and
+// SICS = ||sum of unit vectors||^2 - (number of nonzero keys).
+template <int D>
+__global__ void __launch_bounds__(256) pool_atoms_kernel(PoolParams p) {
+  constexpr int CH = D / 8;                 // lanes per token (16 or 8)
+  constexpr int TPW = 32 / CH;              // tokens per warp step (2 or 4)
+  constexpr int UNROLL = 4;
+  extern __shared__ float pool_sm[];        // [nA][3][D] sums, then [nA][2] counts
+  float* sums = pool_sm;
+  int* cnt = reinterpret_cast<int*>(pool_sm + (size_t)p.nA * 3 * D);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int region = blockIdx.x, bh = blockIdx.y;
+  const int rw = region % p.nRw, rh = (region / p.nRw) % p.nRh, rt = region / (p.nRw * p.nRh);
+  const int t0 = rt * p.Rt, h0 = rh * p.Rh, w0 = rw * p.Rw;
+  const int mAh = p.Rh / p.Ah, mAw = p.Rw / p.Aw;
+  const int A = p.At * p.Ah * p.Aw;         // tokens per atom
+  const int tl = lane / CH, dc = lane % CH;
+  const int N = p.T * p.H * p.W;
+  const __nv_bfloat16* q = p.q + (size_t)bh * N * D;
+  const __nv_bfloat16* k = p.k + (size_t)bh * N * D;
+
+  for (int a = warp; a < p.nA; a += 8) {
+    const int aw = a % mAw, ah = (a / mAw) % mAh, at = a / (mAw * mAh);
+    const int ta = t0 + at * p.At, ha = h0 + ah * p.Ah, wa = w0 + aw * p.Aw;
+    float qs[8], ks[8], us[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { qs[i] = 0.f; ks[i] = 0.f; us[i] = 0.f; }
+    int n_valid = 0, n_unit = 0;
+    for (int s0 = 0; s0 < A; s0 += TPW * UNROLL) {
+      uint4 qv[UNROLL], kv[UNROLL];
+      int tok[UNROLL];
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) {
+        const int s = s0 + u * TPW + tl;
+        const int iw = s % p.Aw, ih = (s / p.Aw) % p.Ah, it = s / (p.Aw * p.Ah);
+        const int t = ta + it, h = ha + ih, w = wa + iw;
+        tok[u] = (s < A && t < p.T && h < p.H && w < p.W) ? (t * p.H + h) * p.W + w : -1;
+        qv[u] = make_uint4(0, 0, 0, 0);
+        kv[u] = make_uint4(0, 0, 0, 0);
+        if (tok[u] >= 0) {
+          qv[u] = __ldg(reinterpret_cast<const uint4*>(q + (size_t)tok[u] * D) + dc);
+          kv[u] = __ldg(reinterpret_cast<const uint4*>(k + (size_t)tok[u] * D) + dc);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) {
+        const __nv_bfloat16* qe = reinterpret_cast<const __nv_bfloat16*>(&qv[u]);
+        const __nv_bfloat16* ke = reinterpret_cast<const __nv_bfloat16*>(&kv[u]);
+        float kf[8], ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          kf[i] = __bfloat162float(ke[i]);
+          ss = fmaf(kf[i], kf[i], ss);
+        }
+        // every lane joins; missing tokens carry zeros
+#pragma unroll
+        for (int o = CH / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (tok[u] < 0) continue;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          qs[i] += __bfloat162float(qe[i]);
+          ks[i] += kf[i];
+        }
+        ++n_valid;
+        if (ss > 0.f) {
+          const float rn = 1.0f / sqrtf(ss);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) us[i] = fmaf(kf[i], rn, us[i]);
+          ++n_unit;
+        }
+      }
+    }
+    // combine the token lanes (same dimensions, lanes dc + CH*t)
+#pragma unroll
+    for (int o = CH; o < 32; o <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        qs[i] += __shfl_xor_sync(0xffffffffu, qs[i], o);
+        ks[i] += __shfl_xor_sync(0xffffffffu, ks[i], o);
+        us[i] += __shfl_xor_sync(0xffffffffu, us[i], o);
+      }
+      n_valid += __shfl_xor_sync(0xffffffffu, n_valid, o);
+      n_unit += __shfl_xor_sync(0xffffffffu, n_unit, o);
+    }
+    if (tl == 0) {
+      float* sa = sums + (size_t)a * 3 * D + dc * 8;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { sa[i] = qs[i]; sa[D + i] = ks[i]; sa[2 * D + i] = us[i]; }
+      if (dc == 0) { cnt[2 * a] = n_valid; cnt[2 * a + 1] = n_unit; }
+    }
+  }
+  __syncthreads();
+
+  // every block of every candidate inside the region: one warp per block,
+  // each lane D/32 dimensions
+  constexpr int DL = D / 32;
+  int first[kMaxCand + 1];
+  first[0] = 0;
+  for (int c = 0; c < p.C; ++c)
+    first[c + 1] = first[c] + (p.Rt / p.cand[c][0]) * (p.Rh / p.cand[c][1]) * (p.Rw / p.cand[c][2]);
+  for (int pi = warp; pi < first[p.C]; pi += 8) {
+    int c = 0;
+    while (pi >= first[c + 1]) ++c;
+    const int bt = p.cand[c][0], bhh = p.cand[c][1], bw = p.cand[c][2];
+    const int lb = pi - first[c];
+    const int mw = p.Rw / bw, mh = p.Rh / bhh;
+    const int lw = lb % mw, lh = (lb / mw) % mh, lt = lb / (mw * mh);
+    const int nt = (p.T + bt - 1) / bt, nh = (p.H + bhh - 1) / bhh, nw = (p.W + bw - 1) / bw;
+    const int tt = rt * (p.Rt / bt) + lt, th = rh * (p.Rh / bhh) + lh, tw = rw * (p.Rw / bw) + lw;
+    if (tt >= nt || th >= nh || tw >= nw) continue;    // warp-uniform
+    const int blk = (tt * nh + th) * nw + tw;
+    float qv[DL], kv[DL], uv[DL];
+#pragma unroll
+    for (int i = 0; i < DL; ++i) { qv[i] = 0.f; kv[i] = 0.f; uv[i] = 0.f; }
+    int nv = 0, nu = 0;
+    const int ft = bt / p.At, fh = bhh / p.Ah, fw = bw / p.Aw;   // atoms per block along each axis
+    for (int x = 0; x < ft * fh * fw; ++x) {
+      const int xw = x % fw, xh = (x / fw) % fh, xt = x / (fw * fh);
+      const int a = ((lt * ft + xt) * mAh + (lh * fh + xh)) * mAw + (lw * fw + xw);
+      const float* sa = sums + (size_t)a * 3 * D + lane * DL;
+#pragma unroll
+      for (int i = 0; i < DL; ++i) { qv[i] += sa[i]; kv[i] += sa[D + i]; uv[i] += sa[2 * D + i]; }
+      nv += cnt[2 * a];
+      nu += cnt[2 * a + 1];
+    }
+    const size_t base = (((size_t)bh * p.C + c) * p.NB + blk);
+    const float inv = nv ? 1.f / (float)nv : 0.f;
+    float usq = 0.f;
+#pragma unroll
+    for (int i = 0; i < DL; ++i) {
+      p.qbar[base * D + lane * DL + i] = nv ? qv[i] * inv : 0.f;
+      p.kbar[base * D + lane * DL + i] = nv ? kv[i] * inv : 0.f;
+      usq = fmaf(uv[i], uv[i], usq);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) usq += __shfl_xor_sync(0xffffffffu, usq, o);
+    if (lane == 0) p.sics[base] = usq - (float)nu;
+  }
+}
+
 // ------------------------------------------------------------------ choose
 __global__ void choose_kernel(ChooseParams p) {
   const int bh = blockIdx.x;
@@ -550,6 +696,23 @@ cudaError_t launch_permute_fm(const PermuteParams& p, int BH, cudaStream_t st) {
 
 cudaError_t launch_pool_sics(const PoolParams& p, int BH, int max_nb, cudaStream_t st) {
   (void)max_nb;
+  if (p.nA > 0 && p.nA <= kMaxPoolAtoms) {
+    const size_t smem = (size_t)p.nA * (3 * p.d + 2) * sizeof(float);
+    dim3 grid(p.nRt * p.nRh * p.nRw, BH);
+    cudaError_t e;
+    if (p.d == 128) {
+      if ((e = cudaFuncSetAttribute(pool_atoms_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem)) != cudaSuccess) return e;
+      pool_atoms_kernel<128><<<grid, 256, smem, st>>>(p);
+    } else if (p.d == 64) {
+      if ((e = cudaFuncSetAttribute(pool_atoms_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem)) != cudaSuccess) return e;
+      pool_atoms_kernel<64><<<grid, 256, smem, st>>>(p);
+    } else {
+      return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+  }
   dim3 grid(p.C, p.nRt * p.nRh * p.nRw, BH);
   if (p.d == 128) pool_sics_kernel<128><<<grid, 256, 0, st>>>(p);
   else if (p.d == 64) pool_sics_kernel<64><<<grid, 256, 0, st>>>(p);

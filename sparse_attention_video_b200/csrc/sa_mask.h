@@ -34,7 +34,12 @@ struct PoolParams {
   int C, NB, T, H, W, d;
   int Rt, Rh, Rw;                   // region: lcm of the candidates' tiles, <= 8 blocks each
   int nRt, nRh, nRw;                // regions covering every candidate's tile grid
+  int At, Ah, Aw;                   // atom: gcd of the candidates' tiles (one block of each)
+  int nA;                           // atoms per region; 0 = per-candidate kernel
 };
+
+// Atoms per region the one-pass pooling kernel holds in shared memory.
+constexpr int kMaxPoolAtoms = 128;
 
 struct ChooseParams {
   const float* sics;
