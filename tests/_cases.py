@@ -54,6 +54,12 @@ SMALL = {
     "spade_d64": Workload(name="spade_d64", config_id=106, T=5, H=9, W=16, heads=2, head_dim=64,
                           kind="spade", block=128, candidates=((1, 8, 16), (8, 4, 4), (2, 8, 8)),
                           top_p=0.9, window=(3, 3, 3)),
+    # candidates whose common region holds 1,024 atoms: the pooling falls back
+    # to the per-candidate kernel
+    "spade_pool_fallback": Workload(name="spade_pool_fallback", config_id=107, T=8, H=6, W=136,
+                                    heads=2, head_dim=128, kind="spade", block=128,
+                                    candidates=((1, 1, 128), (8, 4, 4)), top_p=0.9,
+                                    window=(3, 3, 3)),
 }
 
 
