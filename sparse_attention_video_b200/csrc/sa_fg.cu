@@ -416,30 +416,63 @@ __global__ void fg_pair_count_kernel(FgListParams p) {
   if (lane == 0) p.counts[(size_t)bh * p.P + tile] = c;
 }
 
-__global__ void fg_offsets_kernel(FgListParams p) {
-  const int bh = blockIdx.x;
-  if (threadIdx.x != 0) return;
-  long long run = 0;
-  const long long cap = p.cap_per_head;
-  // Offsets are clamped to the list capacity, so a head whose union lists
-  // would overflow it (only possible with very many ties at tau) writes no
-  // entry out of bounds; that case is flagged in the status word.
-  for (int t = 0; t < p.P; ++t) {
-    p.offsets[(size_t)bh * (p.P + 1) + t] = (uint32_t)(run < cap ? run : cap);
-    run += p.counts[(size_t)bh * p.P + t];
+// Per head: exclusive scan of the tiles' union sizes, 1,024 tiles per pass
+// (warp shuffles, then the warp totals). Offsets are clamped to the list
+// capacity, so a head whose union lists would overflow it (only possible with
+// very many ties at tau) writes no entry out of bounds; that case is flagged
+// in the status word.
+__global__ void __launch_bounds__(1024) fg_offsets_kernel(FgListParams p) {
+  __shared__ unsigned long long wsum[32];
+  const int bh = blockIdx.x, lane = threadIdx.x % 32, wi = threadIdx.x / 32;
+  const uint32_t* cnt = p.counts + (size_t)bh * p.P;
+  uint32_t* off = p.offsets + (size_t)bh * (p.P + 1);
+  const unsigned long long cap = (unsigned long long)p.cap_per_head;
+  unsigned long long carry = 0;
+  for (int t0 = 0; t0 < p.P; t0 += 1024) {
+    const int t = t0 + (int)threadIdx.x;
+    const unsigned long long c = t < p.P ? cnt[t] : 0ull;
+    unsigned long long incl = c;
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[wi] = incl;
+    __syncthreads();
+    unsigned long long before = 0, total = 0;
+    for (int w = 0; w < 32; ++w) {
+      const unsigned long long v = wsum[w];
+      if (w < wi) before += v;
+      total += v;
+    }
+    const unsigned long long run = carry + before + incl - c;
+    if (t < p.P) off[t] = (uint32_t)(run < cap ? run : cap);
+    carry += total;
+    __syncthreads();
   }
-  if (run > cap) atomicOr(p.status, (uint32_t)SA_DEVFLAG_BOUNDS);
-  p.offsets[(size_t)bh * (p.P + 1) + p.P] = (uint32_t)(run < cap ? run : cap);
+  if (threadIdx.x == 0) {
+    off[p.P] = (uint32_t)(carry < cap ? carry : cap);
+    if (carry > cap) atomicOr(p.status, (uint32_t)SA_DEVFLAG_BOUNDS);
+  }
 }
 
-__global__ void fg_compact_kernel(FgListParams p) {
-  const int tile = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+// One warp per (tile, head) lists the tile's union in ascending key order,
+// 1,024 keys (32 bitmask words) at a time: lane l expands the set bits of
+// word l into a per-warp staging buffer in shared memory at its prefix
+// position, then the warp copies the chunk's entries out with consecutive
+// lanes on consecutive list slots (coalesced stores).
+constexpr int kListWarps = 8;
+
+__global__ void __launch_bounds__(32 * kListWarps) fg_compact_kernel(FgListParams p) {
+  __shared__ uint32_t stage[kListWarps][1024];
+  const int wi = threadIdx.x / 32;
+  const int tile = blockIdx.x * kListWarps + wi;
   const int bh = blockIdx.y, lane = threadIdx.x % 32;
   if (tile >= p.P) return;
   const int g0 = tile * p.groups_per_tile;
   const uint32_t* r0 = p.bits + ((size_t)bh * p.G + g0) * p.WN;
   const uint32_t* r1 = (p.groups_per_tile == 2 && g0 + 1 < p.G) ? r0 + p.WN : nullptr;
-  const size_t base = (size_t)bh * p.cap_per_head;
+  uint32_t* out = p.list + (size_t)bh * p.cap_per_head;
+  uint32_t* sb = stage[wi];
   uint32_t pos = p.offsets[(size_t)bh * (p.P + 1) + tile];
   const uint32_t end = p.offsets[(size_t)bh * (p.P + 1) + tile + 1];
   for (int w0 = 0; w0 < p.WN; w0 += 32) {
@@ -447,23 +480,24 @@ __global__ void fg_compact_kernel(FgListParams p) {
     const uint32_t a = w < p.WN ? r0[w] : 0u;
     const uint32_t b = (w < p.WN && r1) ? r1[w] : 0u;
     uint32_t u = a | b;
-    const int c = __popc(u);
-    int incl = c;
+    const uint32_t c = __popc(u);
+    uint32_t incl = c;
     for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += t;
     }
-    uint32_t q = pos + incl - c;
+    uint32_t q = incl - c;
     while (u) {
       const int bit = __ffs(u) - 1;
       u &= u - 1;
-      if (q < end) {
-        const uint32_t key = 32u * w + bit;
-        p.list[base + q] = key | (((a >> bit) & 1u) << 30) | (((b >> bit) & 1u) << 31);
-      }
-      ++q;
+      sb[q++] = (32u * w + bit) | (((a >> bit) & 1u) << 30) | (((b >> bit) & 1u) << 31);
     }
-    pos += __shfl_sync(0xffffffffu, incl, 31);
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+    __syncwarp();
+    for (uint32_t i = lane; i < total; i += 32)
+      if (pos + i < end) out[pos + i] = sb[i];
+    __syncwarp();
+    pos += total;
   }
 }
 
@@ -569,12 +603,12 @@ cudaError_t launch_fg_build(const FgBuildParams& b, EncodeFn enc, cudaStream_t s
 }
 
 cudaError_t launch_fg_lists(const FgListParams& p, cudaStream_t st) {
-  const int warps = 8;
+  const int warps = kListWarps;
   dim3 grid((p.P + warps - 1) / warps, p.BH);
   fg_pair_count_kernel<<<grid, 32 * warps, 0, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  fg_offsets_kernel<<<p.BH, 32, 0, st>>>(p);
+  fg_offsets_kernel<<<p.BH, 1024, 0, st>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   fg_compact_kernel<<<grid, 32 * warps, 0, st>>>(p);
   return cudaGetLastError();

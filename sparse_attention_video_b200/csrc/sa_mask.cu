@@ -475,7 +475,6 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
   if (i >= g.nb) return;
   __shared__ uint32_t bits[kMaxBlocks / 32];
   __shared__ uint32_t vbits[kMaxBlocks / 32];
-  __shared__ unsigned long long keys[kMaxBlocks];
   __shared__ float fbuf[8];
   __shared__ int s_count;
   const int nb = g.nb, W32 = (nb + 31) / 32;
@@ -534,8 +533,16 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
       }
       __syncthreads();
       if (p.kind == SA_MASK_SPADE) {
-        // softmax over valid key blocks, then the shortest prefix by descending
-        // probability (ties to the lower index) whose fp32 running sum reaches top_p
+        // Softmax over the valid key blocks, then the shortest prefix by
+        // descending probability (ties to the lower index) whose mass reaches
+        // top_p. The prefix is found by a radix select over the order key
+        // (probability bits above the complemented block index), 8 bits per
+        // level from the top: each level histograms the count and the mass of
+        // the keys that share the prefix fixed so far, and the bin where the
+        // mass (from the highest bin down) reaches what is still needed
+        // becomes the new prefix. Masses are summed in 2^-40 fixed point, so
+        // the sums, and the cut, do not depend on the order of the atomics;
+        // they differ from a float32 running sum in the last bits only.
         float mx = -INFINITY;
         for (int j = threadIdx.x; j < nb; j += 256)
           if (kvalid(j)) mx = fmaxf(mx, srow[j]);
@@ -544,78 +551,67 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
         for (int j = threadIdx.x; j < nb; j += 256)
           if (kvalid(j)) se += expf(srow[j] - mx);
         se = block_sum(se, fbuf);
-        int npow = 1;
-        while (npow < nb) npow <<= 1;
-        for (int j = threadIdx.x; j < npow; j += 256) {
-          unsigned long long key = 0ull;                 // invalid / padding sorts last
-          if (j < nb && kvalid(j)) {
-            const float pr = expf(srow[j] - mx) / se;
-            key = ((unsigned long long)__float_as_uint(pr) << 32) | (0xFFFFFFFFu - (uint32_t)j);
-          }
-          keys[j] = key;
-        }
-        __syncthreads();
-        // bitonic sort, descending
-        for (int size = 2; size <= npow; size <<= 1)
-          for (int stride = size / 2; stride >= 1; stride >>= 1) {
-            for (int a = threadIdx.x; a < npow; a += 256) {
-              const int b = a ^ stride;
-              if (b > a) {
-                const bool desc = (a & size) == 0;
-                const unsigned long long x = keys[a], y = keys[b];
-                if (desc ? (x < y) : (x > y)) { keys[a] = y; keys[b] = x; }
-              }
+        constexpr float kFix = 1099511627776.f;         // 2^40
+        // order key of valid block j, recomputed (identically) where needed
+        auto order_key = [&](int j) {
+          const float pr = expf(srow[j] - mx) / se;
+          return ((unsigned long long)__float_as_uint(pr) << 32) | (0xFFFFFFFFu - (uint32_t)j);
+        };
+        auto mass = [&](unsigned long long k) {
+          return (unsigned long long)__float2ull_rn(__uint_as_float((uint32_t)(k >> 32)) * kFix);
+        };
+        const unsigned long long target = __float2ull_ru(p.top_p * kFix);
+        __shared__ unsigned long long h_mass[256], w_mass[8], s_above;
+        __shared__ uint32_t h_cnt[256], s_cnt;
+        __shared__ int s_bin, s_all;
+        if (threadIdx.x == 0) s_all = 0;
+        unsigned long long prefix = 0ull, above = 0ull;  // fixed key bits; mass of higher keys
+        int shift = 56;
+        bool all = false;
+        for (;; shift -= 8) {
+          h_mass[threadIdx.x] = 0ull;
+          h_cnt[threadIdx.x] = 0u;
+          __syncthreads();
+          const unsigned long long hi = shift == 56 ? 0ull : (~0ull << (shift + 8));
+          for (int j = threadIdx.x; j < nb; j += 256) {
+            if (!kvalid(j)) continue;
+            const unsigned long long k = order_key(j);
+            if ((k & hi) == prefix) {
+              const int bin = (int)((k >> shift) & 255u);
+              atomicAdd(&h_mass[bin], mass(k));
+              atomicAdd(&h_cnt[bin], 1u);
             }
-            __syncthreads();
           }
-        // Shortest prefix of the sorted order whose fp32 running sum reaches
-        // top_p: a block-wide inclusive scan (thread t sums its 16 consecutive
-        // entries, then a scan over the thread totals), then the first
-        // position whose running sum reaches top_p. Running sums in another
-        // order than one left-to-right pass differ only in the last bits.
-        constexpr int kPer = kMaxBlocks / 256;
-        float cum[kPer];
-        float run = 0.f;
-        const int base = threadIdx.x * kPer;
-#pragma unroll
-        for (int e = 0; e < kPer; ++e) {
-          const int a = base + e;
-          const float pr = (a < npow && keys[a] != 0ull) ? __uint_as_float((uint32_t)(keys[a] >> 32)) : 0.f;
-          run += pr;
-          cum[e] = run;
+          __syncthreads();
+          // thread t takes bin 255 - t: inclusive scan of the mass from the top bin
+          const int bin = 255 - (int)threadIdx.x;
+          const unsigned long long m = h_mass[bin];
+          unsigned long long incl = m;
+          for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
+            if ((threadIdx.x & 31) >= (unsigned)o) incl += t;
+          }
+          if ((threadIdx.x & 31) == 31) w_mass[threadIdx.x >> 5] = incl;
+          __syncthreads();
+          for (int w = 0; w < (int)(threadIdx.x >> 5); ++w) incl += w_mass[w];
+          const unsigned long long need = target - above;  // > 0: above < target
+          if (incl >= need && incl - m < need) {
+            s_bin = bin;
+            s_above = above + (incl - m);
+            s_cnt = h_cnt[bin];
+          }
+          // the whole valid mass falls short of top_p (rounding): keep every valid block
+          if (threadIdx.x == 255 && incl < need) s_all = 1;
+          __syncthreads();
+          if (s_all) { all = true; break; }
+          prefix |= (unsigned long long)s_bin << shift;
+          above = s_above;
+          if (s_cnt == 1u || shift == 0) break;
         }
-        // exclusive scan of the thread totals (warp shuffles, then warp totals)
-        float incl = run;
-        for (int o = 1; o < 32; o <<= 1) {
-          const float t = __shfl_up_sync(0xffffffffu, incl, o);
-          if ((threadIdx.x & 31) >= o) incl += t;
-        }
-        __shared__ float wsum[8];
-        if ((threadIdx.x & 31) == 31) wsum[threadIdx.x >> 5] = incl;
-        if (threadIdx.x == 0) s_count = 0x7fffffff;
-        __syncthreads();
-        float wpre = 0.f;
-        for (int w = 0; w < (int)(threadIdx.x >> 5); ++w) wpre += wsum[w];
-        const float excl = wpre + incl - run;
-        int first = 0x7fffffff;
-#pragma unroll
-        for (int e = kPer - 1; e >= 0; --e) {
-          const int a = base + e;
-          if (a < npow && keys[a] != 0ull && excl + cum[e] >= p.top_p) first = a;
-        }
-        if (first != 0x7fffffff) atomicMin(&s_count, first + 1);
-        __syncthreads();
-        if (threadIdx.x == 0 && s_count == 0x7fffffff) {
-          // the sum never reached top_p (rounding): keep every valid block
-          int nvalid = 0;
-          while (nvalid < npow && keys[nvalid] != 0ull) ++nvalid;
-          s_count = nvalid;
-        }
-        __syncthreads();
-        for (int a = threadIdx.x; a < s_count; a += 256) {
-          const int j = (int)(0xFFFFFFFFu - (uint32_t)(keys[a] & 0xFFFFFFFFull));
-          atomicOr(&bits[j / 32], 1u << (j % 32));
-        }
+        // kept: every key at or above the cut's prefix
+        for (int j = threadIdx.x; j < nb; j += 256)
+          if (kvalid(j) && (all || (order_key(j) >> shift) >= (prefix >> shift)))
+            atomicOr(&bits[j / 32], 1u << (j % 32));
       }
     } else if (p.kind == SA_MASK_SPATIOTEMPORAL) {
       const int N = p.T * p.H * p.W, BS = g.bw, HW = p.H * p.W;
