@@ -486,11 +486,13 @@ __global__ void __launch_bounds__(32 * kListWarps) fg_compact_kernel(FgListParam
       const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += t;
     }
-    uint32_t q = incl - c;
+    uint32_t* dst = sb + (incl - c);
+    const uint32_t kbase = 32u * (uint32_t)w;
     while (u) {
-      const int bit = __ffs(u) - 1;
-      u &= u - 1;
-      sb[q++] = (32u * w + bit) | (((a >> bit) & 1u) << 30) | (((b >> bit) & 1u) << 31);
+      const uint32_t low = u & (0u - u);               // lowest set bit
+      u ^= low;
+      *dst++ = (kbase + (uint32_t)__popc(low - 1u)) | ((a & low) ? (1u << 30) : 0u) |
+               ((b & low) ? (1u << 31) : 0u);
     }
     const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
     __syncwarp();

@@ -230,11 +230,14 @@ __global__ void __launch_bounds__(256) pool_atoms_kernel(PoolParams p) {
   const int rw = region % p.nRw, rh = (region / p.nRw) % p.nRh, rt = region / (p.nRw * p.nRh);
   const int t0 = rt * p.Rt, h0 = rh * p.Rh, w0 = rw * p.Rw;
   const int mAh = p.Rh / p.Ah, mAw = p.Rw / p.Aw;
-  const int A = p.At * p.Ah * p.Aw;         // tokens per atom
   const int tl = lane / CH, dc = lane % CH;
   const int N = p.T * p.H * p.W;
   const __nv_bfloat16* q = p.q + (size_t)bh * N * D;
   const __nv_bfloat16* k = p.k + (size_t)bh * N * D;
+  // This lane's first token of an atom is token tl (atom order t, h, w); its
+  // later ones follow TPW apart. The coordinates inside the atom are the same
+  // for every atom, found once here and then advanced without division.
+  const int iw0 = tl % p.Aw, ih0 = (tl / p.Aw) % p.Ah, it0 = tl / (p.Aw * p.Ah);
 
   for (int a = warp; a < p.nA; a += 8) {
     const int aw = a % mAw, ah = (a / mAw) % mAh, at = a / (mAw * mAh);
@@ -243,15 +246,20 @@ __global__ void __launch_bounds__(256) pool_atoms_kernel(PoolParams p) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) { qs[i] = 0.f; ks[i] = 0.f; us[i] = 0.f; }
     int n_valid = 0, n_unit = 0;
-    for (int s0 = 0; s0 < A; s0 += TPW * UNROLL) {
+    int iw = iw0, ih = ih0, it = it0;
+    // the warp's lanes stay in step: it < At for some lane until the last step
+    while (__any_sync(0xffffffffu, it < p.At)) {
       uint4 qv[UNROLL], kv[UNROLL];
       int tok[UNROLL];
 #pragma unroll
       for (int u = 0; u < UNROLL; ++u) {
-        const int s = s0 + u * TPW + tl;
-        const int iw = s % p.Aw, ih = (s / p.Aw) % p.Ah, it = s / (p.Aw * p.Ah);
         const int t = ta + it, h = ha + ih, w = wa + iw;
-        tok[u] = (s < A && t < p.T && h < p.H && w < p.W) ? (t * p.H + h) * p.W + w : -1;
+        tok[u] = (it < p.At && t < p.T && h < p.H && w < p.W) ? (t * p.H + h) * p.W + w : -1;
+        iw += TPW;
+        while (iw >= p.Aw) {
+          iw -= p.Aw;
+          if (++ih == p.Ah) { ih = 0; ++it; }
+        }
         qv[u] = make_uint4(0, 0, 0, 0);
         kv[u] = make_uint4(0, 0, 0, 0);
         if (tok[u] >= 0) {
@@ -476,7 +484,6 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
   __shared__ uint32_t bits[kMaxBlocks / 32];
   __shared__ uint32_t vbits[kMaxBlocks / 32];
   __shared__ float fbuf[8];
-  __shared__ int s_count;
   const int nb = g.nb, W32 = (nb + 31) / 32;
   for (int w = threadIdx.x; w < W32; w += 256) { bits[w] = 0u; vbits[w] = 0u; }
   __syncthreads();
@@ -540,36 +547,43 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
         // level from the top: each level histograms the count and the mass of
         // the keys that share the prefix fixed so far, and the bin where the
         // mass (from the highest bin down) reaches what is still needed
-        // becomes the new prefix. Masses are summed in 2^-40 fixed point, so
-        // the sums, and the cut, do not depend on the order of the atomics;
-        // they differ from a float32 running sum in the last bits only.
+        // becomes the new prefix. Masses are summed in 2^-31 fixed point
+        // (every probability rounded to a multiple of 2^-31, at most 4,096 of
+        // them: the total stays below 2^32), so the sums, and the cut, do not
+        // depend on the order of the atomics; they differ from a float32
+        // running sum by far less than that sum's own rounding.
         float mx = -INFINITY;
         for (int j = threadIdx.x; j < nb; j += 256)
           if (kvalid(j)) mx = fmaxf(mx, srow[j]);
         mx = block_max(mx, fbuf);
+        // probabilities, once: exp(s - max) first, normalised below
+        __shared__ float prob[kMaxBlocks];
         float se = 0.f;
-        for (int j = threadIdx.x; j < nb; j += 256)
-          if (kvalid(j)) se += expf(srow[j] - mx);
-        se = block_sum(se, fbuf);
-        constexpr float kFix = 1099511627776.f;         // 2^40
-        // order key of valid block j, recomputed (identically) where needed
+        for (int j = threadIdx.x; j < nb; j += 256) {
+          const float e = kvalid(j) ? expf(srow[j] - mx) : 0.f;
+          prob[j] = e;
+          se += e;
+        }
+        se = block_sum(se, fbuf);                       // ends with a barrier
+        for (int j = threadIdx.x; j < nb; j += 256) prob[j] = prob[j] / se;
+        __syncthreads();
+        constexpr float kFix = 2147483648.f;            // 2^31
+        // order key of valid block j: probability bits above ~j
         auto order_key = [&](int j) {
-          const float pr = expf(srow[j] - mx) / se;
-          return ((unsigned long long)__float_as_uint(pr) << 32) | (0xFFFFFFFFu - (uint32_t)j);
+          return ((unsigned long long)__float_as_uint(prob[j]) << 32) | (0xFFFFFFFFu - (uint32_t)j);
         };
-        auto mass = [&](unsigned long long k) {
-          return (unsigned long long)__float2ull_rn(__uint_as_float((uint32_t)(k >> 32)) * kFix);
-        };
-        const unsigned long long target = __float2ull_ru(p.top_p * kFix);
-        __shared__ unsigned long long h_mass[256], w_mass[8], s_above;
+        auto mass = [&](int j) { return __float2uint_rn(prob[j] * kFix); };
+        const uint32_t target = __float2uint_ru(p.top_p * kFix);
+        __shared__ uint32_t h_mass[256], w_mass[8], s_above;
         __shared__ uint32_t h_cnt[256], s_cnt;
         __shared__ int s_bin, s_all;
         if (threadIdx.x == 0) s_all = 0;
-        unsigned long long prefix = 0ull, above = 0ull;  // fixed key bits; mass of higher keys
+        unsigned long long prefix = 0ull;                // fixed key bits
+        uint32_t above = 0u;                             // mass of the keys above them
         int shift = 56;
         bool all = false;
         for (;; shift -= 8) {
-          h_mass[threadIdx.x] = 0ull;
+          h_mass[threadIdx.x] = 0u;
           h_cnt[threadIdx.x] = 0u;
           __syncthreads();
           const unsigned long long hi = shift == 56 ? 0ull : (~0ull << (shift + 8));
@@ -578,23 +592,23 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
             const unsigned long long k = order_key(j);
             if ((k & hi) == prefix) {
               const int bin = (int)((k >> shift) & 255u);
-              atomicAdd(&h_mass[bin], mass(k));
+              atomicAdd(&h_mass[bin], mass(j));
               atomicAdd(&h_cnt[bin], 1u);
             }
           }
           __syncthreads();
           // thread t takes bin 255 - t: inclusive scan of the mass from the top bin
           const int bin = 255 - (int)threadIdx.x;
-          const unsigned long long m = h_mass[bin];
-          unsigned long long incl = m;
+          const uint32_t m = h_mass[bin];
+          uint32_t incl = m;
           for (int o = 1; o < 32; o <<= 1) {
-            const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
+            const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
             if ((threadIdx.x & 31) >= (unsigned)o) incl += t;
           }
           if ((threadIdx.x & 31) == 31) w_mass[threadIdx.x >> 5] = incl;
           __syncthreads();
           for (int w = 0; w < (int)(threadIdx.x >> 5); ++w) incl += w_mass[w];
-          const unsigned long long need = target - above;  // > 0: above < target
+          const uint32_t need = target - above;            // > 0: above < target
           if (incl >= need && incl - m < need) {
             s_bin = bin;
             s_above = above + (incl - m);
