@@ -47,6 +47,13 @@ namespace sa {
 namespace {
 
 constexpr int kThreads = 320;
+// M x 1 slice mode runs 384 threads (two more copy warps) with a register
+// split (setmaxnreg): the softmax warpgroups take 208, warpgroup 2
+// (producer, MMA issuer, copy warps) 88. The shares add up to the launch's
+// 168 per thread.
+constexpr uint32_t kRegsLaunch = 168, kRegsSoftmax = 208, kRegsOther = 88;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther == (kThreads + 64) * kRegsLaunch,
+              "register split must equal the launch total");
 constexpr int kSoftmaxWarps = 8;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
@@ -183,8 +190,8 @@ __device__ __forceinline__ uint32_t site(uint32_t role, uint32_t bar, int j) {
 // kGather = false: blocks of a working layout, kept key blocks from the mask's
 // ascending lists. kGather = true (M x 1 key slices): the query tile is 128
 // contiguous queries (one or two groups); its keys are the union list of those
-// groups, gathered 128 rows at a time with TMA tile::gather4, and each row
-// masks keys outside its own group.
+// groups, copied 128 rows at a time by the copy warps (cp.async), and each
+// row masks keys outside its own group.
 template <int D, int BN, bool kGather>
 __global__ void __launch_bounds__(kGather ? kThreads + 64 : kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
@@ -265,6 +272,10 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   volatile int* abort = &bars->abort;
   uint32_t* status = p.status;
 
+  if (warp >= 8) {
+  // Slice mode: warpgroup 2 gives registers back at one point that dominates
+  // all of its role code; the softmax warpgroups take them in the other branch.
+  if constexpr (kGather) regs_dec<kRegsOther>();
   if (warp == kProducerWarp && kGather) {
     // ------------------------------------------------------------ producer (gather)
     if (n_keys > 0) {
@@ -470,7 +481,9 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     cp_async_wait<0>();
     fence_proxy_async_smem();
     __syncwarp();
+  }
   } else {
+    if constexpr (kGather) regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax + epilogue
     // Group grp = warp / 4 takes the key blocks j with j % 2 == grp; thread r
     // of a group owns row r of those blocks: its own running maximum m, sum
