@@ -52,15 +52,40 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
 }
 
 // ------------------------------------------------------------------ q_avg
-// One CTA per (group, head); thread c owns dimension c (c < d).
-__global__ void fg_qbar_kernel(FgQbarParams p) {
-  const int g = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
+// One CTA of 128 threads per (group, head). d/8 lanes cover one query row
+// with 16-byte loads (8 dimensions each), so 1,024 / d rows are read per
+// step, all of a group's rows in flight at once; the per-lane partial sums
+// are then added in a fixed order through shared memory.
+constexpr int kQbarThreads = 128;
+
+__global__ void __launch_bounds__(kQbarThreads) fg_qbar_kernel(FgQbarParams p) {
+  __shared__ float part[kQbarThreads * 8];          // [row slot][d]
+  const int g = blockIdx.x, bh = blockIdx.y;
+  const int lanes = p.d / 8, rows = kQbarThreads / lanes;
+  const int piece = threadIdx.x % lanes, slot = threadIdx.x / lanes;
+  const int t0 = g * p.group, t1 = min(t0 + p.group, p.N);
+  const __nv_bfloat16* q = p.q + (size_t)bh * p.N * p.d + piece * 8;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 8
+  for (int t = t0 + slot; t < t1; t += rows) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(q + (size_t)t * p.d));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc[2 * e] += __uint_as_float(w[e] << 16);
+      acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) part[slot * p.d + piece * 8 + i] = acc[i];
+  __syncthreads();
+  const int c = threadIdx.x;
   if (c >= p.d) return;
   float s = 0.f;
-  int n = 0;
-  const int t0 = g * p.group;
-  for (int t = t0; t < t0 + p.group && t < p.N; ++t, ++n)
-    s += __bfloat162float(p.q[((size_t)bh * p.N + t) * p.d + c]);
+  for (int r = 0; r < rows; ++r) s += part[r * p.d + c];
+  const int n = t1 > t0 ? t1 - t0 : 0;
   const float mean = n ? s / (float)n : 0.f;
   const __nv_bfloat16 hi = __float2bfloat16_rn(mean);
   const float r1 = mean - __bfloat162float(hi);
@@ -550,7 +575,7 @@ cudaError_t launch_fg_build(const FgBuildParams& b, EncodeFn enc, cudaStream_t s
   // q_avg terms (pad groups stay zero: clear the whole buffer first)
   if ((e = cudaMemsetAsync(b.qsplit, 0, fg_qsplit_bytes(b.BH, b.G, b.d), st)) != cudaSuccess) return e;
   FgQbarParams qp{b.q, b.qsplit, b.BH, b.N, b.d, b.group, b.G, G_pad};
-  fg_qbar_kernel<<<dim3(b.G, b.BH), b.d, 0, st>>>(qp);
+  fg_qbar_kernel<<<dim3(b.G, b.BH), kQbarThreads, 0, st>>>(qp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   CUtensorMap km, qm;

@@ -213,12 +213,14 @@ __global__ void __launch_bounds__(256) pool_sics_kernel(PoolParams p) {
 // least common multiple of the candidates' tiles) is cut into atoms, the
 // greatest common divisor of the tiles along each axis: every atom lies in
 // exactly one block of every candidate. Warps stream the atoms' tokens once
-// (q, k, and the unit vector k / ||k|| with one correctly rounded reciprocal
+// (q, k, and the unit vector k / ||k|| with one approximate reciprocal
 // square root per token), keep per-atom sums in shared memory, then every
 // candidate block adds up its atoms: its mean q, mean k and
 // SICS = ||sum of unit vectors||^2 - (number of nonzero keys).
+constexpr int kPoolAtomThreads = 256;     // 8 warps; two CTAs per SM (shared memory)
+
 template <int D>
-__global__ void __launch_bounds__(256) pool_atoms_kernel(PoolParams p) {
+__global__ void __launch_bounds__(kPoolAtomThreads) pool_atoms_kernel(PoolParams p) {
   constexpr int CH = D / 8;                 // lanes per token (16 or 8)
   constexpr int TPW = 32 / CH;              // tokens per warp step (2 or 4)
   constexpr int UNROLL = 4;
@@ -239,7 +241,8 @@ __global__ void __launch_bounds__(256) pool_atoms_kernel(PoolParams p) {
   // for every atom, found once here and then advanced without division.
   const int iw0 = tl % p.Aw, ih0 = (tl / p.Aw) % p.Ah, it0 = tl / (p.Aw * p.Ah);
 
-  for (int a = warp; a < p.nA; a += 8) {
+  constexpr int kWarps = kPoolAtomThreads / 32;
+  for (int a = warp; a < p.nA; a += kWarps) {
     const int aw = a % mAw, ah = (a / mAw) % mAh, at = a / (mAw * mAh);
     const int ta = t0 + at * p.At, ha = h0 + ah * p.Ah, wa = w0 + aw * p.Aw;
     float qs[8], ks[8], us[8];
@@ -269,28 +272,39 @@ __global__ void __launch_bounds__(256) pool_atoms_kernel(PoolParams p) {
       }
 #pragma unroll
       for (int u = 0; u < UNROLL; ++u) {
-        const __nv_bfloat16* qe = reinterpret_cast<const __nv_bfloat16*>(&qv[u]);
-        const __nv_bfloat16* ke = reinterpret_cast<const __nv_bfloat16*>(&kv[u]);
-        float kf[8], ss = 0.f;
+        // bf16 -> fp32 is a shift: element 2e in the low half of word e
+        const uint32_t* qw = reinterpret_cast<const uint32_t*>(&qv[u]);
+        const uint32_t* kw = reinterpret_cast<const uint32_t*>(&kv[u]);
+        float kf[8], qf[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          kf[i] = __bfloat162float(ke[i]);
-          ss = fmaf(kf[i], kf[i], ss);
+        for (int e = 0; e < 4; ++e) {
+          kf[2 * e] = __uint_as_float(kw[e] << 16);
+          kf[2 * e + 1] = __uint_as_float(kw[e] & 0xFFFF0000u);
+          qf[2 * e] = __uint_as_float(qw[e] << 16);
+          qf[2 * e + 1] = __uint_as_float(qw[e] & 0xFFFF0000u);
         }
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          fma2(kf[2 * e], kf[2 * e + 1], kf[2 * e], kf[2 * e + 1], s0, s1, s0, s1);
+        float ss = s0 + s1;
         // every lane joins; missing tokens carry zeros
 #pragma unroll
         for (int o = CH / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         if (tok[u] < 0) continue;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          qs[i] += __bfloat162float(qe[i]);
-          ks[i] += kf[i];
+        for (int e = 0; e < 4; ++e) {
+          add2(qs[2 * e], qs[2 * e + 1], qf[2 * e], qf[2 * e + 1]);
+          add2(ks[2 * e], ks[2 * e + 1], kf[2 * e], kf[2 * e + 1]);
         }
         ++n_valid;
         if (ss > 0.f) {
-          const float rn = 1.0f / sqrtf(ss);
+          // approximate reciprocal square root (MUFU): the unit vectors
+          // differ from k / sqrt(|k|^2) by a few ulp
+          const float rn = rsqrtf(ss);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) us[i] = fmaf(kf[i], rn, us[i]);
+          for (int e = 0; e < 4; ++e)
+            fma2(kf[2 * e], kf[2 * e + 1], rn, rn, us[2 * e], us[2 * e + 1], us[2 * e], us[2 * e + 1]);
           ++n_unit;
         }
       }
@@ -323,7 +337,7 @@ __global__ void __launch_bounds__(256) pool_atoms_kernel(PoolParams p) {
   first[0] = 0;
   for (int c = 0; c < p.C; ++c)
     first[c + 1] = first[c] + (p.Rt / p.cand[c][0]) * (p.Rh / p.cand[c][1]) * (p.Rw / p.cand[c][2]);
-  for (int pi = warp; pi < first[p.C]; pi += 8) {
+  for (int pi = warp; pi < first[p.C]; pi += kWarps) {
     int c = 0;
     while (pi >= first[c + 1]) ++c;
     const int bt = p.cand[c][0], bhh = p.cand[c][1], bw = p.cand[c][2];
@@ -713,11 +727,11 @@ cudaError_t launch_pool_sics(const PoolParams& p, int BH, int max_nb, cudaStream
     if (p.d == 128) {
       if ((e = cudaFuncSetAttribute(pool_atoms_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)smem)) != cudaSuccess) return e;
-      pool_atoms_kernel<128><<<grid, 256, smem, st>>>(p);
+      pool_atoms_kernel<128><<<grid, kPoolAtomThreads, smem, st>>>(p);
     } else if (p.d == 64) {
       if ((e = cudaFuncSetAttribute(pool_atoms_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)smem)) != cudaSuccess) return e;
-      pool_atoms_kernel<64><<<grid, 256, smem, st>>>(p);
+      pool_atoms_kernel<64><<<grid, kPoolAtomThreads, smem, st>>>(p);
     } else {
       return cudaErrorInvalidValue;
     }
