@@ -34,6 +34,30 @@ def block_means(x, blk):
     return out
 
 
+def block_summaries(x, blk, how="mean"):
+    """Per-channel summary of the valid tokens' vectors in each block, float32 [nb, d].
+
+    SPADE review, minor comment 3 and axiom ledger: a block is summarized by
+    the max, the min or the mean of its tokens along the head dimension (the
+    DSA-SPADE, DSA2-SPADE and MEAN-SPADE variants, whose expressions the pages
+    do not print). Reading: ``how`` applies channel by channel over the
+    block's valid tokens, to Q and K alike; the estimator stays q.k / sqrt(d).
+    A block with no valid token gets a zero summary.
+    """
+    if how == "mean":
+        return block_means(x, blk)
+    if how not in ("max", "min"):
+        raise ValueError(how)
+    nb, _ = blk.shape
+    out = np.zeros((nb, x.shape[1]), dtype=F32)
+    for b in range(nb):
+        idx = blk[b][blk[b] >= 0]
+        if len(idx):
+            v = x[idx].astype(F32)
+            out[b] = v.max(axis=0) if how == "max" else v.min(axis=0)
+    return out
+
+
 def sics(k, blk):
     """Sum of Intra-block Cosine Similarities per block, float32 [nb].
 

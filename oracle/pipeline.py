@@ -47,7 +47,8 @@ def head_mask(wl, q, k, head, force_choice=None):
     valid = masks.valid_blocks(blk)
 
     if wl.kind == "topk":
-        s = masks.pooled_scores(masks.block_means(q, blk), masks.block_means(k, blk), d)
+        s = masks.pooled_scores(masks.block_summaries(q, blk, wl.summarizer),
+                                masks.block_summaries(k, blk, wl.summarizer), d)
         info["scores"] = s
         bm = masks.topk_with_diagonal(s, wl.topk, wl.keep_diagonal, valid, valid)
     elif wl.kind == "sta":
@@ -60,7 +61,8 @@ def head_mask(wl, q, k, head, force_choice=None):
             bm = masks.spatial_rule(blk, wl.T, wl.H, wl.W)
         bm = masks.add_sinks(bm, blk, wl.sink_tokens, wl.block)
     elif wl.kind == "spade":
-        s = masks.pooled_scores(masks.block_means(q, blk), masks.block_means(k, blk), d)
+        s = masks.pooled_scores(masks.block_summaries(q, blk, wl.summarizer),
+                                masks.block_summaries(k, blk, wl.summarizer), d)
         info["scores"] = s
         dims = layout.tile_grid_dims(wl.T, wl.H, wl.W, *tile)
         bm = masks.tile_window(dims, wl.window, valid, valid)

@@ -46,6 +46,7 @@ class Workload:
     fg_group: int = 0
     fg_keep_fraction: float = 0.0
     block: int = 128                               # tokens per block in the working layout
+    summarizer: str = "mean"                       # topk, spade: block summary ("mean", "max", "min")
 
     @property
     def N(self) -> int:

@@ -42,6 +42,63 @@ def test_block_means_all_padding_block_is_zero():
     np.testing.assert_array_equal(masks.block_means(x, blk)[1], 0.0)
 
 
+def _ragged_blocks(seed, n=37, d=8, nb=6, bs=8):
+    g = np.random.default_rng(seed)
+    x = g.standard_normal((n, d)).astype(np.float32)
+    order = np.full(nb * bs, -1)
+    order[:n] = g.permutation(n)
+    return x, order.reshape(nb, bs)
+
+
+@pytest.mark.parametrize("how", ["max", "min"])
+def test_block_summary_extreme_is_attained_and_bounds_every_token(how):
+    # SPADE review, minor comment 3: max / min summaries along the head
+    # dimension. Per channel the summary must bound every valid token of the
+    # block and be one of their values; padding slots take no part.
+    x, blk = _ragged_blocks(3)
+    got = masks.block_summaries(x, blk, how)
+    for b in range(blk.shape[0]):
+        idx = blk[b][blk[b] >= 0]
+        if len(idx) == 0:
+            assert np.all(got[b] == 0.0)
+            continue
+        vals = x[idx]
+        for c in range(x.shape[1]):
+            if how == "max":
+                assert all(got[b, c] >= v for v in vals[:, c])
+            else:
+                assert all(got[b, c] <= v for v in vals[:, c])
+            assert any(got[b, c] == v for v in vals[:, c])
+
+
+def test_block_summaries_ignore_tokens_outside_the_block():
+    x, blk = _ragged_blocks(4)
+    base = {h: masks.block_summaries(x, blk, h) for h in ("mean", "max", "min")}
+    # tokens 37.. do not exist; a token of block 0 changes only block 0
+    y = x.copy()
+    t0 = blk[0][0]
+    y[t0] += 100.0
+    for h in ("mean", "max", "min"):
+        got = masks.block_summaries(y, blk, h)
+        np.testing.assert_array_equal(got[1:], base[h][1:])
+        assert not np.array_equal(got[0], base[h][0]) or h == "min"
+
+
+def test_block_summaries_order_and_single_token():
+    x, blk = _ragged_blocks(5)
+    lo = masks.block_summaries(x, blk, "min")
+    mid = masks.block_summaries(x, blk, "mean")
+    hi = masks.block_summaries(x, blk, "max")
+    assert np.all(lo <= mid + 1e-6) and np.all(mid <= hi + 1e-6)
+    one = np.array([[2], [-1]])
+    z = np.array([[0.0], [0.0], [1.5], [0.0]], np.float32)
+    for h in ("mean", "max", "min"):
+        np.testing.assert_array_equal(masks.block_summaries(z, one, h)[0], [1.5])
+        np.testing.assert_array_equal(masks.block_summaries(z, one, h)[1], [0.0])
+    with pytest.raises(ValueError):
+        masks.block_summaries(x, blk, "median")
+
+
 # ---------------------------------------------------------------- SICS
 def _sics_bruteforce(k, idx):
     u = [k[i].astype(np.float64) / np.linalg.norm(k[i].astype(np.float64)) for i in idx]
