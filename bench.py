@@ -187,7 +187,7 @@ def policy_kwargs(wl):
     """The workload's mask policy as make_policy() arguments."""
     if wl.kind == "topk":
         return dict(kind="topk", block=wl.block, tile=wl.tile, topk=wl.topk,
-                    keep_diagonal=wl.keep_diagonal)
+                    keep_diagonal=wl.keep_diagonal, summarizer=wl.summarizer)
     if wl.kind == "sta":
         return dict(kind="sta", block=wl.block, tile=wl.tile, window=wl.window)
     if wl.kind == "spatiotemporal":
@@ -195,7 +195,7 @@ def policy_kwargs(wl):
                     heads=wl.heads, sink_tokens=wl.sink_tokens, frame_radius=1)
     if wl.kind == "spade":
         return dict(kind="spade", block=wl.block, candidates=wl.candidates, top_p=wl.top_p,
-                    window=wl.window)
+                    window=wl.window, summarizer=wl.summarizer)
     return dict(kind="fg", block=wl.block, fg_group=wl.fg_group,
                 fg_keep_fraction=wl.fg_keep_fraction)
 

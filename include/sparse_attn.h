@@ -98,6 +98,16 @@ enum {
   SA_MASK_EXPLICIT = 6        /* caller-supplied block bitmask                    */
 };
 
+/* Block summaries behind the pooled scores of TOPK and SPADE (SPADE review,
+ * minor comment 3 and axiom ledger: max, min or mean along the head
+ * dimension). Each applies channel by channel over a block's valid tokens,
+ * to Q and K alike; a block with no valid token summarizes to zero. */
+enum {
+  SA_SUMMARIZER_MEAN = 0,     /* MEAN-SPADE (the default)                         */
+  SA_SUMMARIZER_MAX = 1,      /* per-channel maximum                              */
+  SA_SUMMARIZER_MIN = 2       /* per-channel minimum                              */
+};
+
 enum {
   SA_LAYOUT_IDENTITY = 0,     /* blocks of consecutive tokens in original order   */
   SA_LAYOUT_FRAME_MAJOR = 1,  /* slot m = (h*W + w)*T + t                         */
@@ -124,6 +134,7 @@ typedef struct {
   int explicit_layout;        /* EXPLICIT: SA_LAYOUT_*                             */
   const uint32_t* explicit_bits; /* EXPLICIT: device [batch*heads][nb][ceil(nb/32)],
                                  bit j of row i keeps key block j for query block i */
+  int summarizer;             /* TOPK, SPADE: SA_SUMMARIZER_*; other kinds ignore it */
 } sa_policy;
 
 /* ---------------------------------------------------------------- sizes

@@ -18,6 +18,7 @@ SA_MASK_TOPK, SA_MASK_STA, SA_MASK_SPATIOTEMPORAL = 1, 2, 3
 SA_MASK_SPADE, SA_MASK_FG, SA_MASK_EXPLICIT = 4, 5, 6
 
 SA_LAYOUT_IDENTITY, SA_LAYOUT_FRAME_MAJOR, SA_LAYOUT_TILE = 0, 1, 2
+SA_SUMMARIZER_MEAN, SA_SUMMARIZER_MAX, SA_SUMMARIZER_MIN = 0, 1, 2
 
 SA_EXPORT_BLOCK_BITS, SA_EXPORT_HEAD_INFO, SA_EXPORT_FG_BITS, SA_EXPORT_FG_TAU = 1, 2, 3, 4
 SA_EXPORT_FG_TILE_KEYS = 5
@@ -44,7 +45,7 @@ class Policy(ctypes.Structure):
                 ("n_candidates", ctypes.c_int), ("candidates", (ctypes.c_int * 3) * 4),
                 ("top_p", ctypes.c_float), ("fg_group", ctypes.c_int),
                 ("fg_keep_fraction", ctypes.c_float), ("explicit_layout", ctypes.c_int),
-                ("explicit_bits", ctypes.c_void_p)]
+                ("explicit_bits", ctypes.c_void_p), ("summarizer", ctypes.c_int)]
 
 
 class HeadInfo(ctypes.Structure):

@@ -15,9 +15,11 @@ from . import _native as N
 def make_policy(kind, block=128, tile=(1, 1, 128), topk=0, keep_diagonal=False,
                 window=(1, 1, 1), temporal_heads=None, heads=0, sink_tokens=0, frame_radius=1,
                 candidates=(), top_p=0.0, fg_group=64, fg_keep_fraction=0.15,
-                explicit_layout=N.SA_LAYOUT_IDENTITY, explicit_bits=None):
+                explicit_layout=N.SA_LAYOUT_IDENTITY, explicit_bits=None, summarizer="mean"):
     """Fill an ``sa_policy``. ``kind`` is a name ("topk", "sta", "spatiotemporal",
-    "spade", "fg", "explicit") or an SA_MASK_* code."""
+    "spade", "fg", "explicit") or an SA_MASK_* code; ``summarizer`` ("mean",
+    "max", "min" or an SA_SUMMARIZER_* code) picks the block summary behind the
+    pooled scores of "topk" and "spade"."""
     names = {"topk": N.SA_MASK_TOPK, "sta": N.SA_MASK_STA,
              "spatiotemporal": N.SA_MASK_SPATIOTEMPORAL, "spade": N.SA_MASK_SPADE,
              "fg": N.SA_MASK_FG, "explicit": N.SA_MASK_EXPLICIT}
@@ -43,6 +45,8 @@ def make_policy(kind, block=128, tile=(1, 1, 128), topk=0, keep_diagonal=False,
     p.fg_group = fg_group
     p.fg_keep_fraction = fg_keep_fraction
     p.explicit_layout = explicit_layout
+    sums = {"mean": N.SA_SUMMARIZER_MEAN, "max": N.SA_SUMMARIZER_MAX, "min": N.SA_SUMMARIZER_MIN}
+    p.summarizer = sums.get(summarizer, summarizer)
     if explicit_bits is not None:
         p.explicit_bits = explicit_bits.data_ptr()
         p._keep_bits = explicit_bits

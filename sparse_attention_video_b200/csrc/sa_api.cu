@@ -54,6 +54,9 @@ int check_policy(const sa_problem& pr, const sa_policy* po) {
     return SA_OK;
   }
   if (po->block != 128 && !(po->block == 64 && pr.head_dim == 64)) return SA_ERR_UNSUPPORTED;
+  if ((po->kind == SA_MASK_TOPK || po->kind == SA_MASK_SPADE) &&
+      (po->summarizer < SA_SUMMARIZER_MEAN || po->summarizer > SA_SUMMARIZER_MIN))
+    return SA_ERR_INVALID_ARG;
   const long long N = n_tokens(pr);
   switch (po->kind) {
     case SA_MASK_TOPK:
@@ -356,6 +359,7 @@ extern "C" int sparse_attn_build_mask(const sa_problem* problem, const sa_policy
     for (int c = 0; c < C; ++c)
       for (int i = 0; i < 3; ++i) pp.cand[c][i] = po.kind == SA_MASK_SPADE ? po.candidates[c][i] : po.tile[i];
     pp.C = C; pp.NB = M.NB; pp.T = pr.T; pp.H = pr.H; pp.W = pr.W; pp.d = d;
+    pp.summarizer = po.summarizer;
     pool_regions(pp);
     if ((e = cuda_status(launch_pool_sics(pp, BH, M.NB, st)))) return e;
     if (po.kind == SA_MASK_SPADE) {

@@ -90,7 +90,22 @@ __global__ void permute_fm_kernel(PermuteParams p) {
 // runs in a fixed order.
 constexpr int kMaxPoolBlock = 128;   // tokens per block (64 or 128)
 
-template <int D>
+// Block summaries (SA_SUMMARIZER_*): the per-channel sum of the valid tokens
+// (divided by their count at the end: the mean), or their maximum / minimum.
+template <int kSum>
+__device__ __forceinline__ float summ_init() {
+  return kSum == SA_SUMMARIZER_MAX ? -INFINITY : (kSum == SA_SUMMARIZER_MIN ? INFINITY : 0.f);
+}
+template <int kSum>
+__device__ __forceinline__ float summ_add(float a, float b) {
+  return kSum == SA_SUMMARIZER_MAX ? fmaxf(a, b) : (kSum == SA_SUMMARIZER_MIN ? fminf(a, b) : a + b);
+}
+template <int kSum>
+__device__ __forceinline__ float summ_final(float a, int n, float inv_n) {
+  return n == 0 ? 0.f : (kSum == SA_SUMMARIZER_MEAN ? a * inv_n : a);
+}
+
+template <int D, int kSum>
 __global__ void __launch_bounds__(256) pool_sics_kernel(PoolParams p) {
   static_assert(D == 128 || D == 64, "head_dim");
   constexpr int CH = D / 8;                 // lanes per token (16 or 8)
@@ -126,7 +141,7 @@ __global__ void __launch_bounds__(256) pool_sics_kernel(PoolParams p) {
 
   float qs[8], ks[8], us[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) { qs[i] = 0.f; ks[i] = 0.f; us[i] = 0.f; }
+  for (int i = 0; i < 8; ++i) { qs[i] = summ_init<kSum>(); ks[i] = summ_init<kSum>(); us[i] = 0.f; }
   int n_valid = 0, n_unit = 0;
   for (int s0 = 0; s0 < BS; s0 += TPW * UNROLL) {
     uint4 qv[UNROLL], kv[UNROLL];
@@ -158,8 +173,8 @@ __global__ void __launch_bounds__(256) pool_sics_kernel(PoolParams p) {
       if (tok[u] < 0) continue;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        qs[i] += __bfloat162float(qe[i]);
-        ks[i] += kf[i];
+        qs[i] = summ_add<kSum>(qs[i], __bfloat162float(qe[i]));
+        ks[i] = summ_add<kSum>(ks[i], kf[i]);
       }
       ++n_valid;
       if (ss > 0.f) {
@@ -177,8 +192,8 @@ __global__ void __launch_bounds__(256) pool_sics_kernel(PoolParams p) {
   for (int o = CH; o < 32; o <<= 1) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      qs[i] += __shfl_xor_sync(0xffffffffu, qs[i], o);
-      ks[i] += __shfl_xor_sync(0xffffffffu, ks[i], o);
+      qs[i] = summ_add<kSum>(qs[i], __shfl_xor_sync(0xffffffffu, qs[i], o));
+      ks[i] = summ_add<kSum>(ks[i], __shfl_xor_sync(0xffffffffu, ks[i], o));
       us[i] += __shfl_xor_sync(0xffffffffu, us[i], o);
     }
     n_valid += __shfl_xor_sync(0xffffffffu, n_valid, o);
@@ -194,15 +209,17 @@ __global__ void __launch_bounds__(256) pool_sics_kernel(PoolParams p) {
   for (int o = CH / 2; o >= 1; o >>= 1) usq += __shfl_xor_sync(0xffffffffu, usq, o);
   if (tl == 0) {
     const float nv = (float)n_valid;
-    float4* qo = reinterpret_cast<float4*>(p.qbar + base * D + dc * 8);
-    float4* ko = reinterpret_cast<float4*>(p.kbar + base * D + dc * 8);
-    if (n_valid) {
-      qo[0] = make_float4(qs[0] / nv, qs[1] / nv, qs[2] / nv, qs[3] / nv);
-      qo[1] = make_float4(qs[4] / nv, qs[5] / nv, qs[6] / nv, qs[7] / nv);
-      ko[0] = make_float4(ks[0] / nv, ks[1] / nv, ks[2] / nv, ks[3] / nv);
-      ko[1] = make_float4(ks[4] / nv, ks[5] / nv, ks[6] / nv, ks[7] / nv);
-    } else {
-      qo[0] = qo[1] = ko[0] = ko[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float* qo = p.qbar + base * D + dc * 8;
+    float* ko = p.kbar + base * D + dc * 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if constexpr (kSum == SA_SUMMARIZER_MEAN) {
+        qo[i] = n_valid ? qs[i] / nv : 0.f;
+        ko[i] = n_valid ? ks[i] / nv : 0.f;
+      } else {
+        qo[i] = n_valid ? qs[i] : 0.f;
+        ko[i] = n_valid ? ks[i] : 0.f;
+      }
     }
     if (dc == 0) p.sics[base] = usq - (float)n_unit;
   }
@@ -219,7 +236,7 @@ __global__ void __launch_bounds__(256) pool_sics_kernel(PoolParams p) {
 // SICS = ||sum of unit vectors||^2 - (number of nonzero keys).
 constexpr int kPoolAtomThreads = 256;     // 8 warps; two CTAs per SM (shared memory)
 
-template <int D>
+template <int D, int kSum>
 __global__ void __launch_bounds__(kPoolAtomThreads) pool_atoms_kernel(PoolParams p) {
   constexpr int CH = D / 8;                 // lanes per token (16 or 8)
   constexpr int TPW = 32 / CH;              // tokens per warp step (2 or 4)
@@ -247,7 +264,7 @@ __global__ void __launch_bounds__(kPoolAtomThreads) pool_atoms_kernel(PoolParams
     const int ta = t0 + at * p.At, ha = h0 + ah * p.Ah, wa = w0 + aw * p.Aw;
     float qs[8], ks[8], us[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) { qs[i] = 0.f; ks[i] = 0.f; us[i] = 0.f; }
+    for (int i = 0; i < 8; ++i) { qs[i] = summ_init<kSum>(); ks[i] = summ_init<kSum>(); us[i] = 0.f; }
     int n_valid = 0, n_unit = 0;
     int iw = iw0, ih = ih0, it = it0;
     // the warp's lanes stay in step: it < At for some lane until the last step
@@ -292,10 +309,18 @@ __global__ void __launch_bounds__(kPoolAtomThreads) pool_atoms_kernel(PoolParams
 #pragma unroll
         for (int o = CH / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         if (tok[u] < 0) continue;
+        if constexpr (kSum == SA_SUMMARIZER_MEAN) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          add2(qs[2 * e], qs[2 * e + 1], qf[2 * e], qf[2 * e + 1]);
-          add2(ks[2 * e], ks[2 * e + 1], kf[2 * e], kf[2 * e + 1]);
+          for (int e = 0; e < 4; ++e) {
+            add2(qs[2 * e], qs[2 * e + 1], qf[2 * e], qf[2 * e + 1]);
+            add2(ks[2 * e], ks[2 * e + 1], kf[2 * e], kf[2 * e + 1]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            qs[i] = summ_add<kSum>(qs[i], qf[i]);
+            ks[i] = summ_add<kSum>(ks[i], kf[i]);
+          }
         }
         ++n_valid;
         if (ss > 0.f) {
@@ -314,8 +339,8 @@ __global__ void __launch_bounds__(kPoolAtomThreads) pool_atoms_kernel(PoolParams
     for (int o = CH; o < 32; o <<= 1) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        qs[i] += __shfl_xor_sync(0xffffffffu, qs[i], o);
-        ks[i] += __shfl_xor_sync(0xffffffffu, ks[i], o);
+        qs[i] = summ_add<kSum>(qs[i], __shfl_xor_sync(0xffffffffu, qs[i], o));
+        ks[i] = summ_add<kSum>(ks[i], __shfl_xor_sync(0xffffffffu, ks[i], o));
         us[i] += __shfl_xor_sync(0xffffffffu, us[i], o);
       }
       n_valid += __shfl_xor_sync(0xffffffffu, n_valid, o);
@@ -350,7 +375,7 @@ __global__ void __launch_bounds__(kPoolAtomThreads) pool_atoms_kernel(PoolParams
     const int blk = (tt * nh + th) * nw + tw;
     float qv[DL], kv[DL], uv[DL];
 #pragma unroll
-    for (int i = 0; i < DL; ++i) { qv[i] = 0.f; kv[i] = 0.f; uv[i] = 0.f; }
+    for (int i = 0; i < DL; ++i) { qv[i] = summ_init<kSum>(); kv[i] = summ_init<kSum>(); uv[i] = 0.f; }
     int nv = 0, nu = 0;
     const int ft = bt / p.At, fh = bhh / p.Ah, fw = bw / p.Aw;   // atoms per block along each axis
     for (int x = 0; x < ft * fh * fw; ++x) {
@@ -358,7 +383,11 @@ __global__ void __launch_bounds__(kPoolAtomThreads) pool_atoms_kernel(PoolParams
       const int a = ((lt * ft + xt) * mAh + (lh * fh + xh)) * mAw + (lw * fw + xw);
       const float* sa = sums + (size_t)a * 3 * D + lane * DL;
 #pragma unroll
-      for (int i = 0; i < DL; ++i) { qv[i] += sa[i]; kv[i] += sa[D + i]; uv[i] += sa[2 * D + i]; }
+      for (int i = 0; i < DL; ++i) {
+        qv[i] = summ_add<kSum>(qv[i], sa[i]);
+        kv[i] = summ_add<kSum>(kv[i], sa[D + i]);
+        uv[i] += sa[2 * D + i];
+      }
       nv += cnt[2 * a];
       nu += cnt[2 * a + 1];
     }
@@ -367,8 +396,8 @@ __global__ void __launch_bounds__(kPoolAtomThreads) pool_atoms_kernel(PoolParams
     float usq = 0.f;
 #pragma unroll
     for (int i = 0; i < DL; ++i) {
-      p.qbar[base * D + lane * DL + i] = nv ? qv[i] * inv : 0.f;
-      p.kbar[base * D + lane * DL + i] = nv ? kv[i] * inv : 0.f;
+      p.qbar[base * D + lane * DL + i] = summ_final<kSum>(qv[i], nv, inv);
+      p.kbar[base * D + lane * DL + i] = summ_final<kSum>(kv[i], nv, inv);
       usq = fmaf(uv[i], uv[i], usq);
     }
 #pragma unroll
@@ -718,30 +747,37 @@ cudaError_t launch_permute_fm(const PermuteParams& p, int BH, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_pool_sics(const PoolParams& p, int BH, int max_nb, cudaStream_t st) {
-  (void)max_nb;
+template <int D, int kSum>
+static cudaError_t launch_pool(const PoolParams& p, int BH, cudaStream_t st) {
   if (p.nA > 0 && p.nA <= kMaxPoolAtoms) {
     const size_t smem = (size_t)p.nA * (3 * p.d + 2) * sizeof(float);
     dim3 grid(p.nRt * p.nRh * p.nRw, BH);
-    cudaError_t e;
-    if (p.d == 128) {
-      if ((e = cudaFuncSetAttribute(pool_atoms_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)smem)) != cudaSuccess) return e;
-      pool_atoms_kernel<128><<<grid, kPoolAtomThreads, smem, st>>>(p);
-    } else if (p.d == 64) {
-      if ((e = cudaFuncSetAttribute(pool_atoms_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)smem)) != cudaSuccess) return e;
-      pool_atoms_kernel<64><<<grid, kPoolAtomThreads, smem, st>>>(p);
-    } else {
-      return cudaErrorInvalidValue;
-    }
+    cudaError_t e = cudaFuncSetAttribute(pool_atoms_kernel<D, kSum>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    pool_atoms_kernel<D, kSum><<<grid, kPoolAtomThreads, smem, st>>>(p);
     return cudaGetLastError();
   }
   dim3 grid(p.C, p.nRt * p.nRh * p.nRw, BH);
-  if (p.d == 128) pool_sics_kernel<128><<<grid, 256, 0, st>>>(p);
-  else if (p.d == 64) pool_sics_kernel<64><<<grid, 256, 0, st>>>(p);
-  else return cudaErrorInvalidValue;
+  pool_sics_kernel<D, kSum><<<grid, 256, 0, st>>>(p);
   return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_pool_d(const PoolParams& p, int BH, cudaStream_t st) {
+  switch (p.summarizer) {
+    case SA_SUMMARIZER_MEAN: return launch_pool<D, SA_SUMMARIZER_MEAN>(p, BH, st);
+    case SA_SUMMARIZER_MAX: return launch_pool<D, SA_SUMMARIZER_MAX>(p, BH, st);
+    case SA_SUMMARIZER_MIN: return launch_pool<D, SA_SUMMARIZER_MIN>(p, BH, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_pool_sics(const PoolParams& p, int BH, int max_nb, cudaStream_t st) {
+  (void)max_nb;
+  if (p.d == 128) return launch_pool_d<128>(p, BH, st);
+  if (p.d == 64) return launch_pool_d<64>(p, BH, st);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_choose(const ChooseParams& p, int BH, cudaStream_t st) {

@@ -36,6 +36,7 @@ struct PoolParams {
   int nRt, nRh, nRw;                // regions covering every candidate's tile grid
   int At, Ah, Aw;                   // atom: gcd of the candidates' tiles (one block of each)
   int nA;                           // atoms per region; 0 = per-candidate kernel
+  int summarizer;                   // SA_SUMMARIZER_*: per-channel mean, max or min
 };
 
 // Atoms per region the one-pass pooling kernel holds in shared memory.

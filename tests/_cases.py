@@ -18,7 +18,7 @@ REL_TIE = 1e-4
 def policy_kwargs(wl: Workload):
     if wl.kind == "topk":
         return dict(kind="topk", block=wl.block, tile=wl.tile, topk=wl.topk,
-                    keep_diagonal=wl.keep_diagonal)
+                    keep_diagonal=wl.keep_diagonal, summarizer=wl.summarizer)
     if wl.kind == "sta":
         return dict(kind="sta", block=wl.block, tile=wl.tile, window=wl.window)
     if wl.kind == "spatiotemporal":
@@ -26,7 +26,7 @@ def policy_kwargs(wl: Workload):
                     heads=wl.heads, sink_tokens=wl.sink_tokens, frame_radius=1)
     if wl.kind == "spade":
         return dict(kind="spade", block=wl.block, candidates=wl.candidates, top_p=wl.top_p,
-                    window=wl.window)
+                    window=wl.window, summarizer=wl.summarizer)
     if wl.kind == "fg":
         return dict(kind="fg", block=wl.block, fg_group=wl.fg_group,
                     fg_keep_fraction=wl.fg_keep_fraction)
@@ -60,6 +60,18 @@ SMALL = {
                                     heads=2, head_dim=128, kind="spade", block=128,
                                     candidates=((1, 1, 128), (8, 4, 4)), top_p=0.9,
                                     window=(3, 3, 3)),
+    # max / min block summaries (SPADE review, minor comment 3): the atom
+    # pooling kernel, the per-candidate kernel and Top-K
+    "spade_max": Workload(name="spade_max", config_id=108, T=7, H=13, W=24, heads=3,
+                          head_dim=128, kind="spade", block=128,
+                          candidates=((1, 8, 16), (8, 4, 4), (2, 8, 8)), top_p=0.9,
+                          window=(3, 3, 3), summarizer="max"),
+    "spade_fallback_min": Workload(name="spade_fallback_min", config_id=109, T=8, H=6, W=136,
+                                   heads=2, head_dim=128, kind="spade", block=128,
+                                   candidates=((1, 1, 128), (8, 4, 4)), top_p=0.9,
+                                   window=(3, 3, 3), summarizer="min"),
+    "topk_max_d64": CONFIGS["tiny_topk"].with_(name="topk_max_d64", config_id=110,
+                                               summarizer="max"),
 }
 
 
