@@ -7,3 +7,4 @@ inputs made here, so that both sides see identical bits.
 """
 from .configs import CONFIGS, Workload, get_config  # noqa: F401
 from .fields import make_qkv, bf16_bits_to_f32, f32_to_bf16_bits  # noqa: F401
+from .sampling import sample_rows  # noqa: F401
