@@ -236,6 +236,34 @@ SA_API int sparse_attn_mask_export(const sa_problem* problem, const sa_policy* p
  * SA_ERR_DEVICE_BOUNDS. If ``clear`` is nonzero the word is reset. */
 SA_API int sparse_attn_status(void* scratch_ws, void* stream, int clear);
 
+/* ---------------------------------------------------------------- profiler
+ * SVG online head profiler (Sparse VideoGen review, key machinery; Algorithm
+ * 1). For every head, on the sampled query rows ``rows``, attention is
+ * evaluated over all keys, over the spatial pattern's keys and over the
+ * temporal pattern's keys. These are the block masks SA_MASK_SPATIOTEMPORAL
+ * builds for spatial and temporal heads: ``policy->block``,
+ * ``sink_tokens`` and ``frame_radius`` apply, and ``head_is_temporal`` is
+ * not read. A head is temporal when its temporal output's mean squared error
+ * against the full output is below the spatial one's; a tie is spatial.
+ *
+ *   rows         device int32 [batch*heads][n_rows]: token indices in
+ *                original order, 1 <= n_rows <= N. Any order; ascending
+ *                keeps each warp's rows in few frames. A token outside
+ *                [0, N) sets the bounds flag and is skipped.
+ *   row_err      device float [batch*heads][n_rows][2]: per row, the sum over
+ *                head_dim of (O_spatial - O_full)^2, then of (O_temporal - O_full)^2.
+ *   mse          device float [batch*heads][2]: those sums over the rows,
+ *                divided by n_rows * head_dim (fixed summation order).
+ *   is_temporal  device int8 [batch*heads]: the decision.
+ *   scratch_ws   optional (may be null): its status word receives the bounds flag.
+ * Q/K/V as for the forward pass. Asynchronous on ``stream``; the caller owns
+ * every buffer. Returns SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED or
+ * SA_ERR_CUDA. */
+SA_API int sparse_attn_profile_heads(const sa_problem* problem, const sa_policy* policy,
+                                     const void* q, const void* k, const void* v,
+                                     const int32_t* rows, int n_rows, float* row_err, float* mse,
+                                     int8_t* is_temporal, void* scratch_ws, void* stream);
+
 /* Failure-path self-test: launches one CTA on ``stream`` that waits, with the
  * bounded wait every kernel of this library uses, on a barrier that nothing
  * completes. After about one second the wait gives up and records

@@ -27,7 +27,7 @@ EXPORTED = ("sparse_attn_workspace_size", "sparse_attn_build_mask", "sparse_attn
             "sparse_attn_permute", "sparse_attn_attend",
             "sparse_attn_export_bytes", "sparse_attn_mask_export", "sparse_attn_status",
             "sparse_attn_build_mask_static", "sparse_attn_selftest_wait_timeout",
-            "sparse_attn_strerror")
+            "sparse_attn_profile_heads", "sparse_attn_strerror")
 
 SA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
 
@@ -85,6 +85,8 @@ def lib():
         L.sparse_attn_status.argtypes = [vp, vp, ctypes.c_int]
         L.sparse_attn_build_mask_static.argtypes = [P, PP, vp, vp, vp, vp]
         L.sparse_attn_selftest_wait_timeout.argtypes = [vp, vp]
+        L.sparse_attn_profile_heads.argtypes = [P, PP, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp,
+                                                vp, vp]
         L.sparse_attn_strerror.argtypes = [ctypes.c_int]
         L.sparse_attn_strerror.restype = ctypes.c_char_p
         for name in EXPORTED[:-1]:
@@ -132,6 +134,14 @@ def attend(problem, policy, q, k, v, mask_ws, scratch_ws, o, lse, stream=0):
     _check(lib().sparse_attn_attend(ctypes.byref(problem), ctypes.byref(policy), q, k, v,
                                     mask_ws, scratch_ws, o, lse, stream),
            "sparse_attn_attend")
+
+
+def profile_heads(problem, policy, q, k, v, rows, n_rows, row_err, mse, is_temporal,
+                  scratch_ws=None, stream=0):
+    _check(lib().sparse_attn_profile_heads(ctypes.byref(problem), ctypes.byref(policy), q, k, v,
+                                           rows, n_rows, row_err, mse, is_temporal, scratch_ws,
+                                           stream),
+           "sparse_attn_profile_heads")
 
 
 def export_bytes(problem, policy, what):

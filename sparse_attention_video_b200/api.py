@@ -135,3 +135,33 @@ class SparseAttention:
 
     def status(self, clear=False, stream=None):
         return N.status(self.scratch_ws.data_ptr(), _stream_ptr(stream), clear)
+
+
+def profile_heads(q, k, v, rows, T, H, W, block=128, sink_tokens=0, frame_radius=1,
+                  stream=None, scratch_ws=None):
+    """SVG online head profiler (Sparse VideoGen review, key machinery).
+
+    q, k, v: contiguous CUDA bf16 [batch, heads, N, d]; rows: CUDA int32
+    [batch*heads, n_rows] sampled query tokens. Returns (is_temporal int8
+    [batch*heads], mse float32 [batch*heads, 2], row_err float32
+    [batch*heads, n_rows, 2]) as CUDA tensors; the work is queued on
+    ``stream`` and nothing is synchronised.
+    """
+    B, Hh, N_, d = q.shape
+    problem = N.Problem(B, Hh, T, H, W, d)
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        _check_qkv(t, problem, name)
+    if rows.dtype != torch.int32 or not rows.is_cuda or not rows.is_contiguous() \
+            or rows.dim() != 2 or rows.shape[0] != B * Hh:
+        raise ValueError("rows must be a contiguous CUDA int32 tensor [batch*heads, n_rows]")
+    n_rows = rows.shape[1]
+    policy = make_policy("spatiotemporal", block=block, temporal_heads=(), heads=Hh,
+                         sink_tokens=sink_tokens, frame_radius=frame_radius)
+    dev = q.device
+    row_err = torch.empty((B * Hh, n_rows, 2), dtype=torch.float32, device=dev)
+    mse = torch.empty((B * Hh, 2), dtype=torch.float32, device=dev)
+    is_temporal = torch.empty(B * Hh, dtype=torch.int8, device=dev)
+    N.profile_heads(problem, policy, q.data_ptr(), k.data_ptr(), v.data_ptr(), rows.data_ptr(),
+                    n_rows, row_err.data_ptr(), mse.data_ptr(), is_temporal.data_ptr(),
+                    scratch_ws.data_ptr() if scratch_ws is not None else None, _stream_ptr(stream))
+    return is_temporal, mse, row_err

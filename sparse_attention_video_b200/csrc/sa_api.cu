@@ -12,6 +12,7 @@
 #include "sa_fg.h"
 #include "sa_internal.h"
 #include "sa_mask.h"
+#include "sa_profile.h"
 
 using namespace sa;
 
@@ -567,6 +568,45 @@ extern "C" int sparse_attn_mask_export(const sa_problem* problem, const sa_polic
                       cudaMemcpyDeviceToHost, st) != cudaSuccess)
     return SA_ERR_CUDA;
   return cuda_status(cudaStreamSynchronize(st));
+}
+
+extern "C" int sparse_attn_profile_heads(const sa_problem* problem, const sa_policy* policy,
+                                         const void* q, const void* k, const void* v,
+                                         const int32_t* rows, int n_rows, float* row_err,
+                                         float* mse, int8_t* is_temporal, void* scratch_ws,
+                                         void* stream) {
+  int e = check_problem(problem);
+  if (e) return e;
+  if (!policy || policy->kind != SA_MASK_SPATIOTEMPORAL) return SA_ERR_INVALID_ARG;
+  const sa_problem& pr = *problem;
+  const sa_policy& po = *policy;
+  if (po.block != 128 && !(po.block == 64 && pr.head_dim == 64)) return SA_ERR_UNSUPPORTED;
+  if (po.sink_tokens < 0 || po.frame_radius < 0) return SA_ERR_INVALID_ARG;
+  const long long N = n_tokens(pr);
+  if (n_rows < 1 || n_rows > N) return SA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return SA_ERR_INVALID_ARG;
+  if (!aligned(rows, 4) || !aligned(row_err, 4) || !aligned(mse, 4) || !is_temporal)
+    return SA_ERR_INVALID_ARG;
+  if (scratch_ws && !aligned(scratch_ws, 256)) return SA_ERR_WORKSPACE;
+  ProfileParams pp{};
+  pp.q = static_cast<const __nv_bfloat16*>(q);
+  pp.k = static_cast<const __nv_bfloat16*>(k);
+  pp.v = static_cast<const __nv_bfloat16*>(v);
+  pp.rows = rows;
+  pp.row_err = row_err;
+  pp.mse = mse;
+  pp.is_temporal = is_temporal;
+  pp.status = scratch_ws ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(scratch_ws) +
+                                                       ScratchLayout{}.off_status)
+                         : nullptr;
+  pp.BH = pr.batch * pr.heads;
+  pp.N = (int)N; pp.T = pr.T; pp.H = pr.H; pp.W = pr.W; pp.d = pr.head_dim;
+  pp.n_rows = n_rows;
+  pp.block = po.block;
+  pp.sink_blocks = ceil_div(po.sink_tokens, po.block);
+  pp.frame_radius = po.frame_radius;
+  pp.scale_log2 = 1.4426950408889634f / sqrtf((float)pr.head_dim);
+  return cuda_status(launch_profile(pp, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 extern "C" int sparse_attn_status(void* scratch_ws, void* stream, int clear) {
