@@ -44,6 +44,8 @@ def _args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-mask comparison")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-profile", action="store_true",
+                    help="skip the head-profiler timing (spatial/temporal workload only)")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="workload name (synthetic.CONFIGS); the bench line uses the default")
     ap.add_argument("--heads", type=int, default=0,
@@ -394,6 +396,34 @@ def main():
                  "speedup_vs_dense_mask": dense_ms / attn_ms}
         del dsa, words
 
+    # ---- the head profiler (Sparse VideoGen review, key machinery) on 1 % of
+    # each head's query rows; reported beside the step, not part of it
+    prof = {}
+    if not args.no_profile and wl.kind == "spatiotemporal":
+        from sparse_attention_video_b200 import profile_heads
+        from synthetic import sample_rows
+        rows = torch.from_numpy(sample_rows(wl.N, wl.heads, 0.01, seed=2024)).to(dev)
+        for _ in range(2):
+            profile_heads(q, k, v, rows, wl.T, wl.H, wl.W, block=wl.block,
+                          sink_tokens=wl.sink_tokens, stream=stream)
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        p0.record(stream)
+        for _ in range(5):
+            is_t, _, _ = profile_heads(q, k, v, rows, wl.T, wl.H, wl.W, block=wl.block,
+                                       sink_tokens=wl.sink_tokens, stream=stream)
+        p1.record(stream)
+        torch.cuda.synchronize(dev)
+        prof_ms = p0.elapsed_time(p1) / 5
+        # the full pass alone: every sampled row against every key
+        full_flops = 4.0 * wl.head_dim * rows.numel() * wl.N
+        prof = {"profile_heads": {
+            "ms": prof_ms, "rows_per_head": int(rows.shape[1]),
+            "full_pass_tflops": full_flops / (prof_ms * 1e-3) / 1e12,
+            "temporal_heads_found": int(is_t.sum().item()),
+            "kernel": "profile_kernel (mma.sync m16n8k16; all three passes in the time)"}}
+        log("head profiler timed")
+
     if rank != 0:
         if world > 1:
             dist.barrier()
@@ -435,6 +465,7 @@ def main():
         "gpu_launches": LAUNCHES_PER_STEP[wl.kind] * args.steps,
         "clocks": clk,
         **dense,
+        **prof,
     }
     print(json.dumps(line), flush=True)
     if world > 1:
