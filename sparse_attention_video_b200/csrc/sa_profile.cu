@@ -7,13 +7,14 @@
 // layout with frames within +-frame_radius, and frame-major layout with a
 // shared spatial position, both with the sink blocks.
 //
-// One warp owns 16 sampled rows. Keys stream 16 at a time through a
-// double-buffered, XOR-swizzled shared-memory tile filled by cp.async;
-// ldmatrix forms the fragments and mma.sync m16n8k16 (bf16 in, fp32
-// accumulate) computes S = Q K^T and O += P V with an online softmax in
-// registers. The spatial pass walks key blocks in original order and the
-// temporal pass in frame-major order (K/V rows gathered by token); each visits
-// only the blocks that some row of the warp keeps.
+// One warp owns 16 sampled rows. Keys pass through XOR-swizzled shared-memory
+// tiles filled by cp.async (double-buffered); ldmatrix forms the fragments and
+// mma.sync m16n8k16 (bf16 in, fp32 accumulate) computes S = Q K^T and
+// O += P V with an online softmax in registers. The full pass streams every
+// key once per CTA, 64 at a time, for all four warps' rows; the spatial pass
+// then walks key blocks in original order and the temporal pass in
+// frame-major order (K/V rows gathered by token), per warp, each visiting only
+// the blocks that some row of the warp keeps.
 #include "sa_profile.h"
 #include "sa_ptx.cuh"
 
@@ -25,15 +26,22 @@ constexpr int kProfWarps = 4;
 constexpr int kRowsPerWarp = 16;
 constexpr int kStepKeys = 16;
 
+// Shared memory of a CTA: one K/V region, then per warp its Q tile and the
+// O of the full pass. The full pass streams every key through the region as
+// one double-buffered tile of 64 keys read by all warps; the masked passes cut
+// the same bytes into one double-buffered 16-key K/V pair per warp.
 template <int D>
 struct ProfSmem {
-  static constexpr int kTile = kStepKeys * D * 2;          // 16 bf16 rows
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kTile;
-  static constexpr int kOffV = kOffK + 2 * kTile;          // K and V double-buffered
-  static constexpr int kOffO = kOffV + 2 * kTile;          // fp32 [16][D]: O of the full pass
-  static constexpr int kPerWarp = kOffO + kRowsPerWarp * D * 4;
-  static constexpr int kBytes = kProfWarps * kPerWarp;
+  static constexpr int kRow = D * 2;                       // one bf16 row
+  static constexpr int kTile16 = kStepKeys * kRow;         // 16 rows (one step)
+  static constexpr int kCoopKeys = 64;
+  static constexpr int kCoopTile = kCoopKeys * kRow;       // full pass: 64 rows of K or V
+  static constexpr int kKV = 4 * kCoopTile;                // 2 buffers x (K, V)
+  static_assert(kKV == kProfWarps * 4 * kTile16, "masked passes: K, V x 2 buffers per warp");
+  static constexpr int kOffWarp = kKV;
+  static constexpr int kQ = kTile16;
+  static constexpr int kPerWarp = kQ + kRowsPerWarp * D * 4;
+  static constexpr int kBytes = kKV + kProfWarps * kPerWarp;
 };
 
 // Byte offset of 16-byte chunk c of row r in a tile of D bf16 per row: chunks
@@ -98,12 +106,10 @@ __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bh = blockIdx.y;
   const int row0 = (blockIdx.x * kProfWarps + warp) * kRowsPerWarp;
-  if (row0 >= p.n_rows) return;                            // no CTA-wide barrier below
-  uint8_t* ws = prof_smem + warp * L::kPerWarp;
-  uint8_t* sQ = ws + L::kOffQ;
-  uint8_t* sK = ws + L::kOffK;
-  uint8_t* sV = ws + L::kOffV;
-  float* sO = reinterpret_cast<float*>(ws + L::kOffO);
+  const bool has_rows = row0 < p.n_rows;                   // warp-uniform
+  uint8_t* kv = prof_smem;
+  uint8_t* sQ = prof_smem + L::kOffWarp + warp * L::kPerWarp;
+  float* sO = reinterpret_cast<float*>(sQ + L::kQ);
   const size_t head = (size_t)bh * p.N * D;
   const __nv_bfloat16* q = p.q + head;
   const __nv_bfloat16* k = p.k + head;
@@ -114,7 +120,7 @@ __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams 
 
   // lane r < 16 holds the token of the warp's row r (-1: no row)
   int my_tok = -1;
-  if (lane < kRowsPerWarp && row0 + lane < p.n_rows) {
+  if (has_rows && lane < kRowsPerWarp && row0 + lane < p.n_rows) {
     my_tok = p.rows[(size_t)bh * p.n_rows + row0 + lane];
     if (my_tok < 0 || my_tok >= p.N) {
       if (p.status) atomicOr(p.status, SA_DEVFLAG_BOUNDS);
@@ -140,132 +146,77 @@ __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams 
   }
   const int g = lane / 4, cq = 2 * (lane % 4);             // fragment row and column pair
 
-  for (int pass = 0; pass < 3; ++pass) {
-    const bool fm = pass == 2;
-    // rows (bits 0..15) that keep key block b under this pass's pattern
-    auto keeps = [&](int b) -> uint32_t {
-      bool kp = false;
-      if (my_tok >= 0)
-        kp = pass == 0 ? true : (pass == 1 ? spatial_keep(geo, my_tok, b) : temporal_keep(geo, my_tok, b));
-      return __ballot_sync(0xffffffffu, kp) & 0xFFFFu;
-    };
-    auto next_block = [&](int from, uint32_t& rmask) -> int {
-      for (int x = from; x < nb; ++x) {
-        const uint32_t mk = keeps(x);
-        if (mk) { rmask = mk; return x; }
-      }
-      return nb;
-    };
-    // 16 key rows of step (b, sub) into buffer ``buf``; slots past N are zero
-    auto load_step = [&](int buf, int b, int sub) {
-      for (int e = lane; e < kStepKeys * kChunks; e += 32) {
-        const int r = e / kChunks, c = e % kChunks;
-        const int slot = b * p.block + sub * kStepKeys + r;
-        uint8_t* dk = sK + buf * L::kTile + tile_off<D>(r, c);
-        uint8_t* dv = sV + buf * L::kTile + tile_off<D>(r, c);
-        if (slot < p.N) {
-          const int tok = fm ? (slot % p.T) * geo.HW + slot / p.T : slot;
-          cp_async16(dk, k + (size_t)tok * D + c * 8);
-          cp_async16(dv, v + (size_t)tok * D + c * 8);
-        } else {
-          *reinterpret_cast<uint4*>(dk) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(dv) = make_uint4(0, 0, 0, 0);
-        }
-      }
-      cp_async_commit();
-    };
-
-    float acc[D / 8][4];
+  float acc[D / 8][4];
+  float m0, m1, l0, l1;                                    // rows g and g + 8
+  auto reset = [&]() {
 #pragma unroll
     for (int j = 0; j < D / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // rows g and g + 8
-
-    uint32_t rmask = 0;
-    int b = next_block(0, rmask), sub = 0, buf = 0;
-    if (b < nb) load_step(0, b, 0);
-    while (b < nb) {
-      int b2 = b, s2 = sub + 1;
-      uint32_t rm2 = rmask;
-      if (s2 == subs) { s2 = 0; b2 = next_block(b + 1, rm2); }
-      if (b2 < nb) {
-        load_step(buf ^ 1, b2, s2);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
-      __syncwarp();
-      const uint8_t* tK = sK + buf * L::kTile;
-      const uint8_t* tV = sV + buf * L::kTile;
-      // S = Q K^T: keys 0-7 (n-tile 0) and 8-15 (n-tile 1)
-      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-      {
-        const int m = lane / 8, i = lane % 8;
+    m0 = m1 = -INFINITY;
+    l0 = l1 = 0.f;
+  };
+  // One step of 16 keys (slots slot0..slot0+15 of the pass's order) from
+  // 16-row tiles tK, tV; rows outside ``rmask`` and slots past N are masked.
+  auto step16 = [&](const uint8_t* tK, const uint8_t* tV, int slot0, uint32_t rmask) {
+    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      const int m = lane / 8, i = lane % 8;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          uint32_t b00, b01, b10, b11;
-          ldsm_x4(tK + tile_off<D>((m >> 1) * 8 + i, 2 * ks + (m & 1)), b00, b01, b10, b11);
-          mma16816(s0, qa[ks], b00, b01);
-          mma16816(s1, qa[ks], b10, b11);
-        }
+      for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t b00, b01, b10, b11;
+        ldsm_x4(tK + tile_off<D>((m >> 1) * 8 + i, 2 * ks + (m & 1)), b00, b01, b10, b11);
+        mma16816(s0, qa[ks], b00, b01);
+        mma16816(s1, qa[ks], b10, b11);
       }
-      // scores in log2 units; keys past N and rows that drop this block: -inf
-      const int slot0 = b * p.block + sub * kStepKeys;
-      const bool keep0 = (rmask >> g) & 1u, keep1 = (rmask >> (g + 8)) & 1u;
-      float x[8];
-      {
-        const bool v00 = slot0 + cq < p.N, v01 = slot0 + cq + 1 < p.N;
-        const bool v10 = slot0 + 8 + cq < p.N, v11 = slot0 + 8 + cq + 1 < p.N;
-        x[0] = keep0 && v00 ? s0[0] * p.scale_log2 : -INFINITY;   // row g,     key cq
-        x[1] = keep0 && v01 ? s0[1] * p.scale_log2 : -INFINITY;   // row g,     key cq + 1
-        x[2] = keep1 && v00 ? s0[2] * p.scale_log2 : -INFINITY;   // row g + 8, key cq
-        x[3] = keep1 && v01 ? s0[3] * p.scale_log2 : -INFINITY;
-        x[4] = keep0 && v10 ? s1[0] * p.scale_log2 : -INFINITY;   // row g,     key 8 + cq
-        x[5] = keep0 && v11 ? s1[1] * p.scale_log2 : -INFINITY;
-        x[6] = keep1 && v10 ? s1[2] * p.scale_log2 : -INFINITY;   // row g + 8, key 8 + cq
-        x[7] = keep1 && v11 ? s1[3] * p.scale_log2 : -INFINITY;
-      }
-      float mx0 = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[4], x[5]));
-      float mx1 = fmaxf(fmaxf(x[2], x[3]), fmaxf(x[6], x[7]));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-      const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
-      const float a0 = ex2_approx(m0 - u0), a1 = ex2_approx(m1 - u1);   // 0 while m = -inf
-      m0 = n0;
-      m1 = n1;
-      float pr[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) pr[e] = ex2_approx(x[e] - ((e & 2) ? u1 : u0));
-      l0 = l0 * a0 + (pr[0] + pr[1]) + (pr[4] + pr[5]);
-      l1 = l1 * a1 + (pr[2] + pr[3]) + (pr[6] + pr[7]);
-#pragma unroll
-      for (int j = 0; j < D / 8; ++j) {
-        acc[j][0] *= a0; acc[j][1] *= a0;
-        acc[j][2] *= a1; acc[j][3] *= a1;
-      }
-      // P as the A fragment of the 16-key step (the accumulator layout of
-      // the two n-tiles is the A layout of one k16 step)
-      const uint32_t pa[4] = {pack_bf16x2(pr[0], pr[1]), pack_bf16x2(pr[2], pr[3]),
-                              pack_bf16x2(pr[4], pr[5]), pack_bf16x2(pr[6], pr[7])};
-      {
-        const int m = lane / 8, i = lane % 8;
-#pragma unroll
-        for (int np = 0; np < D / 16; ++np) {
-          uint32_t v0, v1, v2, v3;
-          ldsm_x4_t(tV + tile_off<D>((m & 1) * 8 + i, 2 * np + (m >> 1)), v0, v1, v2, v3);
-          mma16816(acc[2 * np], pa, v0, v1);
-          mma16816(acc[2 * np + 1], pa, v2, v3);
-        }
-      }
-      __syncwarp();                                       // tile free for the load two steps on
-      buf ^= 1;
-      b = b2;
-      sub = s2;
-      rmask = rm2;
     }
-    // rows' sums over the four lanes that share them, then O = acc / l
+    const bool keep0 = (rmask >> g) & 1u, keep1 = (rmask >> (g + 8)) & 1u;
+    const bool v00 = slot0 + cq < p.N, v01 = slot0 + cq + 1 < p.N;
+    const bool v10 = slot0 + 8 + cq < p.N, v11 = slot0 + 8 + cq + 1 < p.N;
+    float x[8];
+    x[0] = keep0 && v00 ? s0[0] * p.scale_log2 : -INFINITY;   // row g,     key cq
+    x[1] = keep0 && v01 ? s0[1] * p.scale_log2 : -INFINITY;   // row g,     key cq + 1
+    x[2] = keep1 && v00 ? s0[2] * p.scale_log2 : -INFINITY;   // row g + 8, key cq
+    x[3] = keep1 && v01 ? s0[3] * p.scale_log2 : -INFINITY;
+    x[4] = keep0 && v10 ? s1[0] * p.scale_log2 : -INFINITY;   // row g,     key 8 + cq
+    x[5] = keep0 && v11 ? s1[1] * p.scale_log2 : -INFINITY;
+    x[6] = keep1 && v10 ? s1[2] * p.scale_log2 : -INFINITY;   // row g + 8, key 8 + cq
+    x[7] = keep1 && v11 ? s1[3] * p.scale_log2 : -INFINITY;
+    float mx0 = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[4], x[5]));
+    float mx1 = fmaxf(fmaxf(x[2], x[3]), fmaxf(x[6], x[7]));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+    const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
+    const float a0 = ex2_approx(m0 - u0), a1 = ex2_approx(m1 - u1);   // 0 while m = -inf
+    m0 = n0;
+    m1 = n1;
+    float pr[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) pr[e] = ex2_approx(x[e] - ((e & 2) ? u1 : u0));
+    l0 = l0 * a0 + (pr[0] + pr[1]) + (pr[4] + pr[5]);
+    l1 = l1 * a1 + (pr[2] + pr[3]) + (pr[6] + pr[7]);
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+      acc[j][0] *= a0; acc[j][1] *= a0;
+      acc[j][2] *= a1; acc[j][3] *= a1;
+    }
+    // P as the A fragment of the 16-key step (the accumulator layout of the
+    // two n-tiles is the A layout of one k16 step)
+    const uint32_t pa[4] = {pack_bf16x2(pr[0], pr[1]), pack_bf16x2(pr[2], pr[3]),
+                            pack_bf16x2(pr[4], pr[5]), pack_bf16x2(pr[6], pr[7])};
+    const int m = lane / 8, i = lane % 8;
+#pragma unroll
+    for (int np = 0; np < D / 16; ++np) {
+      uint32_t v0, v1, v2, v3;
+      ldsm_x4_t(tV + tile_off<D>((m & 1) * 8 + i, 2 * np + (m >> 1)), v0, v1, v2, v3);
+      mma16816(acc[2 * np], pa, v0, v1);
+      mma16816(acc[2 * np + 1], pa, v2, v3);
+    }
+  };
+  // rows' sums over the four lanes that share them, O = acc / l; the full
+  // pass keeps O, a masked pass writes each row's squared error against it
+  auto finish = [&](int pass) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
@@ -300,6 +251,115 @@ __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams 
         if (row0 + g + 8 < p.n_rows) re[(size_t)(g + 8) * 2] = e1;
       }
     }
+  };
+
+  // ---- full pass: every key, in original order, 64 keys per CTA step
+  {
+    reset();
+    const uint32_t rmask = __ballot_sync(0xffffffffu, my_tok >= 0) & 0xFFFFu;
+    const int nsteps = (p.N + L::kCoopKeys - 1) / L::kCoopKeys;
+    auto load64 = [&](int buf, int st) {
+      uint8_t* dK = kv + buf * 2 * L::kCoopTile;
+      uint8_t* dV = dK + L::kCoopTile;
+      for (int e = threadIdx.x; e < L::kCoopKeys * kChunks; e += 32 * kProfWarps) {
+        const int r = e / kChunks, c = e % kChunks;
+        const int slot = st * L::kCoopKeys + r;
+        if (slot < p.N) {
+          cp_async16(dK + tile_off<D>(r, c), k + (size_t)slot * D + c * 8);
+          cp_async16(dV + tile_off<D>(r, c), v + (size_t)slot * D + c * 8);
+        } else {
+          *reinterpret_cast<uint4*>(dK + tile_off<D>(r, c)) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(dV + tile_off<D>(r, c)) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      cp_async_commit();
+    };
+    load64(0, 0);
+    for (int st = 0; st < nsteps; ++st) {
+      const int buf = st & 1;
+      if (st + 1 < nsteps) {
+        load64(buf ^ 1, st + 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();
+      if (has_rows) {
+        const uint8_t* tK = kv + buf * 2 * L::kCoopTile;
+        const uint8_t* tV = tK + L::kCoopTile;
+        for (int sub = 0; sub < L::kCoopKeys / kStepKeys; ++sub) {
+          const int slot0 = st * L::kCoopKeys + sub * kStepKeys;
+          if (slot0 < p.N) step16(tK + sub * L::kTile16, tV + sub * L::kTile16, slot0, rmask);
+        }
+      }
+      __syncthreads();                                    // the buffer is refilled next step
+    }
+    if (has_rows) finish(0);
+  }
+  // the shared region becomes four per-warp K/V pairs (every warp is past the
+  // full pass's last read of it)
+  __syncthreads();
+  if (!has_rows) return;
+  uint8_t* sK = kv + warp * 4 * L::kTile16;                // 2 K buffers, then 2 V buffers
+  uint8_t* sV = sK + 2 * L::kTile16;
+
+  // ---- masked passes, per warp: spatial (original order), temporal (frame-major)
+  for (int pass = 1; pass < 3; ++pass) {
+    const bool fm = pass == 2;
+    // rows (bits 0..15) that keep key block b under this pass's pattern
+    auto keeps = [&](int b) -> uint32_t {
+      bool kp = false;
+      if (my_tok >= 0) kp = pass == 1 ? spatial_keep(geo, my_tok, b) : temporal_keep(geo, my_tok, b);
+      return __ballot_sync(0xffffffffu, kp) & 0xFFFFu;
+    };
+    auto next_block = [&](int from, uint32_t& rmask) -> int {
+      for (int x = from; x < nb; ++x) {
+        const uint32_t mk = keeps(x);
+        if (mk) { rmask = mk; return x; }
+      }
+      return nb;
+    };
+    // 16 key rows of step (b, sub) into buffer ``buf``; slots past N are zero
+    auto load_step = [&](int buf, int b, int sub) {
+      for (int e = lane; e < kStepKeys * kChunks; e += 32) {
+        const int r = e / kChunks, c = e % kChunks;
+        const int slot = b * p.block + sub * kStepKeys + r;
+        uint8_t* dk = sK + buf * L::kTile16 + tile_off<D>(r, c);
+        uint8_t* dv = sV + buf * L::kTile16 + tile_off<D>(r, c);
+        if (slot < p.N) {
+          const int tok = fm ? (slot % p.T) * geo.HW + slot / p.T : slot;
+          cp_async16(dk, k + (size_t)tok * D + c * 8);
+          cp_async16(dv, v + (size_t)tok * D + c * 8);
+        } else {
+          *reinterpret_cast<uint4*>(dk) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(dv) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      cp_async_commit();
+    };
+    reset();
+    uint32_t rmask = 0;
+    int b = next_block(0, rmask), sub = 0, buf = 0;
+    if (b < nb) load_step(0, b, 0);
+    while (b < nb) {
+      int b2 = b, s2 = sub + 1;
+      uint32_t rm2 = rmask;
+      if (s2 == subs) { s2 = 0; b2 = next_block(b + 1, rm2); }
+      if (b2 < nb) {
+        load_step(buf ^ 1, b2, s2);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncwarp();
+      step16(sK + buf * L::kTile16, sV + buf * L::kTile16, b * p.block + sub * kStepKeys, rmask);
+      __syncwarp();                                       // tile free for the load two steps on
+      buf ^= 1;
+      b = b2;
+      sub = s2;
+      rmask = rm2;
+    }
+    finish(pass);
   }
 }
 
