@@ -237,10 +237,10 @@ __global__ void __launch_bounds__(256) pool_sics_kernel(PoolParams p) {
 constexpr int kPoolAtomThreads = 256;     // 8 warps; two CTAs per SM (shared memory)
 
 template <int D, int kSum>
-__global__ void __launch_bounds__(kPoolAtomThreads) pool_atoms_kernel(PoolParams p) {
+__global__ void __launch_bounds__(kPoolAtomThreads, 2) pool_atoms_kernel(PoolParams p) {
   constexpr int CH = D / 8;                 // lanes per token (16 or 8)
   constexpr int TPW = 32 / CH;              // tokens per warp step (2 or 4)
-  constexpr int UNROLL = 4;
+  constexpr int UNROLL = 8;                 // a 16-token atom's rows all in flight
   extern __shared__ float pool_sm[];        // [nA][3][D] sums, then [nA][2] counts
   float* sums = pool_sm;
   int* cnt = reinterpret_cast<int*>(pool_sm + (size_t)p.nA * 3 * D);
@@ -259,9 +259,26 @@ __global__ void __launch_bounds__(kPoolAtomThreads) pool_atoms_kernel(PoolParams
   const int iw0 = tl % p.Aw, ih0 = (tl / p.Aw) % p.Ah, it0 = tl / (p.Aw * p.Ah);
 
   constexpr int kWarps = kPoolAtomThreads / 32;
+  // atom a = (at, ah, aw) of the region; this warp takes a = warp, warp + 8,
+  // ... and advances the coordinates without division
+  int aw = warp % mAw, ah = (warp / mAw) % mAh, at = warp / (mAw * mAh);
   for (int a = warp; a < p.nA; a += kWarps) {
-    const int aw = a % mAw, ah = (a / mAw) % mAh, at = a / (mAw * mAh);
     const int ta = t0 + at * p.At, ha = h0 + ah * p.Ah, wa = w0 + aw * p.Aw;
+    aw += kWarps;
+    while (aw >= mAw) {
+      aw -= mAw;
+      if (++ah == mAh) { ah = 0; ++at; }
+    }
+    if (ta >= p.T || ha >= p.H || wa >= p.W) {
+      // an atom wholly in the padding: no token, so the identity summary
+      if (tl == 0) {
+        float* sa = sums + (size_t)a * 3 * D + dc * 8;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { sa[i] = summ_init<kSum>(); sa[D + i] = summ_init<kSum>(); sa[2 * D + i] = 0.f; }
+        if (dc == 0) { cnt[2 * a] = 0; cnt[2 * a + 1] = 0; }
+      }
+      continue;
+    }
     float qs[8], ks[8], us[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) { qs[i] = summ_init<kSum>(); ks[i] = summ_init<kSum>(); us[i] = 0.f; }
@@ -378,19 +395,22 @@ __global__ void __launch_bounds__(kPoolAtomThreads) pool_atoms_kernel(PoolParams
     for (int i = 0; i < DL; ++i) { qv[i] = summ_init<kSum>(); kv[i] = summ_init<kSum>(); uv[i] = 0.f; }
     int nv = 0, nu = 0;
     const int ft = bt / p.At, fh = bhh / p.Ah, fw = bw / p.Aw;   // atoms per block along each axis
-    for (int x = 0; x < ft * fh * fw; ++x) {
-      const int xw = x % fw, xh = (x / fw) % fh, xt = x / (fw * fh);
-      const int a = ((lt * ft + xt) * mAh + (lh * fh + xh)) * mAw + (lw * fw + xw);
-      const float* sa = sums + (size_t)a * 3 * D + lane * DL;
+    for (int xt = 0; xt < ft; ++xt)
+      for (int xh = 0; xh < fh; ++xh) {
+        const int arow = ((lt * ft + xt) * mAh + (lh * fh + xh)) * mAw + lw * fw;
+        for (int xw = 0; xw < fw; ++xw) {
+          const int a = arow + xw;
+          const float* sa = sums + (size_t)a * 3 * D + lane * DL;
 #pragma unroll
-      for (int i = 0; i < DL; ++i) {
-        qv[i] = summ_add<kSum>(qv[i], sa[i]);
-        kv[i] = summ_add<kSum>(kv[i], sa[D + i]);
-        uv[i] += sa[2 * D + i];
+          for (int i = 0; i < DL; ++i) {
+            qv[i] = summ_add<kSum>(qv[i], sa[i]);
+            kv[i] = summ_add<kSum>(kv[i], sa[D + i]);
+            uv[i] += sa[2 * D + i];
+          }
+          nv += cnt[2 * a];
+          nu += cnt[2 * a + 1];
+        }
       }
-      nv += cnt[2 * a];
-      nu += cnt[2 * a + 1];
-    }
     const size_t base = (((size_t)bh * p.C + c) * p.NB + blk);
     const float inv = nv ? 1.f / (float)nv : 0.f;
     float usq = 0.f;
