@@ -236,6 +236,145 @@ __global__ void __launch_bounds__(256) pool_sics_kernel(PoolParams p) {
 // SICS = ||sum of unit vectors||^2 - (number of nonzero keys).
 constexpr int kPoolAtomThreads = 256;     // 8 warps; two CTAs per SM (shared memory)
 
+// One token's 8 dimensions held by this lane (CH = D/8 lanes per token):
+// the summaries of q and k, and the unit vector k / ||k|| for SICS. Every
+// lane joins the ||k||^2 shuffles; lanes of a missing token (zeros) then add
+// nothing.
+template <int D, int kSum>
+__device__ __forceinline__ void pool_token(const uint4& qv, const uint4& kv, bool valid,
+                                           float (&qs)[8], float (&ks)[8], float (&us)[8],
+                                           int& n_valid, int& n_unit) {
+  constexpr int CH = D / 8;
+  // bf16 -> fp32 is a shift: element 2e in the low half of word e
+  const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+  const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+  float kf[8], qf[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    kf[2 * e] = __uint_as_float(kw[e] << 16);
+    kf[2 * e + 1] = __uint_as_float(kw[e] & 0xFFFF0000u);
+    qf[2 * e] = __uint_as_float(qw[e] << 16);
+    qf[2 * e + 1] = __uint_as_float(qw[e] & 0xFFFF0000u);
+  }
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    fma2(kf[2 * e], kf[2 * e + 1], kf[2 * e], kf[2 * e + 1], s0, s1, s0, s1);
+  float ss = s0 + s1;
+#pragma unroll
+  for (int o = CH / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (!valid) return;
+  if constexpr (kSum == SA_SUMMARIZER_MEAN) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      add2(qs[2 * e], qs[2 * e + 1], qf[2 * e], qf[2 * e + 1]);
+      add2(ks[2 * e], ks[2 * e + 1], kf[2 * e], kf[2 * e + 1]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      qs[i] = summ_add<kSum>(qs[i], qf[i]);
+      ks[i] = summ_add<kSum>(ks[i], kf[i]);
+    }
+  }
+  ++n_valid;
+  if (ss > 0.f) {
+    // approximate reciprocal square root (MUFU): the unit vectors differ
+    // from k / sqrt(|k|^2) by a few ulp
+    const float rn = rsqrtf(ss);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      fma2(kf[2 * e], kf[2 * e + 1], rn, rn, us[2 * e], us[2 * e + 1], us[2 * e], us[2 * e + 1]);
+    ++n_unit;
+  }
+}
+
+// The lanes of a warp's token groups combined (same dimensions, lanes
+// dc + CH*t), then group 0 writes atom ``a``'s summaries.
+template <int D, int kSum>
+__device__ __forceinline__ void pool_store_atom(float* sums, int* cnt, int a, int lane,
+                                                float (&qs)[8], float (&ks)[8], float (&us)[8],
+                                                int n_valid, int n_unit) {
+  constexpr int CH = D / 8;
+  const int tl = lane / CH, dc = lane % CH;
+#pragma unroll
+  for (int o = CH; o < 32; o <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      qs[i] = summ_add<kSum>(qs[i], __shfl_xor_sync(0xffffffffu, qs[i], o));
+      ks[i] = summ_add<kSum>(ks[i], __shfl_xor_sync(0xffffffffu, ks[i], o));
+      us[i] += __shfl_xor_sync(0xffffffffu, us[i], o);
+    }
+    n_valid += __shfl_xor_sync(0xffffffffu, n_valid, o);
+    n_unit += __shfl_xor_sync(0xffffffffu, n_unit, o);
+  }
+  if (tl == 0) {
+    float* sa = sums + (size_t)a * 3 * D + dc * 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { sa[i] = qs[i]; sa[D + i] = ks[i]; sa[2 * D + i] = us[i]; }
+    if (dc == 0) { cnt[2 * a] = n_valid; cnt[2 * a + 1] = n_unit; }
+  }
+}
+
+// Every block of every candidate inside the region from the per-atom
+// summaries: one warp per block, each lane D/32 dimensions.
+template <int D, int kSum>
+__device__ __forceinline__ void pool_combine(const PoolParams& p, const float* sums, const int* cnt,
+                                             int warp, int lane, int rt, int rh, int rw, int bh,
+                                             int mAh, int mAw) {
+  constexpr int kWarps = kPoolAtomThreads / 32;
+  constexpr int DL = D / 32;
+  int first[kMaxCand + 1];
+  first[0] = 0;
+  for (int c = 0; c < p.C; ++c)
+    first[c + 1] = first[c] + (p.Rt / p.cand[c][0]) * (p.Rh / p.cand[c][1]) * (p.Rw / p.cand[c][2]);
+  for (int pi = warp; pi < first[p.C]; pi += kWarps) {
+    int c = 0;
+    while (pi >= first[c + 1]) ++c;
+    const int bt = p.cand[c][0], bhh = p.cand[c][1], bw = p.cand[c][2];
+    const int lb = pi - first[c];
+    const int mw = p.Rw / bw, mh = p.Rh / bhh;
+    const int lw = lb % mw, lh = (lb / mw) % mh, lt = lb / (mw * mh);
+    const int nt = (p.T + bt - 1) / bt, nh = (p.H + bhh - 1) / bhh, nw = (p.W + bw - 1) / bw;
+    const int tt = rt * (p.Rt / bt) + lt, th = rh * (p.Rh / bhh) + lh, tw = rw * (p.Rw / bw) + lw;
+    if (tt >= nt || th >= nh || tw >= nw) continue;    // warp-uniform
+    const int blk = (tt * nh + th) * nw + tw;
+    float qv[DL], kv[DL], uv[DL];
+#pragma unroll
+    for (int i = 0; i < DL; ++i) { qv[i] = summ_init<kSum>(); kv[i] = summ_init<kSum>(); uv[i] = 0.f; }
+    int nv = 0, nu = 0;
+    const int ft = bt / p.At, fh = bhh / p.Ah, fw = bw / p.Aw;   // atoms per block along each axis
+    for (int xt = 0; xt < ft; ++xt)
+      for (int xh = 0; xh < fh; ++xh) {
+        const int arow = ((lt * ft + xt) * mAh + (lh * fh + xh)) * mAw + lw * fw;
+        for (int xw = 0; xw < fw; ++xw) {
+          const int a = arow + xw;
+          const float* sa = sums + (size_t)a * 3 * D + lane * DL;
+#pragma unroll
+          for (int i = 0; i < DL; ++i) {
+            qv[i] = summ_add<kSum>(qv[i], sa[i]);
+            kv[i] = summ_add<kSum>(kv[i], sa[D + i]);
+            uv[i] += sa[2 * D + i];
+          }
+          nv += cnt[2 * a];
+          nu += cnt[2 * a + 1];
+        }
+      }
+    const size_t base = (((size_t)bh * p.C + c) * p.NB + blk);
+    const float inv = nv ? 1.f / (float)nv : 0.f;
+    float usq = 0.f;
+#pragma unroll
+    for (int i = 0; i < DL; ++i) {
+      p.qbar[base * D + lane * DL + i] = summ_final<kSum>(qv[i], nv, inv);
+      p.kbar[base * D + lane * DL + i] = summ_final<kSum>(kv[i], nv, inv);
+      usq = fmaf(uv[i], uv[i], usq);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) usq += __shfl_xor_sync(0xffffffffu, usq, o);
+    if (lane == 0) p.sics[base] = usq - (float)nu;
+  }
+}
+
 template <int D, int kSum>
 __global__ void __launch_bounds__(kPoolAtomThreads, 2) pool_atoms_kernel(PoolParams p) {
   constexpr int CH = D / 8;                 // lanes per token (16 or 8)
@@ -305,125 +444,14 @@ __global__ void __launch_bounds__(kPoolAtomThreads, 2) pool_atoms_kernel(PoolPar
         }
       }
 #pragma unroll
-      for (int u = 0; u < UNROLL; ++u) {
-        // bf16 -> fp32 is a shift: element 2e in the low half of word e
-        const uint32_t* qw = reinterpret_cast<const uint32_t*>(&qv[u]);
-        const uint32_t* kw = reinterpret_cast<const uint32_t*>(&kv[u]);
-        float kf[8], qf[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          kf[2 * e] = __uint_as_float(kw[e] << 16);
-          kf[2 * e + 1] = __uint_as_float(kw[e] & 0xFFFF0000u);
-          qf[2 * e] = __uint_as_float(qw[e] << 16);
-          qf[2 * e + 1] = __uint_as_float(qw[e] & 0xFFFF0000u);
-        }
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          fma2(kf[2 * e], kf[2 * e + 1], kf[2 * e], kf[2 * e + 1], s0, s1, s0, s1);
-        float ss = s0 + s1;
-        // every lane joins; missing tokens carry zeros
-#pragma unroll
-        for (int o = CH / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (tok[u] < 0) continue;
-        if constexpr (kSum == SA_SUMMARIZER_MEAN) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            add2(qs[2 * e], qs[2 * e + 1], qf[2 * e], qf[2 * e + 1]);
-            add2(ks[2 * e], ks[2 * e + 1], kf[2 * e], kf[2 * e + 1]);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            qs[i] = summ_add<kSum>(qs[i], qf[i]);
-            ks[i] = summ_add<kSum>(ks[i], kf[i]);
-          }
-        }
-        ++n_valid;
-        if (ss > 0.f) {
-          // approximate reciprocal square root (MUFU): the unit vectors
-          // differ from k / sqrt(|k|^2) by a few ulp
-          const float rn = rsqrtf(ss);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            fma2(kf[2 * e], kf[2 * e + 1], rn, rn, us[2 * e], us[2 * e + 1], us[2 * e], us[2 * e + 1]);
-          ++n_unit;
-        }
-      }
+      for (int u = 0; u < UNROLL; ++u)
+        pool_token<D, kSum>(qv[u], kv[u], tok[u] >= 0, qs, ks, us, n_valid, n_unit);
     }
-    // combine the token lanes (same dimensions, lanes dc + CH*t)
-#pragma unroll
-    for (int o = CH; o < 32; o <<= 1) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        qs[i] = summ_add<kSum>(qs[i], __shfl_xor_sync(0xffffffffu, qs[i], o));
-        ks[i] = summ_add<kSum>(ks[i], __shfl_xor_sync(0xffffffffu, ks[i], o));
-        us[i] += __shfl_xor_sync(0xffffffffu, us[i], o);
-      }
-      n_valid += __shfl_xor_sync(0xffffffffu, n_valid, o);
-      n_unit += __shfl_xor_sync(0xffffffffu, n_unit, o);
-    }
-    if (tl == 0) {
-      float* sa = sums + (size_t)a * 3 * D + dc * 8;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) { sa[i] = qs[i]; sa[D + i] = ks[i]; sa[2 * D + i] = us[i]; }
-      if (dc == 0) { cnt[2 * a] = n_valid; cnt[2 * a + 1] = n_unit; }
-    }
+    pool_store_atom<D, kSum>(sums, cnt, a, lane, qs, ks, us, n_valid, n_unit);
   }
   __syncthreads();
 
-  // every block of every candidate inside the region: one warp per block,
-  // each lane D/32 dimensions
-  constexpr int DL = D / 32;
-  int first[kMaxCand + 1];
-  first[0] = 0;
-  for (int c = 0; c < p.C; ++c)
-    first[c + 1] = first[c] + (p.Rt / p.cand[c][0]) * (p.Rh / p.cand[c][1]) * (p.Rw / p.cand[c][2]);
-  for (int pi = warp; pi < first[p.C]; pi += kWarps) {
-    int c = 0;
-    while (pi >= first[c + 1]) ++c;
-    const int bt = p.cand[c][0], bhh = p.cand[c][1], bw = p.cand[c][2];
-    const int lb = pi - first[c];
-    const int mw = p.Rw / bw, mh = p.Rh / bhh;
-    const int lw = lb % mw, lh = (lb / mw) % mh, lt = lb / (mw * mh);
-    const int nt = (p.T + bt - 1) / bt, nh = (p.H + bhh - 1) / bhh, nw = (p.W + bw - 1) / bw;
-    const int tt = rt * (p.Rt / bt) + lt, th = rh * (p.Rh / bhh) + lh, tw = rw * (p.Rw / bw) + lw;
-    if (tt >= nt || th >= nh || tw >= nw) continue;    // warp-uniform
-    const int blk = (tt * nh + th) * nw + tw;
-    float qv[DL], kv[DL], uv[DL];
-#pragma unroll
-    for (int i = 0; i < DL; ++i) { qv[i] = summ_init<kSum>(); kv[i] = summ_init<kSum>(); uv[i] = 0.f; }
-    int nv = 0, nu = 0;
-    const int ft = bt / p.At, fh = bhh / p.Ah, fw = bw / p.Aw;   // atoms per block along each axis
-    for (int xt = 0; xt < ft; ++xt)
-      for (int xh = 0; xh < fh; ++xh) {
-        const int arow = ((lt * ft + xt) * mAh + (lh * fh + xh)) * mAw + lw * fw;
-        for (int xw = 0; xw < fw; ++xw) {
-          const int a = arow + xw;
-          const float* sa = sums + (size_t)a * 3 * D + lane * DL;
-#pragma unroll
-          for (int i = 0; i < DL; ++i) {
-            qv[i] = summ_add<kSum>(qv[i], sa[i]);
-            kv[i] = summ_add<kSum>(kv[i], sa[D + i]);
-            uv[i] += sa[2 * D + i];
-          }
-          nv += cnt[2 * a];
-          nu += cnt[2 * a + 1];
-        }
-      }
-    const size_t base = (((size_t)bh * p.C + c) * p.NB + blk);
-    const float inv = nv ? 1.f / (float)nv : 0.f;
-    float usq = 0.f;
-#pragma unroll
-    for (int i = 0; i < DL; ++i) {
-      p.qbar[base * D + lane * DL + i] = summ_final<kSum>(qv[i], nv, inv);
-      p.kbar[base * D + lane * DL + i] = summ_final<kSum>(kv[i], nv, inv);
-      usq = fmaf(uv[i], uv[i], usq);
-    }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) usq += __shfl_xor_sync(0xffffffffu, usq, o);
-    if (lane == 0) p.sics[base] = usq - (float)nu;
-  }
+  pool_combine<D, kSum>(p, sums, cnt, warp, lane, rt, rh, rw, bh, mAh, mAw);
 }
 
 // ------------------------------------------------------------------ choose
