@@ -84,6 +84,40 @@ def test_invalid_arguments_are_rejected_on_the_host():
                                         ctypes.byref(s)) == N.SA_ERR_INVALID_ARG
 
 
+def test_summarizer_and_profiler_arguments_are_checked_on_the_host():
+    L = N.lib()
+    m, s = ctypes.c_size_t(), ctypes.c_size_t()
+    wl = CONFIGS["spade_wan21_14b_720p"]
+    pr = N.Problem(1, wl.heads, wl.T, wl.H, wl.W, wl.head_dim)
+    for good in ("mean", "max", "min"):
+        pol = make_policy(**{**C.policy_kwargs(wl), "summarizer": good})
+        assert L.sparse_attn_workspace_size(ctypes.byref(pr), ctypes.byref(pol), ctypes.byref(m),
+                                            ctypes.byref(s)) == N.SA_OK
+    bad = make_policy(**{**C.policy_kwargs(wl), "summarizer": 3})
+    assert L.sparse_attn_workspace_size(ctypes.byref(pr), ctypes.byref(bad), ctypes.byref(m),
+                                        ctypes.byref(s)) == N.SA_ERR_INVALID_ARG
+    # the profiler: spatial/temporal policy only, 1 <= n_rows <= N, aligned device buffers
+    st = CONFIGS["spatiotemporal_hunyuan_720p"]
+    pr = N.Problem(1, st.heads, st.T, st.H, st.W, st.head_dim)
+    ok_pol = make_policy("spatiotemporal", block=128, sink_tokens=226)
+    args = (0x1000, 0x1000, 0x1000, 0x1000, 16, 0x1000, 0x1000, 0x1000, None, None)
+    sta = make_policy("sta", tile=(4, 4, 8), window=(3, 3, 3))
+    assert L.sparse_attn_profile_heads(ctypes.byref(pr), ctypes.byref(sta), *args) == N.SA_ERR_INVALID_ARG
+    for n_rows in (0, st.T * st.H * st.W + 1):
+        a = list(args)
+        a[4] = n_rows
+        assert L.sparse_attn_profile_heads(ctypes.byref(pr), ctypes.byref(ok_pol), *a) == N.SA_ERR_INVALID_ARG
+    a = list(args)
+    a[0] = 0x1008                                                     # q not 16-byte aligned
+    assert L.sparse_attn_profile_heads(ctypes.byref(pr), ctypes.byref(ok_pol), *a) == N.SA_ERR_INVALID_ARG
+    a = list(args)
+    a[7] = None                                                       # no decision buffer
+    assert L.sparse_attn_profile_heads(ctypes.byref(pr), ctypes.byref(ok_pol), *a) == N.SA_ERR_INVALID_ARG
+    a = list(args)
+    a[8] = 0x1010                                                     # scratch not 256-byte aligned
+    assert L.sparse_attn_profile_heads(ctypes.byref(pr), ctypes.byref(ok_pol), *a) == N.SA_ERR_WORKSPACE
+
+
 def test_strerror_covers_every_code():
     for code in range(7):
         assert N.strerror(code) and N.strerror(code) != "unknown status"
