@@ -53,7 +53,10 @@ def head_mask(wl, q, k, head, force_choice=None):
         bm = masks.topk_with_diagonal(s, wl.topk, wl.keep_diagonal, valid, valid)
     elif wl.kind == "sta":
         dims = layout.tile_grid_dims(wl.T, wl.H, wl.W, *wl.tile)
-        bm = masks.tile_window(dims, wl.window, valid, valid)
+        # Sliding Tile Attention review: heads specialize in different window
+        # sizes; a per-head window replaces the policy's one for its head
+        win = wl.head_windows[head] if wl.head_windows else wl.window
+        bm = masks.tile_window(dims, win, valid, valid)
     elif wl.kind == "spatiotemporal":
         if head in wl.temporal_heads:
             bm = masks.temporal_rule(blk, wl.T, wl.H, wl.W)

@@ -47,6 +47,7 @@ class Workload:
     fg_keep_fraction: float = 0.0
     block: int = 128                               # tokens per block in the working layout
     summarizer: str = "mean"                       # topk, spade: block summary ("mean", "max", "min")
+    head_windows: Tuple[Tuple[int, int, int], ...] = ()   # sta: a window per head (empty: window)
 
     @property
     def N(self) -> int:

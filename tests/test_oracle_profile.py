@@ -82,3 +82,45 @@ def test_sample_rows_are_distinct_sorted_and_seeded():
         assert np.all(np.diff(a[h]) > 0) and a[h].min() >= 0 and a[h].max() < 115200
     np.testing.assert_array_equal(a, sample_rows(115200, 3, 0.01, seed=7))
     assert not np.array_equal(a[0], a[1])
+
+
+def test_window_covering_the_grid_is_full_attention_and_wins():
+    # Sliding Tile Attention review, Algorithm 1: a window that spans the
+    # whole tile grid keeps every key, so its error is exactly zero.
+    T, H, W, d = 4, 8, 16, 16
+    tile = (2, 4, 8)                                      # tile grid 2 x 2 x 2
+    q, k, v = _qkv(T * H * W, d, 8)
+    rows = np.array([1, 77, 300, 511])
+    cands = [(1, 1, 1), (3, 3, 3), (1, 3, 1)]
+    assert profile.window_keep(rows, T, H, W, tile, (3, 3, 3)).all()
+    r = profile.sta_window_search(q, k, v, rows, T, H, W, tile, cands)
+    assert r["mse"][1] == 0.0 and r["mse"][0] > 0.0 and r["choice"] == 1
+
+
+def test_window_keep_matches_its_plain_definition():
+    # unit tiles (1, 1, 1) would make blocks of one token; with tiles of one
+    # frame row (1, 1, W) the kept keys of a query at (t, h, w) under window
+    # (wt, wh, 1) are the tokens with |dt| <= wt//2 and |dh| <= wh//2
+    T, H, W = 5, 6, 8
+    tile = (1, 1, W)
+    rows = np.array([0, 13, 100, 239])
+    keep = profile.window_keep(rows, T, H, W, tile, (3, 1, 1))
+    tok = np.arange(T * H * W)
+    t, h = tok // (H * W), (tok // W) % H
+    for r, q_tok in enumerate(rows):
+        want = (np.abs(t - t[q_tok]) <= 1) & (h == h[q_tok])
+        np.testing.assert_array_equal(keep[r], want)
+
+
+def test_per_head_windows_equal_single_window_masks():
+    from oracle import pipeline
+    from synthetic import CONFIGS, Workload, make_qkv, bf16_bits_to_f32
+    base = Workload(name="hw", config_id=130, T=4, H=8, W=16, heads=2, head_dim=32, kind="sta",
+                    tile=(2, 4, 8), block=64, window=(3, 3, 3))
+    per_head = base.with_(head_windows=((1, 1, 1), (1, 3, 3)))
+    x = make_qkv(base)
+    for h, win in enumerate(per_head.head_windows):
+        qf, kf = (bf16_bits_to_f32(x[n][0, h]) for n in "qk")
+        a = pipeline.head_mask(per_head, qf, kf, h)["bmask"]
+        b = pipeline.head_mask(base.with_(window=win), qf, kf, h)["bmask"]
+        np.testing.assert_array_equal(a, b)
