@@ -191,7 +191,8 @@ def policy_kwargs(wl):
         return dict(kind="topk", block=wl.block, tile=wl.tile, topk=wl.topk,
                     keep_diagonal=wl.keep_diagonal, summarizer=wl.summarizer)
     if wl.kind == "sta":
-        return dict(kind="sta", block=wl.block, tile=wl.tile, window=wl.window)
+        return dict(kind="sta", block=wl.block, tile=wl.tile, window=wl.window,
+                    head_windows=wl.head_windows or None)
     if wl.kind == "spatiotemporal":
         return dict(kind="spatiotemporal", block=wl.block, temporal_heads=wl.temporal_heads,
                     heads=wl.heads, sink_tokens=wl.sink_tokens, frame_radius=1)

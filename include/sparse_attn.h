@@ -135,6 +135,10 @@ typedef struct {
   const uint32_t* explicit_bits; /* EXPLICIT: device [batch*heads][nb][ceil(nb/32)],
                                  bit j of row i keeps key block j for query block i */
   int summarizer;             /* TOPK, SPADE: SA_SUMMARIZER_*; other kinds ignore it */
+  const int* head_windows;    /* STA, optional host array [heads][3]: each head's odd
+                                 window extents in tiles (<= 255; null: ``window``
+                                 for every head). Sliding Tile Attention review:
+                                 heads specialize in different window sizes    */
 } sa_policy;
 
 /* ---------------------------------------------------------------- sizes
@@ -222,7 +226,9 @@ typedef struct {
   int32_t nb;                /* blocks of this head's working layout              */
   int32_t kept;              /* kept (query block, key block) pairs               */
   float sics_total[4];       /* SPADE: summed SICS per candidate blocking         */
-  int32_t reserved[2];
+  int32_t window;             /* STA: the head's window, wt | wh << 8 | ww << 16;
+                                 0: the policy's window                        */
+  int32_t reserved;
 } sa_head_info;
 
 SA_API int sparse_attn_export_bytes(const sa_problem* problem, const sa_policy* policy, int what,
@@ -263,6 +269,30 @@ SA_API int sparse_attn_profile_heads(const sa_problem* problem, const sa_policy*
                                      const void* q, const void* k, const void* v,
                                      const int32_t* rows, int n_rows, float* row_err, float* mse,
                                      int8_t* is_temporal, void* scratch_ws, void* stream);
+
+/* STA per-head window search (Sliding Tile Attention review, key machinery;
+ * Algorithm 1: each head's window is the mask that minimizes the MSE to full
+ * attention). For every head, on the sampled query rows ``rows``, attention is
+ * evaluated over all keys and under the sliding tile window of each of the
+ * ``n_candidates`` (1..8) candidates: host int [n_candidates][3], odd
+ * extents in tiles, at most 255. The tile layout is ``policy->tile`` with
+ * ``policy->block`` tokens (kind SA_MASK_STA; ``window`` is not read). The
+ * candidates encode the trade-off; the search returns the lowest error, ties
+ * to the earlier candidate. The result feeds ``sa_policy.head_windows``.
+ *
+ *   rows, scratch_ws  as for sparse_attn_profile_heads.
+ *   row_err     device float [batch*heads][n_rows][n_candidates]: per row and
+ *               candidate, the sum over head_dim of (O_window - O_full)^2.
+ *   mse         device float [batch*heads][n_candidates]: those sums over
+ *               the rows, divided by n_rows * head_dim (fixed order).
+ *   choice      device int8 [batch*heads]: the chosen candidate.
+ * Asynchronous on ``stream``. Returns SA_OK, SA_ERR_INVALID_ARG,
+ * SA_ERR_UNSUPPORTED or SA_ERR_CUDA. */
+SA_API int sparse_attn_sta_window_search(const sa_problem* problem, const sa_policy* policy,
+                                         const void* q, const void* k, const void* v,
+                                         const int32_t* rows, int n_rows, const int* candidates,
+                                         int n_candidates, float* row_err, float* mse,
+                                         int8_t* choice, void* scratch_ws, void* stream);
 
 /* Failure-path self-test: launches one CTA on ``stream`` that waits, with the
  * bounded wait every kernel of this library uses, on a barrier that nothing

@@ -27,7 +27,7 @@ EXPORTED = ("sparse_attn_workspace_size", "sparse_attn_build_mask", "sparse_attn
             "sparse_attn_permute", "sparse_attn_attend",
             "sparse_attn_export_bytes", "sparse_attn_mask_export", "sparse_attn_status",
             "sparse_attn_build_mask_static", "sparse_attn_selftest_wait_timeout",
-            "sparse_attn_profile_heads", "sparse_attn_strerror")
+            "sparse_attn_profile_heads", "sparse_attn_sta_window_search", "sparse_attn_strerror")
 
 SA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
 
@@ -45,7 +45,8 @@ class Policy(ctypes.Structure):
                 ("n_candidates", ctypes.c_int), ("candidates", (ctypes.c_int * 3) * 4),
                 ("top_p", ctypes.c_float), ("fg_group", ctypes.c_int),
                 ("fg_keep_fraction", ctypes.c_float), ("explicit_layout", ctypes.c_int),
-                ("explicit_bits", ctypes.c_void_p), ("summarizer", ctypes.c_int)]
+                ("explicit_bits", ctypes.c_void_p), ("summarizer", ctypes.c_int),
+                ("head_windows", ctypes.POINTER(ctypes.c_int))]
 
 
 class HeadInfo(ctypes.Structure):
@@ -53,7 +54,8 @@ class HeadInfo(ctypes.Structure):
                 ("bt", ctypes.c_int32), ("bh", ctypes.c_int32), ("bw", ctypes.c_int32),
                 ("nt", ctypes.c_int32), ("nh", ctypes.c_int32), ("nw", ctypes.c_int32),
                 ("nb", ctypes.c_int32), ("kept", ctypes.c_int32),
-                ("sics_total", ctypes.c_float * 4), ("reserved", ctypes.c_int32 * 2)]
+                ("sics_total", ctypes.c_float * 4), ("window", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 class SparseAttnError(RuntimeError):
@@ -87,6 +89,8 @@ def lib():
         L.sparse_attn_selftest_wait_timeout.argtypes = [vp, vp]
         L.sparse_attn_profile_heads.argtypes = [P, PP, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp,
                                                 vp, vp]
+        L.sparse_attn_sta_window_search.argtypes = [P, PP, vp, vp, vp, vp, ctypes.c_int, vp,
+                                                    ctypes.c_int, vp, vp, vp, vp, vp]
         L.sparse_attn_strerror.argtypes = [ctypes.c_int]
         L.sparse_attn_strerror.restype = ctypes.c_char_p
         for name in EXPORTED[:-1]:
@@ -142,6 +146,14 @@ def profile_heads(problem, policy, q, k, v, rows, n_rows, row_err, mse, is_tempo
                                            rows, n_rows, row_err, mse, is_temporal, scratch_ws,
                                            stream),
            "sparse_attn_profile_heads")
+
+
+def sta_window_search(problem, policy, q, k, v, rows, n_rows, candidates, n_candidates, row_err,
+                      mse, choice, scratch_ws=None, stream=0):
+    _check(lib().sparse_attn_sta_window_search(ctypes.byref(problem), ctypes.byref(policy), q, k,
+                                               v, rows, n_rows, candidates, n_candidates, row_err,
+                                               mse, choice, scratch_ws, stream),
+           "sparse_attn_sta_window_search")
 
 
 def export_bytes(problem, policy, what):

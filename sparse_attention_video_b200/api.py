@@ -15,11 +15,13 @@ from . import _native as N
 def make_policy(kind, block=128, tile=(1, 1, 128), topk=0, keep_diagonal=False,
                 window=(1, 1, 1), temporal_heads=None, heads=0, sink_tokens=0, frame_radius=1,
                 candidates=(), top_p=0.0, fg_group=64, fg_keep_fraction=0.15,
-                explicit_layout=N.SA_LAYOUT_IDENTITY, explicit_bits=None, summarizer="mean"):
+                explicit_layout=N.SA_LAYOUT_IDENTITY, explicit_bits=None, summarizer="mean",
+                head_windows=None):
     """Fill an ``sa_policy``. ``kind`` is a name ("topk", "sta", "spatiotemporal",
     "spade", "fg", "explicit") or an SA_MASK_* code; ``summarizer`` ("mean",
     "max", "min" or an SA_SUMMARIZER_* code) picks the block summary behind the
-    pooled scores of "topk" and "spade"."""
+    pooled scores of "topk" and "spade"; ``head_windows`` (one odd (wt, wh, ww)
+    per head) gives "sta" a window per head."""
     names = {"topk": N.SA_MASK_TOPK, "sta": N.SA_MASK_STA,
              "spatiotemporal": N.SA_MASK_SPATIOTEMPORAL, "spade": N.SA_MASK_SPADE,
              "fg": N.SA_MASK_FG, "explicit": N.SA_MASK_EXPLICIT}
@@ -47,6 +49,10 @@ def make_policy(kind, block=128, tile=(1, 1, 128), topk=0, keep_diagonal=False,
     p.explicit_layout = explicit_layout
     sums = {"mean": N.SA_SUMMARIZER_MEAN, "max": N.SA_SUMMARIZER_MAX, "min": N.SA_SUMMARIZER_MIN}
     p.summarizer = sums.get(summarizer, summarizer)
+    if head_windows is not None:
+        arr = (ctypes.c_int * (3 * len(head_windows)))(*[int(x) for w in head_windows for x in w])
+        p.head_windows = ctypes.cast(arr, ctypes.POINTER(ctypes.c_int))
+        p._keep_windows = arr
     if explicit_bits is not None:
         p.explicit_bits = explicit_bits.data_ptr()
         p._keep_bits = explicit_bits
@@ -165,3 +171,36 @@ def profile_heads(q, k, v, rows, T, H, W, block=128, sink_tokens=0, frame_radius
                     n_rows, row_err.data_ptr(), mse.data_ptr(), is_temporal.data_ptr(),
                     scratch_ws.data_ptr() if scratch_ws is not None else None, _stream_ptr(stream))
     return is_temporal, mse, row_err
+
+
+def sta_window_search(q, k, v, rows, T, H, W, tile, candidates, block=128, stream=None,
+                      scratch_ws=None):
+    """STA per-head window search (Sliding Tile Attention review, key machinery).
+
+    q, k, v: contiguous CUDA bf16 [batch, heads, N, d]; rows: CUDA int32
+    [batch*heads, n_rows]; tile: (bt, bh, bw) with bt*bh*bw == block;
+    candidates: odd (wt, wh, ww) windows in tiles. Returns (choice int8
+    [batch*heads], mse float32 [batch*heads, n_candidates], row_err float32
+    [batch*heads, n_rows, n_candidates]) as CUDA tensors, queued on ``stream``.
+    ``[candidates[c] for c in choice]`` is a ``head_windows`` for make_policy.
+    """
+    B, Hh, N_, d = q.shape
+    problem = N.Problem(B, Hh, T, H, W, d)
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        _check_qkv(t, problem, name)
+    if rows.dtype != torch.int32 or not rows.is_cuda or not rows.is_contiguous() \
+            or rows.dim() != 2 or rows.shape[0] != B * Hh:
+        raise ValueError("rows must be a contiguous CUDA int32 tensor [batch*heads, n_rows]")
+    n_rows, nc = rows.shape[1], len(candidates)
+    policy = make_policy("sta", block=block, tile=tile, window=(1, 1, 1))
+    cand = (ctypes.c_int * (3 * nc))(*[int(x) for c in candidates for x in c])
+    dev = q.device
+    row_err = torch.empty((B * Hh, n_rows, nc), dtype=torch.float32, device=dev)
+    mse = torch.empty((B * Hh, nc), dtype=torch.float32, device=dev)
+    choice = torch.empty(B * Hh, dtype=torch.int8, device=dev)
+    N.sta_window_search(problem, policy, q.data_ptr(), k.data_ptr(), v.data_ptr(), rows.data_ptr(),
+                        n_rows, cand, nc, row_err.data_ptr(), mse.data_ptr(), choice.data_ptr(),
+                        scratch_ws.data_ptr() if scratch_ws is not None else None,
+                        _stream_ptr(stream))
+    return choice, mse, row_err
+

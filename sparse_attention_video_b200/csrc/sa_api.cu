@@ -66,6 +66,12 @@ int check_policy(const sa_problem& pr, const sa_policy* po) {
     case SA_MASK_STA:
       for (int i = 0; i < 3; ++i)
         if (po->window[i] < 1 || po->window[i] % 2 == 0) return SA_ERR_INVALID_ARG;
+      if (po->head_windows) {
+        if (pr.heads > kMaxHeads) return SA_ERR_UNSUPPORTED;
+        for (int i = 0; i < 3 * pr.heads; ++i)
+          if (po->head_windows[i] < 1 || po->head_windows[i] % 2 == 0 || po->head_windows[i] > 255)
+            return SA_ERR_INVALID_ARG;
+      }
       return check_tile(pr, po->tile, po->block);
     case SA_MASK_SPADE:
       if (po->n_candidates < 1 || po->n_candidates > kMaxCand) return SA_ERR_INVALID_ARG;
@@ -383,6 +389,12 @@ extern "C" int sparse_attn_build_mask(const sa_problem* problem, const sa_policy
       for (int h = 0; h < pr.heads; ++h)
         if (po.head_is_temporal[h]) hp.temporal_bits[h / 32] |= 1u << (h % 32);
     }
+    if (po.kind == SA_MASK_STA && po.head_windows) {
+      hp.has_windows = 1;
+      for (int h = 0; h < pr.heads; ++h)
+        hp.windows[h] = po.head_windows[3 * h] | (po.head_windows[3 * h + 1] << 8) |
+                        (po.head_windows[3 * h + 2] << 16);
+    }
     if ((e = cuda_status(launch_head_init(hp, st)))) return e;
   }
   if (C > 0) {
@@ -595,7 +607,11 @@ extern "C" int sparse_attn_profile_heads(const sa_problem* problem, const sa_pol
   pp.rows = rows;
   pp.row_err = row_err;
   pp.mse = mse;
-  pp.is_temporal = is_temporal;
+  pp.choice = is_temporal;                    // pattern 1 (temporal) beats pattern 0
+  pp.mode = 0;
+  pp.n_pat = 2;
+  pp.tile[0] = pp.tile[1] = 1;
+  pp.tile[2] = po.block;
   pp.status = scratch_ws ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(scratch_ws) +
                                                        ScratchLayout{}.off_status)
                          : nullptr;
@@ -605,6 +621,52 @@ extern "C" int sparse_attn_profile_heads(const sa_problem* problem, const sa_pol
   pp.block = po.block;
   pp.sink_blocks = ceil_div(po.sink_tokens, po.block);
   pp.frame_radius = po.frame_radius;
+  pp.scale_log2 = 1.4426950408889634f / sqrtf((float)pr.head_dim);
+  return cuda_status(launch_profile(pp, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+extern "C" int sparse_attn_sta_window_search(const sa_problem* problem, const sa_policy* policy,
+                                             const void* q, const void* k, const void* v,
+                                             const int32_t* rows, int n_rows,
+                                             const int* candidates, int n_candidates,
+                                             float* row_err, float* mse, int8_t* choice,
+                                             void* scratch_ws, void* stream) {
+  int e = check_problem(problem);
+  if (e) return e;
+  if (!policy || policy->kind != SA_MASK_STA) return SA_ERR_INVALID_ARG;
+  const sa_problem& pr = *problem;
+  const sa_policy& po = *policy;
+  if (po.block != 128 && !(po.block == 64 && pr.head_dim == 64)) return SA_ERR_UNSUPPORTED;
+  if ((e = check_tile(pr, po.tile, po.block))) return e;
+  if (!candidates || n_candidates < 1 || n_candidates > kProfileMaxPatterns) return SA_ERR_INVALID_ARG;
+  for (int i = 0; i < 3 * n_candidates; ++i)
+    if (candidates[i] < 1 || candidates[i] % 2 == 0 || candidates[i] > 255) return SA_ERR_INVALID_ARG;
+  const long long N = n_tokens(pr);
+  if (n_rows < 1 || n_rows > N) return SA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return SA_ERR_INVALID_ARG;
+  if (!aligned(rows, 4) || !aligned(row_err, 4) || !aligned(mse, 4) || !choice)
+    return SA_ERR_INVALID_ARG;
+  if (scratch_ws && !aligned(scratch_ws, 256)) return SA_ERR_WORKSPACE;
+  ProfileParams pp{};
+  pp.q = static_cast<const __nv_bfloat16*>(q);
+  pp.k = static_cast<const __nv_bfloat16*>(k);
+  pp.v = static_cast<const __nv_bfloat16*>(v);
+  pp.rows = rows;
+  pp.row_err = row_err;
+  pp.mse = mse;
+  pp.choice = choice;
+  pp.status = scratch_ws ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(scratch_ws) +
+                                                       ScratchLayout{}.off_status)
+                         : nullptr;
+  pp.BH = pr.batch * pr.heads;
+  pp.N = (int)N; pp.T = pr.T; pp.H = pr.H; pp.W = pr.W; pp.d = pr.head_dim;
+  pp.n_rows = n_rows;
+  pp.block = po.block;
+  pp.mode = 1;
+  pp.n_pat = n_candidates;
+  for (int i = 0; i < 3; ++i) pp.tile[i] = po.tile[i];
+  for (int c = 0; c < n_candidates; ++c)
+    for (int i = 0; i < 3; ++i) pp.win[c][i] = candidates[3 * c + i];
   pp.scale_log2 = 1.4426950408889634f / sqrtf((float)pr.head_dim);
   return cuda_status(launch_profile(pp, reinterpret_cast<cudaStream_t>(stream)));
 }

@@ -13,6 +13,7 @@ namespace sa {
 
 constexpr int kMaxCand = 4;
 constexpr int kMaxBlocks = 4096;  // blocks per head in one working layout
+constexpr int kMaxHeads = 256;    // heads per problem with per-head policy data
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -49,7 +50,8 @@ struct ScratchLayout {
 struct HeadGeom {
   int layout, cand, bt, bh, bw, nt, nh, nw, nb, kept;
   float sics_total[4];
-  int reserved[2];
+  int window;                       // STA: wt | wh << 8 | ww << 16 (0: the policy's window)
+  int reserved;
 };
 static_assert(sizeof(HeadGeom) == sizeof(sa_head_info), "head info layout");
 

@@ -53,6 +53,7 @@ __global__ void head_init_kernel(HeadInitParams p) {
     g.nt = 1; g.nh = 1; g.nw = g.nb;
   }
   g.kept = 0;
+  g.window = p.has_windows ? p.windows[head] : 0;
   p.geo[bh] = g;
 }
 
@@ -619,8 +620,11 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
       if (threadIdx.x == 0 && p.keep_diagonal && i < nb && block_valid(g, i, p.T, p.H, p.W))
         bits[i / 32] |= 1u << (i % 32);
     } else if (p.kind == SA_MASK_STA || p.kind == SA_MASK_SPADE) {
-      // clipped tile window around query tile i
-      const int rt = p.win[0] / 2, rh = p.win[1] / 2, rw = p.win[2] / 2;
+      // clipped tile window around query tile i (the head's own window if it has one)
+      const int wwin = g.window;
+      const int rt = (wwin ? (wwin & 0xFF) : p.win[0]) / 2;
+      const int rh = (wwin ? ((wwin >> 8) & 0xFF) : p.win[1]) / 2;
+      const int rw = (wwin ? ((wwin >> 16) & 0xFF) : p.win[2]) / 2;
       const int iw = i % g.nw, ih = (i / g.nw) % g.nh, it = i / (g.nw * g.nh);
       const int wt = 2 * rt + 1, wh = 2 * rh + 1, ww = 2 * rw + 1;
       for (int e = threadIdx.x; e < wt * wh * ww; e += 256) {

@@ -15,6 +15,8 @@ struct HeadInitParams {
   int bt, bh, bw;                   // tile of SA_LAYOUT_TILE
   int has_temporal_bits;            // SPATIOTEMPORAL: layout per head from the bitset
   uint32_t temporal_bits[8];        // bit h set: head h is temporal (frame-major)
+  int has_windows;                  // STA: a window per head
+  int windows[kMaxHeads];           // wt | wh << 8 | ww << 16
 };
 
 struct PermuteParams {

@@ -1,11 +1,14 @@
-// SVG online head profiler (Sparse VideoGen review, key machinery;
-// Algorithm 1). For every head, on a sample of its query rows, attention is
-// evaluated three times: over all keys, over the spatial pattern's keys and
-// over the temporal pattern's keys. The head takes the pattern whose output
-// has the lower mean squared error against the full output (ties: spatial).
-// The patterns are the block masks of the spatial / temporal heads: identity
-// layout with frames within +-frame_radius, and frame-major layout with a
-// shared spatial position, both with the sink blocks.
+// Sampled-row pattern evaluation. For every head, on a sample of its query
+// rows, attention is evaluated over all keys and under each of several
+// sparse patterns; the head takes the pattern whose output has the lowest
+// mean squared error against the full output (ties: the earlier pattern).
+//   mode 0, SVG online head profiler (Sparse VideoGen review, key machinery;
+//     Algorithm 1): the block masks of the spatial / temporal heads
+//     (identity layout, frames within +-frame_radius; frame-major layout, a
+//     shared spatial position), both with the sink blocks.
+//   mode 1, STA per-head window search (Sliding Tile Attention review, key
+//     machinery; Algorithm 1): one sliding tile window per candidate, on the
+//     3D tile layout.
 //
 // One warp owns 16 sampled rows. Keys pass through XOR-swizzled shared-memory
 // tiles filled by cp.async (double-buffered); ldmatrix forms the fragments and
@@ -98,6 +101,13 @@ __device__ __forceinline__ bool temporal_keep(const PatternGeo& g, int qtok, int
   return !(k_hi < p_lo || p_hi < k_lo);
 }
 
+// STA window: key tile b (raster, tw fastest) against the query's tile.
+__device__ __forceinline__ bool window_keep(int b, int nh, int nw, int qt, int qh, int qw,
+                                            const int (&win)[3]) {
+  const int kt = b / (nh * nw), kh = (b / nw) % nh, kw = b % nw;
+  return abs(kt - qt) <= win[0] / 2 && abs(kh - qh) <= win[1] / 2 && abs(kw - qw) <= win[2] / 2;
+}
+
 template <int D>
 __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams p) {
   using L = ProfSmem<D>;
@@ -154,9 +164,10 @@ __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams 
     m0 = m1 = -INFINITY;
     l0 = l1 = 0.f;
   };
-  // One step of 16 keys (slots slot0..slot0+15 of the pass's order) from
-  // 16-row tiles tK, tV; rows outside ``rmask`` and slots past N are masked.
-  auto step16 = [&](const uint8_t* tK, const uint8_t* tV, int slot0, uint32_t rmask) {
+  // One step of 16 keys from 16-row tiles tK, tV; rows outside ``rmask`` and
+  // keys outside ``kvm`` are masked.
+  // kvm: bit i set when key i of the step exists (not padding)
+  auto step16 = [&](const uint8_t* tK, const uint8_t* tV, uint32_t kvm, uint32_t rmask) {
     float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
     {
       const int m = lane / 8, i = lane % 8;
@@ -169,8 +180,8 @@ __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams 
       }
     }
     const bool keep0 = (rmask >> g) & 1u, keep1 = (rmask >> (g + 8)) & 1u;
-    const bool v00 = slot0 + cq < p.N, v01 = slot0 + cq + 1 < p.N;
-    const bool v10 = slot0 + 8 + cq < p.N, v11 = slot0 + 8 + cq + 1 < p.N;
+    const bool v00 = (kvm >> cq) & 1u, v01 = (kvm >> (cq + 1)) & 1u;
+    const bool v10 = (kvm >> (8 + cq)) & 1u, v11 = (kvm >> (9 + cq)) & 1u;
     float x[8];
     x[0] = keep0 && v00 ? s0[0] * p.scale_log2 : -INFINITY;   // row g,     key cq
     x[1] = keep0 && v01 ? s0[1] * p.scale_log2 : -INFINITY;   // row g,     key cq + 1
@@ -246,9 +257,9 @@ __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams 
       e1 += __shfl_xor_sync(0xffffffffu, e1, 1);
       e1 += __shfl_xor_sync(0xffffffffu, e1, 2);
       if ((lane & 3) == 0) {
-        float* re = p.row_err + ((size_t)bh * p.n_rows + row0) * 2 + (pass - 1);
-        if (row0 + g < p.n_rows) re[(size_t)g * 2] = e0;
-        if (row0 + g + 8 < p.n_rows) re[(size_t)(g + 8) * 2] = e1;
+        float* re = p.row_err + ((size_t)bh * p.n_rows + row0) * p.n_pat + (pass - 1);
+        if (row0 + g < p.n_rows) re[(size_t)g * p.n_pat] = e0;
+        if (row0 + g + 8 < p.n_rows) re[(size_t)(g + 8) * p.n_pat] = e1;
       }
     }
   };
@@ -289,7 +300,10 @@ __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams 
         const uint8_t* tV = tK + L::kCoopTile;
         for (int sub = 0; sub < L::kCoopKeys / kStepKeys; ++sub) {
           const int slot0 = st * L::kCoopKeys + sub * kStepKeys;
-          if (slot0 < p.N) step16(tK + sub * L::kTile16, tV + sub * L::kTile16, slot0, rmask);
+          if (slot0 < p.N) {
+            const uint32_t kvm = slot0 + kStepKeys <= p.N ? 0xFFFFu : ((1u << (p.N - slot0)) - 1u);
+            step16(tK + sub * L::kTile16, tV + sub * L::kTile16, kvm, rmask);
+          }
         }
       }
       __syncthreads();                                    // the buffer is refilled next step
@@ -303,31 +317,63 @@ __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams 
   uint8_t* sK = kv + warp * 4 * L::kTile16;                // 2 K buffers, then 2 V buffers
   uint8_t* sV = sK + 2 * L::kTile16;
 
-  // ---- masked passes, per warp: spatial (original order), temporal (frame-major)
-  for (int pass = 1; pass < 3; ++pass) {
-    const bool fm = pass == 2;
+  // ---- masked passes, per warp. Mode 0: spatial (original order) and
+  // temporal (frame-major order); mode 1: one tile window per candidate (3D
+  // tile order, padding slots inside tiles masked)
+  const int bt = p.tile[0], bhh = p.tile[1], bw = p.tile[2];
+  const int tnh = (p.H + bhh - 1) / bhh, tnw = (p.W + bw - 1) / bw;
+  const int tnb = ((p.T + bt - 1) / bt) * tnh * tnw;
+  int qt = 0, qh = 0, qw = 0;                              // the row's tile (mode 1)
+  if (p.mode == 1 && my_tok >= 0) {
+    qt = my_tok / geo.HW / bt;
+    qh = (my_tok / p.W) % p.H / bhh;
+    qw = my_tok % p.W / bw;
+  }
+  // slot s of the pass's order -> token, or -1 for a padding slot
+  auto slot_token = [&](int pass, int slot) -> int {
+    if (p.mode == 0) {
+      if (slot >= p.N) return -1;
+      return pass == 2 ? (slot % p.T) * geo.HW + slot / p.T : slot;
+    }
+    const int b = slot / p.block, s = slot % p.block;
+    const int t = b / (tnh * tnw) * bt + s / (bhh * bw);
+    const int h = (b / tnw) % tnh * bhh + (s / bw) % bhh;
+    const int w = b % tnw * bw + s % bw;
+    return (t < p.T && h < p.H && w < p.W) ? (t * p.H + h) * p.W + w : -1;
+  };
+  const int nb_pass = p.mode == 0 ? nb : tnb;
+  for (int pass = 1; pass <= p.n_pat; ++pass) {
+    int win[3] = {1, 1, 1};
+    if (p.mode == 1) { win[0] = p.win[pass - 1][0]; win[1] = p.win[pass - 1][1]; win[2] = p.win[pass - 1][2]; }
     // rows (bits 0..15) that keep key block b under this pass's pattern
     auto keeps = [&](int b) -> uint32_t {
       bool kp = false;
-      if (my_tok >= 0) kp = pass == 1 ? spatial_keep(geo, my_tok, b) : temporal_keep(geo, my_tok, b);
+      if (my_tok >= 0) {
+        if (p.mode == 1) kp = window_keep(b, tnh, tnw, qt, qh, qw, win);
+        else kp = pass == 1 ? spatial_keep(geo, my_tok, b) : temporal_keep(geo, my_tok, b);
+      }
       return __ballot_sync(0xffffffffu, kp) & 0xFFFFu;
     };
     auto next_block = [&](int from, uint32_t& rmask) -> int {
-      for (int x = from; x < nb; ++x) {
+      for (int x = from; x < nb_pass; ++x) {
         const uint32_t mk = keeps(x);
         if (mk) { rmask = mk; return x; }
       }
-      return nb;
+      return nb_pass;
     };
-    // 16 key rows of step (b, sub) into buffer ``buf``; slots past N are zero
+    // keys of step (b, sub) that exist
+    auto step_keys = [&](int b, int sub) -> uint32_t {
+      const bool ok = lane < kStepKeys && slot_token(pass, b * p.block + sub * kStepKeys + lane) >= 0;
+      return __ballot_sync(0xffffffffu, ok) & 0xFFFFu;
+    };
+    // 16 key rows of step (b, sub) into buffer ``buf``; padding slots are zero
     auto load_step = [&](int buf, int b, int sub) {
       for (int e = lane; e < kStepKeys * kChunks; e += 32) {
         const int r = e / kChunks, c = e % kChunks;
-        const int slot = b * p.block + sub * kStepKeys + r;
+        const int tok = slot_token(pass, b * p.block + sub * kStepKeys + r);
         uint8_t* dk = sK + buf * L::kTile16 + tile_off<D>(r, c);
         uint8_t* dv = sV + buf * L::kTile16 + tile_off<D>(r, c);
-        if (slot < p.N) {
-          const int tok = fm ? (slot % p.T) * geo.HW + slot / p.T : slot;
+        if (tok >= 0) {
           cp_async16(dk, k + (size_t)tok * D + c * 8);
           cp_async16(dv, v + (size_t)tok * D + c * 8);
         } else {
@@ -340,19 +386,19 @@ __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams 
     reset();
     uint32_t rmask = 0;
     int b = next_block(0, rmask), sub = 0, buf = 0;
-    if (b < nb) load_step(0, b, 0);
-    while (b < nb) {
+    if (b < nb_pass) load_step(0, b, 0);
+    while (b < nb_pass) {
       int b2 = b, s2 = sub + 1;
       uint32_t rm2 = rmask;
       if (s2 == subs) { s2 = 0; b2 = next_block(b + 1, rm2); }
-      if (b2 < nb) {
+      if (b2 < nb_pass) {
         load_step(buf ^ 1, b2, s2);
         cp_async_wait<1>();
       } else {
         cp_async_wait<0>();
       }
       __syncwarp();
-      step16(sK + buf * L::kTile16, sV + buf * L::kTile16, b * p.block + sub * kStepKeys, rmask);
+      step16(sK + buf * L::kTile16, sV + buf * L::kTile16, step_keys(b, sub), rmask);
       __syncwarp();                                       // tile free for the load two steps on
       buf ^= 1;
       b = b2;
@@ -363,26 +409,24 @@ __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams 
   }
 }
 
-// Per head, the rows' errors summed in a fixed order (lane-strided partial
-// sums, then a fixed shuffle tree): the result does not depend on timing.
+// Per head and pattern, the rows' errors summed in a fixed order
+// (lane-strided partial sums, then a fixed shuffle tree), and the pattern
+// with the lowest mean error (ties: the earlier one).
 __global__ void profile_reduce_kernel(ProfileParams p) {
   const int bh = blockIdx.x, lane = threadIdx.x;
-  float s = 0.f, t = 0.f;
-  const float* re = p.row_err + (size_t)bh * p.n_rows * 2;
-  for (int r = lane; r < p.n_rows; r += 32) {
-    s += re[(size_t)r * 2];
-    t += re[(size_t)r * 2 + 1];
+  const float* re = p.row_err + (size_t)bh * p.n_rows * p.n_pat;
+  const float n = (float)p.n_rows * (float)p.d;
+  int best = 0;
+  float best_v = 0.f;
+  for (int c = 0; c < p.n_pat; ++c) {
+    float s = 0.f;
+    for (int r = lane; r < p.n_rows; r += 32) s += re[(size_t)r * p.n_pat + c];
+    for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float m = s / n;
+    if (lane == 0) p.mse[bh * p.n_pat + c] = m;
+    if (c == 0 || m < best_v) { best = c; best_v = m; }
   }
-  for (int o = 16; o >= 1; o >>= 1) {
-    s += __shfl_xor_sync(0xffffffffu, s, o);
-    t += __shfl_xor_sync(0xffffffffu, t, o);
-  }
-  if (lane == 0) {
-    const float n = (float)p.n_rows * (float)p.d;
-    p.mse[bh * 2] = s / n;
-    p.mse[bh * 2 + 1] = t / n;
-    p.is_temporal[bh] = (t / n) < (s / n) ? 1 : 0;
-  }
+  if (lane == 0) p.choice[bh] = (int8_t)best;
 }
 
 }  // namespace

@@ -20,7 +20,8 @@ def policy_kwargs(wl: Workload):
         return dict(kind="topk", block=wl.block, tile=wl.tile, topk=wl.topk,
                     keep_diagonal=wl.keep_diagonal, summarizer=wl.summarizer)
     if wl.kind == "sta":
-        return dict(kind="sta", block=wl.block, tile=wl.tile, window=wl.window)
+        return dict(kind="sta", block=wl.block, tile=wl.tile, window=wl.window,
+                    head_windows=wl.head_windows or None)
     if wl.kind == "spatiotemporal":
         return dict(kind="spatiotemporal", block=wl.block, temporal_heads=wl.temporal_heads,
                     heads=wl.heads, sink_tokens=wl.sink_tokens, frame_radius=1)
@@ -72,6 +73,10 @@ SMALL = {
                                    window=(3, 3, 3), summarizer="min"),
     "topk_max_d64": CONFIGS["tiny_topk"].with_(name="topk_max_d64", config_id=110,
                                                summarizer="max"),
+    # a window per head (Sliding Tile Attention review: head specialization)
+    "sta_head_windows": Workload(name="sta_head_windows", config_id=111, T=9, H=10, W=19, heads=3,
+                                 head_dim=128, kind="sta", tile=(4, 4, 8), block=128,
+                                 window=(3, 3, 3), head_windows=((1, 1, 1), (3, 5, 3), (5, 1, 1))),
 }
 
 

@@ -94,3 +94,44 @@ def test_profile_full_size_sampled():
     rows = np.ascontiguousarray(sample_rows(wl2.N, wl2.heads, fraction=0.01, seed=9)[:, ::18][:, :64])
     x, is_t, mse, row_err = _run(wl2, rows, wl2.sink_tokens)
     _check_heads(wl2, x, rows, is_t, mse, row_err, wl2.sink_tokens, range(wl2.heads))
+
+
+def _run_search(wl, rows, cands):
+    from sparse_attention_video_b200 import sta_window_search
+    x = make_qkv(wl)
+    q, k, v = (_dev(x[n]) for n in "qkv")
+    choice, mse, row_err = sta_window_search(q, k, v, torch.from_numpy(rows).cuda(), wl.T, wl.H,
+                                             wl.W, wl.tile, cands, block=wl.block)
+    torch.cuda.synchronize()
+    return x, choice.cpu().numpy(), mse.cpu().numpy(), row_err.cpu().numpy()
+
+
+def test_sta_window_search_matches_oracle():
+    # Sliding Tile Attention review, Algorithm 1: per head, the candidate
+    # window whose output is closest (MSE) to full attention
+    wl = C.SMALL["sta_ragged"]                      # 9 x 10 x 19, tiles 4 x 4 x 8, 3 heads
+    cands = [(1, 1, 1), (3, 3, 3), (1, 3, 5), (3, 1, 1)]
+    rows = sample_rows(wl.N, wl.heads, fraction=0.1, seed=13)
+    x, choice, mse, row_err = _run_search(wl, rows, cands)
+    for h in range(wl.heads):
+        qf, kf, vf = (bf16_bits_to_f32(x[n][0, h]) for n in "qkv")
+        ref = profile.sta_window_search(qf, kf, vf, rows[h], wl.T, wl.H, wl.W, wl.tile, cands)
+        for c in range(len(cands)):
+            assert abs(mse[h, c] - ref["mse"][c]) <= 0.05 * ref["mse"][c] + 1e-7, (h, c, mse[h], ref["mse"])
+            re = ((ref["o"][c] - ref["o_full"]) ** 2).sum(axis=1)
+            np.testing.assert_allclose(row_err[h, :, c], re, rtol=0.1, atol=0.02 * re.max() + 1e-6)
+        srt = sorted(ref["mse"])
+        if srt[1] - srt[0] > 0.1 * srt[1]:
+            assert choice[h] == ref["choice"], (h, mse[h], ref["mse"])
+
+
+def test_sta_window_search_full_grid_candidate_wins():
+    # a window that spans the tile grid (3 x 3 x 3 tiles) keeps every key; it
+    # visits them in tile order, so its bf16 P rounds differently from the
+    # full pass (order of the online softmax), not to zero error
+    wl = C.SMALL["sta_ragged"]
+    cands = [(3, 3, 3), (5, 5, 5), (1, 1, 1)]
+    rows = sample_rows(wl.N, wl.heads, fraction=0.1, seed=14)
+    _, choice, mse, _ = _run_search(wl, rows, cands)
+    assert np.all(mse[:, 1] < 1e-5 * np.minimum(mse[:, 0], mse[:, 2]))
+    assert np.all(choice == 1)
