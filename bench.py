@@ -424,6 +424,32 @@ def main():
             "temporal_heads_found": int(is_t.sum().item()),
             "kernel": "profile_kernel (mma.sync m16n8k16; all three passes in the time)"}}
         log("head profiler timed")
+    if not args.no_profile and wl.kind == "sta":
+        # the STA per-head window search (Sliding Tile Attention review, key
+        # machinery) on 1 % of each head's rows, four candidate windows
+        from sparse_attention_video_b200 import sta_window_search
+        from synthetic import sample_rows
+        rows = torch.from_numpy(sample_rows(wl.N, wl.heads, 0.01, seed=2024)).to(dev)
+        cands = [(3, 3, 3), (1, 3, 5), (5, 3, 1), (3, 5, 3)]
+        for _ in range(2):
+            sta_window_search(q, k, v, rows, wl.T, wl.H, wl.W, wl.tile, cands, block=wl.block,
+                              stream=stream)
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        p0.record(stream)
+        for _ in range(5):
+            choice, _, _ = sta_window_search(q, k, v, rows, wl.T, wl.H, wl.W, wl.tile, cands,
+                                             block=wl.block, stream=stream)
+        p1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = p0.elapsed_time(p1) / 5
+        full_flops = 4.0 * wl.head_dim * rows.numel() * wl.N
+        prof = {"window_search": {
+            "ms": ms, "rows_per_head": int(rows.shape[1]), "candidates": cands,
+            "full_pass_tflops": full_flops / (ms * 1e-3) / 1e12,
+            "choices": torch.bincount(choice.long().cpu(), minlength=len(cands)).tolist(),
+            "kernel": "profile_kernel, tile-window mode (mma.sync m16n8k16)"}}
+        log("window search timed")
 
     if rank != 0:
         if world > 1:
