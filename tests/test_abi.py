@@ -118,6 +118,36 @@ def test_summarizer_and_profiler_arguments_are_checked_on_the_host():
     assert L.sparse_attn_profile_heads(ctypes.byref(pr), ctypes.byref(ok_pol), *a) == N.SA_ERR_WORKSPACE
 
 
+def test_window_search_and_head_windows_are_checked_on_the_host():
+    L = N.lib()
+    m, s = ctypes.c_size_t(), ctypes.c_size_t()
+    wl = CONFIGS["sta_wan21_1p3b_480p"]
+    pr = N.Problem(1, wl.heads, wl.T, wl.H, wl.W, wl.head_dim)
+    ok = make_policy(**{**C.policy_kwargs(wl), "head_windows": [(3, 3, 3)] * wl.heads})
+    assert L.sparse_attn_workspace_size(ctypes.byref(pr), ctypes.byref(ok), ctypes.byref(m),
+                                        ctypes.byref(s)) == N.SA_OK
+    for bad_w in ((2, 3, 3), (3, 3, 0), (257, 1, 1)):
+        bad = make_policy(**{**C.policy_kwargs(wl), "head_windows": [(3, 3, 3)] * (wl.heads - 1) + [bad_w]})
+        assert L.sparse_attn_workspace_size(ctypes.byref(pr), ctypes.byref(bad), ctypes.byref(m),
+                                            ctypes.byref(s)) == N.SA_ERR_INVALID_ARG, bad_w
+    sta = make_policy("sta", tile=wl.tile, window=(1, 1, 1))
+    cand = (ctypes.c_int * 6)(3, 3, 3, 1, 3, 5)
+    args = [0x1000, 0x1000, 0x1000, 0x1000, 16, cand, 2, 0x1000, 0x1000, 0x1000, None, None]
+    call = lambda pol, a: L.sparse_attn_sta_window_search(ctypes.byref(pr), ctypes.byref(pol), *a)
+    st = make_policy("spatiotemporal", block=128)
+    assert call(st, args) == N.SA_ERR_INVALID_ARG                  # STA policies only
+    for i, val in ((6, 0), (6, 9), (4, 0), (5, None)):               # candidate count, rows, list
+        a = list(args)
+        a[i] = val
+        assert call(sta, a) == N.SA_ERR_INVALID_ARG, (i, val)
+    even = (ctypes.c_int * 6)(3, 3, 3, 1, 2, 5)
+    a = list(args)
+    a[5] = even
+    assert call(sta, a) == N.SA_ERR_INVALID_ARG
+    wrong_tile = make_policy("sta", tile=(4, 4, 4), window=(1, 1, 1))   # 64 tokens != block 128
+    assert call(wrong_tile, args) == N.SA_ERR_INVALID_ARG
+
+
 def test_strerror_covers_every_code():
     for code in range(7):
         assert N.strerror(code) and N.strerror(code) != "unknown status"
