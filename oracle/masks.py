@@ -284,3 +284,29 @@ def fg_threshold(scores, keep_fraction):
 def fg_keep(scores, tau):
     """Slices kept: s >= tau (every slice tied at tau is kept)."""
     return scores >= tau
+
+
+def fg_cached_keep(q, k, group, tau=None):
+    """Slices kept by the cached rule, bool [G, N_keys].
+
+    FG-Attn review (referee summary, minor comment on the thresholds, and the
+    falsifier): the full attention map is computed once, and an M x 1 slice
+    (group g of M contiguous queries, key j) is kept when at least one query
+    of the group gives key j an attention probability above tau_cached, which
+    Sec. 5.1 sets to 0.5/N. N is the number of keys. The probabilities are the
+    float32 softmax of q.k / sqrt(d) over all keys, one query row at a time.
+    The last group holds only the queries that exist. Strictly above: a
+    probability equal to tau does not keep its slice.
+    """
+    n, d = q.shape
+    nk = k.shape[0]
+    if tau is None:
+        tau = 0.5 / nk
+    t = F32(tau)
+    kf = k.astype(F32)
+    scale = F32(1.0 / math.sqrt(d))
+    keep = np.zeros((-(-n // group), nk), dtype=bool)
+    for i in range(n):
+        p = softmax_f32((kf @ q[i].astype(F32)) * scale)
+        keep[i // group] |= p > t
+    return keep

@@ -24,6 +24,10 @@ def head_mask(wl, q, k, head, force_choice=None):
     argmax, for a head whose summed SICS scores tie within the tolerance."""
     d = wl.head_dim
     info = {}
+    if wl.kind == "fg" and wl.fg_rule == "cached":
+        tau = 0.5 / k.shape[0]
+        info.update(tau=tau)
+        return dict(keep_groups=masks.fg_cached_keep(q, k, wl.fg_group, tau), info=info)
     if wl.kind == "fg":
         s = masks.fg_scores(q, k, wl.fg_group)
         tau, r = masks.fg_threshold(s, wl.fg_keep_fraction)

@@ -18,7 +18,10 @@ Mask kinds:
              carries the argument", Eqs. 3-5).
   "fg"       M x 1 key slices: groups of M contiguous queries keep the keys
              whose score against the group's mean query passes a per-head
-             threshold (FG-Attn review, skeptic critique on Sec. 4.4).
+             threshold (FG-Attn review, skeptic critique on Sec. 4.4). With
+             fg_rule "cached", the groups instead keep every key that one of
+             their queries gives a full-attention probability above 0.5/N
+             (FG-Attn review, the cached strategy).
 """
 from dataclasses import dataclass, field
 from typing import Optional, Tuple
@@ -45,6 +48,7 @@ class Workload:
     top_p: float = 0.0
     fg_group: int = 0
     fg_keep_fraction: float = 0.0
+    fg_rule: str = "pooled"                        # fg: "pooled" (q_avg scores) or "cached" (full map)
     block: int = 128                               # tokens per block in the working layout
     summarizer: str = "mean"                       # topk, spade: block summary ("mean", "max", "min")
     head_windows: Tuple[Tuple[int, int, int], ...] = ()   # sta: a window per head (empty: window)

@@ -296,6 +296,89 @@ def test_fg_scores_use_group_mean_query():
     np.testing.assert_allclose(s, qbar @ k.T / 2.0, rtol=1e-5, atol=1e-6)
 
 
+# ---------------------------------------------------------------- FG cached slices
+def _one_hot_qk(n, d, a):
+    # k_j = e_j, q_i = a*sqrt(d)*e_i: score a on the diagonal, 0 elsewhere, so
+    # P_ii = e^a / (e^a + n - 1) and P_ij = 1 / (e^a + n - 1) for j != i
+    k = np.eye(n, d, dtype=np.float32)
+    q = (k * np.float32(a * math.sqrt(d))).astype(np.float32)
+    return q, k
+
+
+@pytest.mark.parametrize("n,group", [(48, 8), (10, 4), (37, 16)])
+def test_fg_cached_one_hot_closed_form(n, group):
+    # off-diagonal P exceeds 0.5/n exactly when e^a < n + 1; the diagonal
+    # always does. Below the crossing every slice is kept; above it each group
+    # keeps exactly the keys of its own queries (the ragged last group too:
+    # padding rows taken as zero queries would keep every key).
+    d = 64
+    q, k = _one_hot_qk(n, d, math.log((n + 1) / 1.5))
+    assert masks.fg_cached_keep(q, k, group).all()
+    q, k = _one_hot_qk(n, d, math.log((n + 1) * 1.5))
+    got = masks.fg_cached_keep(q, k, group)
+    want = np.zeros_like(got)
+    for i in range(n):
+        want[i // group, i] = True
+    assert np.array_equal(got, want)
+
+
+def test_fg_cached_strictly_above_tau():
+    # identical keys: every probability is 1/n; at tau = 1/n nothing is kept,
+    # at the default 0.5/n everything is
+    n, d = 20, 8
+    g = np.random.default_rng(6)
+    q = g.standard_normal((n, d)).astype(np.float32)
+    k = np.tile(g.standard_normal((1, d)).astype(np.float32), (n, 1))
+    assert not masks.fg_cached_keep(q, k, 4, tau=1.0 / n).any()
+    assert masks.fg_cached_keep(q, k, 4).all()
+
+
+def test_fg_cached_matches_torch_softmax_and_group_max_pool():
+    # a different route: float64 torch softmax of the whole map, then the max
+    # over each group of query rows by max_pool1d (ceil_mode covers the ragged
+    # tail); decisions within 1e-4 relative of tau are not compared
+    g = np.random.default_rng(7)
+    n, d, group = 203, 32, 8
+    q = (4.0 * g.standard_normal((n, d))).astype(np.float32)
+    k = g.standard_normal((n, d)).astype(np.float32)
+    got = masks.fg_cached_keep(q, k, group)
+    p = torch.softmax(torch.from_numpy(q).double() @ torch.from_numpy(k).double().T / math.sqrt(d), dim=1)
+    pmax = torch.nn.functional.max_pool1d(p.T[None], group, group, ceil_mode=True)[0].T.numpy()
+    tau = 0.5 / n
+    clear = np.abs(pmax - tau) > 1e-4 * tau
+    assert clear.mean() > 0.99
+    assert np.array_equal(got[clear], (pmax > tau)[clear])
+    assert 0.05 < got.mean() < 0.95                                  # neither rule is trivial here
+
+
+def test_fg_cached_keeps_each_query_argmax_and_bounds_dropped_mass():
+    # P_max >= 1/n > 0.5/n, so every query's top key is kept; every dropped
+    # key has P <= 0.5/n, so a query loses at most half of its mass
+    g = np.random.default_rng(8)
+    n, d, group = 150, 16, 8
+    q = (3.0 * g.standard_normal((n, d))).astype(np.float32)
+    k = g.standard_normal((n, d)).astype(np.float32)
+    keep = masks.fg_cached_keep(q, k, group)
+    s = (q.astype(np.float64) @ k.astype(np.float64).T) / math.sqrt(d)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    for i in range(n):
+        row = keep[i // group]
+        assert row[int(np.argmax(p[i]))]
+        assert p[i][~row].sum() <= 0.5 + 1e-6
+
+
+def test_fg_cached_pipeline_uses_half_over_n():
+    wl = CONFIGS["fg_slices_hunyuan_720p"].with_(name="fg_cached_small", T=2, H=4, W=16, heads=1,
+                                                 fg_rule="cached")
+    x = make_qkv(wl)
+    q, k = (bf16_bits_to_f32(x[c][0, 0]) for c in "qk")
+    out = pipeline.head_mask(wl, q, k, 0)
+    assert out["info"]["tau"] == 0.5 / wl.N
+    assert out["keep_groups"].shape == (math.ceil(wl.N / wl.fg_group), wl.N)
+    assert np.array_equal(out["keep_groups"], masks.fg_cached_keep(q, k, wl.fg_group))
+
+
 # ---------------------------------------------------------------- SPADE pipeline on a small grid
 def test_spade_small_grid_pipeline_invariants():
     from synthetic import Workload
