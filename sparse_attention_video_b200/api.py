@@ -65,12 +65,37 @@ def _stream_ptr(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _check_qkv(t, problem, name):
-    N_ = problem.T * problem.H * problem.W
-    want = (problem.batch, problem.heads, N_, problem.head_dim)
-    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != want:
-        raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {want}, "
-                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+def _check_tensor(t, shape, dtypes, name, device=None):
+    """Raise unless ``t`` is a contiguous CUDA tensor of one of ``dtypes`` and
+    the given shape, on ``device`` when one is given. The kernels see only a
+    pointer, so a wrong size here would read or write past the buffer."""
+    ok = (isinstance(t, torch.Tensor) and t.dtype in dtypes and t.is_cuda and t.is_contiguous()
+          and tuple(t.shape) == tuple(shape) and (device is None or t.device == device))
+    if not ok:
+        kinds = "/".join(str(d).replace("torch.", "") for d in dtypes)
+        where = f" on {device}" if device is not None else ""
+        got = (f"{t.dtype} {tuple(t.shape)} on {t.device}" if isinstance(t, torch.Tensor)
+               else type(t).__name__)
+        raise ValueError(f"{name} must be a contiguous CUDA {kinds} tensor of shape "
+                         f"{tuple(shape)}{where}, got {got}")
+
+
+def _qkv_shape(problem):
+    return (problem.batch, problem.heads, problem.T * problem.H * problem.W, problem.head_dim)
+
+
+def _check_qkv(t, problem, name, device=None):
+    _check_tensor(t, _qkv_shape(problem), (torch.bfloat16,), name, device)
+
+
+def _check_lse(t, problem, device):
+    _check_tensor(t, _qkv_shape(problem)[:3], (torch.float32,), "lse", device)
+
+
+def _check_scratch(ws, device):
+    if not (isinstance(ws, torch.Tensor) and ws.is_cuda and ws.device == device
+            and ws.is_contiguous() and ws.numel() * ws.element_size() >= 256):
+        raise ValueError(f"scratch_ws must be a contiguous CUDA tensor of at least 256 bytes on {device}")
 
 
 class SparseAttention:
@@ -80,10 +105,23 @@ class SparseAttention:
         self.problem = N.Problem(batch, heads, T, H, W, head_dim)
         self.policy = policy
         self.mask_bytes, self.scratch_bytes = N.workspace_size(self.problem, policy)
-        self.device = torch.device(device)
-        self.mask_ws = torch.empty(self.mask_bytes, dtype=torch.uint8, device=self.device)
+        self.mask_ws = torch.empty(self.mask_bytes, dtype=torch.uint8, device=torch.device(device))
+        self.device = self.mask_ws.device                 # "cuda" resolved to its index
         self.scratch_ws = torch.empty(max(self.scratch_bytes, 256), dtype=torch.uint8,
                                       device=self.device)
+        if policy.kind == N.SA_MASK_EXPLICIT:
+            self._check_explicit_bits()
+
+    def _check_explicit_bits(self):
+        bits = getattr(self.policy, "_keep_bits", None)
+        if bits is None or not self.policy.explicit_bits:
+            raise ValueError("an explicit policy needs explicit_bits")
+        need = N.export_bytes(self.problem, self.policy, N.SA_EXPORT_BLOCK_BITS)
+        if not (bits.is_cuda and bits.device == self.device and bits.is_contiguous()
+                and bits.element_size() == 4 and not bits.is_floating_point()
+                and bits.numel() * 4 == need):
+            raise ValueError(f"explicit_bits must be a contiguous CUDA int32/uint32 tensor of "
+                             f"{need // 4} words ([batch*heads][nb][ceil(nb/32)]) on {self.device}")
 
     @property
     def n_tokens(self):
@@ -92,19 +130,21 @@ class SparseAttention:
     def build_mask(self, q, k, stream=None):
         needs = self.policy.kind in (N.SA_MASK_TOPK, N.SA_MASK_SPADE, N.SA_MASK_FG)
         if needs:
-            _check_qkv(q, self.problem, "q")
-            _check_qkv(k, self.problem, "k")
+            _check_qkv(q, self.problem, "q", self.device)
+            _check_qkv(k, self.problem, "k", self.device)
         N.build_mask(self.problem, self.policy, q.data_ptr() if needs else None,
                      k.data_ptr() if needs else None, self.mask_ws.data_ptr(),
                      self.scratch_ws.data_ptr(), _stream_ptr(stream))
 
     def forward(self, q, k, v, out=None, lse=None, stream=None):
         for t, n in ((q, "q"), (k, "k"), (v, "v")):
-            _check_qkv(t, self.problem, n)
+            _check_qkv(t, self.problem, n, self.device)
         if out is None:
             out = torch.empty_like(q)
         if lse is None:
             lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+        _check_qkv(out, self.problem, "out", self.device)
+        _check_lse(lse, self.problem, self.device)
         N.forward(self.problem, self.policy, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                   self.mask_ws.data_ptr(), self.scratch_ws.data_ptr(), out.data_ptr(),
                   lse.data_ptr(), _stream_ptr(stream))
@@ -112,11 +152,15 @@ class SparseAttention:
 
     def permute(self, q, k, v, stream=None):
         for t, n in ((q, "q"), (k, "k"), (v, "v")):
-            _check_qkv(t, self.problem, n)
+            _check_qkv(t, self.problem, n, self.device)
         N.permute(self.problem, self.policy, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                   self.mask_ws.data_ptr(), self.scratch_ws.data_ptr(), _stream_ptr(stream))
 
     def attend(self, q, k, v, out, lse, stream=None):
+        for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+            _check_qkv(t, self.problem, n, self.device)
+        if lse is not None:
+            _check_lse(lse, self.problem, self.device)
         N.attend(self.problem, self.policy, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                  self.mask_ws.data_ptr(), self.scratch_ws.data_ptr(), out.data_ptr(),
                  lse.data_ptr() if lse is not None else None, _stream_ptr(stream))
@@ -143,6 +187,22 @@ class SparseAttention:
         return N.status(self.scratch_ws.data_ptr(), _stream_ptr(stream), clear)
 
 
+def _sampled_problem(q, k, v, rows, T, H, W, scratch_ws):
+    """Problem of a sampled-row call, after checking every tensor it is given."""
+    if not isinstance(q, torch.Tensor) or q.dim() != 4:
+        raise ValueError("q must be a CUDA bf16 tensor [batch, heads, N, head_dim]")
+    B, Hh, _, d = q.shape
+    problem = N.Problem(B, Hh, T, H, W, d)
+    if not (isinstance(rows, torch.Tensor) and rows.dim() == 2 and rows.shape[0] == B * Hh):
+        raise ValueError("rows must be a contiguous CUDA int32 tensor [batch*heads, n_rows]")
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        _check_qkv(t, problem, name, q.device)
+    _check_tensor(rows, tuple(rows.shape), (torch.int32,), "rows", q.device)
+    if scratch_ws is not None:
+        _check_scratch(scratch_ws, q.device)
+    return problem
+
+
 def profile_heads(q, k, v, rows, T, H, W, block=128, sink_tokens=0, frame_radius=1,
                   stream=None, scratch_ws=None):
     """SVG online head profiler (Sparse VideoGen review, key machinery).
@@ -153,13 +213,8 @@ def profile_heads(q, k, v, rows, T, H, W, block=128, sink_tokens=0, frame_radius
     [batch*heads, n_rows, 2]) as CUDA tensors; the work is queued on
     ``stream`` and nothing is synchronised.
     """
-    B, Hh, N_, d = q.shape
-    problem = N.Problem(B, Hh, T, H, W, d)
-    for t, name in ((q, "q"), (k, "k"), (v, "v")):
-        _check_qkv(t, problem, name)
-    if rows.dtype != torch.int32 or not rows.is_cuda or not rows.is_contiguous() \
-            or rows.dim() != 2 or rows.shape[0] != B * Hh:
-        raise ValueError("rows must be a contiguous CUDA int32 tensor [batch*heads, n_rows]")
+    problem = _sampled_problem(q, k, v, rows, T, H, W, scratch_ws)
+    B, Hh = problem.batch, problem.heads
     n_rows = rows.shape[1]
     policy = make_policy("spatiotemporal", block=block, temporal_heads=(), heads=Hh,
                          sink_tokens=sink_tokens, frame_radius=frame_radius)
@@ -184,13 +239,8 @@ def sta_window_search(q, k, v, rows, T, H, W, tile, candidates, block=128, strea
     [batch*heads, n_rows, n_candidates]) as CUDA tensors, queued on ``stream``.
     ``[candidates[c] for c in choice]`` is a ``head_windows`` for make_policy.
     """
-    B, Hh, N_, d = q.shape
-    problem = N.Problem(B, Hh, T, H, W, d)
-    for t, name in ((q, "q"), (k, "k"), (v, "v")):
-        _check_qkv(t, problem, name)
-    if rows.dtype != torch.int32 or not rows.is_cuda or not rows.is_contiguous() \
-            or rows.dim() != 2 or rows.shape[0] != B * Hh:
-        raise ValueError("rows must be a contiguous CUDA int32 tensor [batch*heads, n_rows]")
+    problem = _sampled_problem(q, k, v, rows, T, H, W, scratch_ws)
+    B, Hh = problem.batch, problem.heads
     n_rows, nc = rows.shape[1], len(candidates)
     policy = make_policy("sta", block=block, tile=tile, window=(1, 1, 1))
     cand = (ctypes.c_int * (3 * nc))(*[int(x) for c in candidates for x in c])

@@ -152,3 +152,51 @@ def test_strerror_covers_every_code():
     for code in range(7):
         assert N.strerror(code) and N.strerror(code) != "unknown status"
     assert N.strerror(99) == "unknown status"
+
+
+def test_python_api_checks_tensors_before_any_native_call():
+    # The kernels see bare pointers, so the Python layer must refuse a tensor
+    # of the wrong kind, shape, dtype or device before anything is launched.
+    # CPU tensors stand in for the misplaced ones: every call must raise here.
+    import torch
+    from sparse_attention_video_b200 import api, profile_heads, sta_window_search
+    pr = N.Problem(1, 2, 3, 4, 8, 64)
+    good = (1, 2, 96, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        api._check_qkv(torch.zeros(good, dtype=torch.bfloat16), pr, "q")
+    with pytest.raises(ValueError, match="shape"):
+        api._check_qkv(torch.zeros((1, 2, 95, 64), dtype=torch.bfloat16), pr, "out")
+    with pytest.raises(ValueError, match="float32"):
+        api._check_lse(torch.zeros((1, 2, 96), dtype=torch.float16), pr, None)
+    with pytest.raises(ValueError, match="got list"):
+        api._check_qkv([0.0], pr, "v")
+    with pytest.raises(ValueError, match="scratch_ws"):
+        api._check_scratch(torch.zeros(256, dtype=torch.uint8), torch.device("cpu"))
+    q = torch.zeros(good, dtype=torch.bfloat16)
+    rows = torch.zeros((2, 4), dtype=torch.int32)
+    for fn, extra in ((profile_heads, ()), (sta_window_search, ((1, 1, 64), [(1, 1, 1)]))):
+        with pytest.raises(ValueError):
+            fn(q, q, q, rows, 3, 4, 8, *extra, block=64)
+        with pytest.raises(ValueError, match="rows"):
+            fn(q, q, q, rows[:1], 3, 4, 8, *extra, block=64)
+        with pytest.raises(ValueError, match="q must be"):
+            fn(q[0], q, q, rows, 3, 4, 8, *extra, block=64)
+
+
+def test_explicit_bits_are_checked_against_the_mask_size():
+    import torch
+    from sparse_attention_video_b200 import SparseAttention, make_policy
+    sa = SparseAttention.__new__(SparseAttention)      # no device workspaces on this host
+    sa.problem = N.Problem(1, 2, 3, 4, 128, 64)
+    sa.device = torch.device("cuda", 0)
+    sa.policy = make_policy("explicit", block=128, explicit_layout=N.SA_LAYOUT_IDENTITY)
+    with pytest.raises(ValueError, match="needs explicit_bits"):
+        sa._check_explicit_bits()
+    need = 2 * 12 * 1                                  # [heads][nb = 12 blocks][1 word]
+    for bad in (torch.zeros(need, dtype=torch.int32),           # host memory
+                torch.zeros(need, dtype=torch.float32)):        # not words
+        sa.policy = make_policy("explicit", block=128, explicit_layout=N.SA_LAYOUT_IDENTITY,
+                                explicit_bits=bad)
+        assert N.export_bytes(sa.problem, sa.policy, N.SA_EXPORT_BLOCK_BITS) == 4 * need
+        with pytest.raises(ValueError, match="explicit_bits must be"):
+            sa._check_explicit_bits()
