@@ -41,7 +41,9 @@ int check_problem(const sa_problem* pr) {
 
 int check_tile(const sa_problem& pr, const int* t, int block) {
   if (t[0] < 1 || t[1] < 1 || t[2] < 1) return SA_ERR_INVALID_ARG;
-  if (t[0] * t[1] * t[2] != block) return SA_ERR_INVALID_ARG;
+  // product in 64 bits, stopped once it passes the block: no overflow for any int extents
+  const long long t01 = (long long)t[0] * t[1];
+  if (t01 > block || t01 * t[2] != block) return SA_ERR_INVALID_ARG;
   if (t[0] > 256 || t[1] > 256 || t[2] > 256) return SA_ERR_UNSUPPORTED;
   if (tile_blocks(pr, t) > kMaxBlocks) return SA_ERR_UNSUPPORTED;
   return SA_OK;
@@ -194,17 +196,17 @@ ScratchLayout scratch_layout(const sa_problem& pr, const sa_policy& po, const Ma
 // ------------------------------------------------------------------ tensor maps
 typedef EncodeFn EncodeTiledFn;
 
+// Resolved once, on first use; a function-local static is initialised exactly
+// once even when several host threads make their first call together.
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static const EncodeTiledFn fn = [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+      return reinterpret_cast<EncodeTiledFn>(p);
+    return EncodeTiledFn(nullptr);
+  }();
   return fn;
 }
 

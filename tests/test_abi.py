@@ -74,6 +74,11 @@ def test_invalid_arguments_are_rejected_on_the_host():
     wrong_tile = make_policy("sta", tile=(4, 4, 4), window=(3, 3, 3))  # 64 tokens != block 128
     assert L.sparse_attn_workspace_size(ctypes.byref(pr), ctypes.byref(wrong_tile), ctypes.byref(m),
                                         ctypes.byref(s)) == N.SA_ERR_INVALID_ARG
+    # extents whose product overflows 32 bits are refused, not wrapped around
+    for t in ((1 << 16, 1 << 16, 1), (1 << 11, 1 << 11, 1 << 11), (1, 1 << 30, 1 << 30)):
+        huge = make_policy("sta", tile=t, window=(3, 3, 3))
+        assert L.sparse_attn_workspace_size(ctypes.byref(pr), ctypes.byref(huge), ctypes.byref(m),
+                                            ctypes.byref(s)) == N.SA_ERR_INVALID_ARG, t
     # null / misaligned device pointers never reach the device
     assert L.sparse_attn_forward(ctypes.byref(pr), ctypes.byref(pol), None, None, None, None, None,
                                  None, None, None) == N.SA_ERR_INVALID_ARG
