@@ -841,7 +841,9 @@ cudaError_t launch_pooled_scores(const ScoreParams& p, int BH, int d, cudaStream
   dim3 grid((p.NB + 63) / 64, (p.NB + 63) / 64, BH);
   const size_t sm = 2 * 64 * (d + 1) * sizeof(float);
   if (d == 128) {
-    cudaFuncSetAttribute(pooled_scores_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    const cudaError_t e = cudaFuncSetAttribute(pooled_scores_kernel<128>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
     pooled_scores_kernel<128><<<grid, 256, sm, st>>>(p);
   } else if (d == 64) {
     pooled_scores_kernel<64><<<grid, 256, sm, st>>>(p);
