@@ -286,27 +286,34 @@ def fg_keep(scores, tau):
     return scores >= tau
 
 
-def fg_cached_keep(q, k, group, tau=None):
-    """Slices kept by the cached rule, bool [G, N_keys].
+def fg_cached_pmax(q, k, group):
+    """Largest attention probability of each M x 1 slice, float32 [G, N_keys].
 
-    FG-Attn review (referee summary, minor comment on the thresholds, and the
-    falsifier): the full attention map is computed once, and an M x 1 slice
-    (group g of M contiguous queries, key j) is kept when at least one query
-    of the group gives key j an attention probability above tau_cached, which
-    Sec. 5.1 sets to 0.5/N. N is the number of keys. The probabilities are the
-    float32 softmax of q.k / sqrt(d) over all keys, one query row at a time.
-    The last group holds only the queries that exist. Strictly above: a
-    probability equal to tau does not keep its slice.
+    FG-Attn review (referee summary; the falsifier): the full attention map
+    is computed once. For group g of M contiguous queries and key j this is
+    the maximum over the group's queries of softmax(q.k / sqrt(d))_j, the
+    softmax taken in float32 over all keys, one query row at a time. The
+    last group holds only the queries that exist.
     """
     n, d = q.shape
     nk = k.shape[0]
-    if tau is None:
-        tau = 0.5 / nk
-    t = F32(tau)
     kf = k.astype(F32)
     scale = F32(1.0 / math.sqrt(d))
-    keep = np.zeros((-(-n // group), nk), dtype=bool)
+    pmax = np.zeros((-(-n // group), nk), dtype=F32)
     for i in range(n):
         p = softmax_f32((kf @ q[i].astype(F32)) * scale)
-        keep[i // group] |= p > t
-    return keep
+        np.maximum(pmax[i // group], p, out=pmax[i // group])
+    return pmax
+
+
+def fg_cached_keep(q, k, group, tau=None):
+    """Slices kept by the cached rule, bool [G, N_keys].
+
+    FG-Attn review (minor comment on the thresholds): Sec. 5.1 sets the
+    cached threshold tau_cached to 0.5/N, N the number of keys; a slice is
+    kept when its largest probability (``fg_cached_pmax``) is strictly above
+    tau, so a probability equal to tau does not keep its slice.
+    """
+    if tau is None:
+        tau = 0.5 / k.shape[0]
+    return fg_cached_pmax(q, k, group) > F32(tau)

@@ -344,6 +344,7 @@ def test_fg_cached_matches_torch_softmax_and_group_max_pool():
     got = masks.fg_cached_keep(q, k, group)
     p = torch.softmax(torch.from_numpy(q).double() @ torch.from_numpy(k).double().T / math.sqrt(d), dim=1)
     pmax = torch.nn.functional.max_pool1d(p.T[None], group, group, ceil_mode=True)[0].T.numpy()
+    np.testing.assert_allclose(masks.fg_cached_pmax(q, k, group), pmax, rtol=2e-5, atol=1e-12)
     tau = 0.5 / n
     clear = np.abs(pmax - tau) > 1e-4 * tau
     assert clear.mean() > 0.99
