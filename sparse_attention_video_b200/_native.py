@@ -93,8 +93,9 @@ def lib():
                                                     ctypes.c_int, vp, vp, vp, vp, vp]
         L.sparse_attn_strerror.argtypes = [ctypes.c_int]
         L.sparse_attn_strerror.restype = ctypes.c_char_p
-        for name in EXPORTED[:-1]:
-            getattr(L, name).restype = ctypes.c_int
+        for name in EXPORTED:
+            if name != "sparse_attn_strerror":
+                getattr(L, name).restype = ctypes.c_int
         _LIB = L
     return _LIB
 
