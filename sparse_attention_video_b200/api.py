@@ -136,6 +136,21 @@ class SparseAttention:
                      k.data_ptr() if needs else None, self.mask_ws.data_ptr(),
                      self.scratch_ws.data_ptr(), _stream_ptr(stream))
 
+    def build_mask_fg_cached(self, q, k, lse, tau=0.0, stream=None):
+        """FG cached mask (FG-Attn review, the cached strategy): slices that
+        some query of their group gives a probability above ``tau`` (0: 0.5/N),
+        from ``lse``, the float32 [batch, heads, N] LSE of full attention of q
+        over all keys. The policy must be "fg"; its keep fraction only bounds
+        the size of the union lists."""
+        if self.policy.kind != N.SA_MASK_FG:
+            raise ValueError("build_mask_fg_cached needs an \"fg\" policy")
+        _check_qkv(q, self.problem, "q", self.device)
+        _check_qkv(k, self.problem, "k", self.device)
+        _check_lse(lse, self.problem, self.device)
+        N.build_mask_fg_cached(self.problem, self.policy, q.data_ptr(), k.data_ptr(),
+                               lse.data_ptr(), tau, self.mask_ws.data_ptr(),
+                               self.scratch_ws.data_ptr(), _stream_ptr(stream))
+
     def forward(self, q, k, v, out=None, lse=None, stream=None):
         for t, n in ((q, "q"), (k, "k"), (v, "v")):
             _check_qkv(t, self.problem, n, self.device)
