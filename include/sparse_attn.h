@@ -188,6 +188,22 @@ SA_API int sparse_attn_build_mask_fg_cached(const sa_problem* problem, const sa_
                                            float tau, void* mask_ws, void* scratch_ws,
                                            void* stream);
 
+/* FP8 operands (Sparse VideoGen review: the optional FP8 quantization of
+ * attention). Quantizes n_tensors contiguous bf16 tensors of n_elems elements
+ * each (for attention: each (batch, head) slice of Q, K or V, n_elems =
+ * N * head_dim) to E4M3 ("FP8 Formats for Deep Learning", Micikevicius et al.:
+ * bias 7, 3 mantissa bits, largest finite value 448, no infinity) with one
+ * scale per tensor: inv = 448 / max|x| in float32 (1 for an all-zero tensor)
+ * and code = E4M3 of float32(x * inv), rounded to nearest even and saturating
+ * at 448. The operand an FP8 attention sees is code / inv.
+ *   x      device bf16 [n_tensors][n_elems], 16-byte aligned
+ *   codes  device uint8 [n_tensors][n_elems], 16-byte aligned (written)
+ *   inv    device float [n_tensors] (written)
+ * n_elems must be a positive multiple of 8 and n_tensors at most 65535.
+ * Returns SA_ERR_INVALID_ARG synchronously otherwise. Asynchronous on ``stream``. */
+SA_API int sparse_attn_quantize_e4m3(const void* x, long long n_elems, int n_tensors,
+                                    uint8_t* codes, float* inv, void* stream);
+
 /* ---------------------------------------------------------------- attention
  * O and LSE for the mask in mask_ws (built by sparse_attn_build_mask with the
  * same problem and policy). Equivalent to sparse_attn_permute followed by

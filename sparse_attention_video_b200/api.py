@@ -269,3 +269,20 @@ def sta_window_search(q, k, v, rows, T, H, W, tile, candidates, block=128, strea
                         _stream_ptr(stream))
     return choice, mse, row_err
 
+
+
+def quantize_e4m3(x, stream=None):
+    """E4M3 codes of a contiguous CUDA bf16 tensor [batch, heads, N, d] with one
+    scale per (batch, head) (Sparse VideoGen review: FP8 quantization).
+    Returns (codes uint8, same shape; inv float32 [batch*heads]), queued on
+    ``stream``; the dequantized operand is codes' value / inv."""
+    if not (isinstance(x, torch.Tensor) and x.dim() == 4):
+        raise ValueError("x must be a CUDA bf16 tensor [batch, heads, N, head_dim]")
+    _check_tensor(x, tuple(x.shape), (torch.bfloat16,), "x")
+    n_tensors = x.shape[0] * x.shape[1]
+    n_elems = x.shape[2] * x.shape[3]
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    inv = torch.empty(n_tensors, dtype=torch.float32, device=x.device)
+    N.quantize_e4m3(x.data_ptr(), n_elems, n_tensors, codes.data_ptr(), inv.data_ptr(),
+                    _stream_ptr(stream))
+    return codes, inv

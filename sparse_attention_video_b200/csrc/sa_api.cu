@@ -13,6 +13,7 @@
 #include "sa_internal.h"
 #include "sa_mask.h"
 #include "sa_profile.h"
+#include "sa_quant.h"
 
 using namespace sa;
 
@@ -714,6 +715,20 @@ extern "C" int sparse_attn_sta_window_search(const sa_problem* problem, const sa
     for (int i = 0; i < 3; ++i) pp.win[c][i] = candidates[3 * c + i];
   pp.scale_log2 = 1.4426950408889634f / sqrtf((float)pr.head_dim);
   return cuda_status(launch_profile(pp, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+extern "C" int sparse_attn_quantize_e4m3(const void* x, long long n_elems, int n_tensors,
+                                         uint8_t* codes, float* inv, void* stream) {
+  if (n_elems < 8 || n_elems % 8 != 0 || n_tensors < 1 || n_tensors > 65535)
+    return SA_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(inv, 4)) return SA_ERR_INVALID_ARG;
+  QuantParams qp{};
+  qp.x = static_cast<const __nv_bfloat16*>(x);
+  qp.codes = codes;
+  qp.inv = inv;
+  qp.n_elems = n_elems;
+  qp.n_tensors = n_tensors;
+  return cuda_status(launch_quant_e4m3(qp, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 extern "C" int sparse_attn_status(void* scratch_ws, void* stream, int clear) {
