@@ -35,6 +35,8 @@ def make_policy(kind, block=128, tile=(1, 1, 128), topk=0, keep_diagonal=False,
     if temporal_heads is not None:
         arr = (ctypes.c_int8 * max(1, heads))()
         for h in temporal_heads:
+            if not 0 <= h < heads:
+                raise ValueError(f"temporal head {h} is outside 0..{heads - 1} (pass heads=)")
             arr[h] = 1
         p.head_is_temporal = ctypes.cast(arr, ctypes.POINTER(ctypes.c_int8))
         p._keep_alive = arr
@@ -50,6 +52,8 @@ def make_policy(kind, block=128, tile=(1, 1, 128), topk=0, keep_diagonal=False,
     sums = {"mean": N.SA_SUMMARIZER_MEAN, "max": N.SA_SUMMARIZER_MAX, "min": N.SA_SUMMARIZER_MIN}
     p.summarizer = sums.get(summarizer, summarizer)
     if head_windows is not None:
+        if any(len(w) != 3 for w in head_windows):
+            raise ValueError("each head window is (wt, wh, ww)")
         arr = (ctypes.c_int * (3 * len(head_windows)))(*[int(x) for w in head_windows for x in w])
         p.head_windows = ctypes.cast(arr, ctypes.POINTER(ctypes.c_int))
         p._keep_windows = arr
@@ -92,6 +96,19 @@ def _check_lse(t, problem, device):
     _check_tensor(t, _qkv_shape(problem)[:3], (torch.float32,), "lse", device)
 
 
+def _check_head_arrays(policy, heads):
+    """The library reads one entry per head of the problem from the policy's
+    host arrays; a policy made for fewer heads would be read past its end."""
+    arr = getattr(policy, "_keep_alive", None)
+    if policy.head_is_temporal and (arr is None or len(arr) < heads):
+        raise ValueError(f"the policy's temporal-head flags cover "
+                         f"{0 if arr is None else len(arr)} heads, the problem has {heads}")
+    win = getattr(policy, "_keep_windows", None)
+    if policy.head_windows and (win is None or len(win) < 3 * heads):
+        raise ValueError(f"the policy's head_windows cover "
+                         f"{0 if win is None else len(win) // 3} heads, the problem has {heads}")
+
+
 def _check_scratch(ws, device):
     if not (isinstance(ws, torch.Tensor) and ws.is_cuda and ws.device == device
             and ws.is_contiguous() and ws.numel() * ws.element_size() >= 256):
@@ -104,6 +121,7 @@ class SparseAttention:
     def __init__(self, batch, heads, T, H, W, head_dim, policy, device="cuda"):
         self.problem = N.Problem(batch, heads, T, H, W, head_dim)
         self.policy = policy
+        _check_head_arrays(policy, heads)
         self.mask_bytes, self.scratch_bytes = N.workspace_size(self.problem, policy)
         self.mask_ws = torch.empty(self.mask_bytes, dtype=torch.uint8, device=torch.device(device))
         self.device = self.mask_ws.device                 # "cuda" resolved to its index

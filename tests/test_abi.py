@@ -225,3 +225,24 @@ def test_quantize_and_cached_mask_arguments_are_checked_on_the_host():
         assert call(fg, tau) == N.SA_ERR_INVALID_ARG, tau
     assert call(fg, 0.0, lse=None) == N.SA_ERR_INVALID_ARG
     assert call(fg, 0.0, ws=vp + 16) == N.SA_ERR_WORKSPACE
+
+
+def test_policy_head_arrays_must_cover_the_problem():
+    # the library reads one temporal flag and one window per head of the
+    # problem from the policy's host arrays
+    from sparse_attention_video_b200 import api, make_policy
+    st = make_policy("spatiotemporal", temporal_heads=(1,), heads=2)
+    api._check_head_arrays(st, 2)
+    with pytest.raises(ValueError, match="temporal-head flags cover 2 heads"):
+        api._check_head_arrays(st, 4)
+    with pytest.raises(ValueError, match="outside"):
+        make_policy("spatiotemporal", temporal_heads=(2,), heads=2)
+    sta = make_policy("sta", tile=(4, 4, 8), window=(3, 3, 3), head_windows=[(1, 1, 1), (3, 3, 3)])
+    api._check_head_arrays(sta, 2)
+    with pytest.raises(ValueError, match="head_windows cover 2 heads"):
+        api._check_head_arrays(sta, 3)
+    with pytest.raises(ValueError, match="head_windows cover 0 heads"):
+        api._check_head_arrays(make_policy("sta", tile=(4, 4, 8), head_windows=[]), 1)
+    with pytest.raises(ValueError, match="each head window"):
+        make_policy("sta", tile=(4, 4, 8), head_windows=[(3, 3)])
+    api._check_head_arrays(make_policy("topk", tile=(4, 4, 8), topk=2), 8)   # no head arrays
