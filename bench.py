@@ -48,6 +48,10 @@ def _args():
                     help="skip the head-profiler timing (spatial/temporal workload only)")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="workload name (synthetic.CONFIGS); the bench line uses the default")
+    ap.add_argument("--mask-once", default="",
+                    help="comma-separated workload names: build each one's mask twice through "
+                         "the public API and exit (a short program for ncu launch lists of the "
+                         "mask kernels); prints no bench line")
     ap.add_argument("--heads", type=int, default=0,
                     help="run only this many heads (half of them temporal); for small "
                          "profiler captures, not for bench lines")
@@ -260,6 +264,34 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- mask kernels only
+def mask_once(names, local):
+    """Each named workload's mask built twice (the second build runs with its
+    kernels warm) on the seeded inputs, through SparseAttention.build_mask."""
+    import torch
+
+    from sparse_attention_video_b200 import SparseAttention, make_policy
+    from synthetic import CONFIGS, make_qkv
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    for name in names:
+        wl = CONFIGS[name]
+        x = make_qkv(wl)
+        q, k = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in "qk")
+        sa = SparseAttention(1, wl.heads, wl.T, wl.H, wl.W, wl.head_dim,
+                             make_policy(**policy_kwargs(wl)), device=dev)
+        stream = torch.cuda.current_stream(dev)
+        for _ in range(2):
+            sa.build_mask(q, k, stream)
+        torch.cuda.synchronize(dev)
+        status = sa.status()
+        log(f"{name}: mask built twice, status {status}")
+        if status != 0:
+            raise SystemExit(f"{name}: device status {status}")
+        del q, k, sa
+
+
 # ---------------------------------------------------------------- our arm
 def main():
     args = _args()
@@ -268,6 +300,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.mask_once:
+        mask_once(args.mask_once.split(","), local)
         return
 
     import torch
