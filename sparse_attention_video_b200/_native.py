@@ -98,8 +98,9 @@ def lib():
         L.sparse_attn_quantize_e4m3.argtypes = [vp, ctypes.c_longlong, ctypes.c_int, vp, vp, vp]
         L.sparse_attn_strerror.argtypes = [ctypes.c_int]
         L.sparse_attn_strerror.restype = ctypes.c_char_p
-        for name in EXPORTED[:-1]:
-            getattr(L, name).restype = ctypes.c_int
+        for name in EXPORTED:
+            if name != "sparse_attn_strerror":
+                getattr(L, name).restype = ctypes.c_int
         _LIB = L
     return _LIB
 

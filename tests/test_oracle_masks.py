@@ -271,6 +271,42 @@ def test_top_p_single_dominant_and_uniform():
     assert k.sum() in (9, 10) and k[:9].all()                         # float32 sum of 0.1s
 
 
+def test_top_p_full_mass_and_invalid_blocks():
+    # p = 1: the float32 running sum may stop short of 1, so the scan must run
+    # to the last valid block; invalid blocks are never candidates
+    g = np.random.default_rng(9)
+    row = g.standard_normal(37).astype(np.float32)
+    valid = g.random(37) < 0.7
+    kept = masks.top_p_row(row, valid, 1.0)
+    assert np.array_equal(kept, valid)
+    kept = masks.top_p_row(row, valid, 0.5)
+    assert not (kept & ~valid).any() and kept.any()
+    one = np.zeros(37, bool)
+    one[5] = True
+    assert np.array_equal(masks.top_p_row(row, one, 0.3), one)        # a lone block has mass 1
+
+
+def test_rules_at_degenerate_parameters():
+    T, H, W, block = 5, 4, 24, 64
+    order = layout.identity_order(T, H, W, block)
+    blk = layout.blocks(order, block)
+    valid = masks.valid_blocks(blk)
+    allv = np.outer(valid, valid)
+    # a frame radius covering every frame keeps every valid pair
+    assert np.array_equal(masks.spatial_rule(blk, T, H, W, frame_radius=T), allv)
+    # no sinks: the mask is unchanged
+    m = masks.spatial_rule(blk, T, H, W, frame_radius=0)
+    assert np.array_equal(masks.add_sinks(m.copy(), blk, 0, block), m)
+    # a window spanning the tile grid keeps every valid tile pair; a 1x1x1
+    # window keeps the diagonal only
+    dims = layout.tile_grid_dims(T, H, W, 1, 4, 16)
+    tiles = layout.blocks(layout.tile_order(T, H, W, 1, 4, 16), block)
+    tv = masks.valid_blocks(tiles)
+    span = tuple(2 * n - 1 for n in dims)
+    assert np.array_equal(masks.tile_window(dims, span, tv, tv), np.outer(tv, tv))
+    assert np.array_equal(masks.tile_window(dims, (1, 1, 1), tv, tv), np.diag(tv))
+
+
 # ---------------------------------------------------------------- FG slices
 def test_fg_threshold_keep_count_and_sort():
     g = np.random.default_rng(4)
