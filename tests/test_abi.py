@@ -2,9 +2,11 @@
 symbol include/sparse_attn.h declares, sizes workspaces and rejects bad
 arguments on the host before touching the device."""
 import ctypes
+import math
 import os
 import re
 
+import numpy as np
 import pytest
 
 from sparse_attention_video_b200 import _native as N
@@ -246,3 +248,43 @@ def test_policy_head_arrays_must_cover_the_problem():
     with pytest.raises(ValueError, match="each head window"):
         make_policy("sta", tile=(4, 4, 8), head_windows=[(3, 3)])
     api._check_head_arrays(make_policy("topk", tile=(4, 4, 8), topk=2), 8)   # no head arrays
+
+
+def _layout_bytes(wl):
+    """Mask and scratch bytes from the documented layout: regions in order,
+    each padded to 256 bytes (the mask workspace is at least 256 bytes)."""
+    up = lambda n: (n + 255) // 256 * 256
+    BH, N_, d = wl.batch * wl.heads, wl.N, wl.head_dim
+    cdiv = lambda a, b: -(-a // b)
+    tiles = lambda t: cdiv(wl.T, t[0]) * cdiv(wl.H, t[1]) * cdiv(wl.W, t[2])
+    if wl.kind in ("topk", "sta"):
+        NB = tiles(wl.tile)
+    elif wl.kind == "spade":
+        NB = max(tiles(t) for t in wl.candidates)
+    elif wl.kind == "fg":
+        NB = 0
+    else:
+        NB = cdiv(N_, wl.block)
+    W32 = cdiv(NB, 32)
+    mask = [64 * BH, 4 * BH * NB, 4 * BH * NB * NB, 4 * BH * NB * W32]
+    scratch = [256]
+    if wl.kind == "spatiotemporal" and wl.temporal_heads:
+        scratch.append(3 * up(BH * cdiv(N_, wl.block) * wl.block * d * 2))
+    C = len(wl.candidates) if wl.kind == "spade" else (1 if wl.kind == "topk" else 0)
+    if C:
+        scratch += [4 * BH * C * NB * d, 4 * BH * C * NB * d, 4 * BH * C * NB, 4 * BH * NB * NB]
+    if wl.kind == "fg":
+        G, WN, P = cdiv(N_, wl.fg_group), cdiv(N_, 32), cdiv(N_, 128)
+        cap = math.ceil(float(np.float32(wl.fg_keep_fraction)) * G * N_) + N_ + 32
+        mask += [4 * BH * G * WN, 4 * BH, 4 * BH * P, 4 * BH * (P + 1), 4 * BH * cap]
+        scratch += [3 * BH * cdiv(G, 128) * 128 * d * 2, 4 * BH * 4096, 4 * BH * 4,
+                    8 * BH * 65536 + 8 * BH]
+    return max(sum(up(b) for b in mask), 256), sum(up(b) for b in scratch)
+
+
+@pytest.mark.parametrize("name", list(CONFIGS) + list(C.SMALL))
+def test_workspace_sizes_equal_the_documented_layout(name):
+    wl = CONFIGS[name] if name in CONFIGS else C.SMALL[name]
+    pol = make_policy(**C.policy_kwargs(wl))
+    got = N.workspace_size(N.Problem(wl.batch, wl.heads, wl.T, wl.H, wl.W, wl.head_dim), pol)
+    assert got == _layout_bytes(wl), (name, got, _layout_bytes(wl))
