@@ -23,6 +23,8 @@ codes must match bit for bit.
 """
 import numpy as np
 
+from .attention import masked_attention_rows
+
 F32 = np.float32
 E4M3_MAX = 448.0
 _MIN_NORMAL = 2.0 ** -6
@@ -94,3 +96,11 @@ def dequantize(codes, inv):
 def fp8_operands(q, k, v):
     """Dequantized Q, K, V of one (batch, head), float64 [N, d] each."""
     return tuple(dequantize(*quantize_tensor(x)) for x in (q, k, v))
+
+
+def fp8_attention_rows(q, k, v, rows, keep):
+    """O [r, d] and LSE [r] of FP8 attention for query tokens ``rows``:
+    the exact masked attention (float64) of the dequantized E4M3 operands of
+    one (batch, head)."""
+    qh, kh, vh = fp8_operands(q, k, v)
+    return masked_attention_rows(qh, kh, vh, rows, keep)

@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import quant
+from oracle import attention, quant
 
 
 def _torch_codes(y):
@@ -111,3 +111,44 @@ def test_representable_operands_are_unchanged():
     x[0, 0] = 448.0
     for xh in quant.fp8_operands(x, -x, x):
         assert np.array_equal(np.abs(xh), np.abs(x.astype(np.float64)))
+
+
+def test_fp8_attention_on_grid_operands_is_plain_attention():
+    # operands on the E4M3 grid with 448 present in each: quantization is the
+    # identity, so FP8 attention is the plain attention of the same values
+    g = np.random.default_rng(6)
+    grid = _finite_values()
+    small = grid[np.abs(grid) <= 4.0]
+    q, k, v = (g.choice(small, (40, 16)).astype(np.float32) for _ in range(3))
+    for x in (q, k, v):
+        x[0, 0] = 448.0
+    rows = np.arange(40)
+    keep = g.random((40, 40)) < 0.6
+    keep[:, 0] = True
+    o8, l8 = quant.fp8_attention_rows(q, k, v, rows, keep)
+    o, l = attention.masked_attention_rows(q, k, v, rows, keep)
+    assert np.array_equal(o8, o) and np.array_equal(l8, l)
+
+
+def test_fp8_attention_error_is_bounded_by_the_operand_steps():
+    # each operand moves by at most half a grid step (2^-4 relative for
+    # normals): scores move by at most |dq||k| + |q||dk| + |dq||dk| per
+    # pair (Cauchy-Schwarz), which bounds the LSE shift; O moves by at most
+    # the V step plus the spread of V times the weight change
+    g = np.random.default_rng(7)
+    n, d = 64, 32
+    q, k, v = (g.standard_normal((n, d)).astype(np.float32) for _ in range(3))
+    rows = np.arange(n)
+    keep = np.ones((n, n), bool)
+    o8, l8 = quant.fp8_attention_rows(q, k, v, rows, keep)
+    o, l = attention.masked_attention_rows(q, k, v, rows, keep)
+    qh, kh, vh = quant.fp8_operands(q, k, v)
+    dq = np.linalg.norm(qh - q, axis=1)
+    dk = np.linalg.norm(kh - k, axis=1)
+    nq, nk = np.linalg.norm(q, axis=1), np.linalg.norm(k, axis=1)
+    ds = (np.outer(dq, nk) + np.outer(nq, dk) + np.outer(dq, dk)).max() / np.sqrt(d)
+    assert np.all(np.abs(l8 - l) <= ds + 1e-12)
+    w_change = np.expm1(2 * ds)                       # relative weight change bound
+    spread = np.abs(v).max() + np.abs(vh).max()
+    assert np.all(np.abs(o8 - o) <= np.abs(vh - v).max() + spread * w_change + 1e-12)
+    assert 0 < np.abs(o8 - o).max() < 0.2              # a real, small difference
