@@ -509,7 +509,7 @@ def main():
         ms = c0.elapsed_time(c1) / 2
         from sparse_attention_video_b200 import SA_EXPORT_FG_BITS
         bits = csa.export(SA_EXPORT_FG_BITS)
-        kept = int(np.unpackbits(bits.view(np.uint8)).sum())
+        kept = int(np.bitwise_count(bits).sum(dtype=np.int64))
         G = (wl.N + wl.fg_group - 1) // wl.fg_group
         prof["fg_cached"] = {
             "ms": ms, "status": csa.status(),
