@@ -486,6 +486,57 @@ def main():
             "kernel": "profile_kernel, tile-window mode (mma.sync m16n8k16)"}}
         log("window search timed")
 
+    if wl.kind == "fg" and not args.no_profile and dense:
+        # FG cached mask from the LSE of full attention (an explicit policy
+        # keeping every block); the union lists are sized for every slice
+        nb = (wl.N + wl.block - 1) // wl.block
+        words = torch.full((wl.heads, nb, (nb + 31) // 32), -1, dtype=torch.int32, device=dev)
+        fpol = make_policy("explicit", block=wl.block, explicit_layout=0, explicit_bits=words)
+        fsa = SparseAttention(1, wl.heads, wl.T, wl.H, wl.W, wl.head_dim, fpol, device=dev)
+        fsa.build_mask(q, k, stream)
+        fsa.attend(q, k, v, o, lse, stream)
+        del fsa, words
+        cpol = make_policy("fg", block=wl.block, fg_group=wl.fg_group, fg_keep_fraction=1.0)
+        csa = SparseAttention(1, wl.heads, wl.T, wl.H, wl.W, wl.head_dim, cpol, device=dev)
+        csa.build_mask_fg_cached(q, k, lse, stream=stream)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        c0.record(stream)
+        for _ in range(2):
+            csa.build_mask_fg_cached(q, k, lse, stream=stream)
+        c1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = c0.elapsed_time(c1) / 2
+        from sparse_attention_video_b200 import SA_EXPORT_FG_BITS
+        bits = csa.export(SA_EXPORT_FG_BITS)
+        kept = int(np.bitwise_count(bits).sum(dtype=np.int64))
+        G = (wl.N + wl.fg_group - 1) // wl.fg_group
+        prof["fg_cached"] = {
+            "ms": ms, "status": csa.status(),
+            "score_tflops": 2.0 * wl.head_dim * wl.N * wl.N * wl.heads / (ms * 1e-3) / 1e12,
+            "kept_fraction": kept / (G * wl.N * wl.heads),
+            "kernel": "fg_score_kernel, cached mode (tcgen05), then the union lists"}
+        del csa
+        log("cached mask timed")
+
+    if not args.no_profile:
+        from sparse_attention_video_b200 import quantize_e4m3
+        quantize_e4m3(q, stream)
+        z0, z1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        z0.record(stream)
+        for _ in range(5):
+            quantize_e4m3(q, stream)
+        z1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = z0.elapsed_time(z1) / 5
+        algo = q.numel() * 3                      # 2 bytes read and 1 byte written per element
+        prof["quantize_e4m3"] = {
+            "ms": ms, "algorithmic_gbs": algo / (ms * 1e-3) / 1e9,
+            "frac_of_hbm": algo / (ms * 1e-3) / 1e9 / _peaks()[2],
+            "note": "Q of every head; each element is read twice (amax, then encode)"}
+        log("quantizer timed")
+
     if rank != 0:
         if world > 1:
             dist.barrier()

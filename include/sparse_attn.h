@@ -166,6 +166,44 @@ SA_API int sparse_attn_build_mask(const sa_problem* problem, const sa_policy* po
                            const void* q, const void* k,
                            void* mask_ws, void* scratch_ws, void* stream);
 
+/* FG cached mask (FG-Attn review: referee summary, the minor comment on the
+ * thresholds, and the falsifier): the full attention map is computed once and
+ * an M x 1 slice (group g of fg_group contiguous queries, key j) is kept when
+ * at least one query of g gives key j a probability above tau, i.e. when
+ * q.k / sqrt(d) - lse_q > ln(tau) for some q in g.
+ *   q, k   device bf16 [batch, heads, N, head_dim], as for sparse_attn_build_mask
+ *   lse    device float [batch*heads][N]: the natural-log LSE of FULL attention
+ *          of each query over all N keys, e.g. the ``lse`` output of
+ *          sparse_attn_forward with an EXPLICIT policy that keeps every block
+ *   tau    threshold in (0, 1); 0 selects 0.5 / N, the value the page gives
+ * The policy must be of kind SA_MASK_FG; its fg_keep_fraction is here only an
+ * upper bound on the fraction of slices kept, which sizes the union lists
+ * (more than that sets SA_DEVFLAG_BOUNDS and the lists are cut). Writes the
+ * slice bitmask, tau and the union lists into mask_ws, which
+ * sparse_attn_forward then uses as it uses a mask from sparse_attn_build_mask
+ * with the same problem and policy; the mask may be kept and reused by later
+ * calls. Clears the status word. Asynchronous on ``stream``. */
+SA_API int sparse_attn_build_mask_fg_cached(const sa_problem* problem, const sa_policy* policy,
+                                           const void* q, const void* k, const float* lse,
+                                           float tau, void* mask_ws, void* scratch_ws,
+                                           void* stream);
+
+/* FP8 operands (Sparse VideoGen review: the optional FP8 quantization of
+ * attention). Quantizes n_tensors contiguous bf16 tensors of n_elems elements
+ * each (for attention: each (batch, head) slice of Q, K or V, n_elems =
+ * N * head_dim) to E4M3 ("FP8 Formats for Deep Learning", Micikevicius et al.:
+ * bias 7, 3 mantissa bits, largest finite value 448, no infinity) with one
+ * scale per tensor: inv = 448 / max|x| in float32 (1 for an all-zero tensor)
+ * and code = E4M3 of float32(x * inv), rounded to nearest even and saturating
+ * at 448. The operand an FP8 attention sees is code / inv.
+ *   x      device bf16 [n_tensors][n_elems], 16-byte aligned
+ *   codes  device uint8 [n_tensors][n_elems], 16-byte aligned (written)
+ *   inv    device float [n_tensors] (written)
+ * n_elems must be a positive multiple of 8 and n_tensors at most 65535.
+ * Returns SA_ERR_INVALID_ARG synchronously otherwise. Asynchronous on ``stream``. */
+SA_API int sparse_attn_quantize_e4m3(const void* x, long long n_elems, int n_tensors,
+                                    uint8_t* codes, float* inv, void* stream);
+
 /* ---------------------------------------------------------------- attention
  * O and LSE for the mask in mask_ws (built by sparse_attn_build_mask with the
  * same problem and policy). Equivalent to sparse_attn_permute followed by

@@ -10,4 +10,4 @@ from ._native import (SA_EXPORT_BLOCK_BITS, SA_EXPORT_FG_BITS, SA_EXPORT_FG_TAU,
                       SA_EXPORT_HEAD_INFO, SA_LAYOUT_FRAME_MAJOR, SA_LAYOUT_IDENTITY,
                       SA_LAYOUT_TILE, SparseAttnError, lib)
 from .api import (SparseAttention, make_policy, profile_heads,  # noqa: F401
-                  sta_window_search)
+                  quantize_e4m3, sta_window_search)

@@ -27,7 +27,9 @@ EXPORTED = ("sparse_attn_workspace_size", "sparse_attn_build_mask", "sparse_attn
             "sparse_attn_permute", "sparse_attn_attend",
             "sparse_attn_export_bytes", "sparse_attn_mask_export", "sparse_attn_status",
             "sparse_attn_build_mask_static", "sparse_attn_selftest_wait_timeout",
-            "sparse_attn_profile_heads", "sparse_attn_sta_window_search", "sparse_attn_strerror")
+            "sparse_attn_profile_heads", "sparse_attn_sta_window_search",
+            "sparse_attn_build_mask_fg_cached", "sparse_attn_quantize_e4m3",
+            "sparse_attn_strerror")
 
 SA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
 
@@ -91,6 +93,9 @@ def lib():
                                                 vp, vp]
         L.sparse_attn_sta_window_search.argtypes = [P, PP, vp, vp, vp, vp, ctypes.c_int, vp,
                                                     ctypes.c_int, vp, vp, vp, vp, vp]
+        L.sparse_attn_build_mask_fg_cached.argtypes = [P, PP, vp, vp, vp, ctypes.c_float, vp, vp,
+                                                       vp]
+        L.sparse_attn_quantize_e4m3.argtypes = [vp, ctypes.c_longlong, ctypes.c_int, vp, vp, vp]
         L.sparse_attn_strerror.argtypes = [ctypes.c_int]
         L.sparse_attn_strerror.restype = ctypes.c_char_p
         for name in EXPORTED:
@@ -155,6 +160,17 @@ def sta_window_search(problem, policy, q, k, v, rows, n_rows, candidates, n_cand
                                                v, rows, n_rows, candidates, n_candidates, row_err,
                                                mse, choice, scratch_ws, stream),
            "sparse_attn_sta_window_search")
+
+
+def build_mask_fg_cached(problem, policy, q, k, lse, tau, mask_ws, scratch_ws, stream=0):
+    _check(lib().sparse_attn_build_mask_fg_cached(ctypes.byref(problem), ctypes.byref(policy), q,
+                                                  k, lse, float(tau), mask_ws, scratch_ws, stream),
+           "sparse_attn_build_mask_fg_cached")
+
+
+def quantize_e4m3(x, n_elems, n_tensors, codes, inv, stream=0):
+    _check(lib().sparse_attn_quantize_e4m3(x, n_elems, n_tensors, codes, inv, stream),
+           "sparse_attn_quantize_e4m3")
 
 
 def export_bytes(problem, policy, what):

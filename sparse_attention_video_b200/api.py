@@ -154,6 +154,21 @@ class SparseAttention:
                      k.data_ptr() if needs else None, self.mask_ws.data_ptr(),
                      self.scratch_ws.data_ptr(), _stream_ptr(stream))
 
+    def build_mask_fg_cached(self, q, k, lse, tau=0.0, stream=None):
+        """FG cached mask (FG-Attn review, the cached strategy): slices that
+        some query of their group gives a probability above ``tau`` (0: 0.5/N),
+        from ``lse``, the float32 [batch, heads, N] LSE of full attention of q
+        over all keys. The policy must be "fg"; its keep fraction only bounds
+        the size of the union lists."""
+        if self.policy.kind != N.SA_MASK_FG:
+            raise ValueError("build_mask_fg_cached needs an \"fg\" policy")
+        _check_qkv(q, self.problem, "q", self.device)
+        _check_qkv(k, self.problem, "k", self.device)
+        _check_lse(lse, self.problem, self.device)
+        N.build_mask_fg_cached(self.problem, self.policy, q.data_ptr(), k.data_ptr(),
+                               lse.data_ptr(), tau, self.mask_ws.data_ptr(),
+                               self.scratch_ws.data_ptr(), _stream_ptr(stream))
+
     def forward(self, q, k, v, out=None, lse=None, stream=None):
         for t, n in ((q, "q"), (k, "k"), (v, "v")):
             _check_qkv(t, self.problem, n, self.device)
@@ -272,3 +287,20 @@ def sta_window_search(q, k, v, rows, T, H, W, tile, candidates, block=128, strea
                         _stream_ptr(stream))
     return choice, mse, row_err
 
+
+
+def quantize_e4m3(x, stream=None):
+    """E4M3 codes of a contiguous CUDA bf16 tensor [batch, heads, N, d] with one
+    scale per (batch, head) (Sparse VideoGen review: FP8 quantization).
+    Returns (codes uint8, same shape; inv float32 [batch*heads]), queued on
+    ``stream``; the dequantized operand is codes' value / inv."""
+    if not (isinstance(x, torch.Tensor) and x.dim() == 4):
+        raise ValueError("x must be a CUDA bf16 tensor [batch, heads, N, head_dim]")
+    _check_tensor(x, tuple(x.shape), (torch.bfloat16,), "x")
+    n_tensors = x.shape[0] * x.shape[1]
+    n_elems = x.shape[2] * x.shape[3]
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    inv = torch.empty(n_tensors, dtype=torch.float32, device=x.device)
+    N.quantize_e4m3(x.data_ptr(), n_elems, n_tensors, codes.data_ptr(), inv.data_ptr(),
+                    _stream_ptr(stream))
+    return codes, inv

@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsparse_attn.so")
 SOURCES = ["sa_api.cu", "sa_mask.cu", "sa_attn.cu", "sa_fg.cu", "sa_noalloc.cu", "sa_selftest.cu",
-           "sa_profile.cu"]
+           "sa_profile.cu", "sa_quant.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
               "-Xcompiler", "-fPIC,-fvisibility=hidden", "-cudart", "static"]
 

@@ -13,6 +13,7 @@
 #include "sa_internal.h"
 #include "sa_mask.h"
 #include "sa_profile.h"
+#include "sa_quant.h"
 
 using namespace sa;
 
@@ -275,6 +276,19 @@ void pool_regions(PoolParams& pp) {
 
 int aligned(const void* p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Union lists of the slice bitmask in the mask workspace (FG policies).
+FgListParams fg_lists(const MaskLayout& M, const sa_policy& po, uint8_t* mw, uint32_t* status) {
+  FgListParams lp{};
+  lp.bits = reinterpret_cast<uint32_t*>(mw + M.off_fg_bits);
+  lp.counts = reinterpret_cast<uint32_t*>(mw + M.off_fg_counts);
+  lp.offsets = reinterpret_cast<uint32_t*>(mw + M.off_fg_offsets);
+  lp.list = reinterpret_cast<uint32_t*>(mw + M.off_fg_list);
+  lp.status = status;
+  lp.cap_per_head = M.cap;
+  lp.BH = M.BH; lp.P = M.P; lp.G = M.G; lp.WN = M.WN; lp.groups_per_tile = 128 / po.fg_group;
+  return lp;
+}
+
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
 
 }  // namespace
@@ -334,14 +348,7 @@ extern "C" int sparse_attn_build_mask(const sa_problem* problem, const sa_policy
     fp.status = reinterpret_cast<uint32_t*>(sw + S.off_status);
     fp.BH = BH; fp.N = N; fp.d = d; fp.group = po.fg_group; fp.G = M.G; fp.WN = M.WN;
     fp.keep_fraction = po.fg_keep_fraction;
-    FgListParams& lp = fp.lists;
-    lp.bits = fp.bits;
-    lp.counts = reinterpret_cast<uint32_t*>(mw + M.off_fg_counts);
-    lp.offsets = reinterpret_cast<uint32_t*>(mw + M.off_fg_offsets);
-    lp.list = reinterpret_cast<uint32_t*>(mw + M.off_fg_list);
-    lp.status = fp.status;
-    lp.cap_per_head = M.cap;
-    lp.BH = BH; lp.P = M.P; lp.G = M.G; lp.WN = M.WN; lp.groups_per_tile = 128 / po.fg_group;
+    fp.lists = fg_lists(M, po, mw, fp.status);
     return cuda_status(launch_fg_build(fp, encode_fn(), st));
   }
 
@@ -411,6 +418,43 @@ extern "C" int sparse_attn_build_mask(const sa_problem* problem, const sa_policy
   }
   if (po.kind == SA_MASK_EXPLICIT) sp.explicit_bits = po.explicit_bits;
   return cuda_status(launch_select(sp, BH, st));
+}
+
+extern "C" int sparse_attn_build_mask_fg_cached(const sa_problem* problem,
+                                                const sa_policy* policy, const void* q,
+                                                const void* k, const float* lse, float tau,
+                                                void* mask_ws, void* scratch_ws, void* stream) {
+  int e = check_problem(problem);
+  if (e) return e;
+  e = check_policy(*problem, policy);
+  if (e) return e;
+  if (policy->kind != SA_MASK_FG) return SA_ERR_INVALID_ARG;
+  if (!(tau >= 0.f && tau < 1.f)) return SA_ERR_INVALID_ARG;     // NaN fails too
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(lse, 4)) return SA_ERR_INVALID_ARG;
+  if (!aligned(mask_ws, 256) || !aligned(scratch_ws, 256)) return SA_ERR_WORKSPACE;
+  if (!encode_fn()) return SA_ERR_CUDA;
+  const sa_problem& pr = *problem;
+  const sa_policy& po = *policy;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const MaskLayout M = mask_layout(pr, po);
+  const ScratchLayout S = scratch_layout(pr, po, M);
+  uint8_t* mw = static_cast<uint8_t*>(mask_ws);
+  uint8_t* sw = static_cast<uint8_t*>(scratch_ws);
+  const long long N = n_tokens(pr);
+  if (cudaMemsetAsync(sw + S.off_status, 0, 256, st) != cudaSuccess) return SA_ERR_CUDA;
+  FgCachedParams cp{};
+  cp.q = static_cast<const __nv_bfloat16*>(q);
+  cp.k = static_cast<const __nv_bfloat16*>(k);
+  cp.lse = lse;
+  cp.bits = reinterpret_cast<uint32_t*>(mw + M.off_fg_bits);
+  cp.tau_out = reinterpret_cast<float*>(mw + M.off_fg_tau);
+  cp.status = reinterpret_cast<uint32_t*>(sw + S.off_status);
+  cp.lists = fg_lists(M, po, mw, cp.status);
+  cp.BH = M.BH; cp.N = (int)N; cp.d = pr.head_dim; cp.group = po.fg_group;
+  cp.G = M.G; cp.WN = M.WN;
+  // FG-Attn review, Sec. 5.1 as quoted by the referee: tau_cached = 0.5 / N
+  cp.tau = tau > 0.f ? tau : (float)(0.5 / (double)N);
+  return cuda_status(launch_fg_cached(cp, encode_fn(), st));
 }
 
 namespace {
@@ -671,6 +715,20 @@ extern "C" int sparse_attn_sta_window_search(const sa_problem* problem, const sa
     for (int i = 0; i < 3; ++i) pp.win[c][i] = candidates[3 * c + i];
   pp.scale_log2 = 1.4426950408889634f / sqrtf((float)pr.head_dim);
   return cuda_status(launch_profile(pp, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+extern "C" int sparse_attn_quantize_e4m3(const void* x, long long n_elems, int n_tensors,
+                                         uint8_t* codes, float* inv, void* stream) {
+  if (n_elems < 8 || n_elems % 8 != 0 || n_tensors < 1 || n_tensors > 65535)
+    return SA_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(inv, 4)) return SA_ERR_INVALID_ARG;
+  QuantParams qp{};
+  qp.x = static_cast<const __nv_bfloat16*>(x);
+  qp.codes = codes;
+  qp.inv = inv;
+  qp.n_elems = n_elems;
+  qp.n_tensors = n_tensors;
+  return cuda_status(launch_quant_e4m3(qp, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 extern "C" int sparse_attn_status(void* scratch_ws, void* stream, int clear) {

@@ -143,7 +143,8 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   // Selection state of this head (HIST level > 0 and BITS read the prefix).
   const uint32_t prefix = p.mode == FG_MODE_HIST ? p.sel[bh * 4 + 0] : 0u;
-  const uint32_t tau_key = p.sel[bh * 4 + 0];
+  // (CACHED has no selection state: sel is null there)
+  const uint32_t tau_key = p.mode == FG_MODE_CACHED ? 0u : p.sel[bh * 4 + 0];
   // Bitmask thresholds as floats: the order key is monotonic in the float
   // value, so key >= t  <=>  value >= key_to_float(t) (zeros aside: -0 and
   // +0 compare equal as floats, which only matters when the threshold is a
@@ -167,6 +168,17 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   }
   if (p.mode == FG_MODE_HIST)
     for (int i = threadIdx.x; i < kHists * kBins; i += kScoreThreads) hist[i] = 0u;
+  // CACHED: exp(s/sqrt(d) - lse) > tau  <=>  s > sqrt(d) * (lse + ln tau), one
+  // threshold per query column, staged where the histogram would be. A query
+  // past the end (a zero row of the TMA fill) never keeps a slice.
+  const int n_terms = p.mode == FG_MODE_CACHED ? 1 : 3;
+  if (p.mode == FG_MODE_CACHED) {
+    float* thr = reinterpret_cast<float*>(hist);
+    for (int i = threadIdx.x; i < 128; i += kScoreThreads) {
+      const int qi = gt * 128 + i;
+      thr[i] = qi < p.N ? p.sqrt_d * (p.lse[(size_t)bh * p.N + qi] + p.ln_tau) : INFINITY;
+    }
+  }
   if (warp == 1) {
     __syncwarp();
     tmem_alloc(&bars->tmem_base, 128 * kAcc);
@@ -181,9 +193,10 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
 
   if (warp == 0) {
     if (lane == 0) {
-      // q_avg terms for this group tile: 3 terms x D/64 boxes of (64 x 128 groups)
-      mbar_arrive_expect_tx(&bars->q_full, 3 * L::kTerm);
-      for (int t = 0; t < 3; ++t)
+      // q_avg terms for this group tile: 3 terms x D/64 boxes of (64 x 128
+      // groups); CACHED: one term, the 128 query rows of this tile
+      mbar_arrive_expect_tx(&bars->q_full, n_terms * L::kTerm);
+      for (int t = 0; t < n_terms; ++t)
         for (int h = 0; h < L::kHalves; ++h)
           tma_load_3d(sQ + t * L::kTerm + h * 16384, &qmap, &bars->q_full, h * 64, gt * 128,
                       t * p.BH + bh);
@@ -231,10 +244,12 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         tc_fence_after();
         const uint32_t d_tmem = tmem + ab * 128;
 #pragma unroll
-        for (int t = 0; t < 3; ++t)
+        for (int t = 0; t < 3; ++t) {
+          if (t >= n_terms) break;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             umma_bf16_ss(d_tmem, da[kk], dq[t][kk], idesc, (t > 0 || kk > 0) ? 1u : 0u);
+        }
         umma_commit(&bars->acc_full[ab]);
         umma_commit(&bars->k_empty[st]);
       }
@@ -287,6 +302,20 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
                 atomicAdd(&whist[(kk >> p.bin_shift) & p.bin_mask], 1u);
             }
           }
+        } else if (p.mode == FG_MODE_CACHED) {
+          // this lane's key against the warp's 32 query columns, which all
+          // belong to one group (32 divides the group size): kept when one
+          // of them passes its threshold; lane e of the ballot is key e of
+          // this lane quarter, so the ballot is the bitmask word itself
+          const float* thr = reinterpret_cast<const float*>(hist) + c0;
+          bool any = false;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) any |= v[e] > thr[e];
+          const uint32_t word = __ballot_sync(0xffffffffu, kvalid && any);
+          const int g = (gt * 128 + c0) / p.group;
+          const int kw = ((tile0 + j) * 128 + 32 * quarter) / 32;
+          if (lane == 0 && word != 0u && g < p.G && kw < p.WN)
+            atomicOr(p.bits + ((size_t)bh * p.G + g) * p.WN + kw, word);
         } else {
           const float f_keep = p.mode == FG_MODE_BITS ? f_tau : f_bin_hi;
           bool any_cand = false;
@@ -315,7 +344,7 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->acc_free[ab]);
-      if (p.mode != FG_MODE_HIST) {
+      if (p.mode == FG_MODE_BITS || p.mode == FG_MODE_BITS_COLLECT) {
         // lane e holds this warp's 32 keys for groups half*kCols + 32*i + e
         const int kw = ((tile0 + j) * 128 + 32 * quarter) / 32;
 #pragma unroll
@@ -481,11 +510,15 @@ __global__ void __launch_bounds__(1024) fg_offsets_kernel(FgListParams p) {
 }
 
 // One warp per (tile, head) lists the tile's union in ascending key order,
-// 1,024 keys (32 bitmask words) at a time: lane l expands the set bits of
-// word l into a per-warp staging buffer in shared memory at its prefix
-// position, then the warp copies the chunk's entries out with consecutive
-// lanes on consecutive list slots (coalesced stores).
+// 1,024 keys (32 bitmask words) at a time, through a per-warp staging buffer
+// in shared memory: each word's keys go to its prefix position there, then
+// the warp copies the chunk's entries out with consecutive lanes on
+// consecutive list slots (coalesced stores). Kept keys cluster, so a chunk
+// mixes sparse and dense words: lane l expands word l itself when it has at
+// most kDenseBits set bits, and the whole warp expands each denser word (one
+// bit per lane), so no lane loops over a full word while the others wait.
 constexpr int kListWarps = 8;
+constexpr uint32_t kDenseBits = 12;
 
 __global__ void __launch_bounds__(32 * kListWarps) fg_compact_kernel(FgListParams p) {
   __shared__ uint32_t stage[kListWarps][1024];
@@ -511,13 +544,32 @@ __global__ void __launch_bounds__(32 * kListWarps) fg_compact_kernel(FgListParam
       const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += t;
     }
-    uint32_t* dst = sb + (incl - c);
-    const uint32_t kbase = 32u * (uint32_t)w;
-    while (u) {
-      const uint32_t low = u & (0u - u);               // lowest set bit
-      u ^= low;
-      *dst++ = (kbase + (uint32_t)__popc(low - 1u)) | ((a & low) ? (1u << 30) : 0u) |
-               ((b & low) ? (1u << 31) : 0u);
+    const uint32_t excl = incl - c;
+    // sparse words: each lane expands its own, at most kDenseBits iterations
+    if (c <= kDenseBits) {
+      uint32_t* dst = sb + excl;
+      const uint32_t kbase = 32u * (uint32_t)w;
+      while (u) {
+        const uint32_t low = u & (0u - u);             // lowest set bit
+        u ^= low;
+        *dst++ = (kbase + (uint32_t)__popc(low - 1u)) | ((a & low) ? (1u << 30) : 0u) |
+                 ((b & low) ? (1u << 31) : 0u);
+      }
+    }
+    // dense words: the whole warp on one word at a time, lane l on bit l,
+    // its slot the word's start plus the set bits below it
+    uint32_t dense = __ballot_sync(0xffffffffu, c > kDenseBits);
+    while (dense) {
+      const int src = __ffs(dense) - 1;
+      dense &= dense - 1u;
+      const uint32_t uw = __shfl_sync(0xffffffffu, u, src);
+      const uint32_t aw = __shfl_sync(0xffffffffu, a, src);
+      const uint32_t bw = __shfl_sync(0xffffffffu, b, src);
+      const uint32_t ew = __shfl_sync(0xffffffffu, excl, src);
+      if ((uw >> lane) & 1u)
+        sb[ew + __popc(uw & ((1u << lane) - 1u))] =
+            (32u * (uint32_t)(w0 + src) + (uint32_t)lane) | (((aw >> lane) & 1u) << 30) |
+            (((bw >> lane) & 1u) << 31);
     }
     const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
     __syncwarp();
@@ -551,7 +603,7 @@ cudaError_t launch_score(const CUtensorMap& km, const CUtensorMap& qm, const FgS
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   const int n_tiles = (p.N + 127) / 128;
-  dim3 grid((n_tiles + kKeyTilesPerCta - 1) / kKeyTilesPerCta, (p.G + 127) / 128, p.BH);
+  dim3 grid((n_tiles + kKeyTilesPerCta - 1) / kKeyTilesPerCta, p.row_tiles, p.BH);
   fg_score_kernel<D><<<grid, kScoreThreads, L::kAlloc, st>>>(km, qm, p);
   return cudaGetLastError();
 }
@@ -591,6 +643,7 @@ cudaError_t launch_fg_build(const FgBuildParams& b, EncodeFn enc, cudaStream_t s
   sp.bits = b.bits; sp.hist = b.hist; sp.sel = b.sel; sp.status = b.status;
   sp.cand = b.cand; sp.cand_count = b.cand_count;
   sp.BH = b.BH; sp.N = b.N; sp.G = b.G; sp.WN = b.WN;
+  sp.row_tiles = G_pad / 128;
   const float inv_sqrt_d = 1.0f / sqrtf((float)b.d);
   auto score = [&]() {
     return b.d == 128 ? launch_score<128>(km, qm, sp, st) : launch_score<64>(km, qm, sp, st);
@@ -626,6 +679,36 @@ cudaError_t launch_fg_build(const FgBuildParams& b, EncodeFn enc, cudaStream_t s
   sp.mode = FG_MODE_BITS;
   sp.only_heads = b.fallback;
   if ((e = score()) != cudaSuccess) return e;
+  return launch_fg_lists(b.lists, st);
+}
+
+namespace {
+__global__ void fill_f32_kernel(float* dst, int n, float v) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) dst[i] = v;
+}
+}  // namespace
+
+cudaError_t launch_fg_cached(const FgCachedParams& b, EncodeFn enc, cudaStream_t st) {
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(b.bits, 0, sizeof(uint32_t) * (size_t)b.BH * b.G * b.WN, st)) != cudaSuccess)
+    return e;
+  fill_f32_kernel<<<(b.BH + 255) / 256, 256, 0, st>>>(b.tau_out, b.BH, b.tau);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  CUtensorMap km, qm;
+  if (!encode_3d(&km, b.k, b.d, b.N, b.BH, 128, enc)) return cudaErrorInvalidValue;
+  if (!encode_3d(&qm, b.q, b.d, b.N, b.BH, 128, enc)) return cudaErrorInvalidValue;
+  FgScoreParams sp{};
+  sp.mode = FG_MODE_CACHED;
+  sp.bits = b.bits; sp.status = b.status;
+  sp.lse = b.lse;
+  sp.ln_tau = logf(b.tau);
+  sp.sqrt_d = sqrtf((float)b.d);
+  sp.group = b.group;
+  sp.row_tiles = (b.N + 127) / 128;
+  sp.BH = b.BH; sp.N = b.N; sp.G = b.G; sp.WN = b.WN;
+  e = b.d == 128 ? launch_score<128>(km, qm, sp, st) : launch_score<64>(km, qm, sp, st);
+  if (e != cudaSuccess) return e;
   return launch_fg_lists(b.lists, st);
 }
 

@@ -17,7 +17,10 @@ typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void
 // BITS_COLLECT: bitmask of the keys whose top 24 bits exceed the prefix the
 // first two levels decided, plus a list of the keys that share it (the last
 // 8 bits are then selected among those few by fg_fixup).
-enum { FG_MODE_HIST = 0, FG_MODE_BITS = 1, FG_MODE_BITS_COLLECT = 2 };
+// CACHED: the B operand is 128 query rows instead of q_avg terms; a slice
+// (group, key) is kept when one of the group's queries gives the key a
+// full-attention probability above tau (FG-Attn review, the cached strategy).
+enum { FG_MODE_HIST = 0, FG_MODE_BITS = 1, FG_MODE_BITS_COLLECT = 2, FG_MODE_CACHED = 3 };
 
 // Candidate slots per head for the last select level; more than this (only
 // with very many scores equal in their top 24 bits) falls back to the full
@@ -42,6 +45,11 @@ struct FgScoreParams {
   uint2* cand;             // BITS_COLLECT: [BH][kFgCandCap] (key index, group << 8 | low 8 bits)
   uint32_t* cand_count;    // [BH]
   const uint32_t* only_heads;  // if set: heads whose flag is 0 do nothing
+  const float* lse;        // CACHED: [BH][N] natural-log LSE of full attention
+  float ln_tau;            // CACHED: ln(tau)
+  float sqrt_d;            // CACHED: sqrt(d)
+  int group;               // CACHED: queries per group (64 or 128)
+  int row_tiles;           // 128-row tiles of the B operand (groups, or queries for CACHED)
   int BH, N, G, WN;
 };
 
@@ -72,6 +80,21 @@ struct FgBuildParams {
   float keep_fraction;
 };
 
+// The cached rule's bitmask and union lists from Q, K and the LSE of full
+// attention: a slice is kept when max over its group's queries of
+// exp(q.k / sqrt(d) - lse_q) > tau.
+struct FgCachedParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const float* lse;        // [BH][N]
+  uint32_t* bits;          // [BH][G][WN], cleared here first
+  float* tau_out;          // [BH]: tau, for inspection
+  uint32_t* status;
+  FgListParams lists;
+  int BH, N, d, group, G, WN;
+  float tau;
+};
+
 int fg_g_pad(int G);
 size_t fg_qsplit_bytes(int BH, int G, int d);
 size_t fg_hist_bytes(int BH);
@@ -80,5 +103,6 @@ size_t fg_cand_bytes(int BH);
 long long fg_list_cap_per_head(int G, int N, float keep_fraction);
 cudaError_t launch_fg_build(const FgBuildParams& p, EncodeFn enc, cudaStream_t st);
 cudaError_t launch_fg_lists(const FgListParams& p, cudaStream_t st);
+cudaError_t launch_fg_cached(const FgCachedParams& p, EncodeFn enc, cudaStream_t st);
 
 }  // namespace sa

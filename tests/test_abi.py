@@ -209,6 +209,26 @@ def test_explicit_bits_are_checked_against_the_mask_size():
             sa._check_explicit_bits()
 
 
+def test_quantize_and_cached_mask_arguments_are_checked_on_the_host():
+    L = N.lib()
+    vp = 0x1000                                        # aligned, never dereferenced
+    for n_elems, n_tensors in ((12, 1), (0, 1), (64, 0), (64, 70000)):
+        assert L.sparse_attn_quantize_e4m3(vp, n_elems, n_tensors, vp, vp, None) \
+            == N.SA_ERR_INVALID_ARG, (n_elems, n_tensors)
+    assert L.sparse_attn_quantize_e4m3(vp + 8, 64, 1, vp, vp, None) == N.SA_ERR_INVALID_ARG
+    assert L.sparse_attn_quantize_e4m3(vp, 64, 1, None, vp, None) == N.SA_ERR_INVALID_ARG
+    pr = N.Problem(1, 2, 3, 4, 64, 128)
+    fg = make_policy("fg", fg_group=64, fg_keep_fraction=1.0)
+    sta = make_policy("sta", tile=(1, 2, 64), window=(1, 1, 1))
+    call = lambda pol, tau, lse=vp, ws=vp: L.sparse_attn_build_mask_fg_cached(
+        ctypes.byref(pr), ctypes.byref(pol), vp, vp, lse, tau, ws, ws, None)
+    assert call(sta, 0.0) == N.SA_ERR_INVALID_ARG             # FG policies only
+    for tau in (-0.1, 1.0, float("nan")):
+        assert call(fg, tau) == N.SA_ERR_INVALID_ARG, tau
+    assert call(fg, 0.0, lse=None) == N.SA_ERR_INVALID_ARG
+    assert call(fg, 0.0, ws=vp + 16) == N.SA_ERR_WORKSPACE
+
+
 def test_policy_head_arrays_must_cover_the_problem():
     # the library reads one temporal flag and one window per head of the
     # problem from the policy's host arrays

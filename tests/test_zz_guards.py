@@ -83,3 +83,45 @@ def test_no_write_outside_any_buffer(name):
     assert torch.equal(g["o"].payload(), o_ref.contiguous().view(torch.uint8).reshape(-1))
     assert torch.equal(g["lse"].payload(), lse_ref.contiguous().view(torch.uint8).reshape(-1))
     assert math.isfinite(float(o_ref.float().abs().max()))
+
+
+def test_cached_mask_and_quantizer_write_inside_their_buffers():
+    # the FG cached mask (LSE in, bits and union lists out) and the E4M3
+    # quantizer (codes and scales out), each between guards
+    from sparse_attention_video_b200 import SparseAttention, _native as N, make_policy
+    wl = FG
+    x = make_qkv(wl)
+    q, k, v = (_dev(x[n]) for n in "qkv")
+    policy = make_policy("fg", block=128, fg_group=64, fg_keep_fraction=1.0)
+    sa = SparseAttention(wl.batch, wl.heads, wl.T, wl.H, wl.W, wl.head_dim, policy)
+    lse = torch.zeros((wl.batch, wl.heads, wl.N), dtype=torch.float32, device="cuda")
+    sa.build_mask_fg_cached(q, k, lse + float(np.log(wl.N)))     # a uniform-attention LSE
+    problem = sa.problem
+    mask_bytes, scratch_bytes = N.workspace_size(problem, policy)
+    qkv_bytes = q.numel() * 2
+    g = {"q": Guarded(qkv_bytes), "k": Guarded(qkv_bytes), "lse": Guarded(lse.numel() * 4),
+         "mask": Guarded(mask_bytes), "scratch": Guarded(max(scratch_bytes, 256))}
+    g["q"].payload().copy_(q.view(torch.uint8).reshape(-1))
+    g["k"].payload().copy_(k.view(torch.uint8).reshape(-1))
+    g["lse"].payload().copy_((lse + float(np.log(wl.N))).view(torch.uint8).reshape(-1))
+    stream = torch.cuda.current_stream().cuda_stream
+    N.build_mask_fg_cached(problem, policy, g["q"].ptr, g["k"].ptr, g["lse"].ptr, 0.0,
+                           g["mask"].ptr, g["scratch"].ptr, stream)
+    n_el, n_t = wl.N * wl.head_dim, wl.batch * wl.heads
+    gc, gi = Guarded(n_el * n_t), Guarded(4 * n_t)
+    N.quantize_e4m3(g["q"].ptr, n_el, n_t, gc.ptr, gi.ptr, stream)
+    torch.cuda.synchronize()
+    assert N.status(g["scratch"].ptr, stream) == N.SA_OK
+    bad = [n for n, b in list(g.items()) + [("codes", gc), ("inv", gi)] if not b.intact()]
+    assert not bad, f"written outside {bad}"
+    # the bitmask, tau and union lists match the ordinary run's; the rest of
+    # the mask workspace is not written by this call
+    lay = [(N.SA_EXPORT_FG_BITS, "bits"), (N.SA_EXPORT_FG_TAU, "tau"),
+           (N.SA_EXPORT_FG_TILE_KEYS, "tile keys")]
+    for what, label in lay:
+        nb = N.export_bytes(problem, policy, what)
+        a = np.empty(nb, np.uint8)
+        b = np.empty(nb, np.uint8)
+        N.mask_export(problem, policy, sa.mask_ws.data_ptr(), what, a.ctypes.data, nb, stream)
+        N.mask_export(problem, policy, g["mask"].ptr, what, b.ctypes.data, nb, stream)
+        assert np.array_equal(a, b), label
