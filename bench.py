@@ -44,6 +44,8 @@ def _args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-mask comparison")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-mask-roofline", action="store_true",
+                    help="skip the per-kernel timing of the memory-bound mask kernels")
     ap.add_argument("--no-profile", action="store_true",
                     help="skip the head-profiler timing (spatial/temporal workload only)")
     ap.add_argument("--workload", default=WORKLOAD,
@@ -74,73 +76,186 @@ def _peaks():
 
 
 # ---------------------------------------------------------------- CPU oracle sample
-def cpu_oracle_sample(wl, x, budget_s=20.0):
-    """Time the oracle on a bounded sample of the workload: the full block mask
-    of one spatial and one temporal head and masked attention for sampled query
-    blocks of each. Returns (attended TFLOP/s, description, threads)."""
-    from oracle import attention, pipeline
-    from synthetic import bf16_bits_to_f32
+def _threads():
     try:
         from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
-        threads = os.cpu_count() or 1
-    heads = [0, wl.temporal_heads[0]] if wl.temporal_heads else [0]
-    rng = np.random.default_rng(0)
-    flops = 0.0
-    n_blocks = 0
-    t0 = time.perf_counter()
-    if wl.kind == "fg":
-        q, k, v = (bf16_bits_to_f32(x[n][0, 0]) for n in "qkv")
-        keep = pipeline.head_mask(wl, q, k, 0)["keep_groups"]
-        for g in rng.permutation(keep.shape[0]):
-            attention.slice_attention(q, k, v, keep, wl.fg_group, [int(g)])
-            flops += 4.0 * wl.head_dim * float(keep[g].sum()) * wl.fg_group
-            n_blocks += 1
-            if time.perf_counter() - t0 > budget_s:
-                break
+        return os.cpu_count() or 1
+
+
+def cpu_model():
+    """The host CPU's model name (lscpu, else /proc/cpuinfo)."""
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.startswith("Model name:"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def cpu_oracle_sample(wl, x, budget_s=20.0, single_thread=False):
+    """Time the oracle on a bounded sample of the workload: the full mask of
+    one spatial and one temporal head (FG: of head 0), then masked attention
+    for sampled query blocks (groups) of those heads. Returns a dict with the
+    attended TFLOP/s over the whole sample, the per-query-block attention
+    time and a labelled extrapolation to one full call."""
+    from oracle import attention, pipeline
+    from synthetic import bf16_bits_to_f32
+    limit = None
+    if single_thread:
+        try:
+            from threadpoolctl import threadpool_limits
+            limit = threadpool_limits(limits=1)
+        except Exception:
+            limit = None
+    try:
+        threads = 1 if single_thread else _threads()
+        rng = np.random.default_rng(0)
+        flops = 0.0
+        n_rows = 0
+        mask_s = attn_s = 0.0
+        t0 = time.perf_counter()
+        if wl.kind == "fg":
+            heads = [0]
+            q, k, v = (bf16_bits_to_f32(x[n][0, 0]) for n in "qkv")
+            keep = pipeline.head_mask(wl, q, k, 0)["keep_groups"]
+            mask_s = time.perf_counter() - t0
+            a0 = time.perf_counter()
+            for g in rng.permutation(keep.shape[0]):
+                attention.slice_attention(q, k, v, keep, wl.fg_group, [int(g)])
+                flops += 4.0 * wl.head_dim * float(keep[g].sum()) * wl.fg_group
+                n_rows += 1
+                if time.perf_counter() - t0 > budget_s:
+                    break
+            attn_s = time.perf_counter() - a0
+            unit_rows = wl.fg_group
+            units_per_head = keep.shape[0]
+            what = f"query groups of {wl.fg_group}"
+        else:
+            heads = [0, wl.temporal_heads[0]] if wl.temporal_heads else [0]
+            units_per_head = 0
+            for h in heads:
+                q, k, v = (bf16_bits_to_f32(x[n][0, h]) for n in "qkv")
+                m0 = time.perf_counter()
+                ref = pipeline.head_mask(wl, q, k, h)
+                mask_s += time.perf_counter() - m0
+                blk, bm = ref["order_blocks"], ref["bmask"]
+                units_per_head = max(units_per_head, blk.shape[0])
+                a0 = time.perf_counter()
+                for qb in rng.permutation(blk.shape[0]):
+                    attention.block_sparse_attention(q, k, v, blk, bm, [int(qb)])
+                    flops += 4.0 * wl.head_dim * float(bm[qb].sum()) * wl.block * wl.block
+                    n_rows += 1
+                    if time.perf_counter() - t0 > budget_s * (heads.index(h) + 1) / len(heads):
+                        break
+                attn_s += time.perf_counter() - a0
+            unit_rows = wl.block
+            what = f"query blocks of {wl.block} tokens"
         dt = time.perf_counter() - t0
-        desc = (f"oracle on head 0: slice scores, threshold and mask of the head + masked "
-                f"attention (float64) for {n_blocks} query groups of {wl.fg_group}")
-        return flops / dt / 1e12, desc, threads
-    for h in heads:
-        q, k, v = (bf16_bits_to_f32(x[n][0, h]) for n in "qkv")
-        ref = pipeline.head_mask(wl, q, k, h)
-        blk, bm = ref["order_blocks"], ref["bmask"]
-        for qb in rng.permutation(blk.shape[0]):
-            attention.block_sparse_attention(q, k, v, blk, bm, [int(qb)])
-            flops += 4.0 * wl.head_dim * float(bm[qb].sum()) * wl.block * wl.block
-            n_blocks += 1
-            if time.perf_counter() - t0 > budget_s * (heads.index(h) + 1) / len(heads):
-                break
-    dt = time.perf_counter() - t0
-    desc = (f"oracle on heads {heads}: full block mask per head + masked attention "
-            f"(float64) for {n_blocks} query blocks of 128 tokens")
-    return flops / dt / 1e12, desc, threads
+    finally:
+        if limit is not None:
+            limit.restore_original_limits()
+    per_unit = attn_s / max(n_rows, 1)
+    full_s = mask_s / len(heads) * wl.heads + per_unit * units_per_head * wl.heads
+    desc = (f"oracle on heads {heads}: full mask per head + masked attention (float64) for "
+            f"{n_rows} sampled {what}")
+    return {"value": flops / dt / 1e12, "desc": desc, "threads": threads,
+            "mask_s_per_head": mask_s / len(heads),
+            "attn_s_per_query_block": per_unit, "rows_per_query_block": unit_rows,
+            "extrapolated_full_call_s": full_s}
 
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
+    """SM clock and clock-event reasons of one GPU, sampled during the timed
+    region: NVML every 10 ms from a thread (enough samples even for a
+    fraction of a second), else nvidia-smi every 200 ms."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
 
-    def __init__(self, index):
-        self.index = index
+    def __init__(self, device):
+        self.device = device
         self.proc = None
+        self.thread = None
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.source = None
         self.path = tempfile.mktemp(suffix=".csv")
 
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device)
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            busid = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), bus,
+                                          getattr(props, "pci_device_id", 0))
+            try:
+                return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(busid)
+            except Exception:
+                pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.device.index or 0)
+
     def start(self):
+        import threading
+        try:
+            nv, h = self._nvml_handle()
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                                  getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+            self._stop = threading.Event()
+
+            def loop():
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                        bits = int(get_reasons(h))
+                        for name, bit in self.REASONS:
+                            if bits & bit:
+                                self.reasons.add(name)
+                    except Exception:
+                        pass
+                    self._stop.wait(0.01)
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            self.source = "nvml, 10 ms"
+            return
+        except Exception:
+            self.thread = None
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", "-i", str(self.device.index or 0), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
                 stdout=self.f, stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi, 200 ms"
         except Exception:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=5)
+            if not self.samples:
+                return None
+            return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                    "reasons": sorted(self.reasons), "samples": len(self.samples),
+                    "source": self.source}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -150,7 +265,7 @@ class ClockSampler:
             self.proc.kill()
         self.f.close()
         sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        names = [n for n, _ in self.REASONS]
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
@@ -167,7 +282,45 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": self.source}
+
+
+def kernel_times(fn, device):
+    """Device time of every kernel ``fn`` launches, from one run under the
+    CUDA activity profiler (CUPTI timestamps, not ncu): {name: (launches,
+    total ms)}. Returns {} if the profiler is unavailable."""
+    import torch
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        torch.cuda.synchronize(device)
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            fn()
+            torch.cuda.synchronize(device)
+        out = {}
+        for e in prof.events():
+            dt = getattr(e, "device_time", None)
+            if dt is None:
+                dt = getattr(e, "cuda_time", 0.0)
+            if getattr(e, "device_type", None) is not None and "CUDA" not in str(e.device_type):
+                continue
+            if not dt:
+                continue
+            n, t = out.get(e.name, (0, 0.0))
+            out[e.name] = (n + 1, t + dt / 1e3)
+        return out
+    except Exception as exc:                          # profiler missing or CUPTI refused
+        log(f"kernel timing unavailable: {exc}")
+        return {}
+
+
+def _kernel_ms(times, fragment):
+    """(launches, ms) of the kernels whose name contains ``fragment``."""
+    n, t = 0, 0.0
+    for name, (k, ms) in times.items():
+        if fragment in name:
+            n += k
+            t += ms
+    return n, t
 
 
 def _traffic_per_launch():
@@ -211,6 +364,83 @@ def policy_kwargs(wl):
 LAUNCHES_PER_STEP = {"topk": 5, "sta": 3, "spatiotemporal": 4, "spade": 5, "fg": 13}
 
 
+def _block_valid(info, T, H, W, block):
+    """Valid tokens of each block of a head's working layout (int64 [nb])."""
+    nb = info.nb
+    if info.layout == 2:                      # 3D tile layout, raster tiles
+        b = np.arange(nb)
+        tw, th, tt = b % info.nw, (b // info.nw) % info.nh, b // (info.nw * info.nh)
+        vt = np.minimum(info.bt, T - tt * info.bt)
+        vh = np.minimum(info.bh, H - th * info.bh)
+        vw = np.minimum(info.bw, W - tw * info.bw)
+        return (vt * vh * vw).astype(np.int64)
+    n = T * H * W
+    return np.minimum(block, n - block * np.arange(nb)).astype(np.int64)
+
+
+def useful_flops(wl, sa):
+    """4 * d * (valid query, valid key) pairs of the kept blocks: the work
+    without the pad slots that the tile-granularity count includes."""
+    from sparse_attention_video_b200 import SA_EXPORT_BLOCK_BITS
+    infos = sa.export(2)
+    words = sa.export(SA_EXPORT_BLOCK_BITS)
+    # rows are sized for the largest block count of the policy's layouts,
+    # which may exceed every head's own (SPADE: the candidates not chosen)
+    nbmax = max(i.nb for i in infos)
+    while len(infos) * nbmax * ((nbmax + 31) // 32) < words.size:
+        nbmax += 1
+    w32 = (nbmax + 31) // 32
+    words = words.reshape(len(infos), nbmax, w32)
+    pairs = 0
+    for h, info in enumerate(infos):
+        valid = _block_valid(info, wl.T, wl.H, wl.W, wl.block)
+        bits = np.unpackbits(words[h, :info.nb].view(np.uint8), axis=1,
+                             bitorder="little")[:, :info.nb].astype(np.int64)
+        pairs += int(valid @ bits @ valid)
+    return 4.0 * wl.head_dim * pairs
+
+
+def fg_method_flops(wl, sa):
+    """4 * d * M * kept (group, key) slices: the FG method's own work (each
+    kept slice is one key against the M queries of its group)."""
+    from sparse_attention_video_b200 import SA_EXPORT_FG_BITS
+    bits = sa.export(SA_EXPORT_FG_BITS)
+    kept = int(np.bitwise_count(bits).sum(dtype=np.int64))
+    return 4.0 * wl.head_dim * wl.fg_group * kept, kept
+
+
+# Algorithmic bytes per launch of the memory-bound mask kernels (read + write
+# of what the step must touch once), per workload: name fragment -> bytes.
+def mask_kernel_bytes(wl, n_frame_major_heads=0):
+    tok = wl.N * wl.head_dim * 2                      # one head's tensor, bf16
+    out = {}
+    if n_frame_major_heads:
+        out["permute_fm"] = 3 * 2 * tok * n_frame_major_heads
+    if wl.kind in ("spade", "topk"):
+        out["pool_atoms"] = 2 * tok * wl.heads        # Q and K read once
+    if wl.kind == "fg":
+        out["fg_qbar"] = tok * wl.heads               # Q read once
+    return out
+
+
+def mask_kernel_bytes_entry(wl, times, hbm):
+    fm = len(wl.temporal_heads) if wl.kind == "spatiotemporal" else 0
+    return mask_roofline_entry(wl, times, mask_kernel_bytes(wl, fm), hbm)
+
+
+def mask_roofline_entry(wl, times, nbytes, hbm):
+    res = {}
+    for frag, b in nbytes.items():
+        n, ms = _kernel_ms(times, frag)
+        if n == 0:
+            continue
+        per = ms / n
+        gbs = b / (per * 1e-3) / 1e9
+        res[frag] = {"workload": wl.name, "ms": per, "algorithmic_bytes": b,
+                     "achieved_gbs": gbs, "peak_gbs": hbm, "frac": gbs / hbm}
+    return res
+
+
 # ---------------------------------------------------------------- multi-rank helpers
 def rank_workload(wl, rank):
     """Rank r runs its own problem of the same shape (weak scaling, no data
@@ -247,9 +477,10 @@ def run_reference(args, rank, world):
         xx[n][0, wl.temporal_heads[0]] = x[n][0, 1]
     vals = []
     for i in range(args.warmup + args.steps):
-        v, desc, threads = cpu_oracle_sample(wl, xx, budget_s=max(2.0, 60.0 / (args.steps + args.warmup)))
+        c = cpu_oracle_sample(wl, xx, budget_s=max(2.0, 60.0 / (args.steps + args.warmup)))
+        desc, threads = c["desc"], c["threads"]
         if i >= args.warmup:
-            vals.append(v)
+            vals.append(c["value"])
     value = statistics.mean(vals)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -258,7 +489,7 @@ def run_reference(args, rank, world):
             "config": {"workload": WORKLOAD, "grid": "30x48x80", "tokens": wl.N,
                        "heads": wl.heads, "head_dim": wl.head_dim, "batch": 1},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
-                             "kind": "oracle", "sample": desc},
+                             "kind": "oracle", "sample": desc, "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -352,18 +583,25 @@ def main():
     torch.cuda.synchronize(dev)
     log("warm-up done")
     assert sa.status() == 0, "device status word set during warm-up"
+    method = {}
     if wl.kind == "fg":
         # executed work: every 128-query tile against the union of its groups' kept keys
         from sparse_attention_video_b200 import SA_EXPORT_FG_TILE_KEYS
         keys = float(sa.export(SA_EXPORT_FG_TILE_KEYS).astype(np.float64).sum())
         flops_call = 4.0 * wl.head_dim * keys * 128
+        mflops, kept_slices = fg_method_flops(wl, sa)
+        method = {"method_tflop_per_call": mflops / 1e12, "kept_slices": kept_slices,
+                  "method_note": "4 * d * M * kept slices; the roofline counts the executed "
+                                 "union work of each 128-query tile"}
+        useful = mflops
     else:
         kept = sum(h.kept for h in sa.export(2))
         flops_call = 4.0 * wl.head_dim * kept * wl.block * wl.block
+        useful = useful_flops(wl, sa)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -386,6 +624,30 @@ def main():
     assert sa.status() == 0, "device status word set during the timed steps"
     ms_step = ms_total / args.steps
     value = aggregate_tflops(world, flops_call, ms_step)
+
+    # ---- memory-bound mask kernels: device time of each kernel of one
+    # build_mask (+ permute) from CUPTI, against its algorithmic bytes
+    mask_roof = {}
+    if not args.no_mask_roofline:
+        times = kernel_times(lambda: (sa.build_mask(q, k, stream), sa.permute(q, k, v, stream)), dev)
+        hbm_peak = _peaks()[2]
+        mask_roof.update(mask_kernel_bytes_entry(wl, times, hbm_peak))
+        if wl.name == WORKLOAD and not args.heads:
+            for other in ("spade_wan21_14b_720p", "fg_slices_hunyuan_720p"):
+                owl = rank_workload(CONFIGS[other], rank)
+                ox = make_qkv(owl)
+                oq, ok_ = (torch.from_numpy(ox[n].view(np.int16)).view(torch.bfloat16).to(dev)
+                           for n in "qk")
+                del ox
+                osa = SparseAttention(1, owl.heads, owl.T, owl.H, owl.W, owl.head_dim,
+                                      make_policy(**policy_kwargs(owl)), device=dev)
+                osa.build_mask(oq, ok_, stream)
+                otimes = kernel_times(lambda: osa.build_mask(oq, ok_, stream), dev)
+                assert osa.status() == 0, f"device status word set in the {other} mask build"
+                mask_roof.update(mask_kernel_bytes_entry(owl, otimes, hbm_peak))
+                del oq, ok_, osa
+                torch.cuda.empty_cache()
+        log("mask kernel rooflines done")
 
     # ---- end to end through the public API with host buffers
     o_host = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
@@ -548,10 +810,21 @@ def main():
     traffic = _traffic_per_launch()
     cpu = None
     if not args.no_cpu:
-        v_cpu, desc, threads = cpu_oracle_sample(wl_r, x)
-        log("cpu oracle sample done")
-        cpu = {"value": v_cpu, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": desc}
+        c = cpu_oracle_sample(wl_r, x)
+        c1 = cpu_oracle_sample(wl_r, x, budget_s=6.0, single_thread=True)
+        log("cpu oracle samples done")
+        cpu = {"value": c["value"], "unit": "TFLOP/s", "cores": c["threads"], "kind": "oracle",
+               "sample": c["desc"], "cpu_model": cpu_model(),
+               "single_thread": {"value": c1["value"], "unit": "TFLOP/s", "cores": 1,
+                                 "sample": c1["desc"]},
+               "mask_s_per_head": c["mask_s_per_head"],
+               "attn_s_per_query_block": c["attn_s_per_query_block"],
+               "rows_per_query_block": c["rows_per_query_block"],
+               "extrapolated_full_call_s": c["extrapolated_full_call_s"],
+               "extrapolation_note": ("extrapolated, not measured: the mean mask time per "
+                                      "sampled head x heads + the mean attention time per "
+                                      "sampled query block x query blocks x heads")}
+    sm_mhz = clk["sm_mhz"] if clk else None
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -565,13 +838,23 @@ def main():
         "step_breakdown_ms": {"build_mask": mask_ms, "permute": perm_ms, "attention": attn_ms},
         "attended_tflop_per_call": flops_call / 1e12,
         "attention_ms_per_call": attn_ms,
+        "useful_tflop_per_call": useful / 1e12,
+        "useful_tflops_attention": useful / (attn_ms * 1e-3) / 1e12,
+        **method,
         "roofline": {"kernel": "attn_fwd_kernel<%d,%d,%s>" % (wl.head_dim, wl.block,
                                                                "gather" if wl.kind == "fg" else "block"),
                      "bound": "tensor",
-                     "achieved": achieved, "peak": peak_sust, "unit": "TFLOP/s",
-                     "frac": achieved / peak_sust,
-                     "peak_note": f"{peak_src} sustained cuBLAS bf16 (burst {peak_burst})",
+                     "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s",
+                     "frac": achieved / peak_burst,
+                     "peak_note": (f"{peak_src} burst cuBLAS bf16 (the kernel is timed per call "
+                                   f"inside short steps); the sustained figure is a second number"),
+                     "peak_sustained": peak_sust, "frac_of_sustained": achieved / peak_sust,
+                     "attn_kcycles_per_call": (attn_ms * sm_mhz) if sm_mhz else None,
                      "traffic": traffic if wl.name == WORKLOAD and not args.heads else None},
+        "mask_roofline": mask_roof,
+        **({"method_tflops_attention": method["method_tflop_per_call"] * 1e12 / (attn_ms * 1e-3) / 1e12,
+            "method_frac": method["method_tflop_per_call"] * 1e12 / (attn_ms * 1e-3) / 1e12 / peak_burst}
+           if method else {}),
         "cpu_baseline": cpu,
         "e2e": {"value": aggregate_tflops(world, flops_call, e2e_ms), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
