@@ -357,16 +357,25 @@ SA_API int sparse_attn_selftest_wait_timeout(void* scratch_ws, void* stream);
  * with SA_ERR_UNSUPPORTED before anything is enqueued. No device memory is
  * allocated by this call.
  *
- * The first call on a device looks up the array's device address with that
- * device current; make that first call before any stream capture. All calls
+ * Every call looks up the array's device address in the current device's
+ * context (no allocation; the first lookup on a device may load the library's
+ * device code, so make the first call before any stream capture). All calls
  * share the one array: calls whose work can overlap on the GPU (unordered
- * streams) race on it. The status word of this variant lives in the array and
- * is not reported by sparse_attn_status. Asynchronous on ``stream``.
+ * streams) race on it. The device status word of this variant lives at the
+ * start of the array; read it with sparse_attn_status_static. Each call clears
+ * it first. Asynchronous on ``stream``.
  */
 #define SA_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
 SA_API int sparse_attn_build_mask_static(const sa_problem* problem, const sa_policy* policy,
                                          const void* q, const void* k, void* mask_ws,
                                          void* stream);
+
+/* Device status of the last sparse_attn_build_mask_static work on the current
+ * device, as sparse_attn_status reports it for a caller's scratch workspace:
+ * waits for ``stream``, returns SA_OK, SA_ERR_DEVICE_TIMEOUT or
+ * SA_ERR_DEVICE_BOUNDS (or SA_ERR_CUDA), and with ``clear`` != 0 resets the
+ * word. Copies four bytes to a host variable; allocates nothing. */
+SA_API int sparse_attn_status_static(void* stream, int clear);
 
 /* Static description of a status code. Never NULL. */
 SA_API const char* sparse_attn_strerror(int status);

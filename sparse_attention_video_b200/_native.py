@@ -26,7 +26,8 @@ SA_EXPORT_FG_TILE_KEYS = 5
 EXPORTED = ("sparse_attn_workspace_size", "sparse_attn_build_mask", "sparse_attn_forward",
             "sparse_attn_permute", "sparse_attn_attend",
             "sparse_attn_export_bytes", "sparse_attn_mask_export", "sparse_attn_status",
-            "sparse_attn_build_mask_static", "sparse_attn_selftest_wait_timeout",
+            "sparse_attn_build_mask_static", "sparse_attn_status_static",
+            "sparse_attn_selftest_wait_timeout",
             "sparse_attn_profile_heads", "sparse_attn_sta_window_search",
             "sparse_attn_build_mask_fg_cached", "sparse_attn_quantize_e4m3",
             "sparse_attn_strerror")
@@ -88,6 +89,7 @@ def lib():
         L.sparse_attn_mask_export.argtypes = [P, PP, vp, ctypes.c_int, vp, sz, vp]
         L.sparse_attn_status.argtypes = [vp, vp, ctypes.c_int]
         L.sparse_attn_build_mask_static.argtypes = [P, PP, vp, vp, vp, vp]
+        L.sparse_attn_status_static.argtypes = [vp, ctypes.c_int]
         L.sparse_attn_selftest_wait_timeout.argtypes = [vp, vp]
         L.sparse_attn_profile_heads.argtypes = [P, PP, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp,
                                                 vp, vp]
@@ -191,6 +193,11 @@ def build_mask_static(problem, policy, q, k, mask_ws, stream=0):
     _check(lib().sparse_attn_build_mask_static(ctypes.byref(problem), ctypes.byref(policy), q, k,
                                                mask_ws, stream),
            "sparse_attn_build_mask_static")
+
+
+def status_static(stream=0, clear=False):
+    """Status word of the static-scratch mask build (sparse_attn_status_static)."""
+    return lib().sparse_attn_status_static(stream, 1 if clear else 0)
 
 
 def status(scratch_ws, stream=0, clear=False):

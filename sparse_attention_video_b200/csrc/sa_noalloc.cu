@@ -18,33 +18,21 @@
 // writes itself.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "../../include/sparse_attn.h"
 
 namespace {
 
 static __device__ __align__(256) unsigned char g_static_scratch[SA_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of the array on the current device. In host code the name
-// g_static_scratch is only a host-side stand-in, never a device address, so
-// the address is looked up once per device (with that device current) and
-// cached.
+// Device address of the array in the current device's context. In host code
+// the name g_static_scratch is only a host-side stand-in, never a device
+// address, so the address is looked up with the device current. The lookup
+// runs on every call: it allocates nothing, and a cached address would outlive
+// a cudaDeviceReset or a switch to another context of the same device.
 int static_scratch(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
-      return SA_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return SA_ERR_CUDA;
+  *out = p;
   return SA_OK;
 }
 
@@ -61,4 +49,11 @@ extern "C" int sparse_attn_build_mask_static(const sa_problem* problem, const sa
   e = static_scratch(&scratch);
   if (e != SA_OK) return e;
   return sparse_attn_build_mask(problem, policy, q, k, mask_ws, scratch, stream);
+}
+
+extern "C" int sparse_attn_status_static(void* stream, int clear) {
+  void* scratch = nullptr;
+  const int e = static_scratch(&scratch);
+  if (e != SA_OK) return e;
+  return sparse_attn_status(scratch, stream, clear);
 }
