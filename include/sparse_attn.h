@@ -204,6 +204,43 @@ SA_API int sparse_attn_build_mask_fg_cached(const sa_problem* problem, const sa_
 SA_API int sparse_attn_quantize_e4m3(const void* x, long long n_elems, int n_tensors,
                                     uint8_t* codes, float* inv, void* stream);
 
+/* FP8 attention, step 1 (Sparse VideoGen review: FP8 attention with the
+ * layout transform): sparse_attn_permute for E4M3 codes. For every
+ * frame-major head, writes the frame-major copies of the codes of Q, K and V
+ * into scratch_ws (one byte per element), which sparse_attn_attend_fp8
+ * reads; other heads are not touched.
+ *   q8, k8, v8  device uint8 [batch, heads, N, head_dim] E4M3 codes in the
+ *               original token order (sparse_attn_quantize_e4m3 of each of
+ *               Q, K, V with n_tensors = batch*heads), 16-byte aligned
+ * The mask, problem and policy are those of sparse_attn_build_mask. Returns
+ * SA_ERR_INVALID_ARG / SA_ERR_WORKSPACE / SA_ERR_UNSUPPORTED synchronously.
+ * Asynchronous on ``stream``. */
+SA_API int sparse_attn_permute_fp8(const sa_problem* problem, const sa_policy* policy,
+                                   const void* q8, const void* k8, const void* v8,
+                                   const void* mask_ws, void* scratch_ws, void* stream);
+
+/* FP8 attention, step 2 (Sparse VideoGen review: the optional FP8 attention,
+ * credited with about 1.3x on HunyuanVideo): the block-sparse attention of
+ * sparse_attn_attend over the dequantized operands code / inv, with both
+ * products on E4M3 tensor cores (tcgen05.mma kind::f8f6f4) and fp32
+ * accumulation. The softmax probabilities of the second product are E4M3
+ * codes of 2^4 P (P <= 2^4 relative to the running maximum), so each P
+ * carries at most 2^-4 relative error above 2^-10 and 2^-14 absolute below;
+ * the row sums and LSE use the unrounded fp32 P.
+ *   q8, k8, v8        E4M3 codes as for sparse_attn_permute_fp8
+ *   q_inv, k_inv, v_inv  device float [batch*heads]: each tensor's inverse
+ *                     scale (the ``inv`` output of sparse_attn_quantize_e4m3)
+ *   o, lse            as for sparse_attn_attend (bf16 O, natural-log LSE)
+ * Block policies only (not SA_MASK_FG), head_dim 128 and block 128; others
+ * return SA_ERR_UNSUPPORTED. Frame-major heads read the copies of
+ * sparse_attn_permute_fp8. Asynchronous on ``stream``; device faults set the
+ * status word read by sparse_attn_status. */
+SA_API int sparse_attn_attend_fp8(const sa_problem* problem, const sa_policy* policy,
+                                  const void* q8, const void* k8, const void* v8,
+                                  const float* q_inv, const float* k_inv, const float* v_inv,
+                                  const void* mask_ws, void* scratch_ws, void* o, float* lse,
+                                  void* stream);
+
 /* ---------------------------------------------------------------- attention
  * O and LSE for the mask in mask_ws (built by sparse_attn_build_mask with the
  * same problem and policy). Equivalent to sparse_attn_permute followed by

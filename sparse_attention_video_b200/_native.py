@@ -30,6 +30,7 @@ EXPORTED = ("sparse_attn_workspace_size", "sparse_attn_build_mask", "sparse_attn
             "sparse_attn_selftest_wait_timeout",
             "sparse_attn_profile_heads", "sparse_attn_sta_window_search",
             "sparse_attn_build_mask_fg_cached", "sparse_attn_quantize_e4m3",
+            "sparse_attn_permute_fp8", "sparse_attn_attend_fp8",
             "sparse_attn_strerror")
 
 SA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -98,6 +99,8 @@ def lib():
         L.sparse_attn_build_mask_fg_cached.argtypes = [P, PP, vp, vp, vp, ctypes.c_float, vp, vp,
                                                        vp]
         L.sparse_attn_quantize_e4m3.argtypes = [vp, ctypes.c_longlong, ctypes.c_int, vp, vp, vp]
+        L.sparse_attn_permute_fp8.argtypes = [P, PP, vp, vp, vp, vp, vp, vp]
+        L.sparse_attn_attend_fp8.argtypes = [P, PP, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.sparse_attn_strerror.argtypes = [ctypes.c_int]
         L.sparse_attn_strerror.restype = ctypes.c_char_p
         for name in EXPORTED:
@@ -173,6 +176,19 @@ def build_mask_fg_cached(problem, policy, q, k, lse, tau, mask_ws, scratch_ws, s
 def quantize_e4m3(x, n_elems, n_tensors, codes, inv, stream=0):
     _check(lib().sparse_attn_quantize_e4m3(x, n_elems, n_tensors, codes, inv, stream),
            "sparse_attn_quantize_e4m3")
+
+
+def permute_fp8(problem, policy, q8, k8, v8, mask_ws, scratch_ws, stream=0):
+    _check(lib().sparse_attn_permute_fp8(ctypes.byref(problem), ctypes.byref(policy), q8, k8, v8,
+                                         mask_ws, scratch_ws, stream),
+           "sparse_attn_permute_fp8")
+
+
+def attend_fp8(problem, policy, q8, k8, v8, q_inv, k_inv, v_inv, mask_ws, scratch_ws, o, lse,
+               stream=0):
+    _check(lib().sparse_attn_attend_fp8(ctypes.byref(problem), ctypes.byref(policy), q8, k8, v8,
+                                        q_inv, k_inv, v_inv, mask_ws, scratch_ws, o, lse, stream),
+           "sparse_attn_attend_fp8")
 
 
 def export_bytes(problem, policy, what):

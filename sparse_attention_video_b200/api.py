@@ -199,6 +199,42 @@ class SparseAttention:
                  lse.data_ptr() if lse is not None else None, _stream_ptr(stream))
         return out, lse
 
+    def forward_fp8(self, q, k, v, out=None, lse=None, stream=None):
+        """FP8 attention over the built mask: Q, K and V quantized to E4M3 with
+        one scale per (batch, head) tensor, frame-major copies of the codes,
+        then the block-sparse attention on kind::f8f6f4 tensor cores. Returns
+        (out, lse, (codes, inv) of q, k, v)."""
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            _check_qkv(t, self.problem, n, self.device)
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+        _check_qkv(out, self.problem, "out", self.device)
+        _check_lse(lse, self.problem, self.device)
+        quant = [quantize_e4m3(t, stream) for t in (q, k, v)]
+        (q8, qi), (k8, ki), (v8, vi) = quant
+        N.permute_fp8(self.problem, self.policy, q8.data_ptr(), k8.data_ptr(), v8.data_ptr(),
+                      self.mask_ws.data_ptr(), self.scratch_ws.data_ptr(), _stream_ptr(stream))
+        N.attend_fp8(self.problem, self.policy, q8.data_ptr(), k8.data_ptr(), v8.data_ptr(),
+                     qi.data_ptr(), ki.data_ptr(), vi.data_ptr(), self.mask_ws.data_ptr(),
+                     self.scratch_ws.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                     _stream_ptr(stream))
+        return out, lse, quant
+
+    def attend_fp8(self, q8, k8, v8, q_inv, k_inv, v_inv, out, lse, stream=None):
+        """The FP8 attention step alone on existing codes and scales (after
+        permute_fp8)."""
+        N.attend_fp8(self.problem, self.policy, q8.data_ptr(), k8.data_ptr(), v8.data_ptr(),
+                     q_inv.data_ptr(), k_inv.data_ptr(), v_inv.data_ptr(), self.mask_ws.data_ptr(),
+                     self.scratch_ws.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                     _stream_ptr(stream))
+        return out, lse
+
+    def permute_fp8(self, q8, k8, v8, stream=None):
+        N.permute_fp8(self.problem, self.policy, q8.data_ptr(), k8.data_ptr(), v8.data_ptr(),
+                      self.mask_ws.data_ptr(), self.scratch_ws.data_ptr(), _stream_ptr(stream))
+
     def __call__(self, q, k, v, stream=None):
         self.build_mask(q, k, stream)
         return self.forward(q, k, v, stream=stream)

@@ -211,29 +211,38 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D map over [BH][rows][d] bf16 with a (64, box_rows, 1) box.
-bool map_3d(CUtensorMap* m, const void* base, int BH, long long rows, int d, int box_rows) {
+// 3-D map over [BH][rows][d] with a (128-byte, box_rows, 1) box: bf16 by
+// default, E4M3 codes (one byte each) with ``bytes`` = 1.
+bool map_3d(CUtensorMap* m, const void* base, int BH, long long rows, int d, int box_rows,
+            int bytes = 2) {
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)BH};
-  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)d * bytes, (cuuint64_t)rows * d * bytes};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / bytes), (cuuint32_t)box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+  const CUtensorMapDataType dt = bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                            : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return encode_fn()(m, dt, 3, const_cast<void*>(base), dims,
                      strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 5-D map over [BH][T][H][W][d] bf16 whose box is one (bt, bh, bw) tile x 64 columns.
-bool map_5d(CUtensorMap* m, const void* base, const sa_problem& pr, const int* tile) {
+// 5-D map over [BH][T][H][W][d] whose box is one (bt, bh, bw) tile x 128 bytes
+// of d (bf16, or E4M3 codes with ``bytes`` = 1).
+bool map_5d(CUtensorMap* m, const void* base, const sa_problem& pr, const int* tile,
+            int bytes = 2) {
   const int d = pr.head_dim;
-  const cuuint64_t e = 2;
+  const cuuint64_t e = (cuuint64_t)bytes;
   cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)pr.W, (cuuint64_t)pr.H, (cuuint64_t)pr.T,
                         (cuuint64_t)pr.batch * pr.heads};
   cuuint64_t strides[4] = {d * e, (cuuint64_t)pr.W * d * e, (cuuint64_t)pr.H * pr.W * d * e,
                            (cuuint64_t)pr.T * pr.H * pr.W * d * e};
-  cuuint32_t box[5] = {64, (cuuint32_t)tile[2], (cuuint32_t)tile[1], (cuuint32_t)tile[0], 1};
+  cuuint32_t box[5] = {(cuuint32_t)(128 / bytes), (cuuint32_t)tile[2], (cuuint32_t)tile[1],
+                       (cuuint32_t)tile[0], 1};
   cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims,
+  const CUtensorMapDataType dt = bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                            : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return encode_fn()(m, dt, 5, const_cast<void*>(base), dims,
                      strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -459,6 +468,10 @@ extern "C" int sparse_attn_build_mask_fg_cached(const sa_problem* problem,
 
 namespace {
 
+struct CallCtx;
+bool block_maps(const sa_problem& pr, const sa_policy& po, const CallCtx& c, const void* q,
+                const void* k, const void* v, int bytes, AttnMaps* maps);
+
 struct CallCtx {
   MaskLayout M;
   ScratchLayout S;
@@ -487,6 +500,35 @@ int prepare_call(const sa_problem* problem, const sa_policy* policy, const void*
   c->BH = c->M.BH;
   c->n_pad = policy->kind == SA_MASK_FG ? c->N : ceil_div(c->N, policy->block) * policy->block;
   return SA_OK;
+}
+
+// Tensor maps of the block kernel for Q, K, V (elements of ``bytes`` bytes):
+// the original tensors (3-D), the frame-major copies in the scratch
+// workspace, and one 5-D tile map per blocking candidate.
+bool block_maps(const sa_problem& pr, const sa_policy& po, const CallCtx& c, const void* q,
+                const void* k, const void* v, int bytes, AttnMaps* maps) {
+  const void* src[3] = {q, k, v};
+  const bool fm = needs_frame_major(pr, po);
+  std::memset(maps, 0, sizeof(*maps));
+  CUtensorMap* sets[3] = {maps->q, maps->k, maps->v};
+  const bool tiled = po.kind == SA_MASK_SPADE || is_tile_kind(po.kind) ||
+                     (po.kind == SA_MASK_EXPLICIT && po.explicit_layout == SA_LAYOUT_TILE);
+  const int C = po.kind == SA_MASK_SPADE ? po.n_candidates : 1;
+  for (int i = 0; i < 3; ++i) {
+    if (!map_3d(&sets[i][0], src[i], c.BH, c.N, c.d, po.block, bytes)) return false;
+    if (fm) {
+      const void* perm = c.sw + c.S.off_perm + i * c.S.perm_stride;
+      if (!map_3d(&sets[i][1], perm, c.BH, c.n_pad, c.d, po.block, bytes)) return false;
+    } else {
+      sets[i][1] = sets[i][0];
+    }
+    for (int cc = 0; cc < C; ++cc) {
+      if (!tiled) { sets[i][2 + cc] = sets[i][0]; continue; }
+      const int* tile = po.kind == SA_MASK_SPADE ? po.candidates[cc] : po.tile;
+      if (!map_5d(&sets[i][2 + cc], src[i], pr, tile, bytes)) return false;
+    }
+  }
+  return true;
 }
 
 }  // namespace
@@ -542,28 +584,8 @@ extern "C" int sparse_attn_attend(const sa_problem* problem, const sa_policy* po
     return cuda_status(launch_attn_gather(c.d, maps, ap, c.st));
   }
 
-  const void* src[3] = {q, k, v};
-  const bool fm = needs_frame_major(pr, po);
   AttnMaps maps;
-  std::memset(&maps, 0, sizeof(maps));
-  CUtensorMap* sets[3] = {maps.q, maps.k, maps.v};
-  const bool tiled = po.kind == SA_MASK_SPADE || is_tile_kind(po.kind) ||
-                     (po.kind == SA_MASK_EXPLICIT && po.explicit_layout == SA_LAYOUT_TILE);
-  const int C = po.kind == SA_MASK_SPADE ? po.n_candidates : 1;
-  for (int i = 0; i < 3; ++i) {
-    if (!map_3d(&sets[i][0], src[i], c.BH, c.N, c.d, po.block)) return SA_ERR_CUDA;
-    if (fm) {
-      const void* perm = c.sw + c.S.off_perm + i * c.S.perm_stride;
-      if (!map_3d(&sets[i][1], perm, c.BH, c.n_pad, c.d, po.block)) return SA_ERR_CUDA;
-    } else {
-      sets[i][1] = sets[i][0];
-    }
-    for (int cc = 0; cc < C; ++cc) {
-      if (!tiled) { sets[i][2 + cc] = sets[i][0]; continue; }
-      const int* tile = po.kind == SA_MASK_SPADE ? po.candidates[cc] : po.tile;
-      if (!map_5d(&sets[i][2 + cc], src[i], pr, tile)) return SA_ERR_CUDA;
-    }
-  }
+  if (!block_maps(pr, po, c, q, k, v, 2, &maps)) return SA_ERR_CUDA;
   AttnParams ap{};
   ap.heads = reinterpret_cast<const HeadGeom*>(c.mw + c.M.off_head);
   ap.counts = reinterpret_cast<const int*>(c.mw + c.M.off_counts);
@@ -583,6 +605,58 @@ extern "C" int sparse_attn_forward(const sa_problem* problem, const sa_policy* p
   int e = sparse_attn_permute(problem, policy, q, k, v, mask_ws, scratch_ws, stream);
   if (e) return e;
   return sparse_attn_attend(problem, policy, q, k, v, mask_ws, scratch_ws, o, lse, stream);
+}
+
+extern "C" int sparse_attn_permute_fp8(const sa_problem* problem, const sa_policy* policy,
+                                       const void* q8, const void* k8, const void* v8,
+                                       const void* mask_ws, void* scratch_ws, void* stream) {
+  CallCtx c;
+  int e = prepare_call(problem, policy, q8, k8, v8, mask_ws, scratch_ws, stream, &c);
+  if (e) return e;
+  if (c.d % 32 != 0) return SA_ERR_UNSUPPORTED;
+  if (!needs_frame_major(*problem, *policy)) return SA_OK;
+  // The permutation moves whole rows in 16-byte pieces: a row of d E4M3
+  // codes is moved as a row of d / 2 bf16-sized elements.
+  PermuteParams pp{};
+  pp.heads = reinterpret_cast<const HeadGeom*>(c.mw + c.M.off_head);
+  const void* src[3] = {q8, k8, v8};
+  for (int i = 0; i < 3; ++i) {
+    pp.src[i] = static_cast<const __nv_bfloat16*>(src[i]);
+    pp.dst[i] = reinterpret_cast<__nv_bfloat16*>(c.sw + c.S.off_perm + i * c.S.perm_stride);
+  }
+  pp.T = problem->T; pp.H = problem->H; pp.W = problem->W; pp.d = c.d / 2; pp.n_pad = c.n_pad;
+  return cuda_status(launch_permute_fm(pp, c.BH, c.st));
+}
+
+extern "C" int sparse_attn_attend_fp8(const sa_problem* problem, const sa_policy* policy,
+                                      const void* q8, const void* k8, const void* v8,
+                                      const float* q_inv, const float* k_inv, const float* v_inv,
+                                      const void* mask_ws, void* scratch_ws, void* o, float* lse,
+                                      void* stream) {
+  CallCtx c;
+  int e = prepare_call(problem, policy, q8, k8, v8, mask_ws, scratch_ws, stream, &c);
+  if (e) return e;
+  if (!aligned(o, 16) || (lse && !aligned(lse, 4))) return SA_ERR_INVALID_ARG;
+  if (!q_inv || !k_inv || !v_inv || !aligned(q_inv, 4) || !aligned(k_inv, 4) ||
+      !aligned(v_inv, 4))
+    return SA_ERR_INVALID_ARG;
+  const sa_policy& po = *policy;
+  if (po.kind == SA_MASK_FG || c.d != 128 || po.block != 128) return SA_ERR_UNSUPPORTED;
+  if (!encode_fn()) return SA_ERR_CUDA;
+  AttnMaps maps;
+  if (!block_maps(*problem, po, c, q8, k8, v8, 1, &maps)) return SA_ERR_CUDA;
+  AttnParams ap{};
+  ap.heads = reinterpret_cast<const HeadGeom*>(c.mw + c.M.off_head);
+  ap.counts = reinterpret_cast<const int*>(c.mw + c.M.off_counts);
+  ap.cols = reinterpret_cast<const int*>(c.mw + c.M.off_cols);
+  ap.o = static_cast<__nv_bfloat16*>(o);
+  ap.lse = lse;
+  ap.status = reinterpret_cast<uint32_t*>(c.sw + c.S.off_status);
+  ap.BH = c.BH; ap.NB = c.M.NB; ap.T = problem->T; ap.H = problem->H; ap.W = problem->W;
+  ap.N = c.N;
+  ap.scale_log2 = 1.4426950408889634f / sqrtf((float)c.d);
+  ap.q_inv = q_inv; ap.k_inv = k_inv; ap.v_inv = v_inv;
+  return cuda_status(launch_attn_fwd_fp8(c.d, po.block, maps, ap, c.st));
 }
 
 extern "C" int sparse_attn_export_bytes(const sa_problem* problem, const sa_policy* policy,

@@ -30,13 +30,15 @@
 //               a 3-stage ring. 3D tile layouts are gathered by one 5-D box per
 //               64 columns (no separate permutation pass); identity and
 //               frame-major layouts by a 3-D box.
-//   warp 9      allocates tensor memory; lane 0 issues all MMAs: QK_0, QK_1,
+//   warp 9      allocates tensor memory and issues all MMAs, the whole warp
+//               converged and one elected lane per instruction: QK_0, QK_1,
 //               then PV_j, QK_{j+2} for every j. S_j goes to buffer j % 2,
 //               O_j % 2 accumulates P_j V_j.
 //   warps 10-11 (M x 1 slices only) copy the kept keys' K and V rows with
 //               cp.async; warp 8 then only builds the per-group masks.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "sa_attn.h"
@@ -64,10 +66,18 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows
 // polynomial of sa_ptx.cuh was measured slower on the 115,200-token workload
 // (12.3 / 11.3 against 9.0 ms per call): issue slots, not MUFU, bound it.
 
-template <int D, int BN>
+// FP8 operands (E4M3): every product runs as tcgen05.mma kind::f8f6f4 on
+// the same tiles at one byte per element; P is E4M3 of 2^4 P (the reference
+// moves when a row's maximum passes it by more than 2^4, so 2^4 P <= 2^8 stays
+// below 448 and probabilities down to 2^-13 keep a normal code).
+constexpr float kRescaleThresholdFp8 = 4.0f;
+constexpr float kPOffsetFp8 = 4.0f;
+
+// ES: bytes per element (2 bf16, 1 E4M3). A 128-byte swizzle row holds
+// 128 / ES columns of d.
+template <int D, int BN, int ES = 2>
 struct Smem {
-  static constexpr int kHalvesD = D / 64;                 // 64-column (128-byte) halves
-  static constexpr int kHalvesN = BN / 64;
+  static constexpr int kHalvesD = D * ES / 128;           // 128-byte column groups of d
   static constexpr int kQBytes = kHalvesD * 128 * 128;    // 128 rows, M of the MMA
   static constexpr int kKVHalf = BN * 128;                // one 64-column half of a K/V tile
   static constexpr int kKVBytes = kHalvesD * kKVHalf;
@@ -109,17 +119,18 @@ __device__ __forceinline__ void block_source(const HeadGeom& g, int blk, int BN,
   }
 }
 
-template <int D, int BN>
+template <int D, int BN, int ES = 2>
 __device__ __forceinline__ void load_block(const CUtensorMap* maps, const HeadGeom& g, int bh,
                                            int blk, uint8_t* dst, uint64_t* bar) {
+  constexpr int kBoxCols = 128 / ES;           // one 128-byte swizzle row per box row
   int map, c1, c2, c3;
   block_source(g, blk, BN, map, c1, c2, c3);
   const CUtensorMap* m = maps + map;
 #pragma unroll
-  for (int h = 0; h < D / 64; ++h) {
+  for (int h = 0; h < D / kBoxCols; ++h) {
     uint8_t* d = dst + h * (BN * 128);
-    if (map >= 2) tma_load_5d(d, m, bar, h * 64, c1, c2, c3, bh);
-    else tma_load_3d(d, m, bar, h * 64, c1, bh);
+    if (map >= 2) tma_load_5d(d, m, bar, h * kBoxCols, c1, c2, c3, bh);
+    else tma_load_3d(d, m, bar, h * kBoxCols, c1, bh);
   }
 }
 
@@ -192,10 +203,15 @@ __device__ __forceinline__ uint32_t site(uint32_t role, uint32_t bar, int j) {
 // contiguous queries (one or two groups); its keys are the union list of those
 // groups, copied 128 rows at a time by the copy warps (cp.async), and each
 // row masks keys outside its own group.
-template <int D, int BN, bool kGather>
-__global__ void __launch_bounds__(kGather ? kThreads + 64 : kThreads, 1)
+// kFp8 (block mode, D = BN = 128): Q, K, V are E4M3 codes, one scale per
+// (batch, head) tensor; both products run on kind::f8f6f4.
+template <int D, int BN, bool kGather, bool kFp8 = false>
+__global__ void __launch_bounds__(kGather || kFp8 ? kThreads + 64 : kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
-  using L = Smem<D, BN>;
+  static_assert(!kFp8 || (!kGather && D == 128 && BN == 128), "FP8: block mode, d = 128");
+  constexpr int ES = kFp8 ? 1 : 2;
+  constexpr bool kSplitRegs = kGather || kFp8;
+  using L = Smem<D, BN, ES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -275,7 +291,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   if (warp >= 8) {
   // Slice mode: warpgroup 2 gives registers back at one point that dominates
   // all of its role code; the softmax warpgroups take them in the other branch.
-  if constexpr (kGather) regs_dec<kRegsOther>();
+  if constexpr (kSplitRegs) regs_dec<kRegsOther>();
   if (warp == kProducerWarp && kGather) {
     // ------------------------------------------------------------ producer (gather)
     if (n_keys > 0) {
@@ -330,7 +346,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       const CUtensorMap* kmaps = maps.k;
       const CUtensorMap* vmaps = maps.v;
       mbar_arrive_expect_tx(&bars->q_full, L::kHalvesD * BN * 128);
-      load_block<D, BN>(qmaps, g, bh, qb, sQ, &bars->q_full);
+      load_block<D, BN, ES>(qmaps, g, bh, qb, sQ, &bars->q_full);
       int issued = 0;
       for (int j = 0; j < n_keys; ++j) {
         const int st = j % kStages, rnd = j / kStages;
@@ -338,9 +354,9 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         if (kb < 0 || kb >= g.nb) { atomicOr(status, SA_DEVFLAG_BOUNDS); *abort = 1; break; }
         if (!mbar_wait(&bars->kv_empty[st], (rnd & 1) ^ 1, abort, status, site(1, 1, j))) break;
         mbar_arrive_expect_tx(&bars->k_full[st], L::kKVBytes);
-        load_block<D, BN>(kmaps, g, bh, kb, sK + st * L::kKVBytes, &bars->k_full[st]);
+        load_block<D, BN, ES>(kmaps, g, bh, kb, sK + st * L::kKVBytes, &bars->k_full[st]);
         mbar_arrive_expect_tx(&bars->v_full[st], L::kKVBytes);
-        load_block<D, BN>(vmaps, g, bh, kb, sV + st * L::kKVBytes, &bars->v_full[st]);
+        load_block<D, BN, ES>(vmaps, g, bh, kb, sV + st * L::kKVBytes, &bars->v_full[st]);
         issued = j * 2 + 2;
       }
       if (*abort) {
@@ -354,72 +370,95 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_keys > 0) {
-      constexpr uint32_t idesc_qk = umma_idesc_bf16(128, BN, false, false);
-      constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, false, true);
+    // The whole warp runs this loop (every wait and branch warp-uniform);
+    // one elected lane issues each MMA and commit.
+    if (n_keys > 0) {
+      constexpr uint32_t idesc_qk = kFp8 ? umma_idesc_e4m3(128, BN, false, false)
+                                         : umma_idesc_bf16(128, BN, false, false);
+      constexpr uint32_t idesc_pv = kFp8 ? umma_idesc_e4m3(128, D, false, true)
+                                         : umma_idesc_bf16(128, D, false, true);
+      // Every MMA takes 32 bytes of its K dimension: 16 bf16 or 32 E4M3.
+      constexpr int kKQ = D * ES / 32;             // QK MMAs along d
+      constexpr int kKeysPerMma = 32 / ES;         // PV: keys per MMA
+      constexpr int kKP = BN / kKeysPerMma;        // PV MMAs per block
+      constexpr int kMmaPerChunk = 64 / kKeysPerMma;
+      auto mma_ss = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+        if constexpr (kFp8) umma_e4m3_ss_elect(d, a, b, id, acc);
+        else umma_bf16_ss_elect(d, a, b, id, acc);
+      };
+      auto mma_ts = [&](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
+        if constexpr (kFp8) umma_e4m3_ts_elect(d, a, b, id, acc);
+        else umma_bf16_ts_elect(d, a, b, id, acc);
+      };
       // Descriptors are formed once; each MMA only advances a base by a
       // compile-time offset, so the issuing thread spends its time issuing.
       const uint64_t dQ = umma_desc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dK0 = umma_desc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dV0 = umma_desc_sw128(smem_u32(sV), L::kKVHalf, 1024);
-      uint64_t da[D / 16];
+      uint64_t da[kKQ];
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk)        // 16 bf16 along K inside a 128-byte row
+      for (int kk = 0; kk < kKQ; ++kk)           // 32 bytes of K inside a 128-byte row
         da[kk] = umma_desc_advance(dQ, (kk / 4) * 16384 + (kk % 4) * 32);
       // QK_j into S buffer j & 1 (softmax group j & 1 reads it).
       auto issue_qk = [&](int j) -> bool {
         const int st = j % kStages;
-        if (!mbar_wait<false>(&bars->k_full[st], (j / kStages) & 1, abort, status, site(2, 6, j)))
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(&bars->k_full[st], (j / kStages) & 1, abort,
+                                                      status, site(2, 6, j))))
           return false;
         const uint64_t dk = umma_desc_advance(dK0, st * L::kKVBytes);
-        uint64_t db[D / 16];
+        uint64_t db[kKQ];
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
+        for (int kk = 0; kk < kKQ; ++kk)
           db[kk] = umma_desc_advance(dk, (kk / 4) * L::kKVHalf + (kk % 4) * 32);
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_bf16_ss(tS[j & 1], da[kk], db[kk], idesc_qk, kk > 0 ? 1u : 0u);
-        umma_commit(&bars->s_full[j & 1]);
+        for (int kk = 0; kk < kKQ; ++kk)
+          mma_ss(tS[j & 1], da[kk], db[kk], idesc_qk, kk > 0 ? 1u : 0u);
+        umma_commit_elect(&bars->s_full[j & 1]);
         return true;
       };
       // PV_j: O_{j&1} += P_j V_j, P_j read from S buffer j & 1.
       auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait<false>(&bars->p_full[i & 1], (i >> 1) & 1, abort, status, site(2, 3, i)))
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(&bars->p_full[i & 1], (i >> 1) & 1, abort,
+                                                      status, site(2, 3, i))))
           return false;
-        if (!mbar_wait<false>(&bars->v_full[i % kStages], (i / kStages) & 1, abort, status,
-                              site(2, 4, i)))
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(&bars->v_full[i % kStages], (i / kStages) & 1,
+                                                      abort, status, site(2, 4, i))))
           return false;
         const uint64_t dv = umma_desc_advance(dV0, (i % kStages) * L::kKVBytes);
-        uint64_t db[BN / 16];
+        uint64_t db[kKP];
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) db[kk] = umma_desc_advance(dv, kk * 16 * 128);
+        for (int kk = 0; kk < kKP; ++kk) db[kk] = umma_desc_advance(dv, kk * kKeysPerMma * 128);
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // A = P in tensor memory: 16 keys = 8 packed columns per step. The
-          // P of keys 64c..64c+63 sits at the start of their own S columns
-          // 64c.. (where their scores were). B = V (MN-major: d contiguous).
-          // O_{i&1} is first written by block i & 1.
-          umma_bf16_ts(tO + (i & 1) * D, tS[i & 1] + (kk / 4) * 64 + (kk % 4) * 8, db[kk],
-                       idesc_pv, (i > 1 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kKP; ++kk) {
+          // A = P in tensor memory: 8 packed columns per step (16 bf16 keys,
+          // two per column, or 32 E4M3 keys, four per column). The P of keys
+          // 64c..64c+63 sits at the start of their own S columns 64c.. (where
+          // their scores were). B = V (MN-major: d contiguous). O_{i&1} is
+          // first written by block i & 1.
+          mma_ts(tO + (i & 1) * D,
+                 tS[i & 1] + (kk / kMmaPerChunk) * 64 + (kk % kMmaPerChunk) * 8, db[kk],
+                 idesc_pv, (i > 1 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&bars->kv_empty[i % kStages]);
+        umma_commit_elect(&bars->kv_empty[i % kStages]);
         return true;
       };
       // Order: QK_0, QK_1, then PV_j, QK_{j+2} for every j. S buffer j & 1
       // is rewritten by QK_{j+2} only after PV_j (issued first) read P_j, and
       // the commit of S_{j+2} also covers PV_j: once a softmax group sees
       // S_{j+2}, its O accumulator holds every block before j + 2.
-      bool ok = mbar_wait<false>(&bars->q_full, 0, abort, status, site(2, 5, 0));
+      bool ok = __all_sync(0xffffffffu,
+                           mbar_wait<false>(&bars->q_full, 0, abort, status, site(2, 5, 0)));
       for (int j = 0; ok && j < 2 && j < n_keys; ++j) ok = issue_qk(j);
       for (int j = 0; ok && j < n_keys; ++j) {
         ok = issue_pv(j);
         if (ok && j + 2 < n_keys) ok = issue_qk(j + 2);
       }
       // Every MMA issued above must finish before tensor memory is freed.
-      umma_commit(&bars->drain);
+      umma_commit_elect(&bars->drain);
       mbar_drain(&bars->drain, 0);
+      __syncwarp();
     }
   } else if (kGather && warp >= kCopyWarp0) {
     // ------------------------------------------------------------ K/V row copies (gather)
@@ -483,7 +522,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     __syncwarp();
   }
   } else {
-    if constexpr (kGather) regs_inc<kRegsSoftmax>();
+    if constexpr (kSplitRegs) regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax + epilogue
     // Group grp = warp / 4 takes the key blocks j with j % 2 == grp; thread r
     // of a group owns row r of those blocks: its own running maximum m, sum
@@ -497,7 +536,8 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tSg = tS[grp] + lane_off;
     const uint32_t tOg = tO + grp * D + lane_off;
-    const float scale = p.scale_log2;
+    // FP8: scores of the codes times the two tensors' scales
+    const float scale = kFp8 ? p.scale_log2 / (p.q_inv[bh] * p.k_inv[bh]) : p.scale_log2;
     float m = -INFINITY;                              // reference maximum, log2 units
     float l = 0.f;                                    // sum of P over this group's blocks
     float s[64];
@@ -538,6 +578,75 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       // complete (S_j was committed after PV_{j-2}), and PV_j waits for this
       // group's arrival below, so touching O needs no wait.
       float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (kFp8) {
+        // FP8: the whole row in registers, one maximum and one rescale
+        // decision per block, so no stored E4M3 P is ever rescaled. O is
+        // rescaled before any of P_j is stored (PV_j waits for the arrival
+        // below; O holds this group's blocks up to j - 2, all complete).
+        float sr[BN];
+#pragma unroll
+        for (int c = 0; c < BN; c += 32) tmem_ld32(tSg + c, sr + c);
+        tmem_wait_ld();
+        if (pad) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c) sr[c] = ((pw[c / 32] >> (c % 32)) & 1u) ? sr[c] : -INFINITY;
+        }
+        float mx8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(sr[2 * e], sr[2 * e + 1]);
+#pragma unroll
+        for (int c = 16; c < BN; c += 16) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], sr[c + 2 * e], sr[c + 2 * e + 1]);
+        }
+        const float cm = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7])) * scale;
+        const bool move = cm > m + kRescaleThresholdFp8;
+        const bool had = move && m != -INFINITY;
+        const float alpha = had ? ex2_approx(m - cm) : 1.f;
+        if (move) { l *= alpha; m = cm; }
+        if (__any_sync(0xffffffffu, had)) {
+          float o[16];
+#pragma unroll
+          for (int c = 0; c < D; c += 16) {
+            tmem_ld16(tOg + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] *= alpha;
+            tmem_st16(tOg + c, o);
+          }
+        }
+        // 2^4 P, so that E4M3 keeps probabilities down to 2^-13 in its
+        // normal range; l sums the same values and the epilogue removes 2^4
+        const float neg = (m == -INFINITY ? 0.f : -m) + kPOffsetFp8;
+#pragma unroll
+        for (int ch = 0; ch < kChunks; ++ch) {
+          float* sc = sr + ch * 64;
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            float x0, x1;
+            fma2(sc[c], sc[c + 1], scale, scale, neg, neg, x0, x1);
+            sc[c] = ex2_approx(x0);
+            sc[c + 1] = ex2_approx(x1);
+          }
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            add2(rs4[0], rs4[1], sc[c], sc[c + 1]);
+            add2(rs4[2], rs4[3], sc[c + 2], sc[c + 3]);
+          }
+          // four E4M3 codes per column, key 4i + b in byte b of column i
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(sc[4 * i], sc[4 * i + 1]),
+                                                         __NV_SATFINITE, __NV_E4M3);
+            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(sc[4 * i + 2], sc[4 * i + 3]),
+                                                         __NV_SATFINITE, __NV_E4M3);
+            pk[i] = lo | (hi << 16);
+          }
+          tmem_st16(tSg + ch * 64, reinterpret_cast<const float*>(pk));
+        }
+      } else {
 #pragma unroll
       for (int ch = 0; ch < kChunks; ++ch) {
         tmem_ld32(tSg + ch * 64, s);
@@ -619,6 +728,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(pack_bf16x2(s[2 * c], s[2 * c + 1]));
         tmem_st32(tSg + ch * 64, s);
       }
+      }
       l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       if constexpr (kGather) {
         __syncwarp();
@@ -654,7 +764,9 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       const float a1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mm);
       const float l_tot = a0 * l0 + a1 * l1;
       const float inv_l = (n_keys > 0 && l_tot > 0.f) ? 1.f / l_tot : 0.f;
-      const float w0 = a0 * inv_l, w1 = a1 * inv_l;
+      // FP8: the V codes' scale folds into the output weights
+      const float osc = kFp8 ? 1.f / p.v_inv[bh] : 1.f;
+      const float w0 = a0 * inv_l * osc, w1 = a1 * inv_l * osc;
       const bool use0 = n_keys > 0 && w0 != 0.f, use1 = n_keys > 1 && w1 != 0.f;
       // this thread writes output columns [grp*D/2, grp*D/2 + D/2)
       constexpr int HD = D / 2;
@@ -684,7 +796,9 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       }
       if (tok >= 0 && grp == 0 && p.lse)
         p.lse[(size_t)bh * p.N + tok] =
-            (n_keys > 0 && l_tot > 0.f) ? (mm + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
+            (n_keys > 0 && l_tot > 0.f)
+                ? (mm + __log2f(l_tot) - (kFp8 ? kPOffsetFp8 : 0.f)) * 0.69314718055994530942f
+                : -INFINITY;
     }
   }
 
@@ -699,14 +813,14 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
 
 }  // namespace
 
-template <int D, int BN, bool kGather>
+template <int D, int BN, bool kGather, bool kFp8 = false>
 static cudaError_t launch_one(const AttnMaps& maps, const AttnParams& p, cudaStream_t stream) {
-  using L = Smem<D, BN>;
-  auto kern = attn_fwd_kernel<D, BN, kGather>;
+  using L = Smem<D, BN, kFp8 ? 1 : 2>;
+  auto kern = attn_fwd_kernel<D, BN, kGather, kFp8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   dim3 grid(p.NB, p.BH);
-  kern<<<grid, kGather ? kThreads + 64 : kThreads, L::kAlloc, stream>>>(maps, p);
+  kern<<<grid, kGather || kFp8 ? kThreads + 64 : kThreads, L::kAlloc, stream>>>(maps, p);
   return cudaGetLastError();
 }
 
@@ -715,6 +829,12 @@ cudaError_t launch_attn_fwd(int head_dim, int block, const AttnMaps& maps, const
   if (head_dim == 128 && block == 128) return launch_one<128, 128, false>(maps, p, stream);
   if (head_dim == 64 && block == 128) return launch_one<64, 128, false>(maps, p, stream);
   if (head_dim == 64 && block == 64) return launch_one<64, 64, false>(maps, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_fwd_fp8(int head_dim, int block, const AttnMaps& maps,
+                               const AttnParams& p, cudaStream_t stream) {
+  if (head_dim == 128 && block == 128) return launch_one<128, 128, false, true>(maps, p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -11,7 +11,8 @@ namespace sa {
 // Tensor maps per source tensor. Index 0: the original [BH][N][d] tensor as a
 // 3-D map (identity layout); 1: the frame-major permuted copy [BH][N_pad][d];
 // 2 + c: the original tensor as a 5-D (d, W, H, T, BH) map whose box is the
-// 3D tile of blocking candidate c. All use 64-column boxes, 128-byte swizzle.
+// 3D tile of blocking candidate c. All use 128-byte boxes along d (64 bf16 or
+// 128 E4M3 columns), 128-byte swizzle.
 constexpr int kMapsPerTensor = 6;
 struct AttnMaps {
   CUtensorMap q[kMapsPerTensor];
@@ -35,10 +36,17 @@ struct AttnParams {
   const uint32_t* fg_offsets;  // [BH][NB + 1]
   long long fg_cap;
   int fg_groups_per_tile;      // 2 for groups of 64, 1 for groups of 128
+  // FP8 mode: per-(batch, head) inverse scales of the E4M3 codes (value = code / inv)
+  const float* q_inv;
+  const float* k_inv;
+  const float* v_inv;
 };
 
 cudaError_t launch_attn_fwd(int head_dim, int block, const AttnMaps& maps, const AttnParams& p,
                             cudaStream_t stream);
+// Q, K, V as E4M3 codes (maps over uint8 tensors, 128-column boxes).
+cudaError_t launch_attn_fwd_fp8(int head_dim, int block, const AttnMaps& maps,
+                               const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_attn_gather(int head_dim, const AttnMaps& maps, const AttnParams& p,
                                cudaStream_t stream);
 
