@@ -393,17 +393,10 @@ __global__ void __launch_bounds__(kPoolAtomThreads, 2) pool_atoms_kernel(PoolPar
   const int N = p.T * p.H * p.W;
   const __nv_bfloat16* q = p.q + (size_t)bh * N * D;
   const __nv_bfloat16* k = p.k + (size_t)bh * N * D;
-  // An atom's tokens in atom order (t, h, w): their offsets from the atom's
-  // first token and their coordinates inside it, the same for every atom of
-  // every region. Lane slot tl takes tokens tl, tl + TPW, ... of each atom.
-  __shared__ int2 atom_tok[kMaxAtomTokens];      // {offset, it << 16 | ih << 8 | iw}
-  const int n_tok = p.At * p.Ah * p.Aw;          // <= one block, <= kMaxAtomTokens
-  for (int j = threadIdx.x; j < n_tok; j += kPoolAtomThreads) {
-    const int iw = j % p.Aw, ih = (j / p.Aw) % p.Ah, it = j / (p.Aw * p.Ah);
-    atom_tok[j] = make_int2((it * p.H + ih) * p.W + iw, (it << 16) | (ih << 8) | iw);
-  }
-  __syncthreads();
-  const int n_steps = (n_tok + TPW - 1) / TPW;
+  // This lane's first token of an atom is token tl (atom order t, h, w); its
+  // later ones follow TPW apart. The coordinates inside the atom are the same
+  // for every atom, found once here and then advanced without division.
+  const int iw0 = tl % p.Aw, ih0 = (tl / p.Aw) % p.Ah, it0 = tl / (p.Aw * p.Ah);
 
   constexpr int kWarps = kPoolAtomThreads / 32;
   // atom a = (at, ah, aw) of the region; this warp takes a = warp, warp + 8,
@@ -430,34 +423,30 @@ __global__ void __launch_bounds__(kPoolAtomThreads, 2) pool_atoms_kernel(PoolPar
 #pragma unroll
     for (int i = 0; i < 8; ++i) { qs[i] = summ_init<kSum>(); ks[i] = summ_init<kSum>(); us[i] = 0.f; }
     int n_valid = 0, n_unit = 0;
-    const int base = (ta * p.H + ha) * p.W + wa;
-    // only an atom that crosses the grid's far edge tests its tokens
-    const bool inside = ta + p.At <= p.T && ha + p.Ah <= p.H && wa + p.Aw <= p.W;
-    for (int s0 = 0; s0 < n_steps; s0 += UNROLL) {     // warp-uniform trip count
+    int iw = iw0, ih = ih0, it = it0;
+    // the warp's lanes stay in step: it < At for some lane until the last step
+    while (__any_sync(0xffffffffu, it < p.At)) {
       uint4 qv[UNROLL], kv[UNROLL];
-      bool ok[UNROLL];
+      int tok[UNROLL];
 #pragma unroll
       for (int u = 0; u < UNROLL; ++u) {
-        const int j = (s0 + u) * TPW + tl;
-        ok[u] = j < n_tok;
-        int tok = 0;
-        if (ok[u]) {
-          const int2 e = atom_tok[j];
-          tok = base + e.x;
-          if (!inside)
-            ok[u] = ta + (e.y >> 16) < p.T && ha + ((e.y >> 8) & 0xFF) < p.H &&
-                    wa + (e.y & 0xFF) < p.W;
+        const int t = ta + it, h = ha + ih, w = wa + iw;
+        tok[u] = (it < p.At && t < p.T && h < p.H && w < p.W) ? (t * p.H + h) * p.W + w : -1;
+        iw += TPW;
+        while (iw >= p.Aw) {
+          iw -= p.Aw;
+          if (++ih == p.Ah) { ih = 0; ++it; }
         }
         qv[u] = make_uint4(0, 0, 0, 0);
         kv[u] = make_uint4(0, 0, 0, 0);
-        if (ok[u]) {
-          qv[u] = __ldg(reinterpret_cast<const uint4*>(q + (size_t)tok * D) + dc);
-          kv[u] = __ldg(reinterpret_cast<const uint4*>(k + (size_t)tok * D) + dc);
+        if (tok[u] >= 0) {
+          qv[u] = __ldg(reinterpret_cast<const uint4*>(q + (size_t)tok[u] * D) + dc);
+          kv[u] = __ldg(reinterpret_cast<const uint4*>(k + (size_t)tok[u] * D) + dc);
         }
       }
 #pragma unroll
       for (int u = 0; u < UNROLL; ++u)
-        pool_token<D, kSum>(qv[u], kv[u], ok[u], qs, ks, us, n_valid, n_unit);
+        pool_token<D, kSum>(qv[u], kv[u], tok[u] >= 0, qs, ks, us, n_valid, n_unit);
     }
     pool_store_atom<D, kSum>(sums, cnt, a, lane, qs, ks, us, n_valid, n_unit);
   }

@@ -43,9 +43,6 @@ struct PoolParams {
 
 // Atoms per region the one-pass pooling kernel holds in shared memory.
 constexpr int kMaxPoolAtoms = 128;
-// Tokens of one atom: an atom divides every candidate tile, and a tile holds
-// one block (at most 128 tokens).
-constexpr int kMaxAtomTokens = 128;
 
 struct ChooseParams {
   const float* sics;
