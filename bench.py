@@ -44,6 +44,7 @@ def _args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-mask comparison")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 attention timing")
     ap.add_argument("--no-mask-roofline", action="store_true",
                     help="skip the per-kernel timing of the memory-bound mask kernels")
     ap.add_argument("--no-profile", action="store_true",
@@ -423,9 +424,37 @@ def mask_kernel_bytes(wl, n_frame_major_heads=0):
     return out
 
 
-def mask_kernel_bytes_entry(wl, times, hbm):
+def mask_kernel_bytes_entry(wl, times, hbm, extra=None):
     fm = len(wl.temporal_heads) if wl.kind == "spatiotemporal" else 0
-    return mask_roofline_entry(wl, times, mask_kernel_bytes(wl, fm), hbm)
+    nbytes = mask_kernel_bytes(wl, fm)
+    nbytes.update(extra or {})
+    return mask_roofline_entry(wl, times, nbytes, hbm)
+
+
+def fg_mask_extras(wl, sa):
+    """FG mask kernels beyond fg_qbar: fg_compact's bytes (the slice bitmask
+    read once, the union lists written once: 4 bytes per entry) and
+    fg_score's FLOPs (three bf16 terms of each (group, key) score per pass)."""
+    from sparse_attention_video_b200 import SA_EXPORT_FG_TILE_KEYS
+    G = (wl.N + wl.fg_group - 1) // wl.fg_group
+    words = (wl.N + 31) // 32
+    entries = float(sa.export(SA_EXPORT_FG_TILE_KEYS).astype(np.float64).sum())
+    compact = 4 * G * words * wl.heads + 4 * entries
+    score_pass = 3 * 2.0 * G * wl.N * wl.head_dim * wl.heads
+    return {"fg_compact": compact}, score_pass
+
+
+def fg_score_entry(wl, times, flops_per_pass, peak_tflops, passes=3):
+    n, ms = _kernel_ms(times, "fg_score")
+    if n == 0:
+        return {}
+    tf = passes * flops_per_pass / (ms * 1e-3) / 1e12
+    return {"fg_score": {"workload": wl.name, "ms_all_passes": ms, "launches": n,
+                         "bound": "tensor", "tflop_per_pass": flops_per_pass / 1e12,
+                         "achieved_tflops": tf, "peak_tflops": peak_tflops,
+                         "frac": tf / peak_tflops,
+                         "note": "three passes (two histogram levels, the bitmask); "
+                                 "launches for heads in the tie fallback return at once"}}
 
 
 def mask_roofline_entry(wl, times, nbytes, hbm):
@@ -631,7 +660,10 @@ def main():
     if not args.no_mask_roofline:
         times = kernel_times(lambda: (sa.build_mask(q, k, stream), sa.permute(q, k, v, stream)), dev)
         hbm_peak = _peaks()[2]
-        mask_roof.update(mask_kernel_bytes_entry(wl, times, hbm_peak))
+        extra, score_pass = fg_mask_extras(wl, sa) if wl.kind == "fg" else ({}, 0.0)
+        mask_roof.update(mask_kernel_bytes_entry(wl, times, hbm_peak, extra))
+        if wl.kind == "fg":
+            mask_roof.update(fg_score_entry(wl, times, score_pass, _peaks()[0]))
         if wl.name == WORKLOAD and not args.heads:
             for other in ("spade_wan21_14b_720p", "fg_slices_hunyuan_720p"):
                 owl = rank_workload(CONFIGS[other], rank)
@@ -644,7 +676,10 @@ def main():
                 osa.build_mask(oq, ok_, stream)
                 otimes = kernel_times(lambda: osa.build_mask(oq, ok_, stream), dev)
                 assert osa.status() == 0, f"device status word set in the {other} mask build"
-                mask_roof.update(mask_kernel_bytes_entry(owl, otimes, hbm_peak))
+                extra, score_pass = fg_mask_extras(owl, osa) if owl.kind == "fg" else ({}, 0.0)
+                mask_roof.update(mask_kernel_bytes_entry(owl, otimes, hbm_peak, extra))
+                if owl.kind == "fg":
+                    mask_roof.update(fg_score_entry(owl, otimes, score_pass, _peaks()[0]))
                 del oq, ok_, osa
                 torch.cuda.empty_cache()
         log("mask kernel rooflines done")
@@ -693,6 +728,45 @@ def main():
                  "dense_mask_attn_tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
                  "speedup_vs_dense_mask": dense_ms / attn_ms}
         del dsa, words
+
+    # ---- FP8 attention (Sparse VideoGen review: optional FP8 quantization):
+    # the same mask and kernel structure on E4M3 operands, kind::f8f6f4
+    fp8 = {}
+    if not args.no_fp8 and wl.head_dim == 128 and wl.block == 128 and wl.kind != "fg":
+        from sparse_attention_video_b200 import quantize_e4m3
+        o8 = torch.empty_like(q)
+        l8 = torch.empty_like(lse)
+        _, _, quantized = sa.forward_fp8(q, k, v, o8, l8, stream)
+        (q8, qi), (k8, ki), (v8, vi) = quantized
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        reps = 5
+        torch.cuda.synchronize(dev)
+        ev[0].record(stream)
+        for _ in range(reps):
+            for t in (q, k, v):
+                quantize_e4m3(t, stream)
+        ev[1].record(stream)
+        for _ in range(reps):
+            sa.permute_fp8(q8, k8, v8, stream)
+        ev[2].record(stream)
+        for _ in range(reps):
+            sa.attend_fp8(q8, k8, v8, qi, ki, vi, o8, l8, stream)
+        ev[3].record(stream)
+        torch.cuda.synchronize(dev)
+        assert sa.status() == 0, "device status word set in the FP8 attention"
+        qz_ms, pm_ms, at_ms = (ev[i].elapsed_time(ev[i + 1]) / reps for i in range(3))
+        at_ms = max_over_ranks([at_ms], dist, dev)[0]
+        pb = _peaks()[0]
+        fp8 = {"fp8_attention": {
+            "kernel": "attn_fwd_kernel<128,128,block,fp8> (tcgen05.mma kind::f8f6f4)",
+            "attend_ms": at_ms, "quantize_ms": qz_ms, "permute_ms": pm_ms,
+            "tflops": flops_call / (at_ms * 1e-3) / 1e12,
+            "peak": 2.0 * pb, "frac": flops_call / (at_ms * 1e-3) / 1e12 / (2.0 * pb),
+            "peak_note": "2 x the measured bf16 burst peak (the nominal fp8 : bf16 ratio), "
+                         "not a measured fp8 figure",
+            "speedup_vs_bf16_attention": attn_ms / at_ms}}
+        del o8, l8, quantized, q8, k8, v8, qi, ki, vi
+        log("fp8 attention timed")
 
     # ---- the head profiler (Sparse VideoGen review, key machinery) on 1 % of
     # each head's query rows; reported beside the step, not part of it
@@ -861,6 +935,7 @@ def main():
         "gpu_launches": LAUNCHES_PER_STEP[wl.kind] * args.steps,
         "clocks": clk,
         **dense,
+        **fp8,
         **prof,
     }
     print(json.dumps(line), flush=True)

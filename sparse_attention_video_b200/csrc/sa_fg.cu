@@ -216,7 +216,10 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
           mbar_drain(&bars->k_full[j % kKStages], (j / kKStages) & 1);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    // The whole warp runs the issue loop (waits and branches warp-uniform);
+    // one elected lane issues each MMA and commit, so the descriptors stay
+    // warp-uniform values and the issue keeps ahead of the tensor pipe.
+    {
       constexpr uint32_t idesc = umma_idesc_bf16(128, 128, false, false);
       // Descriptors formed once: the q_avg terms' are fixed, a K stage's
       // differ from stage 0's by a constant; each MMA adds a compile-time
@@ -229,13 +232,16 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         for (int kk = 0; kk < D / 16; ++kk)
           dq[t][kk] = umma_desc_sw128(smem_u32(sQ) + t * L::kTerm + (kk / 4) * 16384 + (kk % 4) * 32,
                                       16, 1024);
-      bool ok = mbar_wait<false>(&bars->q_full, 0, abort, status, 0x05050000u);
+      bool ok = __all_sync(0xffffffffu,
+                           mbar_wait<false>(&bars->q_full, 0, abort, status, 0x05050000u));
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int st = j % kKStages, ab = j % kAcc;
-        if (!mbar_wait<false>(&bars->k_full[st], (j / kKStages) & 1, abort, status, 0x05060000u | j))
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(&bars->k_full[st], (j / kKStages) & 1, abort,
+                                                      status, 0x05060000u | j)))
           break;
-        if (j >= kAcc && !mbar_wait<false>(&bars->acc_free[ab], ((j / kAcc) - 1) & 1, abort, status,
-                                        0x05070000u | j))
+        if (j >= kAcc &&
+            !__all_sync(0xffffffffu, mbar_wait<false>(&bars->acc_free[ab], ((j / kAcc) - 1) & 1,
+                                                      abort, status, 0x05070000u | j)))
           break;
         const uint64_t dk = umma_desc_advance(dK0, st * L::kKTile);
         uint64_t da[D / 16];
@@ -248,13 +254,14 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
           if (t >= n_terms) break;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            umma_bf16_ss(d_tmem, da[kk], dq[t][kk], idesc, (t > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16_ss_elect(d_tmem, da[kk], dq[t][kk], idesc, (t > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&bars->acc_full[ab]);
-        umma_commit(&bars->k_empty[st]);
+        umma_commit_elect(&bars->acc_full[ab]);
+        umma_commit_elect(&bars->k_empty[st]);
       }
-      umma_commit(&bars->drain);
+      umma_commit_elect(&bars->drain);
       mbar_drain(&bars->drain, 0);
+      __syncwarp();
     }
   } else if (warp >= 4) {
     // ---------------------------------------------------------- epilogue
