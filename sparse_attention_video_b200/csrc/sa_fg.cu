@@ -517,15 +517,11 @@ __global__ void __launch_bounds__(1024) fg_offsets_kernel(FgListParams p) {
 }
 
 // One warp per (tile, head) lists the tile's union in ascending key order,
-// 1,024 keys (32 bitmask words) at a time, through a per-warp staging buffer
-// in shared memory: each word's keys go to its prefix position there, then
-// the warp copies the chunk's entries out with consecutive lanes on
-// consecutive list slots (coalesced stores). Kept keys cluster, so a chunk
-// mixes sparse and dense words: lane l expands word l itself when it has at
-// most kDenseBits set bits, and the whole warp expands each denser word (one
-// bit per lane), so no lane loops over a full word while the others wait.
+// 1,024 keys (32 bitmask words) at a time: lane l expands the set bits of
+// word l into a per-warp staging buffer in shared memory at its prefix
+// position, then the warp copies the chunk's entries out with consecutive
+// lanes on consecutive list slots (coalesced stores).
 constexpr int kListWarps = 8;
-constexpr uint32_t kDenseBits = 12;
 
 __global__ void __launch_bounds__(32 * kListWarps) fg_compact_kernel(FgListParams p) {
   __shared__ uint32_t stage[kListWarps][1024];
@@ -551,32 +547,13 @@ __global__ void __launch_bounds__(32 * kListWarps) fg_compact_kernel(FgListParam
       const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += t;
     }
-    const uint32_t excl = incl - c;
-    // sparse words: each lane expands its own, at most kDenseBits iterations
-    if (c <= kDenseBits) {
-      uint32_t* dst = sb + excl;
-      const uint32_t kbase = 32u * (uint32_t)w;
-      while (u) {
-        const uint32_t low = u & (0u - u);             // lowest set bit
-        u ^= low;
-        *dst++ = (kbase + (uint32_t)__popc(low - 1u)) | ((a & low) ? (1u << 30) : 0u) |
-                 ((b & low) ? (1u << 31) : 0u);
-      }
-    }
-    // dense words: the whole warp on one word at a time, lane l on bit l,
-    // its slot the word's start plus the set bits below it
-    uint32_t dense = __ballot_sync(0xffffffffu, c > kDenseBits);
-    while (dense) {
-      const int src = __ffs(dense) - 1;
-      dense &= dense - 1u;
-      const uint32_t uw = __shfl_sync(0xffffffffu, u, src);
-      const uint32_t aw = __shfl_sync(0xffffffffu, a, src);
-      const uint32_t bw = __shfl_sync(0xffffffffu, b, src);
-      const uint32_t ew = __shfl_sync(0xffffffffu, excl, src);
-      if ((uw >> lane) & 1u)
-        sb[ew + __popc(uw & ((1u << lane) - 1u))] =
-            (32u * (uint32_t)(w0 + src) + (uint32_t)lane) | (((aw >> lane) & 1u) << 30) |
-            (((bw >> lane) & 1u) << 31);
+    uint32_t* dst = sb + (incl - c);
+    const uint32_t kbase = 32u * (uint32_t)w;
+    while (u) {
+      const uint32_t low = u & (0u - u);               // lowest set bit
+      u ^= low;
+      *dst++ = (kbase + (uint32_t)__popc(low - 1u)) | ((a & low) ? (1u << 30) : 0u) |
+               ((b & low) ? (1u << 31) : 0u);
     }
     const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
     __syncwarp();
