@@ -62,9 +62,9 @@ constexpr int kMmaWarp = 9;
 constexpr int kCopyWarp0 = 10;             // gather mode: warps 10-11 copy K/V rows
 constexpr int kStages = 3;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows > 2^8
-// Every exp2 runs on MUFU. Moving one in four (or eight) to the FMA-pipe
-// polynomial of sa_ptx.cuh was measured slower on the 115,200-token workload
-// (12.3 / 11.3 against 9.0 ms per call): issue slots, not MUFU, bound it.
+// Every exp2 runs on MUFU. Moving a quarter to three eighths of them to an
+// FMA-pipe polynomial (Cody-Waite split plus a cubic) was measured slower on
+// every workload, with the single-lane and the warp-uniform MMA issuer alike.
 
 // FP8 operands (E4M3): every product runs as tcgen05.mma kind::f8f6f4 on
 // the same tiles at one byte per element; P is E4M3 of 2^4 P (the reference

@@ -9,7 +9,6 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
-#include "sa_exp2_poly.h"
 #include "sa_internal.h"
 
 namespace sa {
@@ -374,21 +373,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x on the FMA pipe, for x <= 127 (x may be -inf). Cody-Waite split
-// x = n + f, n = round(x) taken from the low mantissa bits of x + 1.5*2^23,
-// f in [-1/2, 1/2]; 2^f by the cubic of sa_exp2_poly.h (max relative error
-// about 7.5e-5); 2^n added to the exponent field. x is clamped at -125 so the
-// result stays a normal float (2^-125 instead of 0 for x = -inf).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float magic = 12582912.f;
-  const float t = x + magic;
-  const float f = x - (t - magic);
-  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-  const int n = __float_as_int(t) - __float_as_int(magic);
-  return __int_as_float(__float_as_int(p) + (n << 23));
 }
 
 // Two fp32 lanes per instruction (packed f32x2 FMA / add, sm_100): halves
