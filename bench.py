@@ -787,13 +787,24 @@ def main():
         p1.record(stream)
         torch.cuda.synchronize(dev)
         prof_ms = p0.elapsed_time(p1) / 5
-        # the full pass alone: every sampled row against every key
+        # the full pass alone: every sampled row against every key, on the
+        # attention kernel (its device time from the activity profiler)
         full_flops = 4.0 * wl.head_dim * rows.numel() * wl.N
+        kt = kernel_times(lambda: profile_heads(q, k, v, rows, wl.T, wl.H, wl.W, block=wl.block,
+                                                sink_tokens=wl.sink_tokens, stream=stream), dev)
+        n_a, attn_full_ms = _kernel_ms(kt, "attn_fwd")
+        n_p, masked_ms = _kernel_ms(kt, "profile_kernel")
         prof = {"profile_heads": {
             "ms": prof_ms, "rows_per_head": int(rows.shape[1]),
-            "full_pass_tflops": full_flops / (prof_ms * 1e-3) / 1e12,
+            "full_pass_tflops_over_call": full_flops / (prof_ms * 1e-3) / 1e12,
+            "full_pass_kernel_ms": attn_full_ms if n_a else None,
+            "full_pass_kernel_tflops": (full_flops / (attn_full_ms * 1e-3) / 1e12) if n_a else None,
+            "full_pass_kernel_frac": (full_flops / (attn_full_ms * 1e-3) / 1e12 / _peaks()[0])
+                                     if n_a else None,
+            "masked_passes_ms": masked_ms if n_p else None,
             "temporal_heads_found": int(is_t.sum().item()),
-            "kernel": "profile_kernel (mma.sync m16n8k16; all three passes in the time)"}}
+            "kernel": "full pass: attn_fwd_kernel (tcgen05, dense key list over gathered rows); "
+                      "masked passes: profile_kernel (mma.sync m16n8k16)"}}
         log("head profiler timed")
     if not args.no_profile and wl.kind == "sta":
         # the STA per-head window search (Sliding Tile Attention review, key
@@ -815,11 +826,19 @@ def main():
         torch.cuda.synchronize(dev)
         ms = p0.elapsed_time(p1) / 5
         full_flops = 4.0 * wl.head_dim * rows.numel() * wl.N
+        kt = kernel_times(lambda: sta_window_search(q, k, v, rows, wl.T, wl.H, wl.W, wl.tile, cands,
+                                                    block=wl.block, stream=stream), dev)
+        n_a, attn_full_ms = _kernel_ms(kt, "attn_fwd")
+        n_p, masked_ms = _kernel_ms(kt, "profile_kernel")
         prof = {"window_search": {
             "ms": ms, "rows_per_head": int(rows.shape[1]), "candidates": cands,
-            "full_pass_tflops": full_flops / (ms * 1e-3) / 1e12,
+            "full_pass_tflops_over_call": full_flops / (ms * 1e-3) / 1e12,
+            "full_pass_kernel_ms": attn_full_ms if n_a else None,
+            "full_pass_kernel_tflops": (full_flops / (attn_full_ms * 1e-3) / 1e12) if n_a else None,
+            "masked_passes_ms": masked_ms if n_p else None,
             "choices": torch.bincount(choice.long().cpu(), minlength=len(cands)).tolist(),
-            "kernel": "profile_kernel, tile-window mode (mma.sync m16n8k16)"}}
+            "kernel": "full pass: attn_fwd_kernel (tcgen05); window passes: profile_kernel, "
+                      "tile-window mode (mma.sync m16n8k16)"}}
         log("window search timed")
 
     if wl.kind == "fg" and not args.no_profile and dense:

@@ -336,14 +336,27 @@ SA_API int sparse_attn_status(void* scratch_ws, void* stream, int clear);
  *   mse          device float [batch*heads][2]: those sums over the rows,
  *                divided by n_rows * head_dim (fixed summation order).
  *   is_temporal  device int8 [batch*heads]: the decision.
- *   scratch_ws   optional (may be null): its status word receives the bounds flag.
+ *   scratch_ws   device workspace of at least sparse_attn_profile_workspace_size
+ *                bytes for n_rows, 256-byte aligned (SA_ERR_WORKSPACE if null
+ *                or misaligned); its status word (read by sparse_attn_status)
+ *                receives the bounds and timeout flags.
+ * The full pass runs on the block-sparse attention kernel (tcgen05): the
+ * sampled rows are gathered into 128-row query tiles that visit every key
+ * block, with O kept in fp32; the masked passes measure against it.
  * Q/K/V as for the forward pass. Asynchronous on ``stream``; the caller owns
- * every buffer. Returns SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED or
- * SA_ERR_CUDA. */
+ * every buffer. Returns SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED,
+ * SA_ERR_WORKSPACE or SA_ERR_CUDA. */
 SA_API int sparse_attn_profile_heads(const sa_problem* problem, const sa_policy* policy,
                                      const void* q, const void* k, const void* v,
                                      const int32_t* rows, int n_rows, float* row_err, float* mse,
                                      int8_t* is_temporal, void* scratch_ws, void* stream);
+
+/* Scratch bytes the sampled-row calls (sparse_attn_profile_heads,
+ * sparse_attn_sta_window_search) need for ``n_rows`` rows per head: the
+ * status words, the sampled query rows gathered into 128-row tiles and the
+ * full pass's fp32 output. */
+SA_API int sparse_attn_profile_workspace_size(const sa_problem* problem, int n_rows,
+                                              size_t* bytes);
 
 /* STA per-head window search (Sliding Tile Attention review, key machinery;
  * Algorithm 1: each head's window is the mask that minimizes the MSE to full
@@ -355,7 +368,7 @@ SA_API int sparse_attn_profile_heads(const sa_problem* problem, const sa_policy*
  * candidates encode the trade-off; the search returns the lowest error, ties
  * to the earlier candidate. The result feeds ``sa_policy.head_windows``.
  *
- *   rows, scratch_ws  as for sparse_attn_profile_heads.
+ *   rows, scratch_ws  as for sparse_attn_profile_heads (the same workspace size).
  *   row_err     device float [batch*heads][n_rows][n_candidates]: per row and
  *               candidate, the sum over head_dim of (O_window - O_full)^2.
  *   mse         device float [batch*heads][n_candidates]: those sums over

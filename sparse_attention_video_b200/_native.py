@@ -29,6 +29,7 @@ EXPORTED = ("sparse_attn_workspace_size", "sparse_attn_build_mask", "sparse_attn
             "sparse_attn_build_mask_static", "sparse_attn_status_static",
             "sparse_attn_selftest_wait_timeout",
             "sparse_attn_profile_heads", "sparse_attn_sta_window_search",
+            "sparse_attn_profile_workspace_size",
             "sparse_attn_build_mask_fg_cached", "sparse_attn_quantize_e4m3",
             "sparse_attn_permute_fp8", "sparse_attn_attend_fp8",
             "sparse_attn_strerror")
@@ -94,6 +95,7 @@ def lib():
         L.sparse_attn_selftest_wait_timeout.argtypes = [vp, vp]
         L.sparse_attn_profile_heads.argtypes = [P, PP, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp,
                                                 vp, vp]
+        L.sparse_attn_profile_workspace_size.argtypes = [P, ctypes.c_int, ctypes.POINTER(sz)]
         L.sparse_attn_sta_window_search.argtypes = [P, PP, vp, vp, vp, vp, ctypes.c_int, vp,
                                                     ctypes.c_int, vp, vp, vp, vp, vp]
         L.sparse_attn_build_mask_fg_cached.argtypes = [P, PP, vp, vp, vp, ctypes.c_float, vp, vp,
@@ -149,6 +151,14 @@ def attend(problem, policy, q, k, v, mask_ws, scratch_ws, o, lse, stream=0):
     _check(lib().sparse_attn_attend(ctypes.byref(problem), ctypes.byref(policy), q, k, v,
                                     mask_ws, scratch_ws, o, lse, stream),
            "sparse_attn_attend")
+
+
+def profile_workspace_size(problem, n_rows):
+    n = ctypes.c_size_t()
+    _check(lib().sparse_attn_profile_workspace_size(ctypes.byref(problem), int(n_rows),
+                                                    ctypes.byref(n)),
+           "sparse_attn_profile_workspace_size")
+    return n.value
 
 
 def profile_heads(problem, policy, q, k, v, rows, n_rows, row_err, mse, is_temporal,

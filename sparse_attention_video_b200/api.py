@@ -256,6 +256,18 @@ class SparseAttention:
         return N.status(self.scratch_ws.data_ptr(), _stream_ptr(stream), clear)
 
 
+def _sampled_scratch(problem, n_rows, scratch_ws, device):
+    """The scratch workspace of a sampled-row call: the caller's, checked for
+    size, or a new one of sparse_attn_profile_workspace_size bytes."""
+    need = N.profile_workspace_size(problem, n_rows)
+    if scratch_ws is None:
+        return torch.empty(need, dtype=torch.uint8, device=device)
+    if scratch_ws.numel() * scratch_ws.element_size() < need:
+        raise ValueError(f"scratch_ws holds {scratch_ws.numel() * scratch_ws.element_size()} "
+                         f"bytes, the call needs {need}")
+    return scratch_ws
+
+
 def _sampled_problem(q, k, v, rows, T, H, W, scratch_ws):
     """Problem of a sampled-row call, after checking every tensor it is given."""
     if not isinstance(q, torch.Tensor) or q.dim() != 4:
@@ -280,7 +292,9 @@ def profile_heads(q, k, v, rows, T, H, W, block=128, sink_tokens=0, frame_radius
     [batch*heads, n_rows] sampled query tokens. Returns (is_temporal int8
     [batch*heads], mse float32 [batch*heads, 2], row_err float32
     [batch*heads, n_rows, 2]) as CUDA tensors; the work is queued on
-    ``stream`` and nothing is synchronised.
+    ``stream`` and nothing is synchronised. ``scratch_ws`` (optional here)
+    is the call's workspace; one of sparse_attn_profile_workspace_size bytes
+    is made when it is None.
     """
     problem = _sampled_problem(q, k, v, rows, T, H, W, scratch_ws)
     B, Hh = problem.batch, problem.heads
@@ -291,9 +305,10 @@ def profile_heads(q, k, v, rows, T, H, W, block=128, sink_tokens=0, frame_radius
     row_err = torch.empty((B * Hh, n_rows, 2), dtype=torch.float32, device=dev)
     mse = torch.empty((B * Hh, 2), dtype=torch.float32, device=dev)
     is_temporal = torch.empty(B * Hh, dtype=torch.int8, device=dev)
+    scratch_ws = _sampled_scratch(problem, n_rows, scratch_ws, dev)
     N.profile_heads(problem, policy, q.data_ptr(), k.data_ptr(), v.data_ptr(), rows.data_ptr(),
                     n_rows, row_err.data_ptr(), mse.data_ptr(), is_temporal.data_ptr(),
-                    scratch_ws.data_ptr() if scratch_ws is not None else None, _stream_ptr(stream))
+                    scratch_ws.data_ptr(), _stream_ptr(stream))
     return is_temporal, mse, row_err
 
 
@@ -317,10 +332,10 @@ def sta_window_search(q, k, v, rows, T, H, W, tile, candidates, block=128, strea
     row_err = torch.empty((B * Hh, n_rows, nc), dtype=torch.float32, device=dev)
     mse = torch.empty((B * Hh, nc), dtype=torch.float32, device=dev)
     choice = torch.empty(B * Hh, dtype=torch.int8, device=dev)
+    scratch_ws = _sampled_scratch(problem, n_rows, scratch_ws, dev)
     N.sta_window_search(problem, policy, q.data_ptr(), k.data_ptr(), v.data_ptr(), rows.data_ptr(),
                         n_rows, cand, nc, row_err.data_ptr(), mse.data_ptr(), choice.data_ptr(),
-                        scratch_ws.data_ptr() if scratch_ws is not None else None,
-                        _stream_ptr(stream))
+                        scratch_ws.data_ptr(), _stream_ptr(stream))
     return choice, mse, row_err
 
 

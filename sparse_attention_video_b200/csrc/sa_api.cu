@@ -702,6 +702,82 @@ extern "C" int sparse_attn_mask_export(const sa_problem* problem, const sa_polic
   return cuda_status(cudaStreamSynchronize(st));
 }
 
+// ------------------------------------------------------------------ sampled rows
+namespace {
+
+// Scratch of the sampled-row calls: status words, the gathered query rows
+// [BH][n_pad][d] bf16 (n_pad = n_rows rounded up to 128), and the full pass's
+// fp32 O [BH][n_rows][d].
+struct SampledLayout {
+  size_t off_status = 0, off_qg = 0, off_ofull = 0, total = 0;
+  int n_pad = 0;
+};
+
+SampledLayout sampled_layout(const sa_problem& pr, int n_rows) {
+  SampledLayout L;
+  const size_t BH = (size_t)pr.batch * pr.heads, d = (size_t)pr.head_dim;
+  L.n_pad = ceil_div(n_rows, 128) * 128;
+  L.off_status = 0;
+  L.off_qg = 256;
+  L.off_ofull = align_up(L.off_qg + BH * L.n_pad * d * 2, 256);
+  L.total = align_up(L.off_ofull + BH * (size_t)n_rows * d * 4, 256);
+  return L;
+}
+
+// The full pass of both sampled-row calls on the block-sparse attention
+// kernel: gather the sampled rows into 128-row query tiles, then attend every
+// tile to every key block of the identity layout, O in fp32.
+int sampled_full_pass(const sa_problem& pr, const void* q, const void* k, const void* v,
+                      const int32_t* rows, int n_rows, uint8_t* sw, cudaStream_t st,
+                      const float** o_full) {
+  if (!encode_fn()) return SA_ERR_CUDA;
+  const SampledLayout L = sampled_layout(pr, n_rows);
+  const int BH = pr.batch * pr.heads, d = pr.head_dim;
+  const int N = (int)n_tokens(pr);
+  uint32_t* status = reinterpret_cast<uint32_t*>(sw + L.off_status);
+  __nv_bfloat16* qg = reinterpret_cast<__nv_bfloat16*>(sw + L.off_qg);
+  float* of = reinterpret_cast<float*>(sw + L.off_ofull);
+  if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return SA_ERR_CUDA;
+  int e = cuda_status(launch_gather_rows(static_cast<const __nv_bfloat16*>(q), rows, BH, N, d,
+                                         n_rows, L.n_pad, qg, status, st));
+  if (e) return e;
+  AttnMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  if (!map_3d(&maps.q[0], qg, BH, L.n_pad, d, 128) || !map_3d(&maps.k[0], k, BH, N, d, 128) ||
+      !map_3d(&maps.v[0], v, BH, N, d, 128))
+    return SA_ERR_CUDA;
+  AttnParams ap{};
+  ap.heads = nullptr;
+  HeadGeom g{};
+  g.layout = SA_LAYOUT_IDENTITY;
+  g.bt = 1; g.bh = 1; g.bw = 128;
+  g.nb = ceil_div(N, 128);
+  g.nt = 1; g.nh = 1; g.nw = g.nb;
+  ap.geo0 = g;
+  ap.dense = 1;
+  ap.q_tiles = L.n_pad / 128;
+  ap.q_rows = n_rows;
+  ap.o_f32 = of;
+  ap.status = status;
+  ap.BH = BH; ap.NB = ap.q_tiles; ap.T = pr.T; ap.H = pr.H; ap.W = pr.W; ap.N = N;
+  ap.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
+  e = cuda_status(launch_attn_fwd(d, 128, maps, ap, st));
+  if (e) return e;
+  *o_full = of;
+  return SA_OK;
+}
+
+}  // namespace
+
+extern "C" int sparse_attn_profile_workspace_size(const sa_problem* problem, int n_rows,
+                                                  size_t* bytes) {
+  int e = check_problem(problem);
+  if (e) return e;
+  if (!bytes || n_rows < 1 || n_rows > n_tokens(*problem)) return SA_ERR_INVALID_ARG;
+  *bytes = sampled_layout(*problem, n_rows).total;
+  return SA_OK;
+}
+
 extern "C" int sparse_attn_profile_heads(const sa_problem* problem, const sa_policy* policy,
                                          const void* q, const void* k, const void* v,
                                          const int32_t* rows, int n_rows, float* row_err,
@@ -719,8 +795,13 @@ extern "C" int sparse_attn_profile_heads(const sa_problem* problem, const sa_pol
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return SA_ERR_INVALID_ARG;
   if (!aligned(rows, 4) || !aligned(row_err, 4) || !aligned(mse, 4) || !is_temporal)
     return SA_ERR_INVALID_ARG;
-  if (scratch_ws && !aligned(scratch_ws, 256)) return SA_ERR_WORKSPACE;
+  if (!scratch_ws || !aligned(scratch_ws, 256)) return SA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float* o_full = nullptr;
+  e = sampled_full_pass(pr, q, k, v, rows, n_rows, static_cast<uint8_t*>(scratch_ws), st, &o_full);
+  if (e) return e;
   ProfileParams pp{};
+  pp.o_full = o_full;
   pp.q = static_cast<const __nv_bfloat16*>(q);
   pp.k = static_cast<const __nv_bfloat16*>(k);
   pp.v = static_cast<const __nv_bfloat16*>(v);
@@ -732,9 +813,8 @@ extern "C" int sparse_attn_profile_heads(const sa_problem* problem, const sa_pol
   pp.n_pat = 2;
   pp.tile[0] = pp.tile[1] = 1;
   pp.tile[2] = po.block;
-  pp.status = scratch_ws ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(scratch_ws) +
-                                                       ScratchLayout{}.off_status)
-                         : nullptr;
+  pp.status = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(scratch_ws) +
+                                         sampled_layout(pr, n_rows).off_status);
   pp.BH = pr.batch * pr.heads;
   pp.N = (int)N; pp.T = pr.T; pp.H = pr.H; pp.W = pr.W; pp.d = pr.head_dim;
   pp.n_rows = n_rows;
@@ -742,7 +822,7 @@ extern "C" int sparse_attn_profile_heads(const sa_problem* problem, const sa_pol
   pp.sink_blocks = ceil_div(po.sink_tokens, po.block);
   pp.frame_radius = po.frame_radius;
   pp.scale_log2 = 1.4426950408889634f / sqrtf((float)pr.head_dim);
-  return cuda_status(launch_profile(pp, reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_profile(pp, st));
 }
 
 extern "C" int sparse_attn_sta_window_search(const sa_problem* problem, const sa_policy* policy,
@@ -766,8 +846,13 @@ extern "C" int sparse_attn_sta_window_search(const sa_problem* problem, const sa
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return SA_ERR_INVALID_ARG;
   if (!aligned(rows, 4) || !aligned(row_err, 4) || !aligned(mse, 4) || !choice)
     return SA_ERR_INVALID_ARG;
-  if (scratch_ws && !aligned(scratch_ws, 256)) return SA_ERR_WORKSPACE;
+  if (!scratch_ws || !aligned(scratch_ws, 256)) return SA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float* o_full = nullptr;
+  e = sampled_full_pass(pr, q, k, v, rows, n_rows, static_cast<uint8_t*>(scratch_ws), st, &o_full);
+  if (e) return e;
   ProfileParams pp{};
+  pp.o_full = o_full;
   pp.q = static_cast<const __nv_bfloat16*>(q);
   pp.k = static_cast<const __nv_bfloat16*>(k);
   pp.v = static_cast<const __nv_bfloat16*>(v);
@@ -775,9 +860,8 @@ extern "C" int sparse_attn_sta_window_search(const sa_problem* problem, const sa
   pp.row_err = row_err;
   pp.mse = mse;
   pp.choice = choice;
-  pp.status = scratch_ws ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(scratch_ws) +
-                                                       ScratchLayout{}.off_status)
-                         : nullptr;
+  pp.status = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(scratch_ws) +
+                                         sampled_layout(pr, n_rows).off_status);
   pp.BH = pr.batch * pr.heads;
   pp.N = (int)N; pp.T = pr.T; pp.H = pr.H; pp.W = pr.W; pp.d = pr.head_dim;
   pp.n_rows = n_rows;
@@ -788,7 +872,7 @@ extern "C" int sparse_attn_sta_window_search(const sa_problem* problem, const sa
   for (int c = 0; c < n_candidates; ++c)
     for (int i = 0; i < 3; ++i) pp.win[c][i] = candidates[3 * c + i];
   pp.scale_log2 = 1.4426950408889634f / sqrtf((float)pr.head_dim);
-  return cuda_status(launch_profile(pp, reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_profile(pp, st));
 }
 
 extern "C" int sparse_attn_quantize_e4m3(const void* x, long long n_elems, int n_tensors,

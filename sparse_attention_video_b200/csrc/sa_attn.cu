@@ -237,12 +237,17 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     list = p.fg_list + (size_t)bh * p.fg_cap + begin;
     n_keys = (int)((list_count + BN - 1) / BN);
   } else {
-    g = p.heads[bh];
+    g = p.heads ? p.heads[bh] : p.geo0;
     // uniform across the CTA, before any allocation
-    if (qb >= g.nb || grid_aborted(p.status)) return;
-    const size_t row_base = ((size_t)bh * p.NB + qb);
-    n_keys = p.counts[row_base];
-    cols = p.cols + row_base * p.NB;
+    const int n_q = p.q_tiles > 0 ? p.q_tiles : g.nb;
+    if (qb >= n_q || grid_aborted(p.status)) return;
+    if (p.dense) {
+      n_keys = g.nb;
+    } else {
+      const size_t row_base = ((size_t)bh * p.NB + qb);
+      n_keys = p.counts[row_base];
+      cols = p.cols + row_base * p.NB;
+    }
   }
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -346,11 +351,14 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       const CUtensorMap* kmaps = maps.k;
       const CUtensorMap* vmaps = maps.v;
       mbar_arrive_expect_tx(&bars->q_full, L::kHalvesD * BN * 128);
-      load_block<D, BN, ES>(qmaps, g, bh, qb, sQ, &bars->q_full);
+      // gathered query rows (sampled-row mode) are a plain row tensor
+      HeadGeom gq = g;
+      if (p.q_tiles > 0) gq.layout = SA_LAYOUT_IDENTITY;
+      load_block<D, BN, ES>(qmaps, gq, bh, qb, sQ, &bars->q_full);
       int issued = 0;
       for (int j = 0; j < n_keys; ++j) {
         const int st = j % kStages, rnd = j / kStages;
-        const int kb = cols[j];
+        const int kb = p.dense ? j : cols[j];
         if (kb < 0 || kb >= g.nb) { atomicOr(status, SA_DEVFLAG_BOUNDS); *abort = 1; break; }
         if (!mbar_wait(&bars->kv_empty[st], (rnd & 1) ^ 1, abort, status, site(1, 1, j))) break;
         mbar_arrive_expect_tx(&bars->k_full[st], L::kKVBytes);
@@ -543,7 +551,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     float s[64];
     bool ok = true;
     // key block of this group's next block, loaded one block ahead
-    int kb_next = (!kGather && grp < n_keys) ? cols[grp] : 0;
+    int kb_next = (!kGather && grp < n_keys) ? (p.dense ? grp : cols[grp]) : 0;
     for (int j = grp; j < n_keys; j += 2) {
       const uint32_t par = (uint32_t)(j >> 1) & 1u;
       uint32_t pw[BN / 32];
@@ -559,7 +567,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         // read chunk by chunk below; m_empty is signalled after the block)
       } else {
         const int kb = kb_next;
-        if (j + 2 < n_keys) kb_next = cols[j + 2];
+        if (j + 2 < n_keys) kb_next = p.dense ? j + 2 : cols[j + 2];
         pad = block_pad_mask<BN>(g, kb, p.T, p.H, p.W, pw);
       }
       // a warp either waits out a barrier together or gives up together
@@ -753,7 +761,10 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     named_barrier_sync(1, kSoftmaxWarps * 32);
     const float m_o = xch[((grp ^ 1) * 2 + 0) * 128 + r];
     const float l_o = xch[((grp ^ 1) * 2 + 1) * 128 + r];
-    const int tok = (r < BN) ? slot_to_token(g, qb, r, BN, p.T, p.H, p.W) : -1;
+    // sampled-row mode: row qb*BN + r of the gathered rows, O in fp32
+    const bool rows_f32 = p.o_f32 != nullptr;
+    const int tok = rows_f32 ? ((r < BN && qb * BN + r < p.q_rows) ? qb * BN + r : -1)
+                             : ((r < BN) ? slot_to_token(g, qb, r, BN, p.T, p.H, p.W) : -1);
     if (ok) {
       const float m0 = grp == 0 ? m : m_o, l0 = grp == 0 ? l : l_o;
       const float m1 = grp == 0 ? m_o : m, l1 = grp == 0 ? l_o : l;
@@ -770,7 +781,10 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       const bool use0 = n_keys > 0 && w0 != 0.f, use1 = n_keys > 1 && w1 != 0.f;
       // this thread writes output columns [grp*D/2, grp*D/2 + D/2)
       constexpr int HD = D / 2;
-      __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (tok < 0 ? 0 : tok)) * D + grp * HD;
+      __nv_bfloat16* orow = rows_f32 ? nullptr
+                                     : p.o + ((size_t)bh * p.N + (tok < 0 ? 0 : tok)) * D + grp * HD;
+      float* frow = rows_f32 ? p.o_f32 + ((size_t)bh * p.q_rows + (tok < 0 ? 0 : tok)) * D + grp * HD
+                             : nullptr;
 #pragma unroll
       for (int c = 0; c < HD; c += 16) {
         float o0[16], o1[16];
@@ -778,7 +792,17 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         if (__any_sync(0xffffffffu, use0)) tmem_ld16(tO + lane_off + grp * HD + c, o0);
         if (__any_sync(0xffffffffu, use1)) tmem_ld16(tO + D + lane_off + grp * HD + c, o1);
         tmem_wait_ld();
-        if (tok >= 0) {
+        if (tok >= 0 && rows_f32) {
+#pragma unroll
+          for (int e = 0; e < 16; e += 4) {
+            float4 v;
+            v.x = (use0 ? o0[e] * w0 : 0.f) + (use1 ? o1[e] * w1 : 0.f);
+            v.y = (use0 ? o0[e + 1] * w0 : 0.f) + (use1 ? o1[e + 1] * w1 : 0.f);
+            v.z = (use0 ? o0[e + 2] * w0 : 0.f) + (use1 ? o1[e + 2] * w1 : 0.f);
+            v.w = (use0 ? o0[e + 3] * w0 : 0.f) + (use1 ? o1[e + 3] * w1 : 0.f);
+            *reinterpret_cast<float4*>(frow + c + e) = v;
+          }
+        } else if (tok >= 0) {
 #pragma unroll
           for (int e = 0; e < 16; e += 8) {
             float v[8];
@@ -794,7 +818,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
           }
         }
       }
-      if (tok >= 0 && grp == 0 && p.lse)
+      if (tok >= 0 && grp == 0 && p.lse && !rows_f32)
         p.lse[(size_t)bh * p.N + tok] =
             (n_keys > 0 && l_tot > 0.f)
                 ? (mm + __log2f(l_tot) - (kFp8 ? kPOffsetFp8 : 0.f)) * 0.69314718055994530942f

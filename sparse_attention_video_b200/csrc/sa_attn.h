@@ -40,6 +40,16 @@ struct AttnParams {
   const float* q_inv;
   const float* k_inv;
   const float* v_inv;
+  // Sampled-row mode (the profilers' full pass): every head has geometry geo0
+  // (heads is null), every query tile visits every key block of it in order
+  // (dense), the query tiles are rows of the gathered tensor behind maps.q[0]
+  // (q_tiles of them, q_rows valid per head), and O is written in fp32 to
+  // o_f32 [BH][q_rows][d] (o and lse unused).
+  HeadGeom geo0;
+  int dense;
+  int q_tiles;
+  int q_rows;
+  float* o_f32;
 };
 
 cudaError_t launch_attn_fwd(int head_dim, int block, const AttnMaps& maps, const AttnParams& p,

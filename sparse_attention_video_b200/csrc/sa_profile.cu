@@ -10,14 +10,17 @@
 //     machinery; Algorithm 1): one sliding tile window per candidate, on the
 //     3D tile layout.
 //
-// One warp owns 16 sampled rows. Keys pass through XOR-swizzled shared-memory
-// tiles filled by cp.async (double-buffered); ldmatrix forms the fragments and
-// mma.sync m16n8k16 (bf16 in, fp32 accumulate) computes S = Q K^T and
-// O += P V with an online softmax in registers. The full pass streams every
-// key once per CTA, 64 at a time, for all four warps' rows; the spatial pass
-// then walks key blocks in original order and the temporal pass in
-// frame-major order (K/V rows gathered by token), per warp, each visiting only
-// the blocks that some row of the warp keeps.
+// The full pass (every sampled row against every key, the bulk of the work)
+// runs on the tcgen05 block-sparse attention kernel: the sampled rows are
+// gathered into 128-row query tiles, every tile visits every key block, and
+// the kernel writes O in fp32. The masked passes then run here: one warp owns
+// 16 sampled rows; keys pass through XOR-swizzled shared-memory tiles filled
+// by cp.async (double-buffered); ldmatrix forms the fragments and mma.sync
+// m16n8k16 (bf16 in, fp32 accumulate) computes S = Q K^T and O += P V with an
+// online softmax in registers. The spatial pass walks key blocks in original
+// order and the temporal pass in frame-major order (K/V rows gathered by
+// token), per warp, each visiting only the blocks that some row of the warp
+// keeps.
 #include "sa_profile.h"
 #include "sa_ptx.cuh"
 
@@ -29,18 +32,13 @@ constexpr int kProfWarps = 4;
 constexpr int kRowsPerWarp = 16;
 constexpr int kStepKeys = 16;
 
-// Shared memory of a CTA: one K/V region, then per warp its Q tile and the
-// O of the full pass. The full pass streams every key through the region as
-// one double-buffered tile of 64 keys read by all warps; the masked passes cut
-// the same bytes into one double-buffered 16-key K/V pair per warp.
+// Shared memory of a CTA: one K/V region cut into one double-buffered 16-key
+// K/V pair per warp, then per warp its Q tile and the fp32 O of the full pass.
 template <int D>
 struct ProfSmem {
   static constexpr int kRow = D * 2;                       // one bf16 row
   static constexpr int kTile16 = kStepKeys * kRow;         // 16 rows (one step)
-  static constexpr int kCoopKeys = 64;
-  static constexpr int kCoopTile = kCoopKeys * kRow;       // full pass: 64 rows of K or V
-  static constexpr int kKV = 4 * kCoopTile;                // 2 buffers x (K, V)
-  static_assert(kKV == kProfWarps * 4 * kTile16, "masked passes: K, V x 2 buffers per warp");
+  static constexpr int kKV = kProfWarps * 4 * kTile16;     // K, V x 2 buffers per warp
   static constexpr int kOffWarp = kKV;
   static constexpr int kQ = kTile16;
   static constexpr int kPerWarp = kQ + kRowsPerWarp * D * 4;
@@ -225,8 +223,8 @@ __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams 
       mma16816(acc[2 * np + 1], pa, v2, v3);
     }
   };
-  // rows' sums over the four lanes that share them, O = acc / l; the full
-  // pass keeps O, a masked pass writes each row's squared error against it
+  // rows' sums over the four lanes that share them, O = acc / l; a masked
+  // pass writes each row's squared error against the full pass's O
   auto finish = [&](int pass) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
@@ -237,81 +235,38 @@ __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams 
 #pragma unroll
     for (int j = 0; j < D / 8; ++j) {
       const int col = 8 * j + cq;
-      // rounded products (no contraction into the subtraction below), so a
-      // pattern that visits the full pass's keys reproduces its output exactly
+      // rounded products (no contraction into the subtraction below)
       const float o00 = __fmul_rn(acc[j][0], i0), o01 = __fmul_rn(acc[j][1], i0);
       const float o10 = __fmul_rn(acc[j][2], i1), o11 = __fmul_rn(acc[j][3], i1);
-      float* f0 = sO + g * D + col;
-      float* f1 = sO + (g + 8) * D + col;
-      if (pass == 0) {
-        f0[0] = o00; f0[1] = o01; f1[0] = o10; f1[1] = o11;
-      } else {
-        const float d00 = o00 - f0[0], d01 = o01 - f0[1], d10 = o10 - f1[0], d11 = o11 - f1[1];
-        e0 += d00 * d00 + d01 * d01;
-        e1 += d10 * d10 + d11 * d11;
-      }
+      const float* f0 = sO + g * D + col;
+      const float* f1 = sO + (g + 8) * D + col;
+      const float d00 = o00 - f0[0], d01 = o01 - f0[1], d10 = o10 - f1[0], d11 = o11 - f1[1];
+      e0 += d00 * d00 + d01 * d01;
+      e1 += d10 * d10 + d11 * d11;
     }
-    if (pass > 0) {
-      e0 += __shfl_xor_sync(0xffffffffu, e0, 1);
-      e0 += __shfl_xor_sync(0xffffffffu, e0, 2);
-      e1 += __shfl_xor_sync(0xffffffffu, e1, 1);
-      e1 += __shfl_xor_sync(0xffffffffu, e1, 2);
-      if ((lane & 3) == 0) {
-        float* re = p.row_err + ((size_t)bh * p.n_rows + row0) * p.n_pat + (pass - 1);
-        if (row0 + g < p.n_rows) re[(size_t)g * p.n_pat] = e0;
-        if (row0 + g + 8 < p.n_rows) re[(size_t)(g + 8) * p.n_pat] = e1;
-      }
+    e0 += __shfl_xor_sync(0xffffffffu, e0, 1);
+    e0 += __shfl_xor_sync(0xffffffffu, e0, 2);
+    e1 += __shfl_xor_sync(0xffffffffu, e1, 1);
+    e1 += __shfl_xor_sync(0xffffffffu, e1, 2);
+    if ((lane & 3) == 0) {
+      float* re = p.row_err + ((size_t)bh * p.n_rows + row0) * p.n_pat + (pass - 1);
+      if (row0 + g < p.n_rows) re[(size_t)g * p.n_pat] = e0;
+      if (row0 + g + 8 < p.n_rows) re[(size_t)(g + 8) * p.n_pat] = e1;
     }
   };
 
-  // ---- full pass: every key, in original order, 64 keys per CTA step
-  {
-    reset();
-    const uint32_t rmask = __ballot_sync(0xffffffffu, my_tok >= 0) & 0xFFFFu;
-    const int nsteps = (p.N + L::kCoopKeys - 1) / L::kCoopKeys;
-    auto load64 = [&](int buf, int st) {
-      uint8_t* dK = kv + buf * 2 * L::kCoopTile;
-      uint8_t* dV = dK + L::kCoopTile;
-      for (int e = threadIdx.x; e < L::kCoopKeys * kChunks; e += 32 * kProfWarps) {
-        const int r = e / kChunks, c = e % kChunks;
-        const int slot = st * L::kCoopKeys + r;
-        if (slot < p.N) {
-          cp_async16(dK + tile_off<D>(r, c), k + (size_t)slot * D + c * 8);
-          cp_async16(dV + tile_off<D>(r, c), v + (size_t)slot * D + c * 8);
-        } else {
-          *reinterpret_cast<uint4*>(dK + tile_off<D>(r, c)) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(dV + tile_off<D>(r, c)) = make_uint4(0, 0, 0, 0);
-        }
-      }
-      cp_async_commit();
-    };
-    load64(0, 0);
-    for (int st = 0; st < nsteps; ++st) {
-      const int buf = st & 1;
-      if (st + 1 < nsteps) {
-        load64(buf ^ 1, st + 1);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
-      __syncthreads();
-      if (has_rows) {
-        const uint8_t* tK = kv + buf * 2 * L::kCoopTile;
-        const uint8_t* tV = tK + L::kCoopTile;
-        for (int sub = 0; sub < L::kCoopKeys / kStepKeys; ++sub) {
-          const int slot0 = st * L::kCoopKeys + sub * kStepKeys;
-          if (slot0 < p.N) {
-            const uint32_t kvm = slot0 + kStepKeys <= p.N ? 0xFFFFu : ((1u << (p.N - slot0)) - 1u);
-            step16(tK + sub * L::kTile16, tV + sub * L::kTile16, kvm, rmask);
-          }
-        }
-      }
-      __syncthreads();                                    // the buffer is refilled next step
+  // ---- full pass: every key of every sampled row was attended by the
+  // block-sparse attention kernel (tcgen05, a dense key list over gathered
+  // query rows) before this kernel; its fp32 O of this warp's rows is the
+  // reference the masked passes are measured against.
+  if (has_rows) {
+    for (int e = lane; e < kRowsPerWarp * D; e += 32) {
+      const int r = e / D, c = e % D;
+      sO[r * D + c] = row0 + r < p.n_rows ? p.o_full[((size_t)bh * p.n_rows + row0 + r) * D + c]
+                                          : 0.f;
     }
-    if (has_rows) finish(0);
+    __syncwarp();
   }
-  // the shared region becomes four per-warp K/V pairs (every warp is past the
-  // full pass's last read of it)
   __syncthreads();
   if (!has_rows) return;
   uint8_t* sK = kv + warp * 4 * L::kTile16;                // 2 K buffers, then 2 V buffers
@@ -342,7 +297,9 @@ __global__ void __launch_bounds__(32 * kProfWarps) profile_kernel(ProfileParams 
     return (t < p.T && h < p.H && w < p.W) ? (t * p.H + h) * p.W + w : -1;
   };
   const int nb_pass = p.mode == 0 ? nb : tnb;
-  for (int pass = 1; pass <= p.n_pat; ++pass) {
+  // one pattern per CTA along grid z (the full pass's O is in global memory,
+  // so the patterns are independent)
+  for (int pass = 1 + (int)blockIdx.z; pass <= p.n_pat; pass += (int)gridDim.z) {
     int win[3] = {1, 1, 1};
     if (p.mode == 1) { win[0] = p.win[pass - 1][0]; win[1] = p.win[pass - 1][1]; win[2] = p.win[pass - 1][2]; }
     // rows (bits 0..15) that keep key block b under this pass's pattern
@@ -438,10 +395,43 @@ static cudaError_t launch_profile_d(const ProfileParams& p, cudaStream_t st) {
                                        L::kBytes);
   if (e != cudaSuccess) return e;
   const int rows_per_cta = kProfWarps * kRowsPerWarp;
-  dim3 grid((p.n_rows + rows_per_cta - 1) / rows_per_cta, p.BH);
+  dim3 grid((p.n_rows + rows_per_cta - 1) / rows_per_cta, p.BH, p.n_pat);
   profile_kernel<D><<<grid, 32 * kProfWarps, L::kBytes, st>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   profile_reduce_kernel<<<p.BH, 32, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+namespace {
+
+// One 16-byte piece per thread: piece c of row r of head bh.
+__global__ void gather_rows_kernel(const __nv_bfloat16* src, const int* rows, int N, int d,
+                                   int n_rows, int n_pad, __nv_bfloat16* dst, uint32_t* status) {
+  const int bh = blockIdx.y;
+  const int pieces = d / 8;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int r = (int)(i / pieces), c = (int)(i % pieces);
+  if (r >= n_pad) return;
+  uint4 val = make_uint4(0, 0, 0, 0);
+  if (r < n_rows) {
+    const int t = rows[(size_t)bh * n_rows + r];
+    if (t >= 0 && t < N) {
+      val = __ldg(reinterpret_cast<const uint4*>(src + ((size_t)bh * N + t) * d) + c);
+    } else if (status) {
+      atomicOr(status, SA_DEVFLAG_BOUNDS);
+    }
+  }
+  reinterpret_cast<uint4*>(dst + ((size_t)bh * n_pad + r) * d)[c] = val;
+}
+
+}  // namespace
+
+cudaError_t launch_gather_rows(const __nv_bfloat16* src, const int* rows, int BH, int N, int d,
+                               int n_rows, int n_pad, __nv_bfloat16* dst, uint32_t* status,
+                               cudaStream_t stream) {
+  const long long pieces = (long long)n_pad * (d / 8);
+  dim3 grid((unsigned)((pieces + 255) / 256), BH);
+  gather_rows_kernel<<<grid, 256, 0, stream>>>(src, rows, N, d, n_rows, n_pad, dst, status);
   return cudaGetLastError();
 }
 

@@ -29,8 +29,15 @@ struct ProfileParams {
   int tile[3];               // STA: (bt, bh, bw), bt*bh*bw == block
   int win[kProfileMaxPatterns][3];   // STA: candidate windows (odd, in tiles)
   float scale_log2;          // log2(e) / sqrt(d)
+  const float* o_full;       // [BH][n_rows][d] fp32: full attention of the sampled rows
 };
 
 cudaError_t launch_profile(const ProfileParams& p, cudaStream_t stream);
+
+// dst[bh][r] = src[bh][rows[bh][r]] for r < n_rows, zero rows up to n_pad:
+// the sampled query rows as a contiguous [BH][n_pad][d] bf16 tensor.
+cudaError_t launch_gather_rows(const __nv_bfloat16* src, const int* rows, int BH, int N, int d,
+                               int n_rows, int n_pad, __nv_bfloat16* dst, uint32_t* status,
+                               cudaStream_t stream);
 
 }  // namespace sa

@@ -123,6 +123,17 @@ def test_summarizer_and_profiler_arguments_are_checked_on_the_host():
     a = list(args)
     a[8] = 0x1010                                                     # scratch not 256-byte aligned
     assert L.sparse_attn_profile_heads(ctypes.byref(pr), ctypes.byref(ok_pol), *a) == N.SA_ERR_WORKSPACE
+    # the scratch workspace is required (gathered rows and the full pass's O)
+    assert L.sparse_attn_profile_heads(ctypes.byref(pr), ctypes.byref(ok_pol), *args) == N.SA_ERR_WORKSPACE
+    n_rows = 1152
+    bytes_ = N.profile_workspace_size(pr, n_rows)
+    BH, d = st.heads, st.head_dim
+    n_pad = (n_rows + 127) // 128 * 128
+    up = lambda x: (x + 255) // 256 * 256
+    assert bytes_ == up(up(256 + BH * n_pad * d * 2) + BH * n_rows * d * 4)
+    for bad in (0, st.T * st.H * st.W + 1):
+        with pytest.raises(N.SparseAttnError):
+            N.profile_workspace_size(pr, bad)
 
 
 def test_window_search_and_head_windows_are_checked_on_the_host():

@@ -107,6 +107,15 @@ def test_full_size_sampled(name, heads, qbs):
     run_block_case(CONFIGS[name], heads_check=heads, qblocks_per_head=qbs)
 
 
+@pytest.mark.parametrize("name", ["sta_wan21_1p3b_480p", "spatiotemporal_hunyuan_720p",
+                                  "spade_wan21_14b_720p"])
+def test_full_size_every_head(name):
+    """Every head's whole block mask at full size against the oracle
+    (bit-exact outside the 1e-4 tie band; SPADE's blocking choice and SICS
+    totals), attention on one sampled query block per head."""
+    run_block_case(CONFIGS[name], heads_check=None, qblocks_per_head=1, seed=11)
+
+
 def test_explicit_random_masks_with_empty_rows():
     """Attention alone on random block masks in every layout; rows with no kept
     block must give O = 0 and LSE = -inf."""

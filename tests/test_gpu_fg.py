@@ -90,6 +90,13 @@ def test_fg_full_size_sampled():
     run_fg_case(CONFIGS["fg_slices_hunyuan_720p"], heads_check=[0, 23], groups_per_head=12)
 
 
+def test_fg_full_size_every_head():
+    """Every head of the full-size workload: tau within 1e-4 relative of the
+    oracle's R-th largest score and the whole slice bitmask bit-exact outside
+    the tie band; attention on one sampled group per head."""
+    run_fg_case(CONFIGS["fg_slices_hunyuan_720p"], heads_check=None, groups_per_head=1, seed=5)
+
+
 def test_fg_threshold_ties_fallback():
     """Keys 64.. are copies of key 0 and the first group's queries are 4 x
     key 0, so that group's 73,664 equal scores are the largest of the head:

@@ -5,8 +5,9 @@ Compared per head: the mean squared errors of the spatial and temporal
 outputs against the full output (relative 5 %: the GPU's P is bf16 on the
 tensor cores), the per-row errors, and the decision, which must agree unless
 the oracle's two errors are within 10 % of each other. Where one pattern keeps
-every key, the GPU visits the same keys in the same order as its full pass,
-so that pattern's error must be exactly zero.
+every key it is full attention again, computed by the masked-pass kernel
+while the full pass runs on the tcgen05 attention kernel: its error is
+rounding only, below 1e-3 of the other pattern's.
 """
 import numpy as np
 import pytest
@@ -70,20 +71,22 @@ def test_profile_ragged_rows_and_head_dim_64():
 
 
 def test_profile_exact_patterns():
-    # one frame: the spatial pattern is every key -> spatial error exactly 0
+    # one frame: the spatial pattern is every key -> spatial error at rounding level
     wl = Workload(name="profile_one_frame", config_id=121, T=1, H=16, W=24, heads=2,
                   head_dim=64, kind="spatiotemporal", block=64, sink_tokens=0)
     rows = sample_rows(wl.N, wl.heads, fraction=0.2, seed=5)
     _, is_t, mse, row_err = _run(wl, rows, 0, block=64)
-    assert np.all(row_err[:, :, 0] == 0.0) and np.all(mse[:, 0] == 0.0)
+    assert np.all(mse[:, 0] <= 1e-3 * mse[:, 1])
+    assert np.all(row_err[:, :, 0] <= 1e-3 * row_err[:, :, 1].mean(axis=1, keepdims=True) + 1e-9)
     assert np.all(is_t == 0)
-    # one position per frame: the temporal pattern is every key, visited in
-    # the same order as the full pass -> temporal error exactly 0
+    # one position per frame: the temporal pattern is every key -> temporal
+    # error at rounding level
     wl = Workload(name="profile_one_position", config_id=122, T=256, H=1, W=1, heads=2,
                   head_dim=64, kind="spatiotemporal", block=64, sink_tokens=0)
     rows = sample_rows(wl.N, wl.heads, fraction=0.25, seed=6)
     _, is_t, mse, row_err = _run(wl, rows, 0, block=64)
-    assert np.all(row_err[:, :, 1] == 0.0) and np.all(mse[:, 1] == 0.0)
+    assert np.all(mse[:, 1] <= 1e-3 * mse[:, 0])
+    assert np.all(row_err[:, :, 1] <= 1e-3 * row_err[:, :, 0].mean(axis=1, keepdims=True) + 1e-9)
     assert np.all(mse[:, 0] > 0.0) and np.all(is_t == 1)
 
 
