@@ -352,6 +352,7 @@ extern "C" int sparse_attn_build_mask(const sa_problem* problem, const sa_policy
     fp.cand = reinterpret_cast<uint2*>(sw + S.off_fg_cand);
     fp.cand_count = reinterpret_cast<uint32_t*>(sw + S.off_fg_cand + sizeof(uint2) * (size_t)M.BH * kFgCandCap);
     fp.fallback = fp.cand_count + M.BH;
+    fp.win = fp.fallback + M.BH;
     fp.bits = reinterpret_cast<uint32_t*>(mw + M.off_fg_bits);
     fp.tau = reinterpret_cast<float*>(mw + M.off_fg_tau);
     fp.status = reinterpret_cast<uint32_t*>(sw + S.off_status);

@@ -25,6 +25,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "sa_fg.h"
 #include "sa_ptx.cuh"
 
@@ -136,8 +138,10 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
 
   const int chunk = blockIdx.x, gt = blockIdx.y, bh = blockIdx.z;
   const int n_tiles_total = (p.N + 127) / 128;
-  const int tile0 = chunk * kKeyTilesPerCta;
-  const int n_tiles = min(kKeyTilesPerCta, n_tiles_total - tile0);
+  // key tiles tile0, tile0 + stride, ... (stride > 1: a sample of the keys)
+  const int stride = p.tile_stride > 1 ? p.tile_stride : 1;
+  const int tile0 = chunk * kKeyTilesPerCta * stride;
+  const int n_tiles = min(kKeyTilesPerCta, (n_tiles_total - tile0 + stride - 1) / stride);
   if (n_tiles <= 0 || grid_aborted(p.status)) return;
   if (p.only_heads && p.only_heads[bh] == 0u) return;     // uniform across the CTA
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -152,9 +156,14 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   // BITS: keep >= tau. BITS_COLLECT: keep >= the first key above the 24-bit
   // prefix bin, list the scores inside the bin.
   const float f_tau = key_to_float(tau_key);
-  const uint32_t hi24 = tau_key >> 8;
-  const float f_bin_lo = key_to_float(hi24 << 8);
-  const float f_bin_hi = hi24 >= 0xFFFFFFu ? INFINITY : key_to_float((hi24 + 1u) << 8);
+  const int cs = p.collect_shift > 0 ? p.collect_shift : 8;      // low bits left to fg_fixup
+  const uint32_t hib = tau_key >> cs;
+  const float f_bin_lo = key_to_float(hib << cs);
+  const float f_bin_hi = hib >= (0xFFFFFFFFu >> cs) ? INFINITY : key_to_float((hib + 1u) << cs);
+  // HIST_WIN: the window [win_lo, win_lo + 2^(12 + win_shift)) is histogrammed
+  // in 4,096 bins of 2^win_shift keys; keys above it are counted in registers
+  const uint32_t win_lo = p.mode == FG_MODE_HIST_WIN ? p.sel[bh * 4 + 0] : 0u;
+  uint32_t n_above = 0;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -166,7 +175,7 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
     bars->abort = 0;
     fence_barrier_init();
   }
-  if (p.mode == FG_MODE_HIST)
+  if (p.mode == FG_MODE_HIST || p.mode == FG_MODE_HIST_WIN)
     for (int i = threadIdx.x; i < kHists * kBins; i += kScoreThreads) hist[i] = 0u;
   // CACHED: exp(s/sqrt(d) - lse) > tau  <=>  s > sqrt(d) * (lse + ln tau), one
   // threshold per query column, staged where the histogram would be. A query
@@ -208,7 +217,7 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
         mbar_arrive_expect_tx(&bars->k_full[st], L::kKTile);
         for (int h = 0; h < L::kHalves; ++h)
           tma_load_3d(sK + st * L::kKTile + h * 16384, &kmap, &bars->k_full[st], h * 64,
-                      (tile0 + j) * 128, bh);
+                      (tile0 + j * stride) * 128, bh);
         issued = j + 1;
       }
       if (*abort)
@@ -281,7 +290,7 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
                                              0x06080000u | j)))
         break;
       tc_fence_after();
-      const int key = (tile0 + j) * 128 + r;
+      const int key = (tile0 + j * stride) * 128 + r;
       const bool kvalid = key < p.N;
       uint32_t words[kCols / 32];
 #pragma unroll
@@ -309,6 +318,20 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
                 atomicAdd(&whist[(kk >> p.bin_shift) & p.bin_mask], 1u);
             }
           }
+        } else if (p.mode == FG_MODE_HIST_WIN) {
+          // fine bins: neighbouring keys' scores rarely share one. The
+          // window test is one unsigned compare of the offset (a key below
+          // the window wraps to a large offset) and the count is branch-free:
+          // nested branches here ran the pass 1.5x slower.
+          const uint32_t wsize = 1u << (12 + p.win_shift);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const uint32_t kk = order_key(v[e]);
+            const uint32_t off = kk - win_lo;
+            const bool ok_e = e < n_ok;
+            n_above += (ok_e && off >= wsize && kk >= win_lo) ? 1u : 0u;
+            if (ok_e && off < wsize) atomicAdd(&whist[off >> p.win_shift], 1u);
+          }
         } else if (p.mode == FG_MODE_CACHED) {
           // this lane's key against the warp's 32 query columns, which all
           // belong to one group (32 divides the group size): kept when one
@@ -320,7 +343,7 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
           for (int e = 0; e < 32; ++e) any |= v[e] > thr[e];
           const uint32_t word = __ballot_sync(0xffffffffu, kvalid && any);
           const int g = (gt * 128 + c0) / p.group;
-          const int kw = ((tile0 + j) * 128 + 32 * quarter) / 32;
+          const int kw = ((tile0 + j * stride) * 128 + 32 * quarter) / 32;
           if (lane == 0 && word != 0u && g < p.G && kw < p.WN)
             atomicOr(p.bits + ((size_t)bh * p.G + g) * p.WN + kw, word);
         } else {
@@ -342,7 +365,8 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
                 const uint32_t pos = atomicAdd(p.cand_count + bh, 1u);
                 if (pos < kFgCandCap)
                   p.cand[(size_t)bh * kFgCandCap + pos] = make_uint2(
-                      (uint32_t)key, ((uint32_t)(g_base + c0 + e) << 8) | (order_key(v[e]) & 0xFFu));
+                      (uint32_t)key, ((uint32_t)(g_base + c0 + e) << cs) |
+                                         (order_key(v[e]) & ((1u << cs) - 1u)));
               }
             }
           }
@@ -353,7 +377,7 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       if (lane == 0) mbar_arrive(&bars->acc_free[ab]);
       if (p.mode == FG_MODE_BITS || p.mode == FG_MODE_BITS_COLLECT) {
         // lane e holds this warp's 32 keys for groups half*kCols + 32*i + e
-        const int kw = ((tile0 + j) * 128 + 32 * quarter) / 32;
+        const int kw = ((tile0 + j * stride) * 128 + 32 * quarter) / 32;
 #pragma unroll
         for (int i = 0; i < kCols / 32; ++i) {
           const int gl = half * kCols + lane + 32 * i;
@@ -363,9 +387,14 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
       }
     }
   }
+  if (p.mode == FG_MODE_HIST_WIN) {
+    // this CTA's count of keys above the window, one global add per warp
+    for (int o = 16; o >= 1; o >>= 1) n_above += __shfl_xor_sync(0xffffffffu, n_above, o);
+    if (warp >= 4 && lane == 0 && n_above) atomicAdd(p.above + bh, n_above);
+  }
   tc_fence_before();
   __syncthreads();
-  if (p.mode == FG_MODE_HIST) {
+  if (p.mode == FG_MODE_HIST || p.mode == FG_MODE_HIST_WIN) {
     uint32_t* gh = p.hist + (size_t)bh * kBins;
     for (int b = threadIdx.x; b <= (int)p.bin_mask; b += kScoreThreads) {
       uint32_t c = 0;
@@ -386,8 +415,9 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
 // largest), [2] number of slices kept (after the final level: R plus ties is
 // only known after BITS; [2] holds R).
 __global__ void fg_select_init_kernel(uint32_t* sel, uint32_t* hist, uint32_t* cand_count,
-                                      int BH, uint32_t rank) {
+                                      int BH, uint32_t rank, const uint32_t* only_heads) {
   const int bh = blockIdx.x;
+  if (only_heads && only_heads[bh] == 0u) return;
   if (threadIdx.x == 0) {
     sel[bh * 4 + 0] = 0u; sel[bh * 4 + 1] = rank; sel[bh * 4 + 2] = rank;
     cand_count[bh] = 0u;
@@ -418,31 +448,112 @@ __global__ void fg_select_kernel(uint32_t* sel, uint32_t* hist, int nbins, int s
   }
 }
 
+// ------------------------------------------------------------------ window
+// Level 0 is first taken on a sample of the key tiles (every 8th), which
+// only places tau roughly. The exact pass then counts the keys above a window
+// of four level-0 bins around that place in registers and histograms the
+// keys inside it in 4,096 fine bins; fine bins seldom collide in the
+// shared-memory atomics that bind the full level-0 histogram, and a narrow
+// window keeps most scores out of them. A head whose tau lies outside the
+// window takes the three-level path instead.
+// win arrays: above[BH], miss[BH], hit[BH], ovf[BH] (and fallback[BH]).
+constexpr int kWinBins0 = 4;         // level-0 bins in the window
+constexpr int kWinShift = 10;        // 2^(12 + 10) = 4 level-0 bins of 2^20 keys
+
+__global__ void fg_win_init_kernel(uint32_t* sel, uint32_t* hist, uint32_t* cand_count,
+                                   uint32_t* win, uint32_t* fallback, int BH, uint32_t rank) {
+  const int bh = blockIdx.x;
+  if (threadIdx.x == 0) {
+    sel[bh * 4 + 0] = 0u; sel[bh * 4 + 1] = rank; sel[bh * 4 + 2] = rank;
+    cand_count[bh] = 0u;
+    fallback[bh] = 0u;
+    for (int a = 0; a < 4; ++a) win[a * BH + bh] = 0u;
+  }
+  for (int b = threadIdx.x; b < kBins; b += blockDim.x) hist[(size_t)bh * kBins + b] = 0u;
+}
+
+// From the sampled level-0 histogram: the bin b holding the sampled rank, and
+// the window of four bins around it: b - 1 .. b + 2 when the sampled rank
+// falls in the upper half of b's sampled count, else b - 2 .. b + 1
+// (clamped), so that tau keeps at least a bin and a half of margin.
+__global__ void fg_window_kernel(uint32_t* sel, uint32_t* hist, uint32_t rank_sampled) {
+  const int bh = blockIdx.x;
+  __shared__ uint32_t counts[kBins];
+  uint32_t* h = hist + (size_t)bh * kBins;
+  for (int b = threadIdx.x; b < kBins; b += blockDim.x) { counts[b] = h[b]; h[b] = 0u; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t acc = 0;
+    int b = kBins - 1;
+    for (; b > 0; --b) {
+      if (acc + counts[b] >= rank_sampled) break;
+      acc += counts[b];
+    }
+    const bool upper = rank_sampled - acc <= (counts[b] + 1u) / 2u;   // near b's top
+    const int lo = min(max(upper ? b - 1 : b - 2, 0), kBins - kWinBins0);
+    sel[bh * 4 + 0] = (uint32_t)lo << 20;
+  }
+}
+
+// After the exact windowed pass: tau's fine bin (a 21-bit prefix) and the
+// rank left inside it, or a miss when tau lies above or below the window.
+__global__ void fg_select_win_kernel(uint32_t* sel, uint32_t* hist, uint32_t* win, int BH) {
+  const int bh = blockIdx.x;
+  __shared__ uint32_t counts[kBins];
+  uint32_t* h = hist + (size_t)bh * kBins;
+  for (int b = threadIdx.x; b < kBins; b += blockDim.x) { counts[b] = h[b]; h[b] = 0u; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t rank = sel[bh * 4 + 1];
+    uint32_t acc = win[0 * BH + bh];                    // keys above the window
+    int found = -1;
+    if (acc < rank) {
+      for (int b = kBins - 1; b >= 0; --b) {
+        if (acc + counts[b] >= rank) { found = b; break; }
+        acc += counts[b];
+      }
+    }
+    if (found >= 0) {
+      sel[bh * 4 + 0] += (uint32_t)found << kWinShift;
+      sel[bh * 4 + 1] = rank - acc;
+      win[1 * BH + bh] = 0u;
+      win[2 * BH + bh] = 1u;
+    } else {
+      win[1 * BH + bh] = 1u;
+      win[2 * BH + bh] = 0u;
+    }
+  }
+}
+
 // Last select level over the collected candidates (keys sharing the top 24
 // bits decided so far): histogram of their low 8 bits, the bin holding the
 // rank left is tau's low byte; candidates at or above it get their bit. A
 // head whose list overflowed is flagged for the full third level instead.
+// ``cs`` low key bits are left (8 after the two 12-bit levels, 11 after the
+// window); heads whose only_heads flag is 0 are not touched.
 __global__ void fg_fixup_kernel(uint32_t* sel, const uint2* cand, const uint32_t* cand_count,
                                 uint32_t* fallback, uint32_t* bits, float* tau, float inv_sqrt_d,
-                                int G, int WN) {
+                                int G, int WN, int cs, const uint32_t* only_heads) {
   const int bh = blockIdx.x;
-  __shared__ uint32_t counts[256];
+  if (only_heads && only_heads[bh] == 0u) return;
+  __shared__ uint32_t counts[1 << kWinShift];
   __shared__ uint32_t low;
+  const uint32_t nb = 1u << cs, lmask = nb - 1u;
   const uint32_t n = cand_count[bh];
   if (n > kFgCandCap) {
     if (threadIdx.x == 0) fallback[bh] = 1u;
     return;
   }
-  for (int b = threadIdx.x; b < 256; b += blockDim.x) counts[b] = 0u;
+  for (uint32_t b = threadIdx.x; b < nb; b += blockDim.x) counts[b] = 0u;
   __syncthreads();
   const uint2* c = cand + (size_t)bh * kFgCandCap;
-  for (uint32_t i = threadIdx.x; i < n; i += blockDim.x) atomicAdd(&counts[c[i].y & 0xFFu], 1u);
+  for (uint32_t i = threadIdx.x; i < n; i += blockDim.x) atomicAdd(&counts[c[i].y & lmask], 1u);
   __syncthreads();
   if (threadIdx.x == 0) {
     fallback[bh] = 0u;
     const uint32_t rank = sel[bh * 4 + 1];
     uint32_t acc = 0;
-    int b = 255;
+    int b = (int)nb - 1;
     for (; b > 0; --b) {                     // from the largest keys down
       if (acc + counts[b] >= rank) break;
       acc += counts[b];
@@ -455,8 +566,8 @@ __global__ void fg_fixup_kernel(uint32_t* sel, const uint2* cand, const uint32_t
   __syncthreads();
   for (uint32_t i = threadIdx.x; i < n; i += blockDim.x) {
     const uint2 e = c[i];
-    if ((e.y & 0xFFu) < low) continue;
-    const uint32_t g = e.y >> 8, key = e.x;
+    if ((e.y & lmask) < low) continue;
+    const uint32_t g = e.y >> cs, key = e.x;
     if ((int)g < G && (int)(key >> 5) < WN)
       atomicOr(bits + ((size_t)bh * G + g) * WN + (key >> 5), 1u << (key & 31u));
   }
@@ -587,7 +698,8 @@ cudaError_t launch_score(const CUtensorMap& km, const CUtensorMap& qm, const FgS
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   const int n_tiles = (p.N + 127) / 128;
-  dim3 grid((n_tiles + kKeyTilesPerCta - 1) / kKeyTilesPerCta, p.row_tiles, p.BH);
+  const int per_cta = kKeyTilesPerCta * (p.tile_stride > 1 ? p.tile_stride : 1);
+  dim3 grid((n_tiles + per_cta - 1) / per_cta, p.row_tiles, p.BH);
   fg_score_kernel<D><<<grid, kScoreThreads, L::kAlloc, st>>>(km, qm, p);
   return cudaGetLastError();
 }
@@ -598,8 +710,10 @@ int fg_g_pad(int G) { return (G + 127) / 128 * 128; }
 size_t fg_qsplit_bytes(int BH, int G, int d) { return 3ull * BH * fg_g_pad(G) * d * 2; }
 size_t fg_hist_bytes(int BH) { return sizeof(uint32_t) * (size_t)BH * kBins; }
 size_t fg_sel_bytes(int BH) { return sizeof(uint32_t) * (size_t)BH * 4; }
+// candidates, then cand_count [BH], fallback [BH] and the window state
+// (above, miss, hit, ovf: 4 x [BH])
 size_t fg_cand_bytes(int BH) {
-  return sizeof(uint2) * (size_t)BH * kFgCandCap + 2 * sizeof(uint32_t) * (size_t)BH;
+  return sizeof(uint2) * (size_t)BH * kFgCandCap + 6 * sizeof(uint32_t) * (size_t)BH;
 }
 long long fg_list_cap_per_head(int G, int N, float f) {
   return (long long)ceil((double)f * (double)G * (double)N) + N + 32;
@@ -620,7 +734,12 @@ cudaError_t launch_fg_build(const FgBuildParams& b, EncodeFn enc, cudaStream_t s
 
   const double total = (double)b.G * (double)b.N;
   const uint32_t rank = (uint32_t)ceil((double)b.keep_fraction * total);
-  fg_select_init_kernel<<<b.BH, 256, 0, st>>>(b.sel, b.hist, b.cand_count, b.BH, rank);
+  uint32_t* above = b.win;
+  uint32_t* miss = b.win + b.BH;
+  uint32_t* hit = b.win + 2 * b.BH;
+  uint32_t* ovf = b.win + 3 * b.BH;
+  fg_win_init_kernel<<<b.BH, 256, 0, st>>>(b.sel, b.hist, b.cand_count, b.win, b.fallback, b.BH,
+                                           rank);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   FgScoreParams sp{};
@@ -628,6 +747,7 @@ cudaError_t launch_fg_build(const FgBuildParams& b, EncodeFn enc, cudaStream_t s
   sp.cand = b.cand; sp.cand_count = b.cand_count;
   sp.BH = b.BH; sp.N = b.N; sp.G = b.G; sp.WN = b.WN;
   sp.row_tiles = G_pad / 128;
+  sp.above = above;
   const float inv_sqrt_d = 1.0f / sqrtf((float)b.d);
   auto score = [&]() {
     return b.d == 128 ? launch_score<128>(km, qm, sp, st) : launch_score<64>(km, qm, sp, st);
@@ -637,6 +757,7 @@ cudaError_t launch_fg_build(const FgBuildParams& b, EncodeFn enc, cudaStream_t s
   const int widths[3] = {12, 12, 8};
   auto hist_level = [&](int lv, const uint32_t* only) -> cudaError_t {
     sp.mode = FG_MODE_HIST;
+    sp.tile_stride = 1;
     sp.bin_shift = shifts[lv];
     sp.bin_mask = (1u << widths[lv]) - 1u;
     sp.match_mask = lv == 0 ? 0u : (0xFFFFFFFFu << shifts[lv - 1]);
@@ -647,15 +768,66 @@ cudaError_t launch_fg_build(const FgBuildParams& b, EncodeFn enc, cudaStream_t s
                                            inv_sqrt_d, lv == 2, only);
     return cudaGetLastError();
   };
+
+  // 1. Level 0 on every kSampleStride-th key tile: where tau roughly lies.
+  constexpr int kSampleStride = 8;
+  const int n_tiles = (b.N + 127) / 128;
+  long long n_sampled = 0;
+  for (int t = 0; t < n_tiles; t += kSampleStride) n_sampled += std::min(128, b.N - 128 * t);
+  const uint32_t rank_s = (uint32_t)std::max<double>(
+      1.0, ceil((double)rank * (double)n_sampled / (double)b.N));
+  sp.mode = FG_MODE_HIST;
+  sp.tile_stride = kSampleStride;
+  sp.bin_shift = 20;
+  sp.bin_mask = 0xFFFu;
+  sp.match_mask = 0u;
+  sp.only_heads = nullptr;
+  if ((e = score()) != cudaSuccess) return e;
+  fg_window_kernel<<<b.BH, 256, 0, st>>>(b.sel, b.hist, rank_s);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // 2. Every key: the exact count above the window and its fine histogram.
+  sp.mode = FG_MODE_HIST_WIN;
+  sp.tile_stride = 1;
+  sp.win_shift = kWinShift;
+  if ((e = score()) != cudaSuccess) return e;
+  fg_select_win_kernel<<<b.BH, 256, 0, st>>>(b.sel, b.hist, b.win, b.BH);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // 3. The bitmask pass settles every score outside tau's fine bin and lists
+  // the scores inside it; fg_fixup selects the last 11 bits among them.
+  sp.mode = FG_MODE_BITS_COLLECT;
+  sp.collect_shift = kWinShift;
+  sp.only_heads = hit;
+  if ((e = score()) != cudaSuccess) return e;
+  fg_fixup_kernel<<<b.BH, 256, 0, st>>>(b.sel, b.cand, b.cand_count, ovf, b.bits, b.tau,
+                                        inv_sqrt_d, b.G, b.WN, kWinShift, hit);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // Window heads whose candidate list overflowed: a histogram of the last 11
+  // bits over every key, then the plain bitmask pass.
+  sp.mode = FG_MODE_HIST;
+  sp.bin_shift = 0;
+  sp.bin_mask = (1u << kWinShift) - 1u;
+  sp.match_mask = 0xFFFFFFFFu << kWinShift;
+  sp.only_heads = ovf;
+  if ((e = score()) != cudaSuccess) return e;
+  fg_select_kernel<<<b.BH, 256, 0, st>>>(b.sel, b.hist, 1 << kWinShift, 0, b.tau, inv_sqrt_d, 1,
+                                         ovf);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  sp.mode = FG_MODE_BITS;
+  if ((e = score()) != cudaSuccess) return e;
+
+  // Heads whose tau fell outside the window: the three-level path.
+  fg_select_init_kernel<<<b.BH, 256, 0, st>>>(b.sel, b.hist, b.cand_count, b.BH, rank, miss);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   for (int lv = 0; lv < 2; ++lv)
-    if ((e = hist_level(lv, nullptr)) != cudaSuccess) return e;
+    if ((e = hist_level(lv, miss)) != cudaSuccess) return e;
   // The bitmask pass settles every score outside the 24-bit prefix bin and
   // lists the few inside it; fg_fixup selects the last 8 bits among them.
   sp.mode = FG_MODE_BITS_COLLECT;
-  sp.only_heads = nullptr;
+  sp.collect_shift = 8;
+  sp.only_heads = miss;
   if ((e = score()) != cudaSuccess) return e;
   fg_fixup_kernel<<<b.BH, 256, 0, st>>>(b.sel, b.cand, b.cand_count, b.fallback, b.bits, b.tau,
-                                        inv_sqrt_d, b.G, b.WN);
+                                        inv_sqrt_d, b.G, b.WN, 8, miss);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // Heads whose candidate list overflowed: the full third level and the plain
   // bitmask pass (every other head's CTAs return at once).

@@ -20,7 +20,10 @@ typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void
 // CACHED: the B operand is 128 query rows instead of q_avg terms; a slice
 // (group, key) is kept when one of the group's queries gives the key a
 // full-attention probability above tau (FG-Attn review, the cached strategy).
-enum { FG_MODE_HIST = 0, FG_MODE_BITS = 1, FG_MODE_BITS_COLLECT = 2, FG_MODE_CACHED = 3 };
+// HIST_WIN: exact count of the keys above a per-head window (sel[0] its low
+// end) and a 4,096-bin histogram of the keys inside it.
+enum { FG_MODE_HIST = 0, FG_MODE_BITS = 1, FG_MODE_BITS_COLLECT = 2, FG_MODE_CACHED = 3,
+       FG_MODE_HIST_WIN = 4 };
 
 // Candidate slots per head for the last select level; more than this (only
 // with very many scores equal in their top 24 bits) falls back to the full
@@ -42,7 +45,7 @@ struct FgScoreParams {
   int bin_shift;           // HIST: bin = (key >> bin_shift) & bin_mask
   uint32_t bin_mask;
   uint32_t match_mask;     // HIST: count only keys with (key & match_mask) == prefix
-  uint2* cand;             // BITS_COLLECT: [BH][kFgCandCap] (key index, group << 8 | low 8 bits)
+  uint2* cand;             // BITS_COLLECT: [BH][kFgCandCap] (key index, group << cs | low cs bits)
   uint32_t* cand_count;    // [BH]
   const uint32_t* only_heads;  // if set: heads whose flag is 0 do nothing
   const float* lse;        // CACHED: [BH][N] natural-log LSE of full attention
@@ -51,6 +54,10 @@ struct FgScoreParams {
   int group;               // CACHED: queries per group (64 or 128)
   int row_tiles;           // 128-row tiles of the B operand (groups, or queries for CACHED)
   int BH, N, G, WN;
+  int tile_stride;         // > 1: only every tile_stride-th key tile (a sample)
+  int collect_shift;       // BITS_COLLECT: low key bits left to fg_fixup (0: 8)
+  int win_shift;           // HIST_WIN: log2 of the keys per bin
+  uint32_t* above;         // HIST_WIN: [BH] keys above the window
 };
 
 struct FgListParams {
@@ -72,6 +79,7 @@ struct FgBuildParams {
   uint2* cand;             // [BH][kFgCandCap]
   uint32_t* cand_count;    // [BH]
   uint32_t* fallback;      // [BH]: 1 where the candidate list overflowed
+  uint32_t* win;           // [BH][4]: above-window count, window miss, window hit, overflow
   uint32_t* bits;
   float* tau;
   uint32_t* status;

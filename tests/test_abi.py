@@ -289,7 +289,7 @@ def _layout_bytes(wl):
         cap = math.ceil(float(np.float32(wl.fg_keep_fraction)) * G * N_) + N_ + 32
         mask += [4 * BH * G * WN, 4 * BH, 4 * BH * P, 4 * BH * (P + 1), 4 * BH * cap]
         scratch += [3 * BH * cdiv(G, 128) * 128 * d * 2, 4 * BH * 4096, 4 * BH * 4,
-                    8 * BH * 65536 + 8 * BH]
+                    8 * BH * 65536 + 24 * BH]
     return max(sum(up(b) for b in mask), 256), sum(up(b) for b in scratch)
 
 
