@@ -444,17 +444,19 @@ def fg_mask_extras(wl, sa):
     return {"fg_compact": compact}, score_pass
 
 
-def fg_score_entry(wl, times, flops_per_pass, peak_tflops, passes=3):
+def fg_score_entry(wl, times, flops_per_pass, peak_tflops, passes=2.125):
     n, ms = _kernel_ms(times, "fg_score")
     if n == 0:
         return {}
     tf = passes * flops_per_pass / (ms * 1e-3) / 1e12
     return {"fg_score": {"workload": wl.name, "ms_all_passes": ms, "launches": n,
                          "bound": "tensor", "tflop_per_pass": flops_per_pass / 1e12,
+                         "passes": passes,
                          "achieved_tflops": tf, "peak_tflops": peak_tflops,
                          "frac": tf / peak_tflops,
-                         "note": "three passes (two histogram levels, the bitmask); "
-                                 "launches for heads in the tie fallback return at once"}}
+                         "note": "level 0 on an eighth of the key tiles, the windowed exact "
+                                 "histogram, the bitmask; launches for heads outside the window "
+                                 "or with an overflowing list return at once"}}
 
 
 def mask_roofline_entry(wl, times, nbytes, hbm):
