@@ -11,11 +11,7 @@
 //             float32 operation, then y to E4M3 (round to nearest even,
 //             saturating at 448): eight codes per 16-byte load;
 //   finalize  the inv buffer's amax bits become inv (1 for an all-zero tensor).
-// HBM-bound: 2 bytes read and 1 byte written per element. The two passes
-// run per group of tensors that fits in L2, so the second read of a group
-// comes from L2.
-#include <algorithm>
-
+// HBM-bound: 2 bytes read (twice) and 1 byte written per element.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
@@ -101,26 +97,17 @@ cudaError_t launch_quant_e4m3(const QuantParams& p, cudaStream_t st) {
   uint32_t* amax_bits = reinterpret_cast<uint32_t*>(p.inv);
   cudaError_t e = cudaMemsetAsync(amax_bits, 0, sizeof(uint32_t) * (size_t)p.n_tensors, st);
   if (e != cudaSuccess) return e;
-  // Tensors go through amax and encode in groups of at most about 48 MB, so
-  // that the encode pass reads its group from L2 (126 MB) rather than HBM.
-  const long long tensor_bytes = p.n_elems * 2;
-  const int group = (int)std::max<long long>(1, (48LL << 20) / std::max<long long>(tensor_bytes, 1));
+  // about four CTAs of 256 threads per SM over all tensors, at least one per
+  // tensor, none without a full vector of work
   const long long nv = p.n_elems / 8;
-  for (int t0 = 0; t0 < p.n_tensors; t0 += group) {
-    const int nt = std::min(group, p.n_tensors - t0);
-    // about four CTAs of 256 threads per SM over the group, at least one per
-    // tensor, none without a full vector of work
-    long long per = (4LL * 148 + nt - 1) / nt;
-    per = std::min<long long>(per, (nv + kQuantThreads - 1) / kQuantThreads);
-    per = std::max<long long>(per, 1);
-    const dim3 grid((unsigned)per, (unsigned)nt);
-    const __nv_bfloat16* x = p.x + (size_t)t0 * p.n_elems;
-    amax_kernel<<<grid, kQuantThreads, 0, st>>>(x, p.n_elems, amax_bits + t0);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    encode_kernel<<<grid, kQuantThreads, 0, st>>>(x, p.n_elems, amax_bits + t0,
-                                                  p.codes + (size_t)t0 * p.n_elems);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
+  long long per = (4LL * 148 + p.n_tensors - 1) / p.n_tensors;
+  per = std::min<long long>(per, (nv + kQuantThreads - 1) / kQuantThreads);
+  per = std::max<long long>(per, 1);
+  const dim3 grid((unsigned)per, (unsigned)p.n_tensors);
+  amax_kernel<<<grid, kQuantThreads, 0, st>>>(p.x, p.n_elems, amax_bits);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  encode_kernel<<<grid, kQuantThreads, 0, st>>>(p.x, p.n_elems, amax_bits, p.codes);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   finalize_kernel<<<(p.n_tensors + 255) / 256, 256, 0, st>>>(amax_bits, p.n_tensors);
   return cudaGetLastError();
 }
