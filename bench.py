@@ -324,9 +324,19 @@ def _kernel_ms(times, fragment):
     return n, t
 
 
-def _traffic_per_launch():
+def attn_kernel_name(wl):
+    """The attention kernel a workload's attend() launches: policies that bound
+    a row's kept blocks run the one-warpgroup kernel (two CTAs per SM)."""
+    if wl.kind == "fg":
+        return "attn_fwd_kernel<%d,%d,gather>" % (wl.head_dim, wl.block)
+    if wl.kind in ("topk", "sta", "spatiotemporal"):
+        return "attn_solo_kernel<%d,%d>" % (wl.head_dim, wl.block)
+    return "attn_fwd_kernel<%d,%d,block>" % (wl.head_dim, wl.block)
+
+
+def _traffic_per_launch(kernel):
     """DRAM bytes per attention launch from the committed ncu summary, if it was
-    taken on the current attention source; else None."""
+    taken on the current attention source and of this kernel; else None."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     kv = {}
@@ -335,7 +345,7 @@ def _traffic_per_launch():
             a, b = line.split("=", 1)
             kv[a.strip()] = b.strip()
     src_hash = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()[:16]
-    if kv.get("source_sha256_16") != src_hash:
+    if kv.get("source_sha256_16") != src_hash or kv.get("kernel") != kernel:
         return None
     try:
         return float(kv["dram_bytes_per_launch"])
@@ -902,7 +912,7 @@ def main():
 
     peak_burst, peak_sust, hbm, peak_src = _peaks()
     achieved = flops_call / (attn_ms * 1e-3) / 1e12
-    traffic = _traffic_per_launch()
+    traffic = _traffic_per_launch(attn_kernel_name(wl))
     cpu = None
     if not args.no_cpu:
         c = cpu_oracle_sample(wl_r, x)
@@ -936,8 +946,7 @@ def main():
         "useful_tflop_per_call": useful / 1e12,
         "useful_tflops_attention": useful / (attn_ms * 1e-3) / 1e12,
         **method,
-        "roofline": {"kernel": "attn_fwd_kernel<%d,%d,%s>" % (wl.head_dim, wl.block,
-                                                               "gather" if wl.kind == "fg" else "block"),
+        "roofline": {"kernel": attn_kernel_name(wl),
                      "bound": "tensor",
                      "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s",
                      "frac": achieved / peak_burst,

@@ -835,6 +835,300 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   }
 }
 
+
+// ------------------------------------------------------------------ solo CTAs
+// A lighter block kernel for rows with few kept blocks: one softmax
+// warpgroup, one K and one V stage (freed separately: K after its QK, V after
+// its PV), 256 tensor-memory columns (S and O) and 192 threads, so that two
+// CTAs fit on an SM and one CTA's setup, first loads and epilogue run under
+// the other's blocks. Same arithmetic as attn_fwd_kernel's block mode: S, the
+// lazily rescaled online softmax per 64-column chunk, P over S in tensor
+// memory, O += P V.
+//   warps 0-3  softmax and epilogue (thread r owns row r)
+//   warp 4     TMA producer
+//   warp 5     tensor memory and the MMAs (converged, elect.sync)
+constexpr int kSoloThreads = 192;
+constexpr int kSoloProducer = 4;
+constexpr int kSoloMma = 5;
+
+template <int D, int BN>
+struct SoloSmem {
+  static constexpr int kHalvesD = D / 64;
+  static constexpr int kQBytes = kHalvesD * 128 * 128;
+  static constexpr int kKVHalf = BN * 128;
+  static constexpr int kKVBytes = kHalvesD * kKVHalf;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + kKVBytes;
+  static constexpr int kOffBar = kOffV + kKVBytes;
+  static constexpr int kBytes = kOffBar + 256;
+  static constexpr int kAlloc = kBytes + 1024;
+  static constexpr uint32_t kTmemCols = 256;              // S at 0, O at 128
+};
+
+struct SoloBars {
+  uint64_t q_full, k_full, v_full, k_empty, v_empty, s_full, p_full, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int D, int BN>
+__global__ void __launch_bounds__(kSoloThreads, 2)
+attn_solo_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
+  using L = SoloSmem<D, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem + L::kOffQ;
+  uint8_t* sK = smem + L::kOffK;
+  uint8_t* sV = smem + L::kOffV;
+  SoloBars* bars = reinterpret_cast<SoloBars*>(smem + L::kOffBar);
+  const int qb = blockIdx.x, bh = blockIdx.y;
+  const HeadGeom g = p.heads[bh];
+  if (qb >= g.nb || grid_aborted(p.status)) return;
+  const size_t row_base = (size_t)bh * p.NB + qb;
+  const int n_keys = p.counts[row_base];
+  const int* cols = p.cols + row_base * p.NB;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->k_full, 1); mbar_init(&bars->v_full, 1);
+    mbar_init(&bars->k_empty, 1); mbar_init(&bars->v_empty, 1);
+    mbar_init(&bars->s_full, 1); mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if constexpr (BN < 128) {
+    constexpr int kVecPerHalf = (128 - BN) * 8;
+    for (int i = threadIdx.x; i < kVecPerHalf * L::kHalvesD; i += blockDim.x) {
+      const int h = i / kVecPerHalf, rem = i % kVecPerHalf;
+      reinterpret_cast<uint4*>(sQ + h * 16384 + BN * 128)[rem] = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  if (warp == kSoloMma) {
+    __syncwarp();
+    tmem_alloc(&bars->tmem_base, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const uint32_t tS = tmem, tO = tmem + 128;
+  volatile int* abort = &bars->abort;
+  uint32_t* status = p.status;
+
+  if (warp == kSoloProducer) {
+    if (lane == 0 && n_keys > 0) {
+      mbar_arrive_expect_tx(&bars->q_full, L::kHalvesD * BN * 128);
+      load_block<D, BN>(maps.q, g, bh, qb, sQ, &bars->q_full);
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < n_keys; ++j) {
+        const int kb = cols[j];
+        if (kb < 0 || kb >= g.nb) { atomicOr(status, SA_DEVFLAG_BOUNDS); *abort = 1; break; }
+        // K_j once QK_{j-1} has read the stage, V_j once PV_{j-1} has
+        if (!mbar_wait(&bars->k_empty, (j & 1) ^ 1, abort, status, site(1, 1, j))) break;
+        mbar_arrive_expect_tx(&bars->k_full, L::kKVBytes);
+        load_block<D, BN>(maps.k, g, bh, kb, sK, &bars->k_full);
+        k_issued = j + 1;
+        if (!mbar_wait(&bars->v_empty, (j & 1) ^ 1, abort, status, site(1, 2, j))) break;
+        mbar_arrive_expect_tx(&bars->v_full, L::kKVBytes);
+        load_block<D, BN>(maps.v, g, bh, kb, sV, &bars->v_full);
+        v_issued = j + 1;
+      }
+      if (*abort) {
+        if (k_issued > 0) mbar_drain(&bars->k_full, (k_issued - 1) & 1);
+        if (v_issued > 0) mbar_drain(&bars->v_full, (v_issued - 1) & 1);
+      }
+    }
+  } else if (warp == kSoloMma) {
+    if (n_keys > 0) {
+      constexpr uint32_t idesc_qk = umma_idesc_bf16(128, BN, false, false);
+      constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, false, true);
+      const uint64_t dQ = umma_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dK = umma_desc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dV = umma_desc_sw128(smem_u32(sV), L::kKVHalf, 1024);
+      auto qk = [&](int j) -> bool {
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(&bars->k_full, j & 1, abort, status,
+                                                      site(2, 6, j))))
+          return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16_ss_elect(tS, umma_desc_advance(dQ, (kk / 4) * 16384 + (kk % 4) * 32),
+                             umma_desc_advance(dK, (kk / 4) * L::kKVHalf + (kk % 4) * 32),
+                             idesc_qk, kk > 0 ? 1u : 0u);
+        umma_commit_elect(&bars->s_full);
+        umma_commit_elect(&bars->k_empty);
+        return true;
+      };
+      auto pv = [&](int j) -> bool {
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(&bars->p_full, j & 1, abort, status,
+                                                      site(2, 3, j))))
+          return false;
+        if (!__all_sync(0xffffffffu, mbar_wait<false>(&bars->v_full, j & 1, abort, status,
+                                                      site(2, 4, j))))
+          return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_bf16_ts_elect(tO, tS + (kk / 4) * 64 + (kk % 4) * 8,
+                             umma_desc_advance(dV, kk * 16 * 128), idesc_pv,
+                             (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit_elect(&bars->v_empty);
+        return true;
+      };
+      // QK_0, then PV_j, QK_{j+1}: S is rewritten only after PV_j read P_j,
+      // and S_{j+1}'s commit covers PV_j, so O holds every earlier block
+      // when the softmax sees S_{j+1}.
+      bool ok = __all_sync(0xffffffffu,
+                           mbar_wait<false>(&bars->q_full, 0, abort, status, site(2, 5, 0)));
+      if (ok) ok = qk(0);
+      for (int j = 0; ok && j < n_keys; ++j) {
+        ok = pv(j);
+        if (ok && j + 1 < n_keys) ok = qk(j + 1);
+      }
+      umma_commit_elect(&bars->drain);
+      mbar_drain(&bars->drain, 0);
+      __syncwarp();
+    }
+  } else if (warp < 4) {
+    constexpr int kChunks = BN / 64;
+    const int r = warp * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t tSg = tS + lane_off, tOg = tO + lane_off;
+    const float scale = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    float s[64];
+    bool ok = true;
+    int kb_next = n_keys > 0 ? cols[0] : 0;
+    for (int j = 0; j < n_keys; ++j) {
+      uint32_t pw[BN / 32];
+      const int kb = kb_next;
+      if (j + 1 < n_keys) kb_next = cols[j + 1];
+      const bool pad = block_pad_mask<BN>(g, kb, p.T, p.H, p.W, pw);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, abort, status, site(3, 8, j)))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ch = 0; ch < kChunks; ++ch) {
+        tmem_ld32(tSg + ch * 64, s);
+        tmem_ld32(tSg + ch * 64 + 32, s + 32);
+        tmem_wait_ld();
+        if (pad) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[c] = ((pw[ch * 2 + c / 32] >> (c % 32)) & 1u) ? s[c] : -INFINITY;
+        }
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) {
+          mx4[0] = fmax3(mx4[0], s[c], s[c + 1]);
+          mx4[1] = fmax3(mx4[1], s[c + 2], s[c + 3]);
+          mx4[2] = fmax3(mx4[2], s[c + 4], s[c + 5]);
+          mx4[3] = fmax3(mx4[3], s[c + 6], s[c + 7]);
+        }
+        const float cm = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]) * scale;
+        const bool move = cm > m + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, move)) {
+          const bool had = move && m != -INFINITY;
+          const float alpha = had ? ex2_approx(m - cm) : 1.f;
+          l *= alpha;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) rs4[e] *= alpha;
+          if (__any_sync(0xffffffffu, had)) {
+            float o[32];
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+              tmem_ld32(tOg + c, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] *= alpha;
+              tmem_st32(tOg + c, o);
+            }
+#pragma unroll
+            for (int pc = 0; pc < ch; ++pc) {
+              tmem_ld32(tSg + pc * 64, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const uint32_t b = __float_as_uint(o[e]);
+                o[e] = __uint_as_float(pack_bf16x2(__uint_as_float(b << 16) * alpha,
+                                                   __uint_as_float(b & 0xFFFF0000u) * alpha));
+              }
+              tmem_st32(tSg + pc * 64, o);
+            }
+          }
+          if (move) m = cm;
+        }
+        const float neg = m == -INFINITY ? 0.f : -m;
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          float x0, x1;
+          fma2(s[c], s[c + 1], scale, scale, neg, neg, x0, x1);
+          s[c] = ex2_approx(x0);
+          s[c + 1] = ex2_approx(x1);
+        }
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+          add2(rs4[0], rs4[1], s[c], s[c + 1]);
+          add2(rs4[2], rs4[3], s[c + 2], s[c + 3]);
+        }
+#pragma unroll
+        for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(pack_bf16x2(s[2 * c], s[2 * c + 1]));
+        tmem_st32(tSg + ch * 64, s);
+      }
+      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full);
+    }
+    if (ok && n_keys > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->drain, 0, abort, status, site(3, 10, n_keys)));
+      tc_fence_after();
+    }
+    const int tok = r < BN ? slot_to_token(g, qb, r, BN, p.T, p.H, p.W) : -1;
+    if (ok) {
+      const float inv_l = (n_keys > 0 && l > 0.f) ? 1.f / l : 0.f;
+      const bool use = n_keys > 0;
+      __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (tok < 0 ? 0 : tok)) * D;
+#pragma unroll
+      for (int c = 0; c < D; c += 16) {
+        float o0[16];
+        if (use) tmem_ld16(tOg + c, o0);             // warp-uniform (n_keys is per CTA)
+        tmem_wait_ld();
+        if (tok >= 0) {
+#pragma unroll
+          for (int e = 0; e < 16; e += 8) {
+            uint4 w;
+            w.x = pack_bf16x2(use ? o0[e] * inv_l : 0.f, use ? o0[e + 1] * inv_l : 0.f);
+            w.y = pack_bf16x2(use ? o0[e + 2] * inv_l : 0.f, use ? o0[e + 3] * inv_l : 0.f);
+            w.z = pack_bf16x2(use ? o0[e + 4] * inv_l : 0.f, use ? o0[e + 5] * inv_l : 0.f);
+            w.w = pack_bf16x2(use ? o0[e + 6] * inv_l : 0.f, use ? o0[e + 7] * inv_l : 0.f);
+            *reinterpret_cast<uint4*>(orow + c + e) = w;
+          }
+        }
+      }
+      if (tok >= 0 && p.lse)
+        p.lse[(size_t)bh * p.N + tok] =
+            (n_keys > 0 && l > 0.f) ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kSoloMma) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
 }  // namespace
 
 template <int D, int BN, bool kGather, bool kFp8 = false>
@@ -853,6 +1147,24 @@ cudaError_t launch_attn_fwd(int head_dim, int block, const AttnMaps& maps, const
   if (head_dim == 128 && block == 128) return launch_one<128, 128, false>(maps, p, stream);
   if (head_dim == 64 && block == 128) return launch_one<64, 128, false>(maps, p, stream);
   if (head_dim == 64 && block == 64) return launch_one<64, 64, false>(maps, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+template <int D, int BN>
+static cudaError_t launch_solo(const AttnMaps& maps, const AttnParams& p, cudaStream_t stream) {
+  using L = SoloSmem<D, BN>;
+  auto kern = attn_solo_kernel<D, BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(p.NB, p.BH), kSoloThreads, L::kAlloc, stream>>>(maps, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_fwd_solo(int head_dim, int block, const AttnMaps& maps,
+                                 const AttnParams& p, cudaStream_t stream) {
+  if (head_dim == 128 && block == 128) return launch_solo<128, 128>(maps, p, stream);
+  if (head_dim == 64 && block == 128) return launch_solo<64, 128>(maps, p, stream);
+  if (head_dim == 64 && block == 64) return launch_solo<64, 64>(maps, p, stream);
   return cudaErrorInvalidValue;
 }
 

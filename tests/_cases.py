@@ -73,6 +73,10 @@ SMALL = {
                                    window=(3, 3, 3), summarizer="min"),
     "topk_max_d64": CONFIGS["tiny_topk"].with_(name="topk_max_d64", config_id=110,
                                                summarizer="max"),
+    # head_dim 64 with 128-token blocks on the one-warpgroup kernel
+    "spatiotemporal_d64": Workload(name="spatiotemporal_d64", config_id=112, T=5, H=9, W=16,
+                                   heads=2, head_dim=64, kind="spatiotemporal", block=128,
+                                   sink_tokens=100, temporal_heads=(1,)),
     # a window per head (Sliding Tile Attention review: head specialization)
     "sta_head_windows": Workload(name="sta_head_windows", config_id=111, T=9, H=10, W=19, heads=3,
                                  head_dim=128, kind="sta", tile=(4, 4, 8), block=128,

@@ -154,3 +154,36 @@ def test_explicit_random_masks_with_empty_rows():
             C.check_errors(*e, where=f"explicit layout {lay} head {h}")
             empty_rows = blk[1][blk[1] >= 0]
             assert np.all(o_np[0, h, empty_rows] == 0.0)
+
+
+def test_explicit_head_dim_64_blocks_of_64():
+    """Caller-supplied masks run the two-warpgroup kernel: head_dim 64 with
+    64-token blocks in the identity and 3D tile layouts (the policies that
+    bound their rows run the one-warpgroup kernel at these sizes)."""
+    from sparse_attention_video_b200 import SA_LAYOUT_IDENTITY, SA_LAYOUT_TILE, SparseAttention, make_policy
+    from oracle import layout
+    wl = C.SMALL["sta_d64"]
+    x = make_qkv(wl)
+    q, k, v = (_dev(x[n]) for n in "qkv")
+    rng = np.random.default_rng(9)
+    for lay, tile in ((SA_LAYOUT_IDENTITY, (1, 1, 64)), (SA_LAYOUT_TILE, (2, 4, 8))):
+        if lay == SA_LAYOUT_TILE:
+            order = layout.tile_order(wl.T, wl.H, wl.W, *tile)
+        else:
+            order = layout.identity_order(wl.T, wl.H, wl.W, 64)
+        blk = layout.blocks(order, 64)
+        nb = blk.shape[0]
+        dense = rng.random((wl.heads, nb, nb)) < 0.4
+        dense[:, :, ~masks.valid_blocks(blk)] = False
+        bits_dev = torch.from_numpy(C.pack_rows(dense).view(np.int32)).cuda()
+        pol = make_policy("explicit", block=64, tile=tile, explicit_layout=lay, explicit_bits=bits_dev)
+        sa = SparseAttention(1, wl.heads, wl.T, wl.H, wl.W, wl.head_dim, pol)
+        o, lse = sa(q, k, v)
+        torch.cuda.synchronize()
+        assert sa.status() == 0
+        o_np, lse_np = _bf16_to_np(o), lse.cpu().numpy()
+        for h in range(wl.heads):
+            qf, kf, vf = (bf16_bits_to_f32(x[n][0, h]) for n in "qkv")
+            o_ref, lse_ref = attention.block_sparse_attention(qf, kf, vf, blk, dense[h])
+            e = C.attention_errors(o_np[0, h], lse_np[0, h], o_ref, lse_ref)
+            C.check_errors(*e, where=f"explicit d64 layout {lay} head {h}")
