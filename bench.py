@@ -372,7 +372,14 @@ def policy_kwargs(wl):
 
 
 # kernels of ours launched by one step (build_mask + permute + attend)
-LAUNCHES_PER_STEP = {"topk": 5, "sta": 3, "spatiotemporal": 4, "spade": 5, "fg": 13}
+# (the bench line counts them from one step under the CUDA activity profiler;
+# this table is the fallback when the profiler is unavailable)
+LAUNCHES_PER_STEP = {"topk": 5, "sta": 3, "spatiotemporal": 4, "spade": 5, "fg": 25}
+
+
+def launches_in(times):
+    """Kernel launches in a kernel_times() result (copies and memsets excluded)."""
+    return sum(n for name, (n, _) in times.items() if "kernel" in name)
 
 
 def _block_valid(info, T, H, W, block):
@@ -442,16 +449,20 @@ def mask_kernel_bytes_entry(wl, times, hbm, extra=None):
 
 
 def fg_mask_extras(wl, sa):
-    """FG mask kernels beyond fg_qbar: fg_compact's bytes (the slice bitmask
-    read once, the union lists written once: 4 bytes per entry) and
-    fg_score's FLOPs (three bf16 terms of each (group, key) score per pass)."""
+    """FG mask kernels beyond fg_qbar: fg_pair_count's bytes (the slice
+    bitmask read once, one count per 128-query tile written), fg_compact's
+    (the bitmask read once, the union lists written once: 4 bytes per entry)
+    and fg_score's FLOPs (three bf16 terms of each (group, key) score per
+    pass)."""
     from sparse_attention_video_b200 import SA_EXPORT_FG_TILE_KEYS
     G = (wl.N + wl.fg_group - 1) // wl.fg_group
     words = (wl.N + 31) // 32
+    tiles = (wl.N + 127) // 128
     entries = float(sa.export(SA_EXPORT_FG_TILE_KEYS).astype(np.float64).sum())
-    compact = 4 * G * words * wl.heads + 4 * entries
+    bitmask = 4 * G * words * wl.heads
     score_pass = 3 * 2.0 * G * wl.N * wl.head_dim * wl.heads
-    return {"fg_compact": compact}, score_pass
+    return {"fg_pair_count": bitmask + 4 * tiles * wl.heads,
+            "fg_compact": bitmask + 4 * entries}, score_pass
 
 
 def fg_score_entry(wl, times, flops_per_pass, peak_tflops, passes=2.125):
@@ -623,6 +634,7 @@ def main():
         step()
     torch.cuda.synchronize(dev)
     log("warm-up done")
+    per_step = launches_in(kernel_times(step, dev)) or LAUNCHES_PER_STEP[wl.kind]
     assert sa.status() == 0, "device status word set during warm-up"
     method = {}
     if wl.kind == "fg":
@@ -962,7 +974,7 @@ def main():
         "cpu_baseline": cpu,
         "e2e": {"value": aggregate_tflops(world, flops_call, e2e_ms), "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": LAUNCHES_PER_STEP[wl.kind] * args.steps,
+        "gpu_launches": per_step * args.steps,
         "clocks": clk,
         **dense,
         **fp8,
