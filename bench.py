@@ -782,7 +782,7 @@ def main():
         at_ms = max_over_ranks([at_ms], dist, dev)[0]
         pb = _peaks()[0]
         fp8 = {"fp8_attention": {
-            "kernel": "attn_fwd_kernel<128,128,block,fp8> (tcgen05.mma kind::f8f6f4)",
+            "kernel": attn_kernel_name(wl).replace(">", ",fp8>") + " (tcgen05.mma kind::f8f6f4)",
             "attend_ms": at_ms, "quantize_ms": qz_ms, "permute_ms": pm_ms,
             "tflops": flops_call / (at_ms * 1e-3) / 1e12,
             "peak": 2.0 * pb, "frac": flops_call / (at_ms * 1e-3) / 1e12 / (2.0 * pb),

@@ -283,6 +283,16 @@ void pool_regions(PoolParams& pp) {
   pp.nA = nA <= kMaxPoolAtoms ? (int)nA : 0;    // else the per-candidate kernel
 }
 
+// Top-K, tile windows and frame windows bound how many key blocks a row
+// keeps, to a few dozen at the sizes these policies are used at. Their CTAs
+// spend a large share of their time on setup, the Q load and the epilogue,
+// which the one-warpgroup attention kernel hides by running two CTAs per SM.
+// Top-P and caller-supplied masks can keep most of a row and run the
+// two-warpgroup kernel, whose three K/V stages hide the loads of long rows.
+bool bounded_rows(const sa_policy& po) {
+  return po.kind == SA_MASK_TOPK || po.kind == SA_MASK_STA || po.kind == SA_MASK_SPATIOTEMPORAL;
+}
+
 int aligned(const void* p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Union lists of the slice bitmask in the mask workspace (FG policies).
@@ -596,16 +606,8 @@ extern "C" int sparse_attn_attend(const sa_problem* problem, const sa_policy* po
   ap.status = status;
   ap.BH = c.BH; ap.NB = c.M.NB; ap.T = pr.T; ap.H = pr.H; ap.W = pr.W; ap.N = c.N;
   ap.scale_log2 = scale_log2;
-  // Top-K, tile windows and frame windows bound how many key blocks a row
-  // keeps, to a few dozen at the sizes these policies are used at. Their
-  // CTAs spend a large share of their time on setup, the Q load and the
-  // epilogue, which the one-warpgroup kernel hides by running two CTAs per
-  // SM. Top-P and caller-supplied masks can keep most of a row and run the
-  // two-warpgroup kernel, whose three K/V stages hide the loads of long rows.
-  const bool bounded_rows = po.kind == SA_MASK_TOPK || po.kind == SA_MASK_STA ||
-                            po.kind == SA_MASK_SPATIOTEMPORAL;
-  return cuda_status(bounded_rows ? launch_attn_fwd_solo(c.d, po.block, maps, ap, c.st)
-                                  : launch_attn_fwd(c.d, po.block, maps, ap, c.st));
+  return cuda_status(bounded_rows(po) ? launch_attn_fwd_solo(c.d, po.block, maps, ap, c.st)
+                                      : launch_attn_fwd(c.d, po.block, maps, ap, c.st));
 }
 
 extern "C" int sparse_attn_forward(const sa_problem* problem, const sa_policy* policy,
@@ -666,7 +668,8 @@ extern "C" int sparse_attn_attend_fp8(const sa_problem* problem, const sa_policy
   ap.N = c.N;
   ap.scale_log2 = 1.4426950408889634f / sqrtf((float)c.d);
   ap.q_inv = q_inv; ap.k_inv = k_inv; ap.v_inv = v_inv;
-  return cuda_status(launch_attn_fwd_fp8(c.d, po.block, maps, ap, c.st));
+  return cuda_status(bounded_rows(po) ? launch_attn_fwd_solo_fp8(c.d, po.block, maps, ap, c.st)
+                                      : launch_attn_fwd_fp8(c.d, po.block, maps, ap, c.st));
 }
 
 extern "C" int sparse_attn_export_bytes(const sa_problem* problem, const sa_policy* policy,

@@ -851,9 +851,10 @@ constexpr int kSoloThreads = 192;
 constexpr int kSoloProducer = 4;
 constexpr int kSoloMma = 5;
 
-template <int D, int BN>
+// ES: bytes per element (2 bf16, 1 E4M3 codes).
+template <int D, int BN, int ES = 2>
 struct SoloSmem {
-  static constexpr int kHalvesD = D / 64;
+  static constexpr int kHalvesD = D * ES / 128;           // 128-byte column groups of d
   static constexpr int kQBytes = kHalvesD * 128 * 128;
   static constexpr int kKVHalf = BN * 128;
   static constexpr int kKVBytes = kHalvesD * kKVHalf;
@@ -872,10 +873,16 @@ struct SoloBars {
   int abort;
 };
 
-template <int D, int BN>
+// kFp8 (D = BN = 128): Q, K, V are E4M3 codes with one scale per (batch,
+// head) tensor and both products run on kind::f8f6f4. The softmax takes the
+// block's row maximum first (a pass over S without exponentials), so the
+// reference moves before any P is stored and no stored E4M3 P is rescaled.
+template <int D, int BN, bool kFp8 = false>
 __global__ void __launch_bounds__(kSoloThreads, 2)
 attn_solo_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
-  using L = SoloSmem<D, BN>;
+  static_assert(!kFp8 || (D == 128 && BN == 128), "FP8: d = 128, 128-token blocks");
+  constexpr int ES = kFp8 ? 1 : 2;
+  using L = SoloSmem<D, BN, ES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -924,7 +931,7 @@ attn_solo_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
   if (warp == kSoloProducer) {
     if (lane == 0 && n_keys > 0) {
       mbar_arrive_expect_tx(&bars->q_full, L::kHalvesD * BN * 128);
-      load_block<D, BN>(maps.q, g, bh, qb, sQ, &bars->q_full);
+      load_block<D, BN, ES>(maps.q, g, bh, qb, sQ, &bars->q_full);
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < n_keys; ++j) {
         const int kb = cols[j];
@@ -932,11 +939,11 @@ attn_solo_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         // K_j once QK_{j-1} has read the stage, V_j once PV_{j-1} has
         if (!mbar_wait(&bars->k_empty, (j & 1) ^ 1, abort, status, site(1, 1, j))) break;
         mbar_arrive_expect_tx(&bars->k_full, L::kKVBytes);
-        load_block<D, BN>(maps.k, g, bh, kb, sK, &bars->k_full);
+        load_block<D, BN, ES>(maps.k, g, bh, kb, sK, &bars->k_full);
         k_issued = j + 1;
         if (!mbar_wait(&bars->v_empty, (j & 1) ^ 1, abort, status, site(1, 2, j))) break;
         mbar_arrive_expect_tx(&bars->v_full, L::kKVBytes);
-        load_block<D, BN>(maps.v, g, bh, kb, sV, &bars->v_full);
+        load_block<D, BN, ES>(maps.v, g, bh, kb, sV, &bars->v_full);
         v_issued = j + 1;
       }
       if (*abort) {
@@ -946,8 +953,13 @@ attn_solo_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     }
   } else if (warp == kSoloMma) {
     if (n_keys > 0) {
-      constexpr uint32_t idesc_qk = umma_idesc_bf16(128, BN, false, false);
-      constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, false, true);
+      constexpr uint32_t idesc_qk = kFp8 ? umma_idesc_e4m3(128, BN, false, false)
+                                         : umma_idesc_bf16(128, BN, false, false);
+      constexpr uint32_t idesc_pv = kFp8 ? umma_idesc_e4m3(128, D, false, true)
+                                         : umma_idesc_bf16(128, D, false, true);
+      // every MMA takes 32 bytes of its K dimension: 16 bf16 or 32 E4M3
+      constexpr int kKeysPerMma = 32 / ES;
+      constexpr int kMmaPerChunk = 64 / kKeysPerMma;
       const uint64_t dQ = umma_desc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dK = umma_desc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dV = umma_desc_sw128(smem_u32(sV), L::kKVHalf, 1024);
@@ -957,10 +969,12 @@ attn_solo_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
           return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_bf16_ss_elect(tS, umma_desc_advance(dQ, (kk / 4) * 16384 + (kk % 4) * 32),
-                             umma_desc_advance(dK, (kk / 4) * L::kKVHalf + (kk % 4) * 32),
-                             idesc_qk, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < D * ES / 32; ++kk) {
+          const uint64_t da = umma_desc_advance(dQ, (kk / 4) * 16384 + (kk % 4) * 32);
+          const uint64_t db = umma_desc_advance(dK, (kk / 4) * L::kKVHalf + (kk % 4) * 32);
+          if constexpr (kFp8) umma_e4m3_ss_elect(tS, da, db, idesc_qk, kk > 0 ? 1u : 0u);
+          else umma_bf16_ss_elect(tS, da, db, idesc_qk, kk > 0 ? 1u : 0u);
+        }
         umma_commit_elect(&bars->s_full);
         umma_commit_elect(&bars->k_empty);
         return true;
@@ -974,10 +988,14 @@ attn_solo_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
           return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          umma_bf16_ts_elect(tO, tS + (kk / 4) * 64 + (kk % 4) * 8,
-                             umma_desc_advance(dV, kk * 16 * 128), idesc_pv,
-                             (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BN / kKeysPerMma; ++kk) {
+          // A = P in tensor memory, 8 packed columns per MMA, at the start of
+          // the 64 S columns of its chunk; B = V, MN-major
+          const uint32_t ta = tS + (kk / kMmaPerChunk) * 64 + (kk % kMmaPerChunk) * 8;
+          const uint64_t db = umma_desc_advance(dV, kk * kKeysPerMma * 128);
+          if constexpr (kFp8) umma_e4m3_ts_elect(tO, ta, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          else umma_bf16_ts_elect(tO, ta, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
         umma_commit_elect(&bars->v_empty);
         return true;
       };
@@ -1000,7 +1018,8 @@ attn_solo_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     const int r = warp * 32 + lane;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const uint32_t tSg = tS + lane_off, tOg = tO + lane_off;
-    const float scale = p.scale_log2;
+    // FP8: scores of the codes times the two tensors' scales
+    const float scale = kFp8 ? p.scale_log2 / (p.q_inv[bh] * p.k_inv[bh]) : p.scale_log2;
     float m = -INFINITY, l = 0.f;
     float s[64];
     bool ok = true;
@@ -1016,6 +1035,85 @@ attn_solo_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       }
       tc_fence_after();
       float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (kFp8) {
+        // the block's row maximum (chunk kChunks - 1 stays in registers)
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int ch = 0; ch < kChunks; ++ch) {
+          tmem_ld32(tSg + ch * 64, s);
+          tmem_ld32(tSg + ch * 64 + 32, s + 32);
+          tmem_wait_ld();
+          if (pad) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) s[c] = ((pw[ch * 2 + c / 32] >> (c % 32)) & 1u) ? s[c] : -INFINITY;
+          }
+#pragma unroll
+          for (int c = 0; c < 64; c += 8) {
+            mx4[0] = fmax3(mx4[0], s[c], s[c + 1]);
+            mx4[1] = fmax3(mx4[1], s[c + 2], s[c + 3]);
+            mx4[2] = fmax3(mx4[2], s[c + 4], s[c + 5]);
+            mx4[3] = fmax3(mx4[3], s[c + 6], s[c + 7]);
+          }
+        }
+        const float cm = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]) * scale;
+        const bool move = cm > m + kRescaleThresholdFp8;
+        const bool had = move && m != -INFINITY;
+        const float alpha = had ? ex2_approx(m - cm) : 1.f;
+        if (move) { l *= alpha; m = cm; }
+        if (__any_sync(0xffffffffu, had)) {
+          // O holds the complete earlier blocks (S_j's commit covers PV_{j-1})
+          float o[32];
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            tmem_ld32(tOg + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(tOg + c, o);
+          }
+        }
+        // 2^4 P, so that E4M3 keeps probabilities down to 2^-13 in its
+        // normal range; l sums the same values and the epilogue removes 2^4
+        const float neg = (m == -INFINITY ? 0.f : -m) + kPOffsetFp8;
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i) {
+          const int ch = kChunks - 1 - i;
+          if (i > 0) {
+            tmem_ld32(tSg + ch * 64, s);
+            tmem_ld32(tSg + ch * 64 + 32, s + 32);
+            tmem_wait_ld();
+            if (pad) {
+#pragma unroll
+              for (int c = 0; c < 64; ++c) s[c] = ((pw[ch * 2 + c / 32] >> (c % 32)) & 1u) ? s[c] : -INFINITY;
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            float x0, x1;
+            fma2(s[c], s[c + 1], scale, scale, neg, neg, x0, x1);
+            s[c] = ex2_approx(x0);
+            s[c + 1] = ex2_approx(x1);
+          }
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            add2(rs4[0], rs4[1], s[c], s[c + 1]);
+            add2(rs4[2], rs4[3], s[c + 2], s[c + 3]);
+          }
+          // four E4M3 codes per column, key 4i + b in byte b of column i;
+          // chunk ch's 16 columns start at its own S column 64 ch (the S of
+          // the chunk still to be reloaded is in columns it does not touch)
+          uint32_t pk[16];
+#pragma unroll
+          for (int q4 = 0; q4 < 16; ++q4) {
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(s[4 * q4], s[4 * q4 + 1]),
+                                                         __NV_SATFINITE, __NV_E4M3);
+            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(s[4 * q4 + 2], s[4 * q4 + 3]),
+                                                         __NV_SATFINITE, __NV_E4M3);
+            pk[q4] = lo | (hi << 16);
+          }
+          tmem_st16(tSg + ch * 64, reinterpret_cast<const float*>(pk));
+        }
+      } else {
 #pragma unroll
       for (int ch = 0; ch < kChunks; ++ch) {
         tmem_ld32(tSg + ch * 64, s);
@@ -1083,6 +1181,7 @@ attn_solo_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
         for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(pack_bf16x2(s[2 * c], s[2 * c + 1]));
         tmem_st32(tSg + ch * 64, s);
       }
+      }
       l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       tmem_wait_st();
       tc_fence_before();
@@ -1095,7 +1194,8 @@ attn_solo_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     }
     const int tok = r < BN ? slot_to_token(g, qb, r, BN, p.T, p.H, p.W) : -1;
     if (ok) {
-      const float inv_l = (n_keys > 0 && l > 0.f) ? 1.f / l : 0.f;
+      // FP8: the V codes' scale folds into the output weight
+      const float inv_l = (n_keys > 0 && l > 0.f) ? (kFp8 ? 1.f / (l * p.v_inv[bh]) : 1.f / l) : 0.f;
       const bool use = n_keys > 0;
       __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (tok < 0 ? 0 : tok)) * D;
 #pragma unroll
@@ -1117,7 +1217,9 @@ attn_solo_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       }
       if (tok >= 0 && p.lse)
         p.lse[(size_t)bh * p.N + tok] =
-            (n_keys > 0 && l > 0.f) ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+            (n_keys > 0 && l > 0.f)
+                ? (m + __log2f(l) - (kFp8 ? kPOffsetFp8 : 0.f)) * 0.69314718055994530942f
+                : -INFINITY;
     }
   }
   tc_fence_before();
@@ -1150,10 +1252,10 @@ cudaError_t launch_attn_fwd(int head_dim, int block, const AttnMaps& maps, const
   return cudaErrorInvalidValue;
 }
 
-template <int D, int BN>
+template <int D, int BN, bool kFp8 = false>
 static cudaError_t launch_solo(const AttnMaps& maps, const AttnParams& p, cudaStream_t stream) {
-  using L = SoloSmem<D, BN>;
-  auto kern = attn_solo_kernel<D, BN>;
+  using L = SoloSmem<D, BN, kFp8 ? 1 : 2>;
+  auto kern = attn_solo_kernel<D, BN, kFp8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   kern<<<dim3(p.NB, p.BH), kSoloThreads, L::kAlloc, stream>>>(maps, p);
@@ -1165,6 +1267,12 @@ cudaError_t launch_attn_fwd_solo(int head_dim, int block, const AttnMaps& maps,
   if (head_dim == 128 && block == 128) return launch_solo<128, 128>(maps, p, stream);
   if (head_dim == 64 && block == 128) return launch_solo<64, 128>(maps, p, stream);
   if (head_dim == 64 && block == 64) return launch_solo<64, 64>(maps, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_fwd_solo_fp8(int head_dim, int block, const AttnMaps& maps,
+                                     const AttnParams& p, cudaStream_t stream) {
+  if (head_dim == 128 && block == 128) return launch_solo<128, 128, true>(maps, p, stream);
   return cudaErrorInvalidValue;
 }
 

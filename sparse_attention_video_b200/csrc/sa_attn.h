@@ -57,6 +57,9 @@ cudaError_t launch_attn_fwd(int head_dim, int block, const AttnMaps& maps, const
 // The one-warpgroup block kernel (two CTAs per SM), block mode only.
 cudaError_t launch_attn_fwd_solo(int head_dim, int block, const AttnMaps& maps,
                                  const AttnParams& p, cudaStream_t stream);
+// The one-warpgroup kernel on E4M3 codes (maps over uint8 tensors).
+cudaError_t launch_attn_fwd_solo_fp8(int head_dim, int block, const AttnMaps& maps,
+                                     const AttnParams& p, cudaStream_t stream);
 // Q, K, V as E4M3 codes (maps over uint8 tensors, 128-column boxes).
 cudaError_t launch_attn_fwd_fp8(int head_dim, int block, const AttnMaps& maps,
                                const AttnParams& p, cudaStream_t stream);
