@@ -548,9 +548,10 @@ def run_reference(args, rank, world):
 
 
 # ---------------------------------------------------------------- mask kernels only
-def mask_once(names, local):
+def mask_once(names, local, heads=0):
     """Each named workload's mask built twice (the second build runs with its
-    kernels warm) on the seeded inputs, through SparseAttention.build_mask."""
+    kernels warm) on the seeded inputs, through SparseAttention.build_mask;
+    ``heads`` > 0 keeps only that many heads (a smaller case for profiling)."""
     import torch
 
     from sparse_attention_video_b200 import SparseAttention, make_policy
@@ -560,6 +561,9 @@ def mask_once(names, local):
     dev = torch.device("cuda", local)
     for name in names:
         wl = CONFIGS[name]
+        if heads:
+            th = tuple(h for h in wl.temporal_heads if h < heads)
+            wl = wl.with_(heads=heads, temporal_heads=th)
         x = make_qkv(wl)
         q, k = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in "qk")
         sa = SparseAttention(1, wl.heads, wl.T, wl.H, wl.W, wl.head_dim,
@@ -585,7 +589,7 @@ def main():
         run_reference(args, rank, world)
         return
     if args.mask_once:
-        mask_once(args.mask_once.split(","), local)
+        mask_once(args.mask_once.split(","), local, args.heads)
         return
 
     import torch

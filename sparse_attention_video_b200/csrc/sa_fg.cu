@@ -53,6 +53,20 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
   return __uint_as_float(u);
 }
 
+// The warp's 32 words as a 32 x 32 bit matrix (row = lane), transposed by
+// five block swaps: on return bit l of lane e's word is bit e of lane l's.
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
+  const uint32_t masks[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+  for (int i = 0; i < 5; ++i) {
+    const int j = 16 >> i;
+    const uint32_t m = masks[i];
+    const uint32_t y = __shfl_xor_sync(0xffffffffu, x, j);
+    x = (lane & j) ? ((x & ~m) | ((y & ~m) >> j)) : ((x & m) | ((y & m) << j));
+  }
+  return x;
+}
+
 // ------------------------------------------------------------------ q_avg
 // One CTA of 128 threads per (group, head). d/8 lanes cover one query row
 // with 16-byte loads (8 dimensions each), so 1,024 / d rows are read per
@@ -322,7 +336,9 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
           // fine bins: neighbouring keys' scores rarely share one. The
           // window test is one unsigned compare of the offset (a key below
           // the window wraps to a large offset) and the count is branch-free:
-          // nested branches here ran the pass 1.5x slower.
+          // nested branches here ran the pass 1.5x slower, and so did float
+          // compares against the window's bounds that left the key to the
+          // scores inside it.
           const uint32_t wsize = 1u << (12 + p.win_shift);
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
@@ -348,20 +364,24 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
             atomicOr(p.bits + ((size_t)bh * p.G + g) * p.WN + kw, word);
         } else {
           const float f_keep = p.mode == FG_MODE_BITS ? f_tau : f_bin_hi;
-          bool any_cand = false;
+          // bit e of kb: this lane's key is kept for column c0 + e; of lb:
+          // its score is at least the collected bin's lower edge
+          uint32_t kb = 0u, lb = 0u;
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const bool ok_e = e < n_ok;
-            const bool keep = ok_e && v[e] >= f_keep;
-            const uint32_t ballot = __ballot_sync(0xffffffffu, keep);
-            if (lane == e) words[cc / 32] = ballot;
-            any_cand |= ok_e && v[e] >= f_bin_lo && !(v[e] >= f_keep);
+            if (v[e] >= f_keep) kb |= 1u << e;
+            if (p.mode == FG_MODE_BITS_COLLECT && v[e] >= f_bin_lo) lb |= 1u << e;
           }
-          if (p.mode == FG_MODE_BITS_COLLECT && __any_sync(0xffffffffu, any_cand)) {
+          const uint32_t okm = n_ok >= 32 ? 0xFFFFFFFFu : (n_ok > 0 ? (1u << n_ok) - 1u : 0u);
+          kb &= okm;
+          const uint32_t cand = lb & ~kb & okm;
+          // lane e: the warp's 32 keys for column c0 + e, the bitmask word
+          words[cc / 32] = warp_transpose32(kb, lane);
+          if (p.mode == FG_MODE_BITS_COLLECT && __any_sync(0xffffffffu, cand != 0u)) {
             // rare: scores that share their top 24 bits with the threshold
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              if (e < n_ok && v[e] >= f_bin_lo && !(v[e] >= f_keep)) {
+              if ((cand >> e) & 1u) {
                 const uint32_t pos = atomicAdd(p.cand_count + bh, 1u);
                 if (pos < kFgCandCap)
                   p.cand[(size_t)bh * kFgCandCap + pos] = make_uint2(
