@@ -471,14 +471,14 @@ __global__ void fg_select_kernel(uint32_t* sel, uint32_t* hist, int nbins, int s
 // ------------------------------------------------------------------ window
 // Level 0 is first taken on a sample of the key tiles (every 8th), which
 // only places tau roughly. The exact pass then counts the keys above a window
-// of four level-0 bins around that place in registers and histograms the
+// of two level-0 bins around that place in registers and histograms the
 // keys inside it in 4,096 fine bins; fine bins seldom collide in the
 // shared-memory atomics that bind the full level-0 histogram, and a narrow
 // window keeps most scores out of them. A head whose tau lies outside the
 // window takes the three-level path instead.
 // win arrays: above[BH], miss[BH], hit[BH], ovf[BH] (and fallback[BH]).
-constexpr int kWinBins0 = 4;         // level-0 bins in the window
-constexpr int kWinShift = 10;        // 2^(12 + 10) = 4 level-0 bins of 2^20 keys
+constexpr int kWinBins0 = 2;         // level-0 bins in the window
+constexpr int kWinShift = 9;         // 2^(12 + 9) = 2 level-0 bins of 2^20 keys
 
 __global__ void fg_win_init_kernel(uint32_t* sel, uint32_t* hist, uint32_t* cand_count,
                                    uint32_t* win, uint32_t* fallback, int BH, uint32_t rank) {
@@ -493,9 +493,11 @@ __global__ void fg_win_init_kernel(uint32_t* sel, uint32_t* hist, uint32_t* cand
 }
 
 // From the sampled level-0 histogram: the bin b holding the sampled rank, and
-// the window of four bins around it: b - 1 .. b + 2 when the sampled rank
-// falls in the upper half of b's sampled count, else b - 2 .. b + 1
-// (clamped), so that tau keeps at least a bin and a half of margin.
+// the window of two bins around it: b .. b + 1 when the sampled rank falls
+// in the upper half of b's sampled count, else b - 1 .. b (clamped), so that
+// tau keeps at least half a bin of margin on either side (about 1 % of the
+// scores near a 15 % cut, against a sampling error in the rank of about
+// 10^-4 of them).
 __global__ void fg_window_kernel(uint32_t* sel, uint32_t* hist, uint32_t rank_sampled) {
   const int bh = blockIdx.x;
   __shared__ uint32_t counts[kBins];
@@ -510,12 +512,12 @@ __global__ void fg_window_kernel(uint32_t* sel, uint32_t* hist, uint32_t rank_sa
       acc += counts[b];
     }
     const bool upper = rank_sampled - acc <= (counts[b] + 1u) / 2u;   // near b's top
-    const int lo = min(max(upper ? b - 1 : b - 2, 0), kBins - kWinBins0);
+    const int lo = min(max(upper ? b : b - 1, 0), kBins - kWinBins0);
     sel[bh * 4 + 0] = (uint32_t)lo << 20;
   }
 }
 
-// After the exact windowed pass: tau's fine bin (a 21-bit prefix) and the
+// After the exact windowed pass: tau's fine bin (a 23-bit prefix) and the
 // rank left inside it, or a miss when tau lies above or below the window.
 __global__ void fg_select_win_kernel(uint32_t* sel, uint32_t* hist, uint32_t* win, int BH) {
   const int bh = blockIdx.x;
@@ -549,8 +551,8 @@ __global__ void fg_select_win_kernel(uint32_t* sel, uint32_t* hist, uint32_t* wi
 // bits decided so far): histogram of their low 8 bits, the bin holding the
 // rank left is tau's low byte; candidates at or above it get their bit. A
 // head whose list overflowed is flagged for the full third level instead.
-// ``cs`` low key bits are left (8 after the two 12-bit levels, 11 after the
-// window); heads whose only_heads flag is 0 are not touched.
+// ``cs`` low key bits are left (8 after the two 12-bit levels, kWinShift after
+// the window); heads whose only_heads flag is 0 are not touched.
 __global__ void fg_fixup_kernel(uint32_t* sel, const uint2* cand, const uint32_t* cand_count,
                                 uint32_t* fallback, uint32_t* bits, float* tau, float inv_sqrt_d,
                                 int G, int WN, int cs, const uint32_t* only_heads) {
@@ -813,7 +815,7 @@ cudaError_t launch_fg_build(const FgBuildParams& b, EncodeFn enc, cudaStream_t s
   fg_select_win_kernel<<<b.BH, 256, 0, st>>>(b.sel, b.hist, b.win, b.BH);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 3. The bitmask pass settles every score outside tau's fine bin and lists
-  // the scores inside it; fg_fixup selects the last 11 bits among them.
+  // the scores inside it; fg_fixup selects the last kWinShift bits among them.
   sp.mode = FG_MODE_BITS_COLLECT;
   sp.collect_shift = kWinShift;
   sp.only_heads = hit;
@@ -821,8 +823,8 @@ cudaError_t launch_fg_build(const FgBuildParams& b, EncodeFn enc, cudaStream_t s
   fg_fixup_kernel<<<b.BH, 256, 0, st>>>(b.sel, b.cand, b.cand_count, ovf, b.bits, b.tau,
                                         inv_sqrt_d, b.G, b.WN, kWinShift, hit);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // Window heads whose candidate list overflowed: a histogram of the last 11
-  // bits over every key, then the plain bitmask pass.
+  // Window heads whose candidate list overflowed: a histogram of the last
+  // kWinShift bits over every key, then the plain bitmask pass.
   sp.mode = FG_MODE_HIST;
   sp.bin_shift = 0;
   sp.bin_mask = (1u << kWinShift) - 1u;
