@@ -177,6 +177,8 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
   // HIST_WIN: the window [win_lo, win_lo + 2^(12 + win_shift)) is histogrammed
   // in 4,096 bins of 2^win_shift keys; keys above it are counted in registers
   const uint32_t win_lo = p.mode == FG_MODE_HIST_WIN ? p.sel[bh * 4 + 0] : 0u;
+  const uint32_t win_span = 1u << (12 + p.win_shift);
+  const uint32_t win_hi = win_lo <= 0xFFFFFFFFu - win_span ? win_lo + win_span : 0xFFFFFFFFu;
   uint32_t n_above = 0;
 
   if (threadIdx.x == 0) {
@@ -340,13 +342,26 @@ fg_score_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant_
           // compares against the window's bounds that left the key to the
           // scores inside it.
           const uint32_t wsize = 1u << (12 + p.win_shift);
+          if (n_ok == 32) {
+            // keys at or above win_hi lie above the window (win_hi is the
+            // all-ones key, which no finite score has, when the window
+            // reaches the top)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const uint32_t kk = order_key(v[e]);
-            const uint32_t off = kk - win_lo;
-            const bool ok_e = e < n_ok;
-            n_above += (ok_e && off >= wsize && kk >= win_lo) ? 1u : 0u;
-            if (ok_e && off < wsize) atomicAdd(&whist[off >> p.win_shift], 1u);
+            for (int e = 0; e < 32; ++e) {
+              const uint32_t kk = order_key(v[e]);
+              n_above += kk >= win_hi ? 1u : 0u;
+              const uint32_t off = kk - win_lo;
+              if (off < wsize) atomicAdd(&whist[off >> p.win_shift], 1u);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const uint32_t kk = order_key(v[e]);
+              const uint32_t off = kk - win_lo;
+              const bool ok_e = e < n_ok;
+              n_above += (ok_e && off >= wsize && kk >= win_lo) ? 1u : 0u;
+              if (ok_e && off < wsize) atomicAdd(&whist[off >> p.win_shift], 1u);
+            }
           }
         } else if (p.mode == FG_MODE_CACHED) {
           // this lane's key against the warp's 32 query columns, which all
