@@ -484,7 +484,7 @@ __global__ void fg_select_kernel(uint32_t* sel, uint32_t* hist, int nbins, int s
 }
 
 // ------------------------------------------------------------------ window
-// Level 0 is first taken on a sample of the key tiles (every 8th), which
+// Level 0 is first taken on a sample of the key tiles (every 16th), which
 // only places tau roughly. The exact pass then counts the keys above a window
 // of two level-0 bins around that place in registers and histograms the
 // keys inside it in 4,096 fine bins; fine bins seldom collide in the
@@ -807,7 +807,7 @@ cudaError_t launch_fg_build(const FgBuildParams& b, EncodeFn enc, cudaStream_t s
   };
 
   // 1. Level 0 on every kSampleStride-th key tile: where tau roughly lies.
-  constexpr int kSampleStride = 8;
+  constexpr int kSampleStride = 16;
   const int n_tiles = (b.N + 127) / 128;
   long long n_sampled = 0;
   for (int t = 0; t < n_tiles; t += kSampleStride) n_sampled += std::min(128, b.N - 128 * t);
