@@ -465,7 +465,7 @@ def fg_mask_extras(wl, sa):
             "fg_compact": bitmask + 4 * entries}, score_pass
 
 
-def fg_score_entry(wl, times, flops_per_pass, peak_tflops, passes=2.125):
+def fg_score_entry(wl, times, flops_per_pass, peak_tflops, passes=2.0625):
     n, ms = _kernel_ms(times, "fg_score")
     if n == 0:
         return {}
@@ -475,7 +475,7 @@ def fg_score_entry(wl, times, flops_per_pass, peak_tflops, passes=2.125):
                          "passes": passes,
                          "achieved_tflops": tf, "peak_tflops": peak_tflops,
                          "frac": tf / peak_tflops,
-                         "note": "level 0 on an eighth of the key tiles, the windowed exact "
+                         "note": "level 0 on a sixteenth of the key tiles, the windowed exact "
                                  "histogram, the bitmask; launches for heads outside the window "
                                  "or with an overflowing list return at once"}}
 
