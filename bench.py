@@ -41,7 +41,7 @@ def _args():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-mask comparison")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 attention timing")
@@ -712,22 +712,34 @@ def main():
                 torch.cuda.empty_cache()
         log("mask kernel rooflines done")
 
-    # ---- end to end through the public API with host buffers
-    o_host = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
-    lse_host = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # ---- end to end through the public API with host buffers: each step is
+    # one sparse_attn_forward_host call (Q, K, V copied in, mask, forward, O
+    # and LSE copied out); steps alternate between two streams, each with its
+    # own workspaces and device buffers, so one step's copies overlap the
+    # other's kernels and the other direction's copies
+    sa2 = SparseAttention(1, wl.heads, wl.T, wl.H, wl.W, wl.head_dim,
+                          make_policy(**policy_kwargs(wl)), device=dev)
+    lanes = [(sa, stream), (sa2, torch.cuda.Stream(dev))]
+    outs = [(torch.empty(o.shape, dtype=torch.bfloat16).pin_memory(),
+             torch.empty(lse.shape, dtype=torch.float32).pin_memory()) for _ in lanes]
+    for (obj, st_), (oh, lh) in zip(lanes, outs):        # staging buffers allocated here
+        obj.forward_host(host["q"], host["k"], host["v"], oh, lh, st_)
     torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.e2e_steps):
-        qd, kd, vd = (host[n].to(dev, non_blocking=True) for n in "qkv")
-        sa.build_mask(qd, kd, stream)
-        od, ld = sa.forward(qd, kd, vd, stream=stream)
-        o_host.copy_(od, non_blocking=True)
-        lse_host.copy_(ld, non_blocking=True)
+    lanes[1][1].wait_event(e0)
+    for i in range(args.e2e_steps):
+        (obj, st_), (oh, lh) = lanes[i % 2], outs[i % 2]
+        obj.forward_host(host["q"], host["k"], host["v"], oh, lh, st_)
+    done2 = torch.cuda.Event()
+    done2.record(lanes[1][1])
+    stream.wait_event(done2)
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    assert sa2.status() == 0, "device status word set in the end-to-end steps"
     log("end-to-end steps done")
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    o_host, lse_host = outs[0]
     e2e_ms = max_over_ranks([e2e_ms], dist, dev)[0]
     h2d = sum(host[n].numel() * 2 for n in "qkv")
     d2h = o_host.numel() * 2 + lse_host.numel() * 4
@@ -977,7 +989,8 @@ def main():
            if method else {}),
         "cpu_baseline": cpu,
         "e2e": {"value": aggregate_tflops(world, flops_call, e2e_ms), "unit": "TFLOP/s",
-                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "call": "sparse_attn_forward_host, steps alternating between two streams"},
         "gpu_launches": per_step * args.steps,
         "clocks": clk,
         **dense,

@@ -241,6 +241,32 @@ SA_API int sparse_attn_attend_fp8(const sa_problem* problem, const sa_policy* po
                                   const void* mask_ws, void* scratch_ws, void* o, float* lse,
                                   void* stream);
 
+/* End to end from host memory: copies Q, K and V from host buffers into
+ * qkv_dev, builds the mask (sparse_attn_build_mask), runs sparse_attn_forward
+ * into o_dev / lse_dev and copies O (and LSE) back to host buffers, all queued
+ * on ``stream`` (one cudaMemcpyAsync per tensor). With page-locked host
+ * buffers nothing blocks the host, so a caller can keep two such calls in
+ * flight on two streams (each with its own device buffers and workspaces),
+ * one call's copies overlapping the other's kernels. This library has no
+ * counterpart of it on the pages: it is the transfer-inclusive form of the
+ * same path.
+ *   q_host, k_host, v_host  host bf16 [batch, heads, N, head_dim], original
+ *                           token order (page-locked for asynchronous copies)
+ *   o_host                  host bf16, same shape (written)
+ *   lse_host                host float [batch*heads][N] or NULL (written)
+ *   qkv_dev                 device, 3 x batch*heads*N*head_dim bf16 (Q, K, V
+ *                           in that order), 16-byte aligned, caller-owned
+ *   o_dev, lse_dev          device outputs as for sparse_attn_forward; lse_dev
+ *                           NULL exactly when lse_host is NULL
+ *   mask_ws, scratch_ws     as for sparse_attn_build_mask
+ * Returns SA_ERR_INVALID_ARG for a missing or misaligned buffer, else the
+ * first error of the steps (nothing after it is queued). */
+SA_API int sparse_attn_forward_host(const sa_problem* problem, const sa_policy* policy,
+                                    const void* q_host, const void* k_host, const void* v_host,
+                                    void* o_host, float* lse_host, void* qkv_dev, void* o_dev,
+                                    float* lse_dev, void* mask_ws, void* scratch_ws,
+                                    void* stream);
+
 /* ---------------------------------------------------------------- attention
  * O and LSE for the mask in mask_ws (built by sparse_attn_build_mask with the
  * same problem and policy). Equivalent to sparse_attn_permute followed by

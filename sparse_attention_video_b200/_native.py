@@ -32,7 +32,7 @@ EXPORTED = ("sparse_attn_workspace_size", "sparse_attn_build_mask", "sparse_attn
             "sparse_attn_profile_workspace_size",
             "sparse_attn_build_mask_fg_cached", "sparse_attn_quantize_e4m3",
             "sparse_attn_permute_fp8", "sparse_attn_attend_fp8",
-            "sparse_attn_strerror")
+            "sparse_attn_forward_host", "sparse_attn_strerror")
 
 SA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
 
@@ -85,6 +85,7 @@ def lib():
         L.sparse_attn_workspace_size.argtypes = [P, PP, ctypes.POINTER(sz), ctypes.POINTER(sz)]
         L.sparse_attn_build_mask.argtypes = [P, PP, vp, vp, vp, vp, vp]
         L.sparse_attn_forward.argtypes = [P, PP, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.sparse_attn_forward_host.argtypes = [P, PP, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.sparse_attn_permute.argtypes = [P, PP, vp, vp, vp, vp, vp, vp]
         L.sparse_attn_attend.argtypes = [P, PP, vp, vp, vp, vp, vp, vp, vp, vp]
         L.sparse_attn_export_bytes.argtypes = [P, PP, ctypes.c_int, ctypes.POINTER(sz)]
@@ -139,6 +140,14 @@ def forward(problem, policy, q, k, v, mask_ws, scratch_ws, o, lse, stream=0):
     _check(lib().sparse_attn_forward(ctypes.byref(problem), ctypes.byref(policy), q, k, v,
                                      mask_ws, scratch_ws, o, lse, stream),
            "sparse_attn_forward")
+
+
+def forward_host(problem, policy, q_host, k_host, v_host, o_host, lse_host, qkv_dev, o_dev,
+                 lse_dev, mask_ws, scratch_ws, stream=0):
+    _check(lib().sparse_attn_forward_host(ctypes.byref(problem), ctypes.byref(policy), q_host,
+                                          k_host, v_host, o_host, lse_host, qkv_dev, o_dev,
+                                          lse_dev, mask_ws, scratch_ws, stream),
+           "sparse_attn_forward_host")
 
 
 def permute(problem, policy, q, k, v, mask_ws, scratch_ws, stream=0):

@@ -96,6 +96,18 @@ def _check_lse(t, problem, device):
     _check_tensor(t, _qkv_shape(problem)[:3], (torch.float32,), "lse", device)
 
 
+def _check_host(t, shape, dtype, name):
+    """Raise unless ``t`` is a contiguous CPU tensor of ``dtype`` and the given
+    shape (the library copies exactly that many bytes from or to it)."""
+    ok = (isinstance(t, torch.Tensor) and t.dtype == dtype and t.device.type == "cpu"
+          and t.is_contiguous() and tuple(t.shape) == tuple(shape))
+    if not ok:
+        got = (f"{t.dtype} {tuple(t.shape)} on {t.device}" if isinstance(t, torch.Tensor)
+               else type(t).__name__)
+        raise ValueError(f"{name} must be a contiguous host {dtype} tensor of shape "
+                         f"{tuple(shape)}, got {got}")
+
+
 def _check_head_arrays(policy, heads):
     """The library reads one entry per head of the problem from the policy's
     host arrays; a policy made for fewer heads would be read past its end."""
@@ -181,6 +193,33 @@ class SparseAttention:
         N.forward(self.problem, self.policy, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                   self.mask_ws.data_ptr(), self.scratch_ws.data_ptr(), out.data_ptr(),
                   lse.data_ptr(), _stream_ptr(stream))
+        return out, lse
+
+    def forward_host(self, q, k, v, out, lse=None, stream=None):
+        """Build the mask and run the forward pass on host tensors: Q, K, V
+        are copied in, O (and LSE when given) copied back, all queued on
+        ``stream`` through one library call (sparse_attn_forward_host). The
+        device staging buffers belong to this object, so calls of one object
+        are ordered by their stream; page-locked host tensors keep the copies
+        asynchronous."""
+        shape = _qkv_shape(self.problem)
+        for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+            _check_host(t, shape, torch.bfloat16, n)
+        if lse is not None:
+            _check_host(lse, shape[:3], torch.float32, "lse")
+        if getattr(self, "_stage", None) is None:
+            n = 1
+            for s in shape:
+                n *= s
+            self._stage = (torch.empty(3 * n, dtype=torch.bfloat16, device=self.device),
+                           torch.empty(n, dtype=torch.bfloat16, device=self.device),
+                           torch.empty(shape[:3], dtype=torch.float32, device=self.device))
+        qkv_d, o_d, lse_d = self._stage
+        N.forward_host(self.problem, self.policy, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                       out.data_ptr(), lse.data_ptr() if lse is not None else None,
+                       qkv_d.data_ptr(), o_d.data_ptr(),
+                       lse_d.data_ptr() if lse is not None else None,
+                       self.mask_ws.data_ptr(), self.scratch_ws.data_ptr(), _stream_ptr(stream))
         return out, lse
 
     def permute(self, q, k, v, stream=None):

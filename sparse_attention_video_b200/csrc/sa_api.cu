@@ -619,6 +619,46 @@ extern "C" int sparse_attn_forward(const sa_problem* problem, const sa_policy* p
   return sparse_attn_attend(problem, policy, q, k, v, mask_ws, scratch_ws, o, lse, stream);
 }
 
+extern "C" int sparse_attn_forward_host(const sa_problem* problem, const sa_policy* policy,
+                                        const void* q_host, const void* k_host,
+                                        const void* v_host, void* o_host, float* lse_host,
+                                        void* qkv_dev, void* o_dev, float* lse_dev,
+                                        void* mask_ws, void* scratch_ws, void* stream) {
+  int e = check_problem(problem);
+  if (e) return e;
+  if (!policy) return SA_ERR_INVALID_ARG;
+  if (!q_host || !k_host || !v_host || !o_host || !qkv_dev || !o_dev) return SA_ERR_INVALID_ARG;
+  if ((lse_host == nullptr) != (lse_dev == nullptr)) return SA_ERR_INVALID_ARG;
+  if (!aligned(qkv_dev, 16) || !aligned(o_dev, 16) || (lse_dev && !aligned(lse_dev, 4)))
+    return SA_ERR_INVALID_ARG;
+  const size_t elems = (size_t)problem->batch * problem->heads * (size_t)n_tokens(*problem) *
+                       problem->head_dim;
+  const size_t bytes = elems * 2;                      // bf16
+  uint8_t* qd = static_cast<uint8_t*>(qkv_dev);
+  uint8_t* kd = qd + bytes;
+  uint8_t* vd = kd + bytes;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // one copy per tensor, in and out, on the caller's stream
+  const void* hin[3] = {q_host, k_host, v_host};
+  uint8_t* din[3] = {qd, kd, vd};
+  for (int i = 0; i < 3; ++i)
+    if (cudaMemcpyAsync(din[i], hin[i], bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return SA_ERR_CUDA;
+  e = sparse_attn_build_mask(problem, policy, qd, kd, mask_ws, scratch_ws, stream);
+  if (e) return e;
+  e = sparse_attn_forward(problem, policy, qd, kd, vd, mask_ws, scratch_ws, o_dev, lse_dev, stream);
+  if (e) return e;
+  if (cudaMemcpyAsync(o_host, o_dev, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return SA_ERR_CUDA;
+  if (lse_host) {
+    const size_t lbytes = sizeof(float) * (size_t)problem->batch * problem->heads *
+                          (size_t)n_tokens(*problem);
+    if (cudaMemcpyAsync(lse_host, lse_dev, lbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+
 extern "C" int sparse_attn_permute_fp8(const sa_problem* problem, const sa_policy* policy,
                                        const void* q8, const void* k8, const void* v8,
                                        const void* mask_ws, void* scratch_ws, void* stream) {

@@ -86,6 +86,19 @@ def test_invalid_arguments_are_rejected_on_the_host():
                                  None, None, None) == N.SA_ERR_INVALID_ARG
     assert L.sparse_attn_build_mask(ctypes.byref(pr), ctypes.byref(pol), None, None, 0x1001, 0x2000,
                                     None) == N.SA_ERR_WORKSPACE
+    # the host-buffer call: missing host or device buffers, an LSE on one
+    # side only, a misaligned device buffer; nothing is copied or launched
+    hb = (ctypes.c_char * 64)()
+    h = ctypes.addressof(hb)
+    fh = L.sparse_attn_forward_host
+    assert fh(ctypes.byref(pr), ctypes.byref(pol), None, h, h, h, None, 0x1000, 0x2000, None,
+              0x3000, 0x4000, None) == N.SA_ERR_INVALID_ARG
+    assert fh(ctypes.byref(pr), ctypes.byref(pol), h, h, h, h, None, None, 0x2000, None,
+              0x3000, 0x4000, None) == N.SA_ERR_INVALID_ARG
+    assert fh(ctypes.byref(pr), ctypes.byref(pol), h, h, h, h, h, 0x1000, 0x2000, None,
+              0x3000, 0x4000, None) == N.SA_ERR_INVALID_ARG
+    assert fh(ctypes.byref(pr), ctypes.byref(pol), h, h, h, h, None, 0x1008, 0x2000, None,
+              0x3000, 0x4000, None) == N.SA_ERR_INVALID_ARG
     st = make_policy("spatiotemporal", block=128)                     # head types missing
     assert L.sparse_attn_workspace_size(ctypes.byref(pr), ctypes.byref(st), ctypes.byref(m),
                                         ctypes.byref(s)) == N.SA_ERR_INVALID_ARG
