@@ -113,3 +113,45 @@ def test_fg_threshold_ties_fallback():
         x["k"][:, :, 64:, :] = x["k"][:, :, :1, :]
 
     run_fg_case(wl, groups_per_head=3, transform=tie_keys)
+
+
+def _fg_win_flags(sa, wl):
+    """(miss, hit) flags of the windowed threshold path per head, read from
+    the scratch workspace (status word, three split group means, histograms,
+    selection state, candidate list, then candidate count, fallback and the
+    window state: above, miss, hit, overflow)."""
+    BH, d = wl.batch * wl.heads, wl.head_dim
+    G = math.ceil(wl.N / wl.fg_group)
+    up = lambda n: (n + 255) // 256 * 256
+    off = up(256) + up(3 * BH * math.ceil(G / 128) * 128 * d * 2) + up(4 * BH * 4096) + up(4 * BH * 4)
+    base = off + 8 * BH * 65536
+    raw = sa.scratch_ws[base: base + 24 * BH].cpu().numpy().view(np.uint32).reshape(6, BH)
+    return raw[3], raw[4]
+
+
+def test_fg_window_miss_takes_the_three_level_path():
+    """The level-0 sample reads every 16th key tile. Keys of those tiles are
+    scaled by 3, so the sampled scores overstate the head's and tau lies
+    below the window the sample chooses: the exact pass must find the miss
+    and the three-level path must give the exact threshold and bits."""
+    from sparse_attention_video_b200 import SparseAttention, make_policy
+    wl = Workload(name="fg_window_miss", config_id=115, T=8, H=16, W=20, heads=2,
+                  head_dim=128, kind="fg", fg_group=64, fg_keep_fraction=0.15)
+
+    def loud_sampled_tiles(x):
+        k = bf16_bits_to_f32(x["k"])
+        for t0 in range(0, wl.N, 16 * 128):
+            k[:, :, t0:t0 + 128, :] *= 3.0
+        x["k"][...] = f32_to_bf16_bits(k)
+
+    run_fg_case(wl, groups_per_head=4, transform=loud_sampled_tiles)
+    # the same inputs again, to read the window flags of the build
+    x = make_qkv(wl)
+    loud_sampled_tiles(x)
+    q, k = (_dev(x[n]) for n in "qk")
+    sa = SparseAttention(wl.batch, wl.heads, wl.T, wl.H, wl.W, wl.head_dim,
+                         make_policy(**C.policy_kwargs(wl)))
+    sa.build_mask(q, k)
+    torch.cuda.synchronize()
+    miss, hit = _fg_win_flags(sa, wl)
+    assert miss.all() and not hit.any(), (miss.tolist(), hit.tolist())
