@@ -383,6 +383,7 @@ extern "C" int sparse_attn_build_mask(const sa_problem* problem, const sa_policy
   sp.top_p = po.top_p;
   sp.frame_radius = po.frame_radius;
   sp.sink_blocks = ceil_div(po.sink_tokens, po.block);
+  sp.status = reinterpret_cast<uint32_t*>(sw + S.off_status);
 
   const int C = n_cand(po);
   if (C > 0) {

@@ -491,6 +491,7 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       for (int i = 0; i < 2; ++i) {
         const uint32_t idx = (uint32_t)j * BN + 64 * cw + 32 * i + lane;
         kl[i] = idx < list_count ? (int)(__ldg(list + idx) & 0x3FFFFFFFu) : 0;
+        if (!dbg_in_range(kl[i], p.N, status)) kl[i] = 0;
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->kv_empty[st], (rnd & 1) ^ 1, abort, status,
                                              site(4, 1, j)))) {
@@ -763,8 +764,9 @@ attn_fwd_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     const float l_o = xch[((grp ^ 1) * 2 + 1) * 128 + r];
     // sampled-row mode: row qb*BN + r of the gathered rows, O in fp32
     const bool rows_f32 = p.o_f32 != nullptr;
-    const int tok = rows_f32 ? ((r < BN && qb * BN + r < p.q_rows) ? qb * BN + r : -1)
+    int tok = rows_f32 ? ((r < BN && qb * BN + r < p.q_rows) ? qb * BN + r : -1)
                              : ((r < BN) ? slot_to_token(g, qb, r, BN, p.T, p.H, p.W) : -1);
+    if (tok >= 0 && !dbg_in_range(tok, rows_f32 ? p.q_rows : p.N, status)) tok = -1;
     if (ok) {
       const float m0 = grp == 0 ? m : m_o, l0 = grp == 0 ? l : l_o;
       const float m1 = grp == 0 ? m_o : m, l1 = grp == 0 ? l_o : l;
@@ -1192,7 +1194,8 @@ attn_solo_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->drain, 0, abort, status, site(3, 10, n_keys)));
       tc_fence_after();
     }
-    const int tok = r < BN ? slot_to_token(g, qb, r, BN, p.T, p.H, p.W) : -1;
+    int tok = r < BN ? slot_to_token(g, qb, r, BN, p.T, p.H, p.W) : -1;
+    if (tok >= 0 && !dbg_in_range(tok, p.N, status)) tok = -1;
     if (ok) {
       // FP8: the V codes' scale folds into the output weight
       const float inv_l = (n_keys > 0 && l > 0.f) ? (kFp8 ? 1.f / (l * p.v_inv[bh]) : 1.f / l) : 0.f;

@@ -772,7 +772,8 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
     int pos = wcount[w];
     while (word) {
       const int b = __ffs(word) - 1;
-      crow[pos++] = 32 * w + b;
+      if (dbg_in_range(pos, p.NB, p.status)) crow[pos] = 32 * w + b;
+      ++pos;
       word &= word - 1;
     }
   }

@@ -72,6 +72,7 @@ struct SelectParams {
   int win[3];
   float top_p;
   int frame_radius, sink_blocks;
+  uint32_t* status;                 // debug builds: index checks flag it
 };
 
 cudaError_t launch_head_init(const HeadInitParams& p, cudaStream_t st);

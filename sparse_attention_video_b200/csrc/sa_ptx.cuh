@@ -13,6 +13,24 @@
 
 namespace sa {
 
+// Debug builds (compiled with SA_DEBUG_CHECKS) test indices that come from
+// data (mask lists, slot maps, union lists) before they address memory: a
+// failed test sets the bounds flag of the status word and the access is
+// skipped or redirected to index 0. Release builds compile the test to true.
+#ifdef SA_DEBUG_CHECKS
+__device__ __forceinline__ bool dbg_in_range(long long i, long long n, uint32_t* status) {
+  const bool ok = i >= 0 && i < n;
+  if (!ok && status) atomicOr(status, SA_DEVFLAG_BOUNDS);
+  return ok;
+}
+#else
+__device__ __forceinline__ bool dbg_in_range(long long, long long, uint32_t*) { return true; }
+#endif
+
+}  // namespace sa
+
+namespace sa {
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
