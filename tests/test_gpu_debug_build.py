@@ -47,7 +47,7 @@ def debug_lib():
     import sparse_attention_video_b200._native as N
     from sparse_attention_video_b200 import build as B
     if not os.path.exists(B.LIB_DEBUG):
-        pytest.fail(f"{B.LIB_DEBUG} is missing: build it with build.py --debug")
+        B.build(debug=True)                 # nvcc is on every machine the suite runs on
     release = (N.lib(), N.LIB_PATH)
     yield N, B.LIB_DEBUG
     N._LIB, N.LIB_PATH = release
