@@ -292,7 +292,11 @@ SA_API int sparse_attn_permute(const sa_problem* problem, const sa_policy* polic
 
 /* Attention step of the forward pass (the flash-style kernel with online
  * softmax over the kept key blocks or key slices). Frame-major heads read the
- * copies sparse_attn_permute left in scratch_ws. Asynchronous on ``stream``. */
+ * copies sparse_attn_permute left in scratch_ws. Policies that bound a row's
+ * kept blocks (TOPK, STA, SPATIOTEMPORAL) run the one-warpgroup kernel, two
+ * CTAs per SM; SPADE and EXPLICIT masks the two-warpgroup kernel; FG slices
+ * its gather mode. The choice changes speed only: every kernel computes the
+ * same masked softmax attention. Asynchronous on ``stream``. */
 SA_API int sparse_attn_attend(const sa_problem* problem, const sa_policy* policy,
                               const void* q, const void* k, const void* v,
                               const void* mask_ws, void* scratch_ws,
